@@ -1,0 +1,214 @@
+// libkda C ABI: host-side validation, planning and dispatch to the kernels.
+// Every argument error is caught here, before anything is enqueued.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "kda_internal.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+kda_status_t fail(kda_status_t st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+kda_status_t fail(kda_status_t st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+kda_status_t ok() {
+    g_last_error.clear();
+    return KDA_OK;
+}
+
+kda_status_t cuda_fail(cudaError_t e, const char *where) {
+    return fail(KDA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool supported_d(int32_t d) { return d == 32 || d == 64 || d == 128; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr size_t kStatusBytes = 256;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Checks shared by the prefill entry points. On success returns KDA_OK.
+kda_status_t check_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const float *beta, const float *initial_state,
+                           const int32_t *cu_dev, const int32_t *cu_host, int32_t num_seqs,
+                           int64_t total_tokens, int32_t H, int32_t d_k, int32_t d_v,
+                           kda_dtype_t dtype, const void *out, const float *final_state) {
+    if (dtype != KDA_F32 && dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "dtype %d is not KDA_F32 or KDA_BF16", (int)dtype);
+    if (H <= 0 || H > 65535) return fail(KDA_ERR_INVALID_ARGUMENT, "H=%d outside [1, 65535]", H);
+    if (!supported_d(d_k) || !supported_d(d_v))
+        return fail(KDA_ERR_INVALID_ARGUMENT, "d_k=%d, d_v=%d: each must be 32, 64 or 128", d_k, d_v);
+    if (num_seqs < 0) return fail(KDA_ERR_INVALID_ARGUMENT, "num_seqs=%d < 0", num_seqs);
+    if (total_tokens < 0 || total_tokens > INT32_MAX)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "total_tokens=%lld outside [0, 2^31)",
+                    (long long)total_tokens);
+    if (num_seqs == 0) {
+        if (total_tokens != 0)
+            return fail(KDA_ERR_INVALID_ARGUMENT, "num_seqs=0 but total_tokens=%lld",
+                        (long long)total_tokens);
+        return ok();
+    }
+    if (!cu_dev || !cu_host)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "cu_seqlens_dev and cu_seqlens_host are required");
+    if (cu_host[0] != 0) return fail(KDA_ERR_INVALID_ARGUMENT, "cu_seqlens[0]=%d != 0", cu_host[0]);
+    for (int32_t n = 0; n < num_seqs; ++n)
+        if (cu_host[n + 1] < cu_host[n])
+            return fail(KDA_ERR_INVALID_ARGUMENT, "cu_seqlens decreases at %d (%d -> %d)", n,
+                        cu_host[n], cu_host[n + 1]);
+    if ((int64_t)cu_host[num_seqs] != total_tokens)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "cu_seqlens[%d]=%d != total_tokens=%lld", num_seqs,
+                    cu_host[num_seqs], (long long)total_tokens);
+    if (total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !out))
+        return fail(KDA_ERR_INVALID_ARGUMENT, "q, k, v, log_alpha, beta and out are required");
+    const void *ptrs[] = {q, k, v, log_alpha, out, initial_state, final_state};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p))
+            return fail(KDA_ERR_INVALID_ARGUMENT, "tensor pointer %p is not 16-byte aligned", p);
+    if (out && (out == q || out == k || out == v))
+        return fail(KDA_ERR_INVALID_ARGUMENT, "out must not alias q, k or v");
+    return ok();
+}
+
+kda::Problem make_problem(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, const float *initial_state, const int32_t *cu_dev,
+                          int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
+                          int32_t d_v, kda_dtype_t dtype, void *out, float *final_state) {
+    kda::Problem p;
+    p.q = q; p.k = k; p.v = v;
+    p.log_alpha = log_alpha; p.beta = beta;
+    p.initial_state = initial_state;
+    p.cu_seqlens = cu_dev;
+    p.num_seqs = num_seqs; p.total_tokens = total_tokens;
+    p.H = H; p.dk = d_k; p.dv = d_v; p.dtype = dtype;
+    p.out = out; p.final_state = final_state;
+    return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
+                                  int32_t d_v, kda_dtype_t dtype) {
+    if (num_seqs < 0 || total_tokens < 0 || H <= 0 || !supported_d(d_k) || !supported_d(d_v) ||
+        (dtype != KDA_F32 && dtype != KDA_BF16))
+        return 0;
+    // [0, 256): device status word; then the per-sequence schedule (int32 each).
+    return kStatusBytes + round_up((size_t)num_seqs * sizeof(int32_t), 256);
+}
+
+kda_status_t kda_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
+                         const float *beta, const float *initial_state,
+                         const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                         int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
+                         int32_t d_v, kda_dtype_t dtype, void *out, float *final_state,
+                         void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+    kda_status_t st = check_prefill(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev,
+                                    cu_seqlens_host, num_seqs, total_tokens, H, d_k, d_v, dtype,
+                                    out, final_state);
+    if (st != KDA_OK || num_seqs == 0) return st;
+    const size_t need = kda_prefill_workspace_size(num_seqs, total_tokens, H, d_k, d_v, dtype);
+    if (!workspace || workspace_bytes < need)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "workspace %p of %zu bytes < required %zu",
+                    workspace, workspace_bytes, need);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "workspace is not 256-byte aligned");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_prefill: clearing the status word");
+    kda::Problem p = make_problem(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev,
+                                  num_seqs, total_tokens, H, d_k, d_v, dtype, out, final_state);
+    e = kda::launch_prefill_recurrent(p, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_prefill: launch");
+    return ok();
+}
+
+kda_status_t kda_prefill_recurrent(const void *q, const void *k, const void *v,
+                                   const float *log_alpha, const float *beta,
+                                   const float *initial_state, const int32_t *cu_seqlens_dev,
+                                   const int32_t *cu_seqlens_host, int32_t num_seqs,
+                                   int64_t total_tokens, int32_t H, int32_t d_k, int32_t d_v,
+                                   kda_dtype_t dtype, void *out, float *final_state,
+                                   kda_stream_t stream) {
+    kda_status_t st = check_prefill(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev,
+                                    cu_seqlens_host, num_seqs, total_tokens, H, d_k, d_v, dtype,
+                                    out, final_state);
+    if (st != KDA_OK || num_seqs == 0) return st;
+    kda::Problem p = make_problem(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev,
+                                  num_seqs, total_tokens, H, d_k, d_v, dtype, out, final_state);
+    cudaError_t e = kda::launch_prefill_recurrent(p, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kda_prefill_recurrent: launch");
+    return ok();
+}
+
+kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                             const float *beta, float *state, int32_t num_seqs, int32_t H,
+                             int32_t d_k, int32_t d_v, kda_dtype_t dtype, void *out,
+                             void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+    (void)workspace;
+    (void)workspace_bytes;
+    if (dtype != KDA_F32 && dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "dtype %d is not KDA_F32 or KDA_BF16", (int)dtype);
+    if (H <= 0) return fail(KDA_ERR_INVALID_ARGUMENT, "H=%d <= 0", H);
+    if (!supported_d(d_k) || !supported_d(d_v))
+        return fail(KDA_ERR_INVALID_ARGUMENT, "d_k=%d, d_v=%d: each must be 32, 64 or 128", d_k, d_v);
+    if (num_seqs < 0) return fail(KDA_ERR_INVALID_ARGUMENT, "num_seqs=%d < 0", num_seqs);
+    if ((int64_t)num_seqs * H > INT32_MAX)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "num_seqs * H exceeds 2^31 - 1");
+    if (num_seqs == 0) return ok();
+    if (!q || !k || !v || !log_alpha || !beta || !state || !out)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "q, k, v, log_alpha, beta, state and out are required");
+    const void *ptrs[] = {q, k, v, log_alpha, state, out};
+    for (const void *p : ptrs)
+        if (!aligned16(p))
+            return fail(KDA_ERR_INVALID_ARGUMENT, "tensor pointer %p is not 16-byte aligned", p);
+    if (out == q || out == k || out == v || out == (void *)state)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "out must not alias an input or the state");
+    kda::DecodeProblem p;
+    p.q = q; p.k = k; p.v = v; p.log_alpha = log_alpha; p.beta = beta; p.state = state;
+    p.num_seqs = num_seqs; p.H = H; p.dk = d_k; p.dv = d_v; p.dtype = dtype; p.out = out;
+    cudaError_t e = kda::launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step: launch");
+    return ok();
+}
+
+const char *kda_status_string(kda_status_t s) {
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARGUMENT: return "KDA_ERR_INVALID_ARGUMENT";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+const char *kda_last_error(void) { return g_last_error.c_str(); }
+
+kda_status_t kda_read_device_status(const void *workspace, kda_stream_t stream) {
+    if (!workspace) return fail(KDA_ERR_INVALID_ARGUMENT, "workspace is NULL");
+    int32_t word = 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof word, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_read_device_status");
+    if (word == 0) return ok();
+    return fail(KDA_ERR_TIMEOUT, "device status word 0x%x: a bounded on-device wait gave up",
+                (unsigned)word);
+}
+
+int32_t kda_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,49 @@
+// Internal declarations shared by the libkda translation units (not part of the ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+// ---- element access for the two input dtypes -------------------------------------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// ---- problem description passed from the API layer to the launchers --------------------
+struct Problem {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta;
+    const float *initial_state;
+    const int32_t *cu_seqlens;  // device
+    int32_t num_seqs;
+    int64_t total_tokens;
+    int32_t H, dk, dv;
+    kda_dtype_t dtype;
+    void *out;
+    float *final_state;
+};
+
+// Each launcher enqueues its kernel(s) on `stream` and returns the launch's cudaError_t.
+cudaError_t launch_prefill_recurrent(const Problem &p, cudaStream_t stream);
+
+struct DecodeProblem {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta;
+    float *state;
+    int32_t num_seqs, H, dk, dv;
+    kda_dtype_t dtype;
+    void *out;
+};
+cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream);
+
+}  // namespace kda

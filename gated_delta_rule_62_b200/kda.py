@@ -1,0 +1,207 @@
+"""ctypes binding of libkda (argument marshalling only; every step runs in the CUDA library).
+
+PyTorch provides device memory and the current CUDA stream. There is no CPU
+fallback: if ``libkda.so`` is missing or fails to load, every call raises.
+
+Layouts follow ``include/kda.h``: q, k, log_alpha [T, H, d_k]; v, out [T, H, d_v];
+beta [T, H]; states [N, H, d_k, d_v] fp32; cu_seqlens [N + 1] int32. Dense
+[B, T, ...] inputs are accepted and packed as B sequences of T tokens.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_OK, KDA_ERR_INVALID_ARGUMENT, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
+KDA_F32, KDA_BF16 = 0, 1
+
+_lock = threading.Lock()
+_lib = None
+
+_vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+
+SIGNATURES = {
+    "kda_prefill_workspace_size": (_sz, [_i32, _i64, _i32, _i32, _i32, _i32]),
+    "kda_prefill": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
+                           _i32, _vp, _vp, _vp, _sz, _vp]),
+    "kda_prefill_recurrent": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32,
+                                     _i32, _i32, _i32, _vp, _vp, _vp]),
+    "kda_decode_step": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp,
+                               _vp, _sz, _vp]),
+    "kda_status_string": (ctypes.c_char_p, [_i32]),
+    "kda_last_error": (ctypes.c_char_p, []),
+    "kda_read_device_status": (_i32, [_vp, _vp]),
+    "kda_version": (_i32, []),
+}
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        super().__init__(message)
+
+
+def lib():
+    """Load libkda.so (raises if it is missing: there is no fallback path)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} not built; run python -m gated_delta_rule_62_b200.build")
+            L = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(L, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = L
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != KDA_OK:
+        L = lib()
+        name = L.kda_status_string(status).decode()
+        msg = L.kda_last_error().decode()
+        raise KdaError(status, f"{what}: {name}: {msg}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return KDA_BF16
+    if dt == torch.float32:
+        return KDA_F32
+    raise TypeError(f"unsupported input dtype {dt}; use bfloat16 or float32")
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, ndim=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+
+
+def workspace_size(num_seqs: int, total_tokens: int, H: int, dk: int, dv: int, dtype) -> int:
+    return int(lib().kda_prefill_workspace_size(num_seqs, total_tokens, H, dk, dv,
+                                                _dtype_code(dtype)))
+
+
+def prefill(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, cu_seqlens_dev=None,
+            out=None, final_state=None, workspace=None, output_final_state=True,
+            algo: str = "auto", stream=None):
+    """Chunked KDA prefill over packed sequences (``kda_prefill``).
+
+    q, k, log_alpha: [T, H, d_k] (or [B, T, H, d_k]); v: [T, H, d_v]; beta [T, H].
+    cu_seqlens: host int32 offsets [N + 1] (default: one sequence, or B equal ones
+    for 4-D inputs); cu_seqlens_dev: the same on the device (copied if omitted).
+    algo: "auto" (``kda_prefill``) or "recurrent" (``kda_prefill_recurrent``).
+    Returns (out, final_state or None).
+    """
+    dense = q.dim() == 4
+    if dense:
+        B, T = q.shape[:2]
+        q, k, v = q.reshape(B * T, *q.shape[2:]), k.reshape(B * T, *k.shape[2:]), v.reshape(B * T, *v.shape[2:])
+        log_alpha = log_alpha.reshape(B * T, *log_alpha.shape[2:])
+        beta = beta.reshape(B * T, *beta.shape[2:])
+        if cu_seqlens is None:
+            cu_seqlens = torch.arange(0, (B + 1) * T, T, dtype=torch.int32)
+    dtype = q.dtype
+    _need(q, "q", ndim=3)
+    Ttot, H, dk = q.shape
+    dv = v.shape[-1]
+    _need(k, "k", dtype, 3)
+    _need(v, "v", dtype, 3)
+    _need(log_alpha, "log_alpha", torch.float32, 3)
+    _need(beta, "beta", torch.float32, 2)
+    if k.shape != q.shape or log_alpha.shape != q.shape or v.shape[:2] != (Ttot, H) or beta.shape != (Ttot, H):
+        raise ValueError("inconsistent shapes among q, k, v, log_alpha, beta")
+    if cu_seqlens is None:
+        cu_seqlens = torch.tensor([0, Ttot], dtype=torch.int32)
+    cu_host = torch.as_tensor(cu_seqlens, dtype=torch.int32).cpu().contiguous()
+    N = cu_host.numel() - 1
+    if cu_seqlens_dev is None:
+        cu_seqlens_dev = cu_host.to(q.device, non_blocking=False)
+    _need(cu_seqlens_dev, "cu_seqlens_dev", torch.int32, 1)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", torch.float32, 4)
+        if tuple(initial_state.shape) != (N, H, dk, dv):
+            raise ValueError(f"initial_state must be {(N, H, dk, dv)}")
+    if out is None:
+        out = torch.empty(Ttot, H, dv, dtype=dtype, device=q.device)
+    _need(out, "out", dtype, 3)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+    if final_state is not None:
+        _need(final_state, "final_state", torch.float32, 4)
+    L = lib()
+    code = _dtype_code(dtype)
+    common = [_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
+              _ptr(cu_seqlens_dev), ctypes.c_void_p(cu_host.data_ptr()), N, Ttot, H, dk, dv, code,
+              _ptr(out), _ptr(final_state)]
+    if algo == "recurrent":
+        _check(L.kda_prefill_recurrent(*common, _stream(stream)), "kda_prefill_recurrent")
+    elif algo == "auto":
+        need = workspace_size(N, Ttot, H, dk, dv, dtype)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _need(workspace, "workspace", torch.uint8, 1)
+        _check(L.kda_prefill(*common, _ptr(workspace), workspace.numel(), _stream(stream)),
+               "kda_prefill")
+    else:
+        raise ValueError(f"unknown algo {algo!r}")
+    if dense:
+        out = out.reshape(B, T, H, dv)
+    return out, final_state
+
+
+def decode_step(q, k, v, log_alpha, beta, state, out=None, stream=None):
+    """One decode token per sequence (``kda_decode_step``); ``state`` is updated in place.
+
+    q, k, log_alpha: [N, H, d_k]; v: [N, H, d_v]; beta: [N, H]; state [N, H, d_k, d_v] fp32.
+    Returns out [N, H, d_v].
+    """
+    dtype = q.dtype
+    _need(q, "q", ndim=3)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    _need(k, "k", dtype, 3)
+    _need(v, "v", dtype, 3)
+    _need(log_alpha, "log_alpha", torch.float32, 3)
+    _need(beta, "beta", torch.float32, 2)
+    _need(state, "state", torch.float32, 4)
+    if k.shape != q.shape or log_alpha.shape != q.shape or tuple(state.shape) != (N, H, dk, dv):
+        raise ValueError("inconsistent shapes among q, k, log_alpha, state")
+    if out is None:
+        out = torch.empty(N, H, dv, dtype=dtype, device=q.device)
+    _need(out, "out", dtype, 3)
+    _check(lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                 _ptr(state), N, H, dk, dv, _dtype_code(dtype), _ptr(out), None, 0,
+                                 _stream(stream)), "kda_decode_step")
+    return out
+
+
+def read_device_status(workspace, stream=None) -> int:
+    """Status word of the last kda_prefill that used ``workspace`` (synchronises the stream)."""
+    st = lib().kda_read_device_status(_ptr(workspace), _stream(stream))
+    return int(st)

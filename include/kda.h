@@ -1,0 +1,181 @@
+/*
+ * kda.h -- C ABI of libkda: the Kimi Delta Attention (KDA) recurrence on B200 (sm_100a).
+ *
+ * The operation (per sequence n and head h; state S is d_k x d_v fp32, row c =
+ * key channel, column j = value channel), for each token t in order:
+ *
+ *     S   <- Diag(alpha_t) S,            alpha_t = exp(log_alpha_t), one gate per key channel
+ *     S   <- S + beta_t k_t (v_t - S^T k_t)^T                   (delta rule: write only the error)
+ *     o_t  = S^T q_t                                             (read after the write)
+ *
+ * Sources: "Kimi K3 -- the architecture and infrastructure, explained"
+ * (shivam2003.com), sections "How the delta rule actually works" (the update
+ * S <- S - beta (S k - v) k^T, written there for the transposed d_v x d_k
+ * state) and "Kimi Delta Attention: the load-bearing choice" (channel-wise
+ * gating; blockwise computation that maps onto matrix units; constant per-token
+ * decode cost); aitrending.vip "Inside Kimi K3", section "Technical Details"
+ * (beta = writing strength, alpha = forgetting factor, 128 dials per head);
+ * same shivam2003.com article, section "Serving infrastructure: supernodes and
+ * the prefill cache" (a cached prefill state is restored so a returning request
+ * only pays for the new suffix: initial/final state I/O).
+ *
+ * Conventions shared by every entry point
+ *   - Device pointers unless a name ends in _host. All tensors are dense and
+ *     row-major with the last dimension contiguous, 16-byte aligned base.
+ *   - q, k: [T, H, d_k]; v, out: [T, H, d_v] in the input dtype (fp32 or bf16).
+ *     log_alpha: [T, H, d_k] fp32 (must be <= 0); beta: [T, H] fp32 (in [0, 1]);
+ *     states: [N, H, d_k, d_v] fp32. q and k are used as given (the caller
+ *     normalises them; no 1/sqrt(d_k) scale is applied).
+ *   - Ownership: the caller allocates and frees every buffer, including the
+ *     workspace. The library does not allocate, free or synchronise inside
+ *     kda_prefill / kda_decode_step: both only enqueue work on `stream` and
+ *     return. Buffers must stay valid until the stream has run the work.
+ *   - Aliasing: final_state may alias initial_state (in-place resume); the
+ *     decode state is updated in place; out must not alias any input.
+ *   - Errors: arguments are checked on the host before anything is enqueued;
+ *     a non-OK status means nothing was enqueued (except KDA_ERR_CUDA, which
+ *     reports a failed launch). kda_last_error() returns a message for the
+ *     calling thread's last non-OK status. No C++ exception crosses this ABI.
+ *   - Values are not checked on the device: inputs must be finite, log_alpha <= 0
+ *     and beta in [0, 1]; otherwise results are unspecified (but memory-safe).
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *kda_stream_t;
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARGUMENT = 1, /* bad pointer, size, shape, or cu_seqlens            */
+    KDA_ERR_UNSUPPORTED = 2,      /* a dtype / head-size combination with no kernel       */
+    KDA_ERR_CUDA = 3,             /* a CUDA runtime call or launch failed                 */
+    KDA_ERR_TIMEOUT = 4           /* a bounded on-device wait gave up (device status word) */
+} kda_status_t;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
+
+/* Supported head sizes: d_k, d_v in {32, 64, 128}. */
+
+/*
+ * Bytes of device workspace kda_prefill needs for this problem (>= 256; a
+ * multiple of 256). Pure host function; never fails (returns 0 only for
+ * arguments kda_prefill would reject).
+ */
+KDA_API size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H,
+                                  int32_t d_k, int32_t d_v, kda_dtype_t dtype);
+
+/*
+ * Chunked prefill over packed variable-length sequences.
+ *
+ *   q, k        [total_tokens, H, d_k]  dtype
+ *   v           [total_tokens, H, d_v]  dtype
+ *   log_alpha   [total_tokens, H, d_k]  fp32
+ *   beta        [total_tokens, H]       fp32
+ *   initial_state [num_seqs, H, d_k, d_v] fp32, or NULL for a zero start
+ *   cu_seqlens_dev  [num_seqs + 1] int32 device copy of the token offsets
+ *   cu_seqlens_host [num_seqs + 1] int32 host copy of the same offsets (read
+ *                   during the call only; used to validate and plan)
+ *   out         [total_tokens, H, d_v]  dtype  (written)
+ *   final_state [num_seqs, H, d_k, d_v] fp32, or NULL if not wanted (written;
+ *               may alias initial_state)
+ *   workspace   >= kda_prefill_workspace_size(...) bytes of device memory,
+ *               256-byte aligned; contents on entry are ignored.
+ *
+ * cu_seqlens must start at 0, be non-decreasing and end at total_tokens.
+ * Zero-length sequences are allowed (their final state is their initial state).
+ * A dense [B, T] batch is cu_seqlens = {0, T, 2T, ..., B*T}.
+ *
+ * Tokens are processed in chunks of 64 per sequence: bf16 inputs with
+ * d_k = d_v = 128 run on the tensor-core chunk kernel; every other supported
+ * combination runs the token-serial fp32 kernel (see kda_prefill_recurrent).
+ * The result does not depend on that choice beyond rounding.
+ *
+ * Status: KDA_ERR_INVALID_ARGUMENT for a NULL required pointer, H <= 0,
+ * num_seqs < 0, an unsupported d_k/d_v, bad cu_seqlens_host, or a workspace
+ * smaller than required; KDA_ERR_CUDA if a launch fails.
+ */
+KDA_API kda_status_t kda_prefill(const void *q, const void *k, const void *v,
+                         const float *log_alpha, const float *beta,
+                         const float *initial_state,
+                         const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                         int32_t num_seqs, int64_t total_tokens, int32_t H,
+                         int32_t d_k, int32_t d_v, kda_dtype_t dtype,
+                         void *out, float *final_state,
+                         void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * The same operation as kda_prefill, always on the token-serial kernel: one
+ * thread block per (sequence, head, 32-wide slice of d_v) walks the tokens in
+ * order with the state slice in registers and fp32 arithmetic throughout. It
+ * needs no workspace. Arguments and status as kda_prefill.
+ */
+KDA_API kda_status_t kda_prefill_recurrent(const void *q, const void *k, const void *v,
+                                   const float *log_alpha, const float *beta,
+                                   const float *initial_state,
+                                   const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                                   int32_t num_seqs, int64_t total_tokens, int32_t H,
+                                   int32_t d_k, int32_t d_v, kda_dtype_t dtype,
+                                   void *out, float *final_state, kda_stream_t stream);
+
+/*
+ * One decode step: one new token for each of num_seqs sequences, state updated
+ * in place (constant cost per token: the state of each head is read once and
+ * written once).
+ *
+ *   q, k        [num_seqs, H, d_k]  dtype
+ *   v           [num_seqs, H, d_v]  dtype
+ *   log_alpha   [num_seqs, H, d_k]  fp32
+ *   beta        [num_seqs, H]       fp32
+ *   state       [num_seqs, H, d_k, d_v] fp32, read and written in place
+ *   out         [num_seqs, H, d_v]  dtype (written)
+ *   workspace   may be NULL with workspace_bytes == 0 (the decode kernel has no
+ *               on-device waits and needs no scratch); reserved for future use.
+ *
+ * Status: KDA_ERR_INVALID_ARGUMENT for a NULL required pointer, num_seqs < 0,
+ * H <= 0 or unsupported head sizes; KDA_ERR_CUDA if the launch fails.
+ * num_seqs == 0 is a no-op.
+ */
+KDA_API kda_status_t kda_decode_step(const void *q, const void *k, const void *v,
+                             const float *log_alpha, const float *beta,
+                             float *state, int32_t num_seqs, int32_t H,
+                             int32_t d_k, int32_t d_v, kda_dtype_t dtype,
+                             void *out, void *workspace, size_t workspace_bytes,
+                             kda_stream_t stream);
+
+/* Static string naming a status code. Never NULL. */
+KDA_API const char *kda_status_string(kda_status_t status);
+
+/* Message for the calling thread's last non-OK status ("" if none). The
+ * pointer stays valid until the thread's next call into the library. */
+KDA_API const char *kda_last_error(void);
+
+/*
+ * Reads the device status word that kda_prefill keeps at the start of its
+ * workspace: KDA_OK, or KDA_ERR_TIMEOUT if a bounded on-device wait of the
+ * last prefill that used this workspace gave up (its outputs are then
+ * invalid). Synchronises `stream` (this is the only call that does).
+ */
+KDA_API kda_status_t kda_read_device_status(const void *workspace, kda_stream_t stream);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+KDA_API int32_t kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,125 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad arguments
+on the host before any CUDA call (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from gated_delta_rule_62_b200 import kda as K
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"KDA_API\s+[\w\s\*]+?\b(kda_\w+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_symbols()
+    for must in ["kda_prefill", "kda_prefill_workspace_size", "kda_decode_step", "kda_status_string",
+                 "kda_last_error", "kda_read_device_status"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(K.LIB_PATH)
+    missing = [n for n in declared_symbols() if not hasattr(L, n)]
+    assert not missing, missing
+    # and the binding knows every one of them
+    assert set(declared_symbols()) <= set(K.SIGNATURES)
+
+
+def test_status_strings():
+    L = K.lib()
+    assert L.kda_status_string(0) == b"KDA_OK"
+    assert L.kda_status_string(4) == b"KDA_ERR_TIMEOUT"
+    assert L.kda_status_string(99) == b"KDA_ERR_UNKNOWN"
+    assert L.kda_version() >= 100
+
+
+def test_workspace_size():
+    assert K.workspace_size(1, 64, 2, 32, 32, torch.float32) >= 256
+    assert K.workspace_size(24, 10**6, 32, 128, 128, torch.bfloat16) % 256 == 0
+    L = K.lib()
+    assert L.kda_prefill_workspace_size(1, 10, 2, 48, 32, 0) == 0  # unsupported d_k
+    assert L.kda_prefill_workspace_size(1, 10, 0, 32, 32, 0) == 0
+
+
+def _prefill_raw(**over):
+    """Call kda_prefill with fake (never dereferenced) pointers; validation fails first."""
+    L = K.lib()
+    cu = (ctypes.c_int32 * 3)(*over.pop("cu", [0, 5, 9]))
+    fake = ctypes.c_void_p(0x10000)
+    a = dict(q=fake, k=fake, v=fake, la=fake, beta=fake, s0=None, cud=fake, cuh=cu, N=2, T=9, H=2,
+             dk=32, dv=32, dt=0, out=ctypes.c_void_p(0x20000), fs=None, ws=None, wsb=0, st=None)
+    a.update(over)
+    rc = L.kda_prefill(a["q"], a["k"], a["v"], a["la"], a["beta"], a["s0"], a["cud"],
+                       ctypes.cast(a["cuh"], ctypes.c_void_p), a["N"], a["T"], a["H"], a["dk"],
+                       a["dv"], a["dt"], a["out"], a["fs"], a["ws"], a["wsb"], a["st"])
+    return rc, L.kda_last_error().decode()
+
+
+@pytest.mark.parametrize("over,needle", [
+    (dict(H=0), "H=0"),
+    (dict(dk=48), "d_k=48"),
+    (dict(dv=256), "d_v=256"),
+    (dict(dt=7), "dtype"),
+    (dict(N=-1), "num_seqs"),
+    (dict(cu=[1, 5, 9]), "cu_seqlens[0]"),
+    (dict(cu=[0, 5, 4], T=4), "decreases"),
+    (dict(T=10), "total_tokens"),
+    (dict(q=None), "required"),
+    (dict(cud=None), "cu_seqlens_dev"),
+    (dict(q=ctypes.c_void_p(0x10004)), "16-byte"),
+    (dict(out=ctypes.c_void_p(0x10000)), "alias"),
+    (dict(), "workspace"),  # all else valid: the missing workspace is reported
+    (dict(ws=ctypes.c_void_p(0x30000), wsb=16), "workspace"),
+    (dict(ws=ctypes.c_void_p(0x30010), wsb=1 << 20), "256-byte"),
+])
+def test_prefill_rejects_bad_arguments(over, needle):
+    rc, msg = _prefill_raw(**over)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT
+    assert needle in msg, msg
+
+
+def test_decode_rejects_bad_arguments():
+    L = K.lib()
+    fake = ctypes.c_void_p(0x10000)
+    rc = L.kda_decode_step(fake, fake, fake, fake, fake, fake, 4, 2, 64, 100, 1,
+                           ctypes.c_void_p(0x20000), None, 0, None)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and b"d_v=100" in L.kda_last_error()
+    rc = L.kda_decode_step(fake, fake, fake, fake, fake, None, 4, 2, 64, 64, 1,
+                           ctypes.c_void_p(0x20000), None, 0, None)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and b"required" in L.kda_last_error()
+    # zero sequences: a no-op that needs no pointers
+    assert L.kda_decode_step(None, None, None, None, None, None, 0, 2, 64, 64, 1, None, None, 0,
+                             None) == K.KDA_OK
+
+
+def test_zero_sequences_is_a_noop():
+    L = K.lib()
+    rc = L.kda_prefill(None, None, None, None, None, None, None, None, 0, 0, 4, 128, 128, 1, None,
+                       None, None, 0, None)
+    assert rc == K.KDA_OK
+
+
+def test_binding_requires_cuda_tensors():
+    x = torch.zeros(4, 2, 32)
+    with pytest.raises(ValueError, match="CUDA"):
+        K.prefill(x, x, x, x, torch.zeros(4, 2))
+
+
+def test_product_path_does_not_import_oracle():
+    """The library binding and package never import the oracle (no CPU fallback)."""
+    pkg = os.path.join(ROOT, "gated_delta_rule_62_b200")
+    for fn in os.listdir(pkg):
+        if fn.endswith(".py"):
+            src = open(os.path.join(pkg, fn)).read()
+            assert not re.search(r"^\s*(from|import)\s+oracle", src, re.M), fn

@@ -1,0 +1,74 @@
+"""Decode step on the GPU vs the fp64 oracle (a decode step is a one-token prefill)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_62_b200 import kda as K
+from gated_delta_rule_62_b200 import workloads as W
+from tests.gpu_helpers import TOL, assert_close, f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from gated_delta_rule_62_b200 import build
+    build.build()
+    oracle.build()
+
+
+def _oracle_step(d, s):
+    N = d["q"].shape[0]
+    cu = np.arange(N + 1, dtype=np.int64)
+    s = f64(s) if isinstance(s, torch.Tensor) else np.asarray(s, dtype=np.float64)
+    return oracle.forward(f64(d["q"]), f64(d["k"]), f64(d["v"]), f64(d["log_alpha"]), f64(d["beta"]),
+                          s, cu)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(32, 32), (64, 64), (128, 128), (32, 128), (128, 64), (64, 32)])
+def test_decode_steps(dtype, dk, dv):
+    wl = W.custom((1,) * 5, 3, dk, dv, dtype, seed=dk + 3 * dv)
+    g = torch.Generator(device=DEV).manual_seed(17)
+    state = torch.randn(5, 3, dk, dv, device=DEV, generator=g)
+    steps = W.make_decode_steps(wl, g, 4, DEV)
+    ref_s = f64(state)
+    for t in range(4):
+        d = {n: steps[n][t] for n in steps}
+        out = K.decode_step(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], state)
+        ro, ref_s = _oracle_step(d, ref_s)
+        scale = float(d["v"].abs().max())
+        assert_close(out, ro, TOL[dtype], scale, f"decode out step {t}")
+        assert_close(state, ref_s, TOL[dtype], scale, f"decode state step {t}")
+        ref_s = f64(state)  # continue from the GPU state (no drift across steps)
+
+
+def test_decode_equals_one_token_prefill():
+    wl = W.custom((1,) * 7, 4, 128, 128, "bf16", seed=21, init_state="normal")
+    inp = W.make_inputs(wl, DEV)
+    s = inp["initial_state"].clone()
+    out_d = K.decode_step(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], s)
+    out_p, fs = K.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                          inp["initial_state"], inp["cu_seqlens"], inp["cu_seqlens_dev"])
+    assert torch.allclose(out_d.float(), out_p.float(), atol=2e-2, rtol=0)
+    assert torch.allclose(s, fs, atol=1e-4, rtol=0)
+
+
+def test_decode_256_sequences_from_prefill_state():
+    """The 256-sequence, 32-head decode workload: state seeded by a 512-token GPU prefill, then
+    decode steps checked against the oracle started from the GPU's seeded state."""
+    wl = W.DECODE_256
+    inp = W.make_inputs(wl, DEV)
+    _, state = K.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], None,
+                         inp["cu_seqlens"], inp["cu_seqlens_dev"])
+    steps = W.make_decode_steps(wl, inp["_gen"], 3, DEV)
+    ref_s = f64(state)
+    for t in range(3):
+        d = {n: steps[n][t] for n in steps}
+        out = K.decode_step(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], state)
+        ro, ref_s = _oracle_step(d, ref_s)
+        scale = float(d["v"].abs().max())
+        assert_close(out, ro, TOL["bf16"], scale, f"decode256 out step {t}")
+        assert_close(state, ref_s, TOL["bf16"], scale, f"decode256 state step {t}")
