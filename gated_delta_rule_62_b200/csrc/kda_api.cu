@@ -106,7 +106,7 @@ size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_
         (dtype != KDA_F32 && dtype != KDA_BF16))
         return 0;
     // [0, 256): device status word; then the per-sequence schedule (int32 each).
-    return kStatusBytes + round_up((size_t)num_seqs * sizeof(int32_t), 256);
+    return kda::chunk_workspace_bytes(num_seqs);
 }
 
 kda_status_t kda_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -126,11 +126,16 @@ kda_status_t kda_prefill(const void *q, const void *k, const void *v, const floa
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(KDA_ERR_INVALID_ARGUMENT, "workspace is not 256-byte aligned");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
-    if (e != cudaSuccess) return cuda_fail(e, "kda_prefill: clearing the status word");
     kda::Problem p = make_problem(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev,
                                   num_seqs, total_tokens, H, d_k, d_v, dtype, out, final_state);
-    e = kda::launch_prefill_recurrent(p, s);
+    cudaError_t e;
+    if (kda::chunk_supported(p)) {
+        // the planning kernel clears the status word
+        e = kda::launch_prefill_chunk(p, workspace, s, kda::kWaitTimeoutNs);
+    } else {
+        e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
+        if (e == cudaSuccess) e = kda::launch_prefill_recurrent(p, s);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "kda_prefill: launch");
     return ok();
 }
@@ -207,6 +212,20 @@ kda_status_t kda_read_device_status(const void *workspace, kda_stream_t stream) 
     if (word == 0) return ok();
     return fail(KDA_ERR_TIMEOUT, "device status word 0x%x: a bounded on-device wait gave up",
                 (unsigned)word);
+}
+
+kda_status_t kda_selftest_bounded_wait(void *workspace, size_t workspace_bytes,
+                                       uint64_t timeout_ns, kda_stream_t stream) {
+    if (!workspace || workspace_bytes < kStatusBytes)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "workspace of at least %zu bytes is required",
+                    kStatusBytes);
+    if (timeout_ns == 0 || timeout_ns > 10000000000ull)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "timeout_ns must be in (0, 1e10]");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
+    if (e == cudaSuccess) e = kda::launch_bounded_wait_probe(workspace, timeout_ns, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_selftest_bounded_wait: launch");
+    return ok();
 }
 
 int32_t kda_version(void) { return 100; }

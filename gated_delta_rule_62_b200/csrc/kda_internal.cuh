@@ -36,6 +36,17 @@ struct Problem {
 // Each launcher enqueues its kernel(s) on `stream` and returns the launch's cudaError_t.
 cudaError_t launch_prefill_recurrent(const Problem &p, cudaStream_t stream);
 
+// Tensor-core chunk kernel: bf16 inputs with d_k = d_v = 128 and at least one token.
+bool chunk_supported(const Problem &p);
+size_t chunk_workspace_bytes(int32_t num_seqs);
+// workspace: [0, 256) status word, then the longest-first sequence order (int32 each).
+cudaError_t launch_prefill_chunk(const Problem &p, void *workspace, cudaStream_t stream,
+                                 uint64_t timeout_ns);
+cudaError_t launch_bounded_wait_probe(void *workspace, uint64_t timeout_ns, cudaStream_t stream);
+
+// Upper bound on any single on-device wait before a kernel gives up (ns).
+constexpr uint64_t kWaitTimeoutNs = 4000000000ull;
+
 struct DecodeProblem {
     const void *q, *k, *v;
     const float *log_alpha, *beta;

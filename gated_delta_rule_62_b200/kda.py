@@ -39,6 +39,7 @@ SIGNATURES = {
     "kda_last_error": (ctypes.c_char_p, []),
     "kda_read_device_status": (_i32, [_vp, _vp]),
     "kda_version": (_i32, []),
+    "kda_selftest_bounded_wait": (_i32, [_vp, _sz, ctypes.c_uint64, _vp]),
 }
 
 
@@ -199,6 +200,12 @@ def decode_step(q, k, v, log_alpha, beta, state, out=None, stream=None):
                                  _ptr(state), N, H, dk, dv, _dtype_code(dtype), _ptr(out), None, 0,
                                  _stream(stream)), "kda_decode_step")
     return out
+
+
+def selftest_bounded_wait(workspace, timeout_ns: int, stream=None):
+    """Launch the bounded-wait probe (a wait nothing releases); see kda.h."""
+    _check(lib().kda_selftest_bounded_wait(_ptr(workspace), workspace.numel(), int(timeout_ns),
+                                           _stream(stream)), "kda_selftest_bounded_wait")
 
 
 def read_device_status(workspace, stream=None) -> int:

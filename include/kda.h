@@ -171,6 +171,17 @@ KDA_API const char *kda_last_error(void);
  */
 KDA_API kda_status_t kda_read_device_status(const void *workspace, kda_stream_t stream);
 
+/*
+ * Diagnostic: launches a one-block kernel that waits on an on-device barrier
+ * nothing will ever release, using the same bounded wait as the prefill
+ * kernels, so callers can check that a stuck wait ends by itself: after
+ * timeout_ns (in (0, 1e10]) the kernel records KDA_ERR_TIMEOUT in the status
+ * word at the start of `workspace` (>= 256 bytes) and exits, leaving the
+ * context usable; kda_read_device_status then reports KDA_ERR_TIMEOUT.
+ */
+KDA_API kda_status_t kda_selftest_bounded_wait(void *workspace, size_t workspace_bytes,
+                                               uint64_t timeout_ns, kda_stream_t stream);
+
 /* Library version: major * 10000 + minor * 100 + patch. */
 KDA_API int32_t kda_version(void);
 
