@@ -317,11 +317,13 @@ def run_ours(args, rank, local, ws):
         host_out.copy_(out, non_blocking=True)
         host_fs.copy_(fs, non_blocking=True)
 
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier(ws)
-    e2e_ms = max_over_ranks(time_events(e2e_step, max(3, args.steps // 2), stream), ws)
+    e2e_ms = None
+    if not args.no_e2e:
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(ws)
+        e2e_ms = max_over_ranks(time_events(e2e_step, max(3, args.steps // 2), stream), ws)
     del host, dev
 
     dec = bench_decode(args, K, stream, ws) if not args.no_decode else None
@@ -347,8 +349,9 @@ def run_ours(args, rank, local, ws):
                      "frac": gbs / pk["hbm_gbs"], "traffic": args.traffic,
                      "bytes_per_token_head": PREFILL_BYTES_PER_TOKEN_HEAD,
                      "kernel_ms": kern_ms, "peak_source": pk["source"]},
-        "e2e": {"value": T * ws / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "e2e": None if e2e_ms is None else {
+            "value": T * ws / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "decode": dec,
         "gpu_launches": args.steps * kernels_per_step,
         "clocks": clocks,
@@ -366,6 +369,7 @@ def main():
     ap.add_argument("--workload", default=W.PREFILL_8K.name, choices=sorted(W.WORKLOADS))
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-tokens", type=int, default=2048)
