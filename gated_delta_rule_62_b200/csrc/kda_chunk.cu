@@ -296,10 +296,12 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const float gC = s_psum[c] + s_psum[D + c];
         if (hf == 0) {
             s_gamma[c] = __expf(gC);
-            atomicMax(&s_flags[1], __float_as_uint(-gC));
+            // Any channel decaying by more than e^kFastLimit sends the chunk down the exact path.
+            // (Also taken for non-finite gates: the comparison below is false for NaN.)
+            if (!(-gC <= kFastLimit)) s_flags[1] = 1u;
         }
         __syncthreads();
-        const bool safe = __uint_as_float(s_flags[1]) > kFastLimit;
+        const bool safe = s_flags[1] != 0u;
 
         if (safe) {
             // Exact path: A and L formed pairwise from raw q, k and g (no factored exponentials).
