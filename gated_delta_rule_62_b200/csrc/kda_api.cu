@@ -98,6 +98,10 @@ kda::Problem make_problem(const void *q, const void *k, const void *v, const flo
 
 }  // namespace
 
+namespace kda {
+kda_status_t record_error(kda_status_t st, const char *msg) { return fail(st, "%s", msg); }
+}  // namespace kda
+
 extern "C" {
 
 size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,

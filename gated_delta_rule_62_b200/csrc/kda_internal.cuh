@@ -44,6 +44,9 @@ cudaError_t launch_prefill_chunk(const Problem &p, void *workspace, cudaStream_t
                                  uint64_t timeout_ns);
 cudaError_t launch_bounded_wait_probe(void *workspace, uint64_t timeout_ns, cudaStream_t stream);
 
+// Records `msg` as the calling thread's kda_last_error() and returns `st`.
+kda_status_t record_error(kda_status_t st, const char *msg);
+
 // Upper bound on any single on-device wait before a kernel gives up (ns).
 constexpr uint64_t kWaitTimeoutNs = 4000000000ull;
 

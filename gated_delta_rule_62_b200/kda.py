@@ -40,6 +40,8 @@ SIGNATURES = {
     "kda_read_device_status": (_i32, [_vp, _vp]),
     "kda_version": (_i32, []),
     "kda_selftest_bounded_wait": (_i32, [_vp, _sz, ctypes.c_uint64, _vp]),
+    "kda_prefill_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
+                                   _i32, _i32, _vp, _vp, _vp]),
 }
 
 

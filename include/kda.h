@@ -182,6 +182,33 @@ KDA_API kda_status_t kda_read_device_status(const void *workspace, kda_stream_t 
 KDA_API kda_status_t kda_selftest_bounded_wait(void *workspace, size_t workspace_bytes,
                                                uint64_t timeout_ns, kda_stream_t stream);
 
+/*
+ * kda_prefill without a workspace argument, for callers that cannot allocate
+ * device memory when they run a prefill (code inside an allocator or pool
+ * callback, a serving loop whose memory is fixed at start-up). The pages
+ * describe no counterpart; this is a library convenience.
+ *
+ * The scratch kda_prefill keeps in its workspace lives instead in a fixed
+ * 64 KiB array in the library's device memory, held on every GPU that loads
+ * the library until the process exits. That caps num_seqs at 16320; larger
+ * values return KDA_ERR_INVALID_ARGUMENT. No device memory is allocated or
+ * freed. The first call on a device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Every call shares the one array and rewrites all of it that it uses, so
+ * calls that overlap on the GPU (different streams, or different host threads)
+ * race and must be serialised by the caller. The device status word is kept in
+ * that array and is not readable by the caller. Other arguments, results and
+ * status codes are those of kda_prefill.
+ */
+KDA_API kda_status_t kda_prefill_noalloc(const void *q, const void *k, const void *v,
+                                         const float *log_alpha, const float *beta,
+                                         const float *initial_state,
+                                         const int32_t *cu_seqlens_dev,
+                                         const int32_t *cu_seqlens_host,
+                                         int32_t num_seqs, int64_t total_tokens, int32_t H,
+                                         int32_t d_k, int32_t d_v, kda_dtype_t dtype,
+                                         void *out, float *final_state, kda_stream_t stream);
+
 /* Library version: major * 10000 + minor * 100 + patch. */
 KDA_API int32_t kda_version(void);
 
