@@ -2,34 +2,33 @@
 //
 // "KDA's update is organized blockwise ... so it maps onto GPU matrix units"
 // (shivam2003.com Kimi K3 article, section "Kimi Delta Attention: the
-// load-bearing choice"). The blockwise form used here is derived from the
-// per-token recurrence (decay, delta-rule write, read after the write):
+// load-bearing choice"). The blockwise form is derived from the per-token
+// recurrence (channel-wise decay, delta-rule write of the error, read after
+// the write). For a chunk of C = 64 tokens entered with state S (d_k x d_v),
+// g_i = sum_{s<=i} log_alpha_s (inclusive, per key channel), gamma = e^(g_{C-1}):
 //
-// For a chunk of C = 64 tokens starting from state S (d_k x d_v), with
-// g_i = sum_{s<=i} log_alpha_s (inclusive, per key channel), gamma = exp(g_{C-1}),
-//   Q~ = q * e^g,  K~ = k * e^g,  K- = k * e^-g,  K^ = k * e^(g_{C-1} - g)      (rows = tokens)
-//   A  = tril(Q~ K-^T)        (j <= i),    L = diag(beta) strictly_tril(K~ K-^T)
-//   T  = (I + L)^-1,  W = T diag(beta) K~,  U~ = T diag(beta) V
-//   U  = U~ - W S                          (the errors the delta rule writes)
+//   Q~ = q*e^g,  K~ = k*e^g,  K- = k*e^-g                       (rows = tokens)
+//   A  = tril(Q~ K-^T)          (j <= i)
+//   L  = diag(beta) strictly_tril(K~ K-^T),   T' = (I + L)^-1 diag(beta)
+//   W  = T' K~,   U~ = T' V,    U = U~ - W S           (the errors the delta rule writes)
 //   O  = Q~ S + A U
-//   S' = diag(gamma) S + K^^T U
-// which is the WY/UT form of the product of the per-token transitions
-// (I - beta k k^T) Diag(alpha) over the chunk. Every product is computed
-// transposed so that M = 128 (d_v or d_k) fills the tensor core's 128 lanes:
-//   U^T = (beta V)^T T^T - S^T W^T,  O^T = S^T Q~^T + U^T A^T,
-//   S'^T = S^T diag(gamma) + U^T K^,  W^T = (beta K~)^T T^T,  [Q~; K~] K-^T.
-// The fp32 master state S^T stays in TMEM for the whole sequence (lane = value
-// channel, column = key channel); a bf16 copy in shared memory feeds the MMAs.
+//   S_next = diag(gamma) (S + K-^T U)
+//
+// the WY/UT form of the product of the per-token transitions (I - beta k k^T) Diag(alpha).
+// Tokens are the M dimension of the token-row products (M = 64); the state update
+// has M = 128 key channels. K~, V, U and S enter the MMAs as MN-major operands
+// straight from the tiles TMA or the epilogues write, so no tile is transposed.
+// The fp32 master state S stays in TMEM for the whole sequence (lane = key channel).
 //
 // Factoring e^(g_i - g_j) = e^(g_i) e^(-g_j) overflows when a chunk decays by more
-// than ~e^88 in some channel. Chunks whose total decay exceeds e^60 take an
-// exact path that forms A and L pairwise on CUDA cores instead.
+// than ~e^88 in some channel. A chunk whose decay exceeds e^60 in any channel takes
+// an exact path: A and L are formed pairwise on CUDA cores, the K- tile holds
+// K^ = k e^(g_{C-1} - g), and S is scaled by gamma before S += K^^T U.
 //
-// One CTA (256 threads, 1 per SM) per (sequence, head); TMA brings each chunk's
-// q, k (128-byte swizzled, directly in the MMA operand layout), v and
-// log_alpha tiles into shared memory, prefetching the next chunk while the
-// current one computes. Every on-device wait is bounded; on timeout the
-// kernel records KDA_ERR_TIMEOUT in the workspace status word and returns.
+// One CTA of 256 threads per (sequence, head, d_v slice); DS = 128 / NSPLIT value
+// channels per CTA (NSPLIT = 2 doubles the CTAs for workloads with few heads, at the
+// price of repeating the key-side work). Every on-device wait is bounded; on timeout
+// the kernel records KDA_ERR_TIMEOUT in the workspace status word and returns.
 #include <cuda.h>
 
 #include <mutex>
@@ -47,31 +46,171 @@ constexpr int D = 128;   // d_k = d_v
 constexpr int NT = 256;  // threads per CTA
 constexpr float kFastLimit = 60.f;  // max in-chunk decay exponent for the factored path
 
-// Shared-memory map (byte offsets from a 1024-aligned base). bf16 operand tiles are
-// K-major with the 128-byte swizzle; a tile with K = 128 is two 64-wide K atoms.
-constexpr uint32_t OFF_QK = 0;                   // [Q~; K~] 128 rows x K=128 (raw q/k on arrival)
-constexpr uint32_t OFF_KI = OFF_QK + 32768;      // K- [j][c] 64 x 128, later W [i][c]
-constexpr uint32_t OFF_KBT = OFF_KI + 16384;     // (beta K~)^T [c][j] 128 x 64, later U^T [d][j]
-constexpr uint32_t OFF_VBT = OFF_KBT + 16384;    // (beta V)^T [d][j] 128 x 64
-constexpr uint32_t OFF_KHT = OFF_VBT + 16384;    // K^^T [c][j] 128 x 64
-constexpr uint32_t OFF_AQK = OFF_KHT + 16384;    // A [i][j] 64 x 64
-constexpr uint32_t OFF_TT = OFF_AQK + 8192;      // T [i][j] 64 x 64
-constexpr uint32_t OFF_ST = OFF_TT + 8192;       // S^T bf16 [d][c] 128 x 128
-constexpr uint32_t OFF_VR = OFF_ST + 32768;      // raw v [t][d] bf16 (TMA, unswizzled)
-constexpr uint32_t OFF_LA = OFF_VR + 16384;      // raw log_alpha [t][c] fp32 (TMA), then g
-constexpr uint32_t LT_LD = 68;                   // fp32 pitch of the L / T scratch
-constexpr uint32_t OFF_LT = OFF_LA + 32768;      // L -> T fp32 [64][68]
-constexpr uint32_t OFF_P = OFF_LT + 64 * LT_LD * 4;  // 3 x 16 x 16 fp32 block products
-constexpr uint32_t OFF_MISC = OFF_P + 3 * 256 * 4;
-constexpr uint32_t MISC_BYTES = 64 * 4 + 128 * 4 + 256 * 4 + 64 + 64;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+// ---------------------------------------------------------------- tile addressing
+// bf16 tiles use the 128-byte swizzle: 128-byte rows of 64 elements, 8-row groups
+// 1024 bytes apart, 16-byte chunk index XOR (row % 8); 64-column blocks `bs` bytes apart.
+__device__ __forceinline__ uint32_t tchunk(uint32_t bs, uint32_t row, uint32_t col) {
+    return (col >> 6) * bs + (row >> 3) * 1024 + (row & 7) * 128 +
+           ((((col & 63) >> 3) ^ (row & 7)) << 4);
+}
+__device__ __forceinline__ uint32_t telem(uint32_t bs, uint32_t row, uint32_t col) {
+    return tchunk(bs, row, col) + ((col & 7) << 1);
+}
 
-// TMEM columns (fp32, 128 lanes).
-constexpr uint32_t TM_S = 0, TM_D1 = 128, TM_W = 192, TM_U = 256, TM_O = 320, TM_COLS = 512;
+// Operand descriptors for K step kk (16 elements along K).
+// K-major tile (rows = M/N, columns = K): K advances 32 bytes inside a row, K blocks at bs.
+__device__ __forceinline__ uint64_t desc_k(uint32_t base, uint32_t bs, uint32_t kk) {
+    return smem_desc_sw128(base + (kk >> 2) * bs + (kk & 3) * 32, 16, 1024);
+}
+// MN-major tile (rows = K, columns = M/N): K advances two 8-row groups, MN blocks at bs.
+__device__ __forceinline__ uint64_t desc_mn(uint32_t base, uint32_t bs, uint32_t kk) {
+    return smem_desc_sw128(base + kk * 2048, bs, 1024);
+}
 
-constexpr uint32_t IDESC_N64 = idesc_bf16_f32(128, 64);
-constexpr uint32_t IDESC_N64_NEG = idesc_bf16_f32(128, 64, true);
-constexpr uint32_t IDESC_N128 = idesc_bf16_f32(128, 128);
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ void st_chunk(uint8_t *p, const float *v) {
+    *reinterpret_cast<uint4 *>(p) = make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]),
+                                               pack2(v[4], v[5]), pack2(v[6], v[7]));
+}
+__device__ __forceinline__ float2 ld_bf2(const uint8_t *p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+}
+__device__ __forceinline__ void st_bf2(uint8_t *p, float a, float b) {
+    *reinterpret_cast<uint32_t *>(p) = pack2(a, b);
+}
+__device__ __forceinline__ float ld_bf(const uint8_t *p) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p));
+}
+__device__ __forceinline__ void st_bf(uint8_t *p, float x) {
+    *reinterpret_cast<__nv_bfloat16 *>(p) = __float2bfloat16_rn(x);
+}
+
+// ---------------------------------------------------------------- 64x64 unit lower-triangular inverse
+constexpr int LT_LD = 68;  // fp32 pitch of the L / T scratch
+constexpr int PB_LD = 36;  // fp32 pitch of the 32x32 block-product scratch
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// acc (a 16x16 tile as two m16n8 fragments) += A[16][K] * B[K][16], fp32 in shared memory,
+// multiplied with tf32 operands by the warp-level mma.sync m16n8k8.
+__device__ __forceinline__ void warp_mm16(float (&acc)[2][4], const float *A, int pa,
+                                          const float *B, int pb, int K) {
+    const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+    for (int k = 0; k < K; k += 8) {
+        const uint32_t a0 = to_tf32(A[gid * pa + k + tig]);
+        const uint32_t a1 = to_tf32(A[(gid + 8) * pa + k + tig]);
+        const uint32_t a2 = to_tf32(A[gid * pa + k + tig + 4]);
+        const uint32_t a3 = to_tf32(A[(gid + 8) * pa + k + tig + 4]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t b0 = to_tf32(B[(k + tig) * pb + 8 * nt + gid]);
+            const uint32_t b1 = to_tf32(B[(k + tig + 4) * pb + 8 * nt + gid]);
+            asm volatile(
+                "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, "
+                "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
+                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+}
+__device__ __forceinline__ void warp_store16(float *X, int px, const float (&acc)[2][4], float s) {
+    const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        X[gid * px + 8 * nt + 2 * tig] = s * acc[nt][0];
+        X[gid * px + 8 * nt + 2 * tig + 1] = s * acc[nt][1];
+        X[(gid + 8) * px + 8 * nt + 2 * tig] = s * acc[nt][2];
+        X[(gid + 8) * px + 8 * nt + 2 * tig + 1] = s * acc[nt][3];
+    }
+}
+
+// T = (I + L)^-1 in place for strictly lower-triangular L (fp32, pitch LT_LD, zeros on and
+// above the diagonal). Blocks of 16: the diagonal blocks by forward substitution, then the
+// block inverse [[A,0],[B,C]]^-1 = [[A^-1,0],[-C^-1 B A^-1, C^-1]] at 16 and then at 32.
+// Called by all NT threads (contains __syncthreads).
+__device__ void invert_unit_lower(float *LT, float *PB, int tid) {
+    const int warp = tid >> 5, lane = tid & 31;
+    if (warp < 4 && lane < 16) {
+        float *Lb = LT + (16 * warp) * LT_LD + 16 * warp;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float s = (i == lane) ? 1.f : 0.f;
+#pragma unroll
+            for (int j = 0; j < i; ++j) s = fmaf(-Lb[i * LT_LD + j], x[j], s);
+            x[i] = s;
+        }
+        __syncwarp(0x0000ffffu);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Lb[i * LT_LD + lane] = x[i];
+    }
+    __syncthreads();
+    if (warp < 2) {
+        // warp 0: T10 = -T11 (L10 T00); warp 1: T32 = -T33 (L32 T22)
+        const int r0 = warp ? 48 : 16, c0 = warp ? 32 : 0;
+        float *P = PB + warp * 16 * PB_LD;
+        float acc[2][4] = {};
+        warp_mm16(acc, LT + r0 * LT_LD + c0, LT_LD, LT + c0 * LT_LD + c0, LT_LD, 16);
+        warp_store16(P, PB_LD, acc, 1.f);
+        __syncwarp();
+        float acc2[2][4] = {};
+        warp_mm16(acc2, LT + r0 * LT_LD + r0, LT_LD, P, PB_LD, 16);
+        warp_store16(LT + r0 * LT_LD + c0, LT_LD, acc2, -1.f);
+    }
+    __syncthreads();
+    // rows 32..63 x cols 0..31: P = L[32:64, 0:32] T[0:32, 0:32];  T[32:64, 0:32] = -T[32:64, 32:64] P
+    const int rt = (warp >> 1) & 1, ct = warp & 1;
+    if (warp < 4) {
+        float acc[2][4] = {};
+        warp_mm16(acc, LT + (32 + 16 * rt) * LT_LD, LT_LD, LT + 16 * ct, LT_LD, 32);
+        warp_store16(PB + (16 * rt) * PB_LD + 16 * ct, PB_LD, acc, 1.f);
+    }
+    __syncthreads();
+    if (warp < 4) {
+        float acc[2][4] = {};
+        warp_mm16(acc, LT + (32 + 16 * rt) * LT_LD + 32, LT_LD, PB + 16 * ct, PB_LD, 32);
+        warp_store16(LT + (32 + 16 * rt) * LT_LD + 16 * ct, LT_LD, acc, -1.f);
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------- shared memory map
+template <int DS>
+struct Smem {
+    static constexpr uint32_t QK = 0;                       // [q~ ; k~] 128 rows x 128, blocks 16 KB
+    static constexpr uint32_t KI = QK + 32768;              // K- (or K^) [j][c] 64 x 128, blocks 8 KB
+    static constexpr uint32_t W = KI + 16384;               // W [i][c] 64 x 128, blocks 8 KB
+    static constexpr uint32_t S = W + 16384;                // S [c][d] bf16 128 x DS, blocks 16 KB
+    static constexpr uint32_t V = S + 256 * DS;             // V [j][d] 64 x DS, blocks 8 KB
+    static constexpr uint32_t U = V + 128 * DS;             // U [j][d] 64 x DS, blocks 8 KB
+    static constexpr uint32_t AQK = U + 128 * DS;           // A [i][j] 64 x 64
+    static constexpr uint32_t TT = AQK + 8192;              // T' [i][j] 64 x 64
+    static constexpr uint32_t LA = TT + 8192;               // log_alpha [t][c] fp32, then g
+    static constexpr uint32_t LT = LA + 32768;              // L -> T fp32 [64][LT_LD]
+    static constexpr uint32_t PB = LT + 64 * LT_LD * 4;     // 32 x PB_LD fp32
+    static constexpr uint32_t MISC = PB + 32 * PB_LD * 4;   // beta, gamma, psum, flags, barriers
+    static constexpr uint32_t MISC_BYTES = 64 * 4 + 128 * 4 + 4 * 128 * 4 + 64 + 64;
+    static constexpr uint32_t BYTES = MISC + MISC_BYTES + 1024;  // + alignment slack
+};
+
+// TMEM columns (fp32, 128 lanes). DS <= 64: O has its own columns; DS = 128: O reuses W's.
+template <int DS>
+struct Tmem {
+    static constexpr uint32_t S = 0;
+    static constexpr uint32_t D1 = 128;
+    static constexpr uint32_t U = 192;
+    static constexpr uint32_t W = U + DS;
+    static constexpr uint32_t O = DS <= 64 ? W + 128 : W;
+    static constexpr uint32_t COLS = 512;
+    static_assert(O + DS <= COLS && W + 128 <= COLS, "TMEM overflow");
+};
 
 struct ChunkParams {
     const int32_t *cu_seqlens;
@@ -85,113 +224,54 @@ struct ChunkParams {
     uint64_t timeout_ns;
 };
 
-// Byte offset of element (row, k) in a K-major SW128 bf16 tile of `rows` rows.
-__device__ __forceinline__ uint32_t sw_off(uint32_t rows, uint32_t row, uint32_t k) {
-    const uint32_t kk = k & 63;
-    return (k >> 6) * rows * 128 + (row >> 3) * 1024 + (row & 7) * 128 +
-           (((kk >> 3) ^ (row & 7)) << 4) + ((kk & 7) << 1);
-}
-// Byte offset of the 16-byte chunk holding elements (row, k .. k+7), k % 8 == 0.
-__device__ __forceinline__ uint32_t sw_chunk(uint32_t rows, uint32_t row, uint32_t k) {
-    const uint32_t kk = k & 63;
-    return (k >> 6) * rows * 128 + (row >> 3) * 1024 + (row & 7) * 128 +
-           (((kk >> 3) ^ (row & 7)) << 4);
-}
-
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-__device__ __forceinline__ void st_chunk(uint8_t *p, const float *v) {
-    uint4 u = make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]),
-                         pack2(v[6], v[7]));
-    *reinterpret_cast<uint4 *>(p) = u;
-}
-__device__ __forceinline__ float ld_bf(const uint8_t *p) {
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p));
-}
-__device__ __forceinline__ void st_bf(uint8_t *p, float x) {
-    *reinterpret_cast<__nv_bfloat16 *>(p) = __float2bfloat16_rn(x);
-}
-
-// Descriptor of K-step kk (16 elements) of a K-major SW128 tile with `rows` rows.
-__device__ __forceinline__ uint64_t kdesc(uint32_t base, uint32_t rows, uint32_t kk) {
-    return smem_desc_sw128(base + (kk >> 2) * rows * 128 + (kk & 3) * 32);
-}
-
-// T = (I + L)^-1 for strictly lower-triangular L (fp32, pitch LT_LD), in place.
-// Diagonal 16x16 blocks by forward substitution (one column per lane), then the
-// off-diagonal blocks row by row: T_rc = -T_rr sum_{k=c}^{r-1} L_rk T_kc.
-__device__ void invert_unit_lower(float *LT, float *P, int tid) {
-    if (tid < 128 && (tid & 31) < 16) {
-        const int w = tid >> 5, l = tid & 31;
-        float *Lb = LT + (16 * w) * LT_LD + 16 * w;
-        float x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float s = (i == l) ? 1.f : 0.f;
-#pragma unroll
-            for (int j = 0; j < i; ++j) s = fmaf(-Lb[i * LT_LD + j], x[j], s);
-            x[i] = s;
-        }
-        __syncwarp(0x0000ffffu);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) Lb[i * LT_LD + l] = x[i];
-    }
-    __syncthreads();
-    for (int r = 1; r < 4; ++r) {
-        for (int e = tid; e < r * 256; e += NT) {
-            const int cb = e >> 8, i = (e >> 4) & 15, j = e & 15;
-            const float *Lrow = LT + (16 * r + i) * LT_LD;
-            float s = 0.f;
-            for (int k = 16 * cb; k < 16 * r; ++k) s = fmaf(Lrow[k], LT[k * LT_LD + 16 * cb + j], s);
-            P[e] = s;
-        }
-        __syncthreads();
-        for (int e = tid; e < r * 256; e += NT) {
-            const int cb = e >> 8, i = (e >> 4) & 15, j = e & 15;
-            const float *Trow = LT + (16 * r + i) * LT_LD + 16 * r;
-            float s = 0.f;
-#pragma unroll
-            for (int m = 0; m < 16; ++m) s = fmaf(Trow[m], P[cb * 256 + m * 16 + j], s);
-            LT[(16 * r + i) * LT_LD + 16 * cb + j] = -s;
-        }
-        __syncthreads();
-    }
-}
-
+template <int DS>
 __global__ void __launch_bounds__(NT, 1)
 chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
              const ChunkParams p) {
+    using SM = Smem<DS>;
+    using TM = Tmem<DS>;
+    constexpr int NSPLIT = D / DS;
+    constexpr uint32_t I_D1 = idesc_bf16_f32(128, 64);               // [Q~;K~] x K-
+    constexpr uint32_t I_W = idesc_bf16_f32(64, 128, false, 0, 1);    // T' x K~ (B MN-major)
+    constexpr uint32_t I_UT = idesc_bf16_f32(64, DS, false, 0, 1);    // T' x V, Q~ x S, A x U
+    constexpr uint32_t I_UWS = idesc_bf16_f32(64, DS, true, 0, 1);    // -W x S
+    constexpr uint32_t I_S = idesc_bf16_f32(128, DS, false, 1, 1);    // K-^T x U (A MN-major)
+    constexpr int SCOLS = DS / 2;  // TMEM columns of S / U / O per thread (two threads per lane)
+
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-    float *s_beta = reinterpret_cast<float *>(sm + OFF_MISC);  // [64]
-    float *s_gamma = s_beta + 64;                                // [128]
-    float *s_psum = s_gamma + 128;                               // [2][128]
-    uint32_t *s_flags = reinterpret_cast<uint32_t *>(s_psum + 256);  // abort, maxdecay, tmem
-    uint64_t *bars = reinterpret_cast<uint64_t *>(s_flags + 16);     // qk, lv, mma
-    uint64_t *bar_qk = bars, *bar_lv = bars + 1, *bar_mma = bars + 2;
-    float *LA = reinterpret_cast<float *>(sm + OFF_LA);
-    float *LT = reinterpret_cast<float *>(sm + OFF_LT);
-    float *P = reinterpret_cast<float *>(sm + OFF_P);
-    const uint32_t sbase = smem_u32(sm);
+    float *s_beta = reinterpret_cast<float *>(sm + SM::MISC);  // [64]
+    float *s_gamma = s_beta + 64;                               // [128]
+    float *s_psum = s_gamma + 128;                              // [4][128]
+    uint32_t *s_flags = reinterpret_cast<uint32_t *>(s_psum + 512);  // abort, exact path, tmem
+    uint64_t *bars = reinterpret_cast<uint64_t *>(s_flags + 16);     // qk, la, v, mma
+    uint64_t *bar_qk = bars, *bar_la = bars + 1, *bar_v = bars + 2, *bar_mma = bars + 3;
+    float *LA = reinterpret_cast<float *>(sm + SM::LA);
+    float *LT = reinterpret_cast<float *>(sm + SM::LT);
+    float *PB = reinterpret_cast<float *>(sm + SM::PB);
+    const uint32_t sb = smem_u32(sm);
 
-    const int tid = threadIdx.x;
-    const int r = tid & 127, hf = tid >> 7, warp = tid >> 5;
-    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
     const int H = p.H;
-    const int slot = blockIdx.x / H, h = blockIdx.x % H;
+    const int split = blockIdx.x % NSPLIT;
+    const int hs = blockIdx.x / NSPLIT;
+    const int slot = hs / H, h = hs % H;
     const int n = p.order ? p.order[slot] : slot;
+    const int d0 = split * DS;  // first value channel of this CTA
     const int64_t bos = p.cu_seqlens[n], eos = p.cu_seqlens[n + 1];
     const int nchunks = (int)((eos - bos + C - 1) / C);
     const size_t state_off = ((size_t)n * H + h) * (size_t)(D * D);
+    const int c_me = 32 * quad + lane;  // key channel = TMEM lane of this thread
 
     if (tid == 0) {
         s_flags[0] = 0;
         mbar_init(bar_qk, 1);
-        mbar_init(bar_lv, 1);
+        mbar_init(bar_la, 1);
+        mbar_init(bar_v, 1);
         mbar_init(bar_mma, 1);
         fence_mbarrier_init();
         prefetch_tmap(&tm_q);
@@ -200,7 +280,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         prefetch_tmap(&tm_la);
     }
     if (warp == 0) {
-        tmem_alloc(&s_flags[2], TM_COLS);
+        tmem_alloc(&s_flags[2], TM::COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -210,43 +290,58 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
     auto issue_qk = [&](int64_t t0) {
         mbar_arrive_expect_tx(bar_qk, 32768);
-        tma_load_3d(sm + OFF_QK, &tm_q, bar_qk, 0, h, (int32_t)t0);
-        tma_load_3d(sm + OFF_QK + 8192, &tm_k, bar_qk, 0, h, (int32_t)t0);
-        tma_load_3d(sm + OFF_QK + 16384, &tm_q, bar_qk, 64, h, (int32_t)t0);
-        tma_load_3d(sm + OFF_QK + 24576, &tm_k, bar_qk, 64, h, (int32_t)t0);
+        tma_load_3d(sm + SM::QK, &tm_q, bar_qk, 0, h, (int32_t)t0);
+        tma_load_3d(sm + SM::QK + 8192, &tm_k, bar_qk, 0, h, (int32_t)t0);
+        tma_load_3d(sm + SM::QK + 16384, &tm_q, bar_qk, 64, h, (int32_t)t0);
+        tma_load_3d(sm + SM::QK + 24576, &tm_k, bar_qk, 64, h, (int32_t)t0);
     };
-    auto issue_lv = [&](int64_t t0) {
-        mbar_arrive_expect_tx(bar_lv, 32768 + 16384);
-        tma_load_3d(sm + OFF_LA, &tm_la, bar_lv, 0, h, (int32_t)t0);
-        tma_load_3d(sm + OFF_VR, &tm_v, bar_lv, 0, h, (int32_t)t0);
+    auto issue_la = [&](int64_t t0) {
+        mbar_arrive_expect_tx(bar_la, 32768);
+        tma_load_3d(sm + SM::LA, &tm_la, bar_la, 0, h, (int32_t)t0);
     };
-    bool qk_pending = false, lv_pending = false;
-    if (nchunks > 0 && tid == 0) {
-        issue_qk(bos);
-        issue_lv(bos);
-    }
-    if (nchunks > 0) qk_pending = lv_pending = true;
-
-    // Initial state -> S^T (TMEM fp32, lane d, column c) and its bf16 copy (rows d).
-    {
-        const int d = r;
+    auto issue_v = [&](int64_t t0) {
+        mbar_arrive_expect_tx(bar_v, 128 * DS);
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            const int c0 = 64 * hf + 32 * part;
+        for (int b = 0; b < DS / 64; ++b)
+            tma_load_3d(sm + SM::V + 8192 * b, &tm_v, bar_v, d0 + 64 * b, h, (int32_t)t0);
+    };
+    bool qk_pending = false, la_pending = false, v_pending = false;
+    if (nchunks > 0) {
+        if (tid == 0) {
+            issue_qk(bos);
+            issue_la(bos);
+            issue_v(bos);
+        }
+        qk_pending = la_pending = v_pending = true;
+    }
+
+    // Initial state -> S (TMEM fp32, lane c, columns d) and its bf16 tile [c][d].
+    {
+        const size_t row = state_off + (size_t)c_me * D + d0 + half * SCOLS;
+        const float *src = p.s0 ? p.s0 + row : nullptr;
+        float *dst = p.sT ? p.sT + row : nullptr;
+#pragma unroll
+        for (int part = 0; part < SCOLS / 32; ++part) {
             float v[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-                v[e] = p.s0 ? p.s0[state_off + (size_t)(c0 + e) * D + d] : 0.f;
+            for (int e = 0; e < 32; e += 4) {
+                float4 f = src ? *reinterpret_cast<const float4 *>(src + 32 * part + e)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[e] = f.x; v[e + 1] = f.y; v[e + 2] = f.z; v[e + 3] = f.w;
+            }
             if (nchunks == 0) {
-                if (p.sT) {
+                if (dst) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) p.sT[state_off + (size_t)(c0 + e) * D + d] = v[e];
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4 *>(dst + 32 * part + e) =
+                            make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
                 }
             } else {
-                tmem_st32(tmem + lane_base + TM_S + c0, v);
+                const int col = half * SCOLS + 32 * part;
+                tmem_st32(tmem + lane_base + TM::S + col, v);
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8)
-                    st_chunk(sm + OFF_ST + sw_chunk(128, d, c0 + 8 * q8), v + 8 * q8);
+                    st_chunk(sm + SM::S + tchunk(16384, c_me, col + 8 * q8), v + 8 * q8);
             }
         }
         tmem_wait_st();
@@ -255,10 +350,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     tc_fence_before();
     __syncthreads();
 
-    uint32_t ph_qk = 0, ph_lv = 0, ph_mma = 0;
-    const uint64_t deadline_step = p.timeout_ns;
+    uint32_t ph_qk = 0, ph_la = 0, ph_v = 0, ph_mma = 0;
     auto wait_bar = [&](uint64_t *bar, uint32_t &ph) {
-        const bool ok = mbar_wait_bounded(bar, ph, globaltimer_ns() + deadline_step);
+        const bool ok = mbar_wait_bounded(bar, ph, globaltimer_ns() + p.timeout_ns);
         ph ^= 1u;
         if (!ok) {
             s_flags[0] = 1;
@@ -266,56 +360,71 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         }
     };
 
+    // gating thread mapping: channel pair (cA, cA + 1), token quarter tq
+    const int tq = tid >> 6, cA = 2 * (tid & 63);
+
     for (int ci = 0; ci < nchunks; ++ci) {
         const int64_t t0 = bos + (int64_t)ci * C;
         const int valid = (int)(eos - t0 < C ? eos - t0 : C);
         const bool has_next = ci + 1 < nchunks;
         if (tid < C) s_beta[tid] = (tid < valid) ? p.beta[(size_t)(t0 + tid) * H + h] : 0.f;
         if (tid == 0) s_flags[1] = 0;
-        wait_bar(bar_lv, ph_lv);
+        wait_bar(bar_la, ph_la);
         wait_bar(bar_qk, ph_qk);
-        lv_pending = qk_pending = false;
+        la_pending = qk_pending = false;
         __syncthreads();
         if (s_flags[0]) break;
 
-        // ---- gate cumsum: thread (c = r, half hf) scans tokens [32 hf, 32 hf + 32)
-        const int c = r, i0 = 32 * hf;
+        // ---- gate cumsum: local prefix over this thread's 16 tokens of two channels
         {
-            float acc = 0.f;
-#pragma unroll 8
-            for (int i = 0; i < 32; ++i) {
-                const int t = i0 + i;
-                const float x = (t < valid) ? LA[t * D + c] : 0.f;
-                acc += x;
-                LA[t * D + c] = acc;
+            float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 4
+            for (int i = 0; i < 16; ++i) {
+                const int t = 16 * tq + i;
+                float2 *pl = reinterpret_cast<float2 *>(LA + t * D + cA);
+                const float2 x = (t < valid) ? *pl : make_float2(0.f, 0.f);
+                acc.x += x.x;
+                acc.y += x.y;
+                *pl = acc;
             }
-            s_psum[hf * D + c] = acc;
+            s_psum[tq * D + cA] = acc.x;
+            s_psum[tq * D + cA + 1] = acc.y;
         }
         __syncthreads();
-        float goff = hf ? s_psum[c] : 0.f;
-        const float gC = s_psum[c] + s_psum[D + c];
-        if (hf == 0) {
-            s_gamma[c] = __expf(gC);
-            // Any channel decaying by more than e^kFastLimit sends the chunk down the exact path.
-            // (Also taken for non-finite gates: the comparison below is false for NaN.)
-            if (!(-gC <= kFastLimit)) s_flags[1] = 1u;
+        float2 goff = make_float2(0.f, 0.f), gC = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float a = s_psum[q * D + cA], b = s_psum[q * D + cA + 1];
+            if (q < tq) { goff.x += a; goff.y += b; }
+            gC.x += a;
+            gC.y += b;
+        }
+        if (tq == 0) {
+            s_gamma[cA] = __expf(gC.x);
+            s_gamma[cA + 1] = __expf(gC.y);
+            // Any channel decaying by more than e^kFastLimit sends the chunk down the exact
+            // path (also non-finite gates: the comparison is false for NaN).
+            if (!(-gC.x <= kFastLimit) || !(-gC.y <= kFastLimit)) s_flags[1] = 1u;
         }
         __syncthreads();
         const bool safe = s_flags[1] != 0u;
 
         if (safe) {
-            // Exact path: A and L formed pairwise from raw q, k and g (no factored exponentials).
-            if (hf) {
-                for (int i = 0; i < 32; ++i) LA[(i0 + i) * D + c] += goff;
+            // Exact path: A and L pairwise from raw q, k and the full g (no factored exponentials).
+            if (tq > 0) {
+                for (int i = 0; i < 16; ++i) {
+                    float2 *pl = reinterpret_cast<float2 *>(LA + (16 * tq + i) * D + cA);
+                    const float2 x = *pl;
+                    *pl = make_float2(x.x + goff.x, x.y + goff.y);
+                }
             }
-            goff = 0.f;
+            goff = make_float2(0.f, 0.f);
             for (int e = tid; e < 64 * 64; e += NT) {
                 const int i = e >> 6, j = e & 63;
-                st_bf(sm + OFF_AQK + sw_off(64, i, j), 0.f);
+                st_bf(sm + SM::AQK + telem(8192, i, j), 0.f);
                 LT[i * LT_LD + j] = 0.f;
             }
             __syncthreads();
-            const int lane = tid & 31;
             for (int e = warp; e < 64 * 64; e += NT / 32) {
                 const int i = e >> 6, j = e & 63;
                 if (j > i || i >= valid) continue;
@@ -324,9 +433,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 for (int m = 0; m < 4; ++m) {
                     const int cc = lane + 32 * m;
                     const float ex = __expf(LA[i * D + cc] - LA[j * D + cc]);
-                    const float kj = ld_bf(sm + OFF_QK + sw_off(128, 64 + j, cc)) * ex;
-                    a = fmaf(ld_bf(sm + OFF_QK + sw_off(128, i, cc)), kj, a);
-                    l = fmaf(ld_bf(sm + OFF_QK + sw_off(128, 64 + i, cc)), kj, l);
+                    const float kj = ld_bf(sm + SM::QK + telem(16384, 64 + j, cc)) * ex;
+                    a = fmaf(ld_bf(sm + SM::QK + telem(16384, i, cc)), kj, a);
+                    l = fmaf(ld_bf(sm + SM::QK + telem(16384, 64 + i, cc)), kj, l);
                 }
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) {
@@ -334,98 +443,91 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     l += __shfl_xor_sync(0xffffffffu, l, off);
                 }
                 if (lane == 0) {
-                    st_bf(sm + OFF_AQK + sw_off(64, i, j), a);
+                    st_bf(sm + SM::AQK + telem(8192, i, j), a);
                     if (j < i) LT[i * LT_LD + j] = s_beta[i] * l;
                 }
             }
+            // S <- diag(gamma) S ahead of S += K^^T U
+            const float gm = s_gamma[c_me];
+#pragma unroll
+            for (int part = 0; part < SCOLS / 32; ++part) {
+                const uint32_t ta = tmem + lane_base + TM::S + half * SCOLS + 32 * part;
+                float v[32];
+                tmem_ld32(ta, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] *= gm;
+                tmem_st32(ta, v);
+            }
+            tmem_wait_st();
+            tc_fence_before();
             __syncthreads();
         }
 
-        // ---- gated operands for tokens [i0, i0 + 32) of channel c (and value channel d = r)
-        {
-            const float gam = s_gamma[c];
-            float khat[8], kbt[8], vbt[8];
-#pragma unroll 1
-            for (int i8 = 0; i8 < 32; i8 += 8) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int t = i0 + i8 + u;
-                    const bool ok = t < valid;
-                    const float g = goff + LA[t * D + c];
-                    const float eg = __expf(g), emg = __expf(-g);
-                    uint8_t *qp = sm + OFF_QK + sw_off(128, t, c);
-                    uint8_t *kp = sm + OFF_QK + sw_off(128, 64 + t, c);
-                    const float qv = ok ? ld_bf(qp) : 0.f;
-                    const float kv = ok ? ld_bf(kp) : 0.f;
-                    const float bt = s_beta[t];
-                    st_bf(qp, qv * eg);
-                    st_bf(kp, kv * eg);
-                    if (!safe) st_bf(sm + OFF_KI + sw_off(64, t, c), kv * emg);
-                    khat[u] = safe ? kv * __expf(gC - g) : kv * emg * gam;
-                    kbt[u] = bt * kv * eg;
-                    const __nv_bfloat16 vr =
-                        reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_VR)[t * D + r];
-                    vbt[u] = ok ? bt * __bfloat162float(vr) : 0.f;
-                }
-                st_chunk(sm + OFF_KHT + sw_chunk(128, c, i0 + i8), khat);
-                st_chunk(sm + OFF_KBT + sw_chunk(128, c, i0 + i8), kbt);
-                st_chunk(sm + OFF_VBT + sw_chunk(128, r, i0 + i8), vbt);
-            }
+        // ---- gated operands: Q~, K~ in place; K- (fast) or K^ (exact) into the KI tile
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+            const int t = 16 * tq + i;
+            const bool ok = t < valid;
+            const float2 lg = *reinterpret_cast<const float2 *>(LA + t * D + cA);
+            const float g0 = goff.x + lg.x, g1 = goff.y + lg.y;
+            const float e0 = __expf(g0), e1 = __expf(g1);
+            uint8_t *qp = sm + SM::QK + telem(16384, t, cA);
+            uint8_t *kp = sm + SM::QK + telem(16384, 64 + t, cA);
+            float2 qv = ld_bf2(qp), kv = ld_bf2(kp);
+            if (!ok) qv = kv = make_float2(0.f, 0.f);
+            st_bf2(qp, qv.x * e0, qv.y * e1);
+            st_bf2(kp, kv.x * e0, kv.y * e1);
+            const float m0 = __expf(safe ? gC.x - g0 : -g0), m1 = __expf(safe ? gC.y - g1 : -g1);
+            st_bf2(sm + SM::KI + telem(8192, t, cA), kv.x * m0, kv.y * m1);
         }
         fence_proxy_async_smem();
         __syncthreads();
 
         if (tid == 0) {
-            if (has_next) {
-                fence_proxy_async_smem();
-                issue_lv(t0 + C);
-            }
+            if (has_next) issue_la(t0 + C);
             tc_fence_after();
             if (!safe) {
 #pragma unroll
                 for (uint32_t kk = 0; kk < 8; ++kk)
-                    mma_bf16_ss(tmem + TM_D1, kdesc(sbase + OFF_QK, 128, kk),
-                                kdesc(sbase + OFF_KI, 64, kk), IDESC_N64, kk > 0);
+                    mma_bf16_ss(tmem + TM::D1, desc_k(sb + SM::QK, 16384, kk),
+                                desc_k(sb + SM::KI, 8192, kk), I_D1, kk > 0);
             }
+            if (DS <= 64) {  // O = Q~ S now (own TMEM columns)
 #pragma unroll
-            for (uint32_t kk = 0; kk < 8; ++kk)
-                mma_bf16_ss(tmem + TM_O, kdesc(sbase + OFF_ST, 128, kk),
-                            kdesc(sbase + OFF_QK, 128, kk), IDESC_N64, kk > 0);
+                for (uint32_t kk = 0; kk < 8; ++kk)
+                    mma_bf16_ss(tmem + TM::O, desc_k(sb + SM::QK, 16384, kk),
+                                desc_mn(sb + SM::S, 16384, kk), I_UT, kk > 0);
+            }
             mma_commit(bar_mma);
         }
-        lv_pending = has_next;
+        la_pending = has_next;
         wait_bar(bar_mma, ph_mma);
         tc_fence_after();
-        if (tid == 0 && has_next) {
-            fence_proxy_async_smem();
-            issue_qk(t0 + C);
-        }
-        qk_pending = has_next;
 
-        // ---- A (rows 0..63 of D1) to bf16, L (rows 64..127) to fp32 scratch
+        // ---- A (D1 rows 0..63) to bf16, L (rows 64..127, times beta_i, j < i) to fp32
         if (!safe) {
+            const int r = c_me;
             float v[32];
-            tmem_ld32(tmem + lane_base + TM_D1 + 32 * hf, v);
+            tmem_ld32(tmem + lane_base + TM::D1 + 32 * half, v);
             tmem_wait_ld();
             if (r < 64) {
-                const int i = r;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = (32 * hf + e <= i) ? v[e] : 0.f;
+                for (int e = 0; e < 32; ++e) v[e] = (32 * half + e <= r) ? v[e] : 0.f;
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8)
-                    st_chunk(sm + OFF_AQK + sw_chunk(64, i, 32 * hf + 8 * q8), v + 8 * q8);
+                    st_chunk(sm + SM::AQK + tchunk(8192, r, 32 * half + 8 * q8), v + 8 * q8);
             } else {
                 const int i = r - 64;
                 const float b = s_beta[i];
-                float4 *dst = reinterpret_cast<float4 *>(LT + i * LT_LD + 32 * hf);
+                float4 *dst = reinterpret_cast<float4 *>(LT + i * LT_LD + 32 * half);
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
-                    float4 w;
-                    w.x = (32 * hf + 4 * e4 + 0 < i) ? b * v[4 * e4 + 0] : 0.f;
-                    w.y = (32 * hf + 4 * e4 + 1 < i) ? b * v[4 * e4 + 1] : 0.f;
-                    w.z = (32 * hf + 4 * e4 + 2 < i) ? b * v[4 * e4 + 2] : 0.f;
-                    w.w = (32 * hf + 4 * e4 + 3 < i) ? b * v[4 * e4 + 3] : 0.f;
-                    dst[e4] = w;
+                    const int j = 32 * half + 4 * e4;
+                    dst[e4] = make_float4(j + 0 < i ? b * v[4 * e4 + 0] : 0.f,
+                                          j + 1 < i ? b * v[4 * e4 + 1] : 0.f,
+                                          j + 2 < i ? b * v[4 * e4 + 2] : 0.f,
+                                          j + 3 < i ? b * v[4 * e4 + 3] : 0.f);
                 }
             }
         }
@@ -433,122 +535,158 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         __syncthreads();
         if (s_flags[0]) break;
 
-        // ---- T = (I + L)^-1, then bf16 into the MMA tile
-        invert_unit_lower(LT, P, tid);
+        // ---- T = (I + L)^-1; T' = T diag(beta) to bf16
+        invert_unit_lower(LT, PB, tid);
         {
             const int i = tid >> 2, j0 = (tid & 3) * 16;
             float v[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = LT[i * LT_LD + j0 + e];
-            st_chunk(sm + OFF_TT + sw_chunk(64, i, j0), v);
-            st_chunk(sm + OFF_TT + sw_chunk(64, i, j0 + 8), v + 8);
+            for (int e = 0; e < 16; ++e) v[e] = LT[i * LT_LD + j0 + e] * s_beta[j0 + e];
+            st_chunk(sm + SM::TT + tchunk(8192, i, j0), v);
+            st_chunk(sm + SM::TT + tchunk(8192, i, j0 + 8), v + 8);
         }
         fence_proxy_async_smem();
         __syncthreads();
 
+        wait_bar(bar_v, ph_v);  // V of this chunk
+        v_pending = false;
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_W, kdesc(sbase + OFF_KBT, 128, kk),
-                            kdesc(sbase + OFF_TT, 64, kk), IDESC_N64, kk > 0);
+            for (uint32_t kk = 0; kk < 4; ++kk)  // W = T' K~
+                mma_bf16_ss(tmem + TM::W, desc_k(sb + SM::TT, 8192, kk),
+                            desc_mn(sb + SM::QK + 8192, 16384, kk), I_W, kk > 0);
 #pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_U, kdesc(sbase + OFF_VBT, 128, kk),
-                            kdesc(sbase + OFF_TT, 64, kk), IDESC_N64, kk > 0);
+            for (uint32_t kk = 0; kk < 4; ++kk)  // U~ = T' V
+                mma_bf16_ss(tmem + TM::U, desc_k(sb + SM::TT, 8192, kk),
+                            desc_mn(sb + SM::V, 8192, kk), I_UT, kk > 0);
             mma_commit(bar_mma);
         }
         wait_bar(bar_mma, ph_mma);
         tc_fence_after();
+        if (tid == 0 && has_next) {
+            issue_v(t0 + C);
+            if (DS <= 64) issue_qk(t0 + C);  // Q~ and K~ are consumed
+        }
+        v_pending = has_next;
+        if (DS <= 64) qk_pending = has_next;
 
-        // ---- W^T (lane c, column i) -> W [i][c] bf16 (reuses the K- tile)
-        {
+        // ---- W (TMEM, M=64: row 16*quad + lane for lane < 16) -> bf16 tile [i][c]
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int col = 64 * half + 32 * part;
             float v[32];
-            tmem_ld32(tmem + lane_base + TM_W + 32 * hf, v);
+            tmem_ld32(tmem + lane_base + TM::W + col, v);
             tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) st_bf(sm + OFF_KI + sw_off(64, 32 * hf + e, c), v[e]);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (s_flags[0]) break;
-
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (uint32_t kk = 0; kk < 8; ++kk)
-                mma_bf16_ss(tmem + TM_U, kdesc(sbase + OFF_ST, 128, kk),
-                            kdesc(sbase + OFF_KI, 64, kk), IDESC_N64_NEG, 1);
-            mma_commit(bar_mma);
-        }
-        wait_bar(bar_mma, ph_mma);
-        tc_fence_after();
-
-        // ---- U^T (lane d, column j) -> bf16 tile (reuses the (beta K~)^T tile); S^T *= gamma
-        {
-            float v[32];
-            tmem_ld32(tmem + lane_base + TM_U + 32 * hf, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8)
-                st_chunk(sm + OFF_KBT + sw_chunk(128, r, 32 * hf + 8 * q8), v + 8 * q8);
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int c0 = 64 * hf + 32 * part;
-                tmem_ld32(tmem + lane_base + TM_S + c0, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] *= s_gamma[c0 + e];
-                tmem_st32(tmem + lane_base + TM_S + c0, v);
-            }
-            tmem_wait_st();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (s_flags[0]) break;
-
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_O, kdesc(sbase + OFF_KBT, 128, kk),
-                            kdesc(sbase + OFF_AQK, 64, kk), IDESC_N64, 1);
-#pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_S, kdesc(sbase + OFF_KBT, 128, kk),
-                            kdesc(sbase + OFF_KHT, 128, kk), IDESC_N128, 1);
-            mma_commit(bar_mma);
-        }
-        wait_bar(bar_mma, ph_mma);
-        tc_fence_after();
-
-        // ---- outputs (O^T: lane d, column i) and the new state's bf16 copy
-        {
-            const int d = r;
-            float v[32];
-            tmem_ld32(tmem + lane_base + TM_O + 32 * hf, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int i = 32 * hf + e;
-                if (i < valid) p.out[((size_t)(t0 + i) * H + h) * D + d] = __float2bfloat16_rn(v[e]);
-            }
-            const bool last = ci + 1 == nchunks;
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int c0 = 64 * hf + 32 * part;
-                tmem_ld32(tmem + lane_base + TM_S + c0, v);
-                tmem_wait_ld();
+            if (lane < 16) {
+                const int i = 16 * quad + lane;
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8)
-                    st_chunk(sm + OFF_ST + sw_chunk(128, d, c0 + 8 * q8), v + 8 * q8);
-                if (last && p.sT) {
+                    st_chunk(sm + SM::W + tchunk(8192, i, col + 8 * q8), v + 8 * q8);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (s_flags[0]) break;
+
+        if (tid == 0) {
+            tc_fence_after();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) p.sT[state_off + (size_t)(c0 + e) * D + d] = v[e];
+            for (uint32_t kk = 0; kk < 8; ++kk)  // U = U~ - W S
+                mma_bf16_ss(tmem + TM::U, desc_k(sb + SM::W, 8192, kk),
+                            desc_mn(sb + SM::S, 16384, kk), I_UWS, 1);
+            if (DS > 64) {  // O = Q~ S (W's columns are free now)
+#pragma unroll
+                for (uint32_t kk = 0; kk < 8; ++kk)
+                    mma_bf16_ss(tmem + TM::O, desc_k(sb + SM::QK, 16384, kk),
+                                desc_mn(sb + SM::S, 16384, kk), I_UT, kk > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        wait_bar(bar_mma, ph_mma);
+        tc_fence_after();
+        if (DS > 64) {
+            if (tid == 0 && has_next) issue_qk(t0 + C);
+            qk_pending = has_next;
+        }
+
+        // ---- U (TMEM, M=64) -> bf16 tile [j][d]
+#pragma unroll
+        for (int part = 0; part < SCOLS / 32; ++part) {
+            const int col = half * SCOLS + 32 * part;
+            float v[32];
+            tmem_ld32(tmem + lane_base + TM::U + col, v);
+            tmem_wait_ld();
+            if (lane < 16) {
+                const int j = 16 * quad + lane;
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8)
+                    st_chunk(sm + SM::U + tchunk(8192, j, col + 8 * q8), v + 8 * q8);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (s_flags[0]) break;
+
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)  // O += A U
+                mma_bf16_ss(tmem + TM::O, desc_k(sb + SM::AQK, 8192, kk),
+                            desc_mn(sb + SM::U, 8192, kk), I_UT, 1);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)  // S += K-^T U   (K^^T U on the exact path)
+                mma_bf16_ss(tmem + TM::S, desc_mn(sb + SM::KI, 8192, kk),
+                            desc_mn(sb + SM::U, 8192, kk), I_S, 1);
+            mma_commit(bar_mma);
+        }
+        wait_bar(bar_mma, ph_mma);
+        tc_fence_after();
+
+        // ---- outputs (O: M=64 rows) and the next state (S *= gamma on the fast path)
+        {
+            float v[32];
+#pragma unroll
+            for (int part = 0; part < SCOLS / 32; ++part) {
+                const int col = half * SCOLS + 32 * part;
+                tmem_ld32(tmem + lane_base + TM::O + col, v);
+                tmem_wait_ld();
+                const int i = 16 * quad + lane;
+                if (lane < 16 && i < valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(
+                        p.out + ((size_t)(t0 + i) * H + h) * D + d0 + col);
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8)
+                        dst[q8] = make_uint4(pack2(v[8 * q8], v[8 * q8 + 1]),
+                                             pack2(v[8 * q8 + 2], v[8 * q8 + 3]),
+                                             pack2(v[8 * q8 + 4], v[8 * q8 + 5]),
+                                             pack2(v[8 * q8 + 6], v[8 * q8 + 7]));
                 }
             }
+            const float gm = safe ? 1.f : s_gamma[c_me];
+#pragma unroll
+            for (int part = 0; part < SCOLS / 32; ++part) {
+                const int col = half * SCOLS + 32 * part;
+                const uint32_t ta = tmem + lane_base + TM::S + col;
+                tmem_ld32(ta, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] *= gm;
+                if (!safe) tmem_st32(ta, v);
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8)
+                    st_chunk(sm + SM::S + tchunk(16384, c_me, col + 8 * q8), v + 8 * q8);
+                if (!has_next && p.sT) {
+                    float *dst = p.sT + state_off + (size_t)c_me * D + d0 + col;
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4 *>(dst + e) =
+                            make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                }
+            }
+            tmem_wait_st();
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -558,9 +696,10 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
     // ---- teardown: on an abort, let in-flight copies and MMAs land before freeing TMEM
     if (s_flags[0] && tid == 0) {
-        const uint64_t dl = globaltimer_ns() + deadline_step;
+        const uint64_t dl = globaltimer_ns() + p.timeout_ns;
         if (qk_pending) mbar_wait_bounded(bar_qk, ph_qk, dl);
-        if (lv_pending) mbar_wait_bounded(bar_lv, ph_lv, dl);
+        if (la_pending) mbar_wait_bounded(bar_la, ph_la, dl);
+        if (v_pending) mbar_wait_bounded(bar_v, ph_v, dl);
         mma_commit(bar_mma);
         mbar_wait_bounded(bar_mma, ph_mma, dl);
     }
@@ -568,7 +707,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, TM_COLS);
+        tmem_dealloc(tmem, TM::COLS);
     }
 }
 
@@ -636,6 +775,21 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint32_t
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int DS>
+cudaError_t launch_ds(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                      const CUtensorMap &mla, const ChunkParams &cp, unsigned grid,
+                      cudaStream_t stream) {
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(chunk_kernel<DS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)Smem<DS>::BYTES);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    chunk_kernel<DS><<<grid, NT, Smem<DS>::BYTES, stream>>>(mq, mk, mv, mla, cp);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_bounded_wait_probe(void *workspace, uint64_t timeout_ns, cudaStream_t stream) {
@@ -653,20 +807,22 @@ size_t chunk_workspace_bytes(int32_t num_seqs) {
 
 cudaError_t launch_prefill_chunk(const Problem &p, void *workspace, cudaStream_t stream,
                                  uint64_t timeout_ns) {
+    // Few (sequence, head) pairs cannot fill the GPU: split d_v across two CTAs per head.
+    int sms = 148;
+    {
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    const int64_t heads = (int64_t)p.num_seqs * p.H;
+    const int nsplit = heads * 2 <= sms ? 2 : 1;
     CUtensorMap mq, mk, mv, mla;
     const uint64_t T = (uint64_t)p.total_tokens, H = (uint64_t)p.H;
     if (!make_map(&mq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, H, T, 64, true) ||
         !make_map(&mk, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, H, T, 64, true) ||
-        !make_map(&mv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, H, T, D, false) ||
+        !make_map(&mv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, H, T, 64, true) ||
         !make_map(&mla, p.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, H, T, D, false))
         return cudaErrorInvalidValue;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)SMEM_BYTES);
-    });
-    if (attr_err != cudaSuccess) return attr_err;
     int32_t *status = reinterpret_cast<int32_t *>(workspace);
     int32_t *order = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + 256);
     const int plan_threads = 256;
@@ -684,9 +840,9 @@ cudaError_t launch_prefill_chunk(const Problem &p, void *workspace, cudaStream_t
     cp.status = status;
     cp.H = p.H;
     cp.timeout_ns = timeout_ns;
-    const unsigned grid = (unsigned)p.num_seqs * (unsigned)p.H;
-    chunk_kernel<<<grid, NT, SMEM_BYTES, stream>>>(mq, mk, mv, mla, cp);
-    return cudaGetLastError();
+    const unsigned grid = (unsigned)(heads * nsplit);
+    return nsplit == 2 ? launch_ds<64>(mq, mk, mv, mla, cp, grid, stream)
+                       : launch_ds<128>(mq, mk, mv, mla, cp, grid, stream);
 }
 
 }  // namespace kda

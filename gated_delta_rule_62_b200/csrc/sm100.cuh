@@ -103,26 +103,30 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 }
 
 // ---------------------------------------------------------------- descriptors
-// K-major operand tile in the 128-byte swizzled canonical layout: rows of 128 B
-// (64 bf16 along K), 8-row groups 1024 B apart, 16-byte chunk index XOR (row % 8).
-// start: shared address (16-byte units in the descriptor); SBO = 1024 B; LBO unused.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+// Shared-memory operand descriptor for the 128-byte swizzled canonical layouts: rows of
+// 128 B, 8-row swizzle atoms 1024 B apart. For a K-major operand `lbo` is unused and `sbo`
+// is the pitch of 8-row (M/N) groups; for an MN-major operand `lbo` is the pitch of
+// 64-element M/N blocks and `sbo` the pitch of 8-row (K) groups.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = 0;
-    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);         // start address
-    d |= (uint64_t)(1u) << 16;                         // leading byte offset (unused for SW128 K-major)
-    d |= (uint64_t)((1024u >> 4) & 0x3FFFu) << 32;     // stride byte offset: 8-row group pitch
-    d |= (uint64_t)1u << 46;                           // descriptor version (sm_100)
-    d |= (uint64_t)2u << 61;                           // layout: SWIZZLE_128B
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);            // start address
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;        // leading byte offset
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;        // stride byte offset
+    d |= (uint64_t)1u << 46;                            // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                            // layout: SWIZZLE_128B
     return d;
 }
 
-// kind::f16 instruction descriptor: bf16 A and B (K-major), fp32 accumulator.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool negate_a = false) {
+// kind::f16 instruction descriptor: bf16 A and B, fp32 accumulator; a_mn / b_mn select
+// MN-major operands; negate_a negates A.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool negate_a = false,
+                                                      int a_mn = 0, int b_mn = 0) {
     return (1u << 4)                      // D format: f32
            | (1u << 7)                    // A format: bf16
            | (1u << 10)                   // B format: bf16
            | ((negate_a ? 1u : 0u) << 13) // negate A
-           | (0u << 15) | (0u << 16)      // A, B K-major
+           | ((uint32_t)a_mn << 15)       // A major: 0 = K, 1 = MN
+           | ((uint32_t)b_mn << 16)       // B major
            | ((uint32_t)(N >> 3) << 17)   // N / 8
            | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
