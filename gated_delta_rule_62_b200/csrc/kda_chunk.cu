@@ -131,25 +131,51 @@ __device__ __forceinline__ void warp_store16(float *X, int px, const float (&acc
     }
 }
 
-// T = (I + L)^-1 in place for strictly lower-triangular L (fp32, pitch LT_LD, zeros on and
-// above the diagonal). Blocks of 16: the diagonal blocks by forward substitution, then the
-// block inverse [[A,0],[B,C]]^-1 = [[A^-1,0],[-C^-1 B A^-1, C^-1]] at 16 and then at 32.
-// Called by all NT threads (contains __syncthreads).
-__device__ void invert_unit_lower(float *LT, float *PB, int tid) {
+// Writes rows of a 16x16 fragment tile as bf16 T' = T diag(beta) into the TT tile at (r0, c0).
+__device__ __forceinline__ void frag_to_tt(uint8_t *TT, int r0, int c0, const float (&acc)[2][4],
+                                           float s, const float *beta) {
+    const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int c = c0 + 8 * nt + 2 * tig;
+        const float b0 = s * beta[c], b1 = s * beta[c + 1];
+        st_bf2(TT + telem(8192, r0 + gid, c), acc[nt][0] * b0, acc[nt][1] * b1);
+        st_bf2(TT + telem(8192, r0 + gid + 8, c), acc[nt][2] * b0, acc[nt][3] * b1);
+    }
+}
+
+// T = (I + L)^-1 for strictly lower-triangular L (fp32 in LT, pitch LT_LD, zeros on and
+// above the diagonal), written as bf16 T' = T diag(beta) into the lower blocks of TT (its
+// strictly upper 16x16 blocks must already be zero). Blocks of 16: the diagonal blocks by
+// forward substitution, then the block inverse [[A,0],[B,C]]^-1 = [[A^-1,0],[-C^-1 B A^-1,
+// C^-1]] at 16 and then at 32, on the tensor cores (tf32 mma.sync). LT keeps the fp32 blocks
+// later stages need. Called by all NT threads; ends with the TT stores issued (no barrier).
+__device__ void invert_unit_lower(float *LT, float *PB, uint8_t *TT, const float *beta, int tid) {
     const int warp = tid >> 5, lane = tid & 31;
     if (warp < 4 && lane < 16) {
-        float *Lb = LT + (16 * warp) * LT_LD + 16 * warp;
+        const int b0 = 16 * warp;
+        const float *Lb = LT + b0 * LT_LD + b0;
+        // all 120 sub-diagonal values first (independent loads), then a dependency chain of 15
+        float lv[120];
+#pragma unroll
+        for (int j = 0, e = 0; j < 15; ++j)
+#pragma unroll
+            for (int i = j + 1; i < 16; ++i, ++e) lv[e] = Lb[i * LT_LD + j];
         float x[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float s = (i == lane) ? 1.f : 0.f;
+        for (int i = 0; i < 16; ++i) x[i] = (i == lane) ? 1.f : 0.f;
 #pragma unroll
-            for (int j = 0; j < i; ++j) s = fmaf(-Lb[i * LT_LD + j], x[j], s);
-            x[i] = s;
-        }
+        for (int j = 0, e = 0; j < 15; ++j)
+#pragma unroll
+            for (int i = j + 1; i < 16; ++i, ++e) x[i] = fmaf(-lv[e], x[j], x[i]);
         __syncwarp(0x0000ffffu);
+        float *Tb = LT + b0 * LT_LD + b0;
+        const float bl = beta[b0 + lane];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) Lb[i * LT_LD + lane] = x[i];
+        for (int i = 0; i < 16; ++i) {
+            Tb[i * LT_LD + lane] = x[i];
+            st_bf(TT + telem(8192, b0 + i, b0 + lane), x[i] * bl);
+        }
     }
     __syncthreads();
     if (warp < 2) {
@@ -163,6 +189,7 @@ __device__ void invert_unit_lower(float *LT, float *PB, int tid) {
         float acc2[2][4] = {};
         warp_mm16(acc2, LT + r0 * LT_LD + r0, LT_LD, P, PB_LD, 16);
         warp_store16(LT + r0 * LT_LD + c0, LT_LD, acc2, -1.f);
+        frag_to_tt(TT, r0, c0, acc2, -1.f, beta);
     }
     __syncthreads();
     // rows 32..63 x cols 0..31: P = L[32:64, 0:32] T[0:32, 0:32];  T[32:64, 0:32] = -T[32:64, 32:64] P
@@ -176,9 +203,8 @@ __device__ void invert_unit_lower(float *LT, float *PB, int tid) {
     if (warp < 4) {
         float acc[2][4] = {};
         warp_mm16(acc, LT + (32 + 16 * rt) * LT_LD + 32, LT_LD, PB + 16 * ct, PB_LD, 32);
-        warp_store16(LT + (32 + 16 * rt) * LT_LD + 16 * ct, LT_LD, acc, -1.f);
+        frag_to_tt(TT, 32 + 16 * rt, 16 * ct, acc, -1.f, beta);
     }
-    __syncthreads();
 }
 
 // ---------------------------------------------------------------- shared memory map
@@ -315,6 +341,10 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         qk_pending = la_pending = v_pending = true;
     }
 
+    // The strictly upper 16x16 blocks of T' are zero for every chunk.
+    for (int e = tid; e < 8192 / 16; e += NT)
+        reinterpret_cast<uint4 *>(sm + SM::TT)[e] = make_uint4(0u, 0u, 0u, 0u);
+
     // Initial state -> S (TMEM fp32, lane c, columns d) and its bf16 tile [c][d].
     {
         const size_t row = state_off + (size_t)c_me * D + d0 + half * SCOLS;
@@ -352,7 +382,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
     uint32_t ph_qk = 0, ph_la = 0, ph_v = 0, ph_mma = 0;
     auto wait_bar = [&](uint64_t *bar, uint32_t &ph) {
-        const bool ok = mbar_wait_bounded(bar, ph, globaltimer_ns() + p.timeout_ns);
+        const bool ok = mbar_wait_bounded(bar, ph, p.timeout_ns);
         ph ^= 1u;
         if (!ok) {
             s_flags[0] = 1;
@@ -360,37 +390,43 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         }
     };
 
-    // gating thread mapping: channel pair (cA, cA + 1), token quarter tq
+    // gating thread mapping: channel pair (cA, cA + 1), token quarter tq (tokens 16 tq .. +15)
     const int tq = tid >> 6, cA = 2 * (tid & 63);
+    // beta of the next chunk is loaded one chunk ahead (one value per thread < C)
+    float beta_next = 0.f;
+    if (nchunks > 0 && tid < C && bos + tid < eos) beta_next = p.beta[(size_t)(bos + tid) * H + h];
 
     for (int ci = 0; ci < nchunks; ++ci) {
         const int64_t t0 = bos + (int64_t)ci * C;
         const int valid = (int)(eos - t0 < C ? eos - t0 : C);
         const bool has_next = ci + 1 < nchunks;
-        if (tid < C) s_beta[tid] = (tid < valid) ? p.beta[(size_t)(t0 + tid) * H + h] : 0.f;
-        if (tid == 0) s_flags[1] = 0;
+        if (tid < C) {
+            s_beta[tid] = beta_next;
+            beta_next = (has_next && t0 + C + tid < eos) ? p.beta[(size_t)(t0 + C + tid) * H + h] : 0.f;
+        }
         wait_bar(bar_la, ph_la);
         wait_bar(bar_qk, ph_qk);
         la_pending = qk_pending = false;
-        __syncthreads();
-        if (s_flags[0]) break;
 
-        // ---- gate cumsum: local prefix over this thread's 16 tokens of two channels
-        {
-            float2 acc = make_float2(0.f, 0.f);
-#pragma unroll 4
-            for (int i = 0; i < 16; ++i) {
-                const int t = 16 * tq + i;
-                float2 *pl = reinterpret_cast<float2 *>(LA + t * D + cA);
-                const float2 x = (t < valid) ? *pl : make_float2(0.f, 0.f);
-                acc.x += x.x;
-                acc.y += x.y;
-                *pl = acc;
-            }
-            s_psum[tq * D + cA] = acc.x;
-            s_psum[tq * D + cA + 1] = acc.y;
+        // ---- gates: log_alpha of 16 tokens x 2 channels into registers, quarter totals
+        float2 la[16];
+        float2 tot = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int t = 16 * tq + i;
+            la[i] = (t < valid) ? *reinterpret_cast<const float2 *>(LA + t * D + cA)
+                                : make_float2(0.f, 0.f);
+            tot.x += la[i].x;
+            tot.y += la[i].y;
         }
-        __syncthreads();
+        s_psum[tq * D + cA] = tot.x;
+        s_psum[tq * D + cA + 1] = tot.y;
+        // A quarter decaying by more than e^(kFastLimit/4) in some channel sends the chunk
+        // down the exact path; otherwise the whole chunk decays by at most e^kFastLimit.
+        // (NaN gates also take the exact path: the comparisons are false for NaN.)
+        const int unsafe = !(-tot.x <= 0.25f * kFastLimit) || !(-tot.y <= 0.25f * kFastLimit);
+        const bool safe = __syncthreads_or(unsafe) != 0;
+        if (s_flags[0]) break;
         float2 goff = make_float2(0.f, 0.f), gC = make_float2(0.f, 0.f);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -402,23 +438,19 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         if (tq == 0) {
             s_gamma[cA] = __expf(gC.x);
             s_gamma[cA + 1] = __expf(gC.y);
-            // Any channel decaying by more than e^kFastLimit sends the chunk down the exact
-            // path (also non-finite gates: the comparison is false for NaN).
-            if (!(-gC.x <= kFastLimit) || !(-gC.y <= kFastLimit)) s_flags[1] = 1u;
         }
-        __syncthreads();
-        const bool safe = s_flags[1] != 0u;
 
         if (safe) {
             // Exact path: A and L pairwise from raw q, k and the full g (no factored exponentials).
-            if (tq > 0) {
+            {
+                float2 g = goff;
+#pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    float2 *pl = reinterpret_cast<float2 *>(LA + (16 * tq + i) * D + cA);
-                    const float2 x = *pl;
-                    *pl = make_float2(x.x + goff.x, x.y + goff.y);
+                    g.x += la[i].x;
+                    g.y += la[i].y;
+                    *reinterpret_cast<float2 *>(LA + (16 * tq + i) * D + cA) = g;
                 }
             }
-            goff = make_float2(0.f, 0.f);
             for (int e = tid; e < 64 * 64; e += NT) {
                 const int i = e >> 6, j = e & 63;
                 st_bf(sm + SM::AQK + telem(8192, i, j), 0.f);
@@ -448,6 +480,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 }
             }
             // S <- diag(gamma) S ahead of S += K^^T U
+            __syncthreads();
             const float gm = s_gamma[c_me];
 #pragma unroll
             for (int part = 0; part < SCOLS / 32; ++part) {
@@ -464,22 +497,39 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             __syncthreads();
         }
 
-        // ---- gated operands: Q~, K~ in place; K- (fast) or K^ (exact) into the KI tile
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-            const int t = 16 * tq + i;
-            const bool ok = t < valid;
-            const float2 lg = *reinterpret_cast<const float2 *>(LA + t * D + cA);
-            const float g0 = goff.x + lg.x, g1 = goff.y + lg.y;
-            const float e0 = __expf(g0), e1 = __expf(g1);
-            uint8_t *qp = sm + SM::QK + telem(16384, t, cA);
-            uint8_t *kp = sm + SM::QK + telem(16384, 64 + t, cA);
-            float2 qv = ld_bf2(qp), kv = ld_bf2(kp);
-            if (!ok) qv = kv = make_float2(0.f, 0.f);
-            st_bf2(qp, qv.x * e0, qv.y * e1);
-            st_bf2(kp, kv.x * e0, kv.y * e1);
-            const float m0 = __expf(safe ? gC.x - g0 : -g0), m1 = __expf(safe ? gC.y - g1 : -g1);
-            st_bf2(sm + SM::KI + telem(8192, t, cA), kv.x * m0, kv.y * m1);
+        // ---- gated operands. With alpha = e^log_alpha, prefix products P_i and suffix
+        // products R_i (within the quarter): e^g_i = e^goff P_i; e^-g_i = e^(-goff-tot) R_i;
+        // e^(g_C - g_i) = e^(g_C-goff-tot) R_i. Q~, K~ overwrite q, k in place; the KI tile
+        // gets K- (fast path) or K^ (exact path).
+        {
+            float2 al[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) al[i] = make_float2(__expf(la[i].x), __expf(la[i].y));
+            const float2 eA = make_float2(__expf(goff.x), __expf(goff.y));
+            const float2 eB = safe ? make_float2(__expf(gC.x - goff.x - tot.x), __expf(gC.y - goff.y - tot.y))
+                                   : make_float2(__expf(-goff.x - tot.x), __expf(-goff.y - tot.y));
+            float2 R[16];
+            float2 run = make_float2(1.f, 1.f);
+#pragma unroll
+            for (int i = 15; i >= 0; --i) {
+                R[i] = run;
+                run.x *= al[i].x;
+                run.y *= al[i].y;
+            }
+            float2 P = eA;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int t = 16 * tq + i;
+                P.x *= al[i].x;
+                P.y *= al[i].y;
+                uint8_t *qp = sm + SM::QK + telem(16384, t, cA);
+                uint8_t *kp = sm + SM::QK + telem(16384, 64 + t, cA);
+                float2 qv = ld_bf2(qp), kv = ld_bf2(kp);
+                if (t >= valid) qv = kv = make_float2(0.f, 0.f);
+                st_bf2(qp, qv.x * P.x, qv.y * P.y);
+                st_bf2(kp, kv.x * P.x, kv.y * P.y);
+                st_bf2(sm + SM::KI + telem(8192, t, cA), kv.x * (eB.x * R[i].x), kv.y * (eB.y * R[i].y));
+            }
         }
         fence_proxy_async_smem();
         __syncthreads();
@@ -535,16 +585,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         __syncthreads();
         if (s_flags[0]) break;
 
-        // ---- T = (I + L)^-1; T' = T diag(beta) to bf16
-        invert_unit_lower(LT, PB, tid);
-        {
-            const int i = tid >> 2, j0 = (tid & 3) * 16;
-            float v[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = LT[i * LT_LD + j0 + e] * s_beta[j0 + e];
-            st_chunk(sm + SM::TT + tchunk(8192, i, j0), v);
-            st_chunk(sm + SM::TT + tchunk(8192, i, j0 + 8), v + 8);
-        }
+        // ---- T' = (I + L)^-1 diag(beta), bf16, into the TT tile
+        invert_unit_lower(LT, PB, sm + SM::TT, s_beta, tid);
         fence_proxy_async_smem();
         __syncthreads();
 
@@ -696,12 +738,11 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
     // ---- teardown: on an abort, let in-flight copies and MMAs land before freeing TMEM
     if (s_flags[0] && tid == 0) {
-        const uint64_t dl = globaltimer_ns() + p.timeout_ns;
-        if (qk_pending) mbar_wait_bounded(bar_qk, ph_qk, dl);
-        if (la_pending) mbar_wait_bounded(bar_la, ph_la, dl);
-        if (v_pending) mbar_wait_bounded(bar_v, ph_v, dl);
+        if (qk_pending) mbar_wait_bounded(bar_qk, ph_qk, p.timeout_ns);
+        if (la_pending) mbar_wait_bounded(bar_la, ph_la, p.timeout_ns);
+        if (v_pending) mbar_wait_bounded(bar_v, ph_v, p.timeout_ns);
         mma_commit(bar_mma);
-        mbar_wait_bounded(bar_mma, ph_mma, dl);
+        mbar_wait_bounded(bar_mma, ph_mma, p.timeout_ns);
     }
     tc_fence_before();
     __syncthreads();
@@ -737,7 +778,7 @@ __global__ void bounded_wait_probe(int32_t *status, uint64_t timeout_ns) {
         fence_mbarrier_init();
     }
     __syncthreads();
-    if (!mbar_wait_bounded(&bar, 0, globaltimer_ns() + timeout_ns) && threadIdx.x == 0)
+    if (!mbar_wait_bounded(&bar, 0, timeout_ns) && threadIdx.x == 0)
         atomicOr(status, 1);
 }
 

@@ -51,14 +51,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
-// Bounded wait: spins until the phase with `parity` completes or `deadline_ns`
-// (a %globaltimer value) passes. Returns false on timeout.
+// Bounded wait: spins until the phase with `parity` completes or `timeout_ns` have passed
+// (measured on %globaltimer, read only once the phase is found incomplete). Returns false on
+// timeout.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
-                                                  uint64_t deadline_ns) {
+                                                  uint64_t timeout_ns) {
     if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t deadline = globaltimer_ns() + timeout_ns;
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() > deadline_ns) return false;
+        if (globaltimer_ns() > deadline) return false;
     }
 }
 
