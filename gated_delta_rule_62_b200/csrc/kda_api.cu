@@ -109,8 +109,15 @@ size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_
     if (num_seqs < 0 || total_tokens < 0 || H <= 0 || !supported_d(d_k) || !supported_d(d_v) ||
         (dtype != KDA_F32 && dtype != KDA_BF16))
         return 0;
-    // [0, 256): device status word; then the per-sequence schedule (int32 each).
-    return kda::chunk_workspace_bytes(num_seqs);
+    // [0, 256): device status word; then the per-sequence schedule (int32 each). Few-head
+    // problems also get room for the split-role kernel's ring of chunk images.
+    const size_t fused = kda::chunk_workspace_bytes(num_seqs);
+    const int64_t heads = (int64_t)num_seqs * H;
+    if (kda::split_eligible(heads, dtype, d_k, d_v)) {
+        const size_t split = kda::split_workspace_bytes(heads);
+        return split > fused ? split : fused;
+    }
+    return fused;
 }
 
 kda_status_t kda_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -123,7 +130,9 @@ kda_status_t kda_prefill(const void *q, const void *k, const void *v, const floa
                                     cu_seqlens_host, num_seqs, total_tokens, H, d_k, d_v, dtype,
                                     out, final_state);
     if (st != KDA_OK || num_seqs == 0) return st;
-    const size_t need = kda_prefill_workspace_size(num_seqs, total_tokens, H, d_k, d_v, dtype);
+    // Any workspace of the minimum size is accepted; a larger one (as sized by
+    // kda_prefill_workspace_size) lets few-head problems use the split-role kernel.
+    const size_t need = kda::chunk_workspace_bytes(num_seqs);
     if (!workspace || workspace_bytes < need)
         return fail(KDA_ERR_INVALID_ARGUMENT, "workspace %p of %zu bytes < required %zu",
                     workspace, workspace_bytes, need);
@@ -133,7 +142,17 @@ kda_status_t kda_prefill(const void *q, const void *k, const void *v, const floa
     kda::Problem p = make_problem(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev,
                                   num_seqs, total_tokens, H, d_k, d_v, dtype, out, final_state);
     cudaError_t e;
-    if (kda::chunk_supported(p)) {
+    int32_t max_chunks = 0;
+    for (int32_t n = 0; n < num_seqs; ++n) {
+        const int32_t c = (cu_seqlens_host[n + 1] - cu_seqlens_host[n] + 63) / 64;
+        max_chunks = c > max_chunks ? c : max_chunks;
+    }
+    const int64_t heads = (int64_t)num_seqs * H;
+    if (kda::chunk_supported(p) && max_chunks >= 2 && kda::split_eligible(heads, dtype, d_k, d_v) &&
+        workspace_bytes >= kda::split_workspace_bytes(heads)) {
+        // few heads: consumer CTAs run the state chains, producer CTAs fill the other SMs
+        e = kda::launch_prefill_split(p, max_chunks, workspace, s, kda::kWaitTimeoutNs);
+    } else if (kda::chunk_supported(p)) {
         // the planning kernel clears the status word
         e = kda::launch_prefill_chunk(p, workspace, s, kda::kWaitTimeoutNs);
     } else {

@@ -1,0 +1,376 @@
+// Device building blocks shared by the chunked-prefill kernels (kda_chunk.cu, kda_chunk_split.cu):
+// 128-byte-swizzled tile addressing, tcgen05 operand descriptors, bf16 packing, the 64x64 unit
+// lower-triangular inverse, the gating of one chunk, and TMEM epilogues. See kda_chunk.cu for the
+// chunk algebra these implement.
+#pragma once
+
+#include <cuda.h>
+
+#include "kda_internal.cuh"
+#include "sm100.cuh"
+
+namespace kda {
+namespace chunk {
+
+using namespace sm100;
+
+constexpr int C = 64;    // chunk length
+constexpr int D = 128;   // d_k = d_v
+constexpr int NT = 256;  // compute threads per CTA
+constexpr float kFastLimit = 60.f;  // max in-chunk decay exponent for the factored path
+
+// ---------------------------------------------------------------- tile addressing
+// bf16 tiles use the 128-byte swizzle: 128-byte rows of 64 elements, 8-row groups
+// 1024 bytes apart, 16-byte chunk index XOR (row % 8); 64-column blocks `bs` bytes apart.
+__device__ __forceinline__ uint32_t tchunk(uint32_t bs, uint32_t row, uint32_t col) {
+    return (col >> 6) * bs + (row >> 3) * 1024 + (row & 7) * 128 +
+           ((((col & 63) >> 3) ^ (row & 7)) << 4);
+}
+__device__ __forceinline__ uint32_t telem(uint32_t bs, uint32_t row, uint32_t col) {
+    return tchunk(bs, row, col) + ((col & 7) << 1);
+}
+
+// Operand descriptors for K step kk (16 elements along K).
+// K-major tile (rows = M/N, columns = K): K advances 32 bytes inside a row, K blocks at bs.
+__device__ __forceinline__ uint64_t desc_k(uint32_t base, uint32_t bs, uint32_t kk) {
+    return smem_desc_sw128(base + (kk >> 2) * bs + (kk & 3) * 32, 16, 1024);
+}
+// MN-major tile (rows = K, columns = M/N): K advances two 8-row groups, MN blocks at bs.
+__device__ __forceinline__ uint64_t desc_mn(uint32_t base, uint32_t bs, uint32_t kk) {
+    return smem_desc_sw128(base + kk * 2048, bs, 1024);
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ void st_chunk(uint8_t *p, const float *v) {
+    *reinterpret_cast<uint4 *>(p) = make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]),
+                                               pack2(v[4], v[5]), pack2(v[6], v[7]));
+}
+__device__ __forceinline__ float2 ld_bf2(const uint8_t *p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+}
+__device__ __forceinline__ void st_bf2(uint8_t *p, float a, float b) {
+    *reinterpret_cast<uint32_t *>(p) = pack2(a, b);
+}
+__device__ __forceinline__ float ld_bf(const uint8_t *p) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p));
+}
+__device__ __forceinline__ void st_bf(uint8_t *p, float x) {
+    *reinterpret_cast<__nv_bfloat16 *>(p) = __float2bfloat16_rn(x);
+}
+
+// ---------------------------------------------------------------- 64x64 unit lower-triangular inverse
+constexpr int LT_LD = 68;  // fp32 pitch of the L / T scratch
+constexpr int PB_LD = 36;  // fp32 pitch of the 32x32 block-product scratch
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// acc (a 16x16 tile as two m16n8 fragments) += A[16][K] * B[K][16], fp32 in shared memory,
+// multiplied with tf32 operands by the warp-level mma.sync m16n8k8.
+__device__ __forceinline__ void warp_mm16(float (&acc)[2][4], const float *A, int pa,
+                                          const float *B, int pb, int K) {
+    const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+    for (int k = 0; k < K; k += 8) {
+        const uint32_t a0 = to_tf32(A[gid * pa + k + tig]);
+        const uint32_t a1 = to_tf32(A[(gid + 8) * pa + k + tig]);
+        const uint32_t a2 = to_tf32(A[gid * pa + k + tig + 4]);
+        const uint32_t a3 = to_tf32(A[(gid + 8) * pa + k + tig + 4]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t b0 = to_tf32(B[(k + tig) * pb + 8 * nt + gid]);
+            const uint32_t b1 = to_tf32(B[(k + tig + 4) * pb + 8 * nt + gid]);
+            asm volatile(
+                "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, "
+                "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
+                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+}
+__device__ __forceinline__ void warp_store16(float *X, int px, const float (&acc)[2][4], float s) {
+    const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        X[gid * px + 8 * nt + 2 * tig] = s * acc[nt][0];
+        X[gid * px + 8 * nt + 2 * tig + 1] = s * acc[nt][1];
+        X[(gid + 8) * px + 8 * nt + 2 * tig] = s * acc[nt][2];
+        X[(gid + 8) * px + 8 * nt + 2 * tig + 1] = s * acc[nt][3];
+    }
+}
+
+// Writes rows of a 16x16 fragment tile as bf16 T' = T diag(beta) into the TT tile at (r0, c0).
+__device__ __forceinline__ void frag_to_tt(uint8_t *TT, int r0, int c0, const float (&acc)[2][4],
+                                           float s, const float *beta) {
+    const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int c = c0 + 8 * nt + 2 * tig;
+        const float b0 = s * beta[c], b1 = s * beta[c + 1];
+        st_bf2(TT + telem(8192, r0 + gid, c), acc[nt][0] * b0, acc[nt][1] * b1);
+        st_bf2(TT + telem(8192, r0 + gid + 8, c), acc[nt][2] * b0, acc[nt][3] * b1);
+    }
+}
+
+// T = (I + L)^-1 for strictly lower-triangular L (fp32 in LT, pitch LT_LD, zeros on and
+// above the diagonal), written as bf16 T' = T diag(beta) into the lower blocks of TT (its
+// strictly upper 16x16 blocks must already be zero). Blocks of 16: the diagonal blocks by
+// forward substitution, then the block inverse [[A,0],[B,C]]^-1 = [[A^-1,0],[-C^-1 B A^-1,
+// C^-1]] at 16 and then at 32, on the tensor cores (tf32 mma.sync). LT keeps the fp32 blocks
+// later stages need. Called by all NT threads; ends with the TT stores issued (no barrier).
+static __device__ void invert_unit_lower(float *LT, float *PB, uint8_t *TT, const float *beta, int tid) {
+    const int warp = tid >> 5, lane = tid & 31;
+    if (warp < 4 && lane < 16) {
+        const int b0 = 16 * warp;
+        const float *Lb = LT + b0 * LT_LD + b0;
+        // all 120 sub-diagonal values first (independent loads), then a dependency chain of 15
+        float lv[120];
+#pragma unroll
+        for (int j = 0, e = 0; j < 15; ++j)
+#pragma unroll
+            for (int i = j + 1; i < 16; ++i, ++e) lv[e] = Lb[i * LT_LD + j];
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = (i == lane) ? 1.f : 0.f;
+#pragma unroll
+        for (int j = 0, e = 0; j < 15; ++j)
+#pragma unroll
+            for (int i = j + 1; i < 16; ++i, ++e) x[i] = fmaf(-lv[e], x[j], x[i]);
+        __syncwarp(0x0000ffffu);
+        float *Tb = LT + b0 * LT_LD + b0;
+        const float bl = beta[b0 + lane];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            Tb[i * LT_LD + lane] = x[i];
+            st_bf(TT + telem(8192, b0 + i, b0 + lane), x[i] * bl);
+        }
+    }
+    __syncthreads();
+    if (warp < 2) {
+        // warp 0: T10 = -T11 (L10 T00); warp 1: T32 = -T33 (L32 T22)
+        const int r0 = warp ? 48 : 16, c0 = warp ? 32 : 0;
+        float *P = PB + warp * 16 * PB_LD;
+        float acc[2][4] = {};
+        warp_mm16(acc, LT + r0 * LT_LD + c0, LT_LD, LT + c0 * LT_LD + c0, LT_LD, 16);
+        warp_store16(P, PB_LD, acc, 1.f);
+        __syncwarp();
+        float acc2[2][4] = {};
+        warp_mm16(acc2, LT + r0 * LT_LD + r0, LT_LD, P, PB_LD, 16);
+        warp_store16(LT + r0 * LT_LD + c0, LT_LD, acc2, -1.f);
+        frag_to_tt(TT, r0, c0, acc2, -1.f, beta);
+    }
+    __syncthreads();
+    // rows 32..63 x cols 0..31: P = L[32:64, 0:32] T[0:32, 0:32];  T[32:64, 0:32] = -T[32:64, 32:64] P
+    const int rt = (warp >> 1) & 1, ct = warp & 1;
+    if (warp < 4) {
+        float acc[2][4] = {};
+        warp_mm16(acc, LT + (32 + 16 * rt) * LT_LD, LT_LD, LT + 16 * ct, LT_LD, 32);
+        warp_store16(PB + (16 * rt) * PB_LD + 16 * ct, PB_LD, acc, 1.f);
+    }
+    __syncthreads();
+    if (warp < 4) {
+        float acc[2][4] = {};
+        warp_mm16(acc, LT + (32 + 16 * rt) * LT_LD + 32, LT_LD, PB + 16 * ct, PB_LD, 32);
+        frag_to_tt(TT, 32 + 16 * rt, 16 * ct, acc, -1.f, beta);
+    }
+}
+
+
+// ---------------------------------------------------------------- gating of one chunk
+// All NT threads. In: QK holds raw q (rows 0..63) and k (rows 64..127) as a K-major tile with
+// 16 KB blocks, LA the chunk's raw log_alpha [t][c] fp32, s_beta the chunk's beta (0 past `valid`).
+// Out: QK holds Q~ and K~ in place, KI holds K- (factored path) or K^ (exact path), s_gamma =
+// e^(g_{C-1}); the exact path also writes A into AQK and beta-scaled L into LT (zeros elsewhere).
+// Thread mapping: channel pair (cA, cA + 1), token quarter tq (tokens 16 tq .. 16 tq + 15).
+// Returns 1 for the exact path, 0 for the factored path, -1 if *s_abort was set.
+__device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK, float *LA,
+                                          float *LT, const float *s_beta, float *s_gamma,
+                                          float *s_psum, const uint32_t *s_abort, int valid,
+                                          int tid) {
+    const int tq = tid >> 6, cA = 2 * (tid & 63);
+    const int warp = tid >> 5, lane = tid & 31;
+    // ---- gates: log_alpha of 16 tokens x 2 channels into registers, quarter totals
+    float2 la[16];
+    float2 tot = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int t = 16 * tq + i;
+        la[i] = (t < valid) ? *reinterpret_cast<const float2 *>(LA + t * D + cA)
+                            : make_float2(0.f, 0.f);
+        tot.x += la[i].x;
+        tot.y += la[i].y;
+    }
+    s_psum[tq * D + cA] = tot.x;
+    s_psum[tq * D + cA + 1] = tot.y;
+    // A quarter decaying by more than e^(kFastLimit/4) in some channel sends the chunk
+    // down the exact path; otherwise the whole chunk decays by at most e^kFastLimit.
+    // (NaN gates also take the exact path: the comparisons are false for NaN.)
+    const int unsafe = !(-tot.x <= 0.25f * kFastLimit) || !(-tot.y <= 0.25f * kFastLimit);
+    const bool safe = __syncthreads_or(unsafe) != 0;
+    if (*s_abort) return -1;
+    float2 goff = make_float2(0.f, 0.f), gC = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float a = s_psum[q * D + cA], b = s_psum[q * D + cA + 1];
+        if (q < tq) { goff.x += a; goff.y += b; }
+        gC.x += a;
+        gC.y += b;
+    }
+    if (tq == 0) {
+        s_gamma[cA] = __expf(gC.x);
+        s_gamma[cA + 1] = __expf(gC.y);
+    }
+
+    if (safe) {
+        // Exact path: A and L pairwise from raw q, k and the full g (no factored exponentials).
+        {
+            float2 g = goff;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                g.x += la[i].x;
+                g.y += la[i].y;
+                *reinterpret_cast<float2 *>(LA + (16 * tq + i) * D + cA) = g;
+            }
+        }
+        for (int e = tid; e < 64 * 64; e += NT) {
+            const int i = e >> 6, j = e & 63;
+            st_bf(AQK + telem(8192, i, j), 0.f);
+            LT[i * LT_LD + j] = 0.f;
+        }
+        __syncthreads();
+        for (int e = warp; e < 64 * 64; e += NT / 32) {
+            const int i = e >> 6, j = e & 63;
+            if (j > i || i >= valid) continue;
+            float a = 0.f, l = 0.f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int cc = lane + 32 * m;
+                const float ex = __expf(LA[i * D + cc] - LA[j * D + cc]);
+                const float kj = ld_bf(QK + telem(16384, 64 + j, cc)) * ex;
+                a = fmaf(ld_bf(QK + telem(16384, i, cc)), kj, a);
+                l = fmaf(ld_bf(QK + telem(16384, 64 + i, cc)), kj, l);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                a += __shfl_xor_sync(0xffffffffu, a, off);
+                l += __shfl_xor_sync(0xffffffffu, l, off);
+            }
+            if (lane == 0) {
+                st_bf(AQK + telem(8192, i, j), a);
+                if (j < i) LT[i * LT_LD + j] = s_beta[i] * l;
+            }
+        }
+        __syncthreads();  // raw q, k are read above and overwritten below
+    }
+
+    // ---- gated operands. With alpha = e^log_alpha, prefix products P_i and suffix
+    // products R_i (within the quarter): e^g_i = e^goff P_i; e^-g_i = e^(-goff-tot) R_i;
+    // e^(g_C - g_i) = e^(g_C-goff-tot) R_i. Q~, K~ overwrite q, k in place; the KI tile
+    // gets K- (fast path) or K^ (exact path).
+    {
+        float2 al[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) al[i] = make_float2(__expf(la[i].x), __expf(la[i].y));
+        const float2 eA = make_float2(__expf(goff.x), __expf(goff.y));
+        const float2 eB = safe ? make_float2(__expf(gC.x - goff.x - tot.x), __expf(gC.y - goff.y - tot.y))
+                               : make_float2(__expf(-goff.x - tot.x), __expf(-goff.y - tot.y));
+        float2 R[16];
+        float2 run = make_float2(1.f, 1.f);
+#pragma unroll
+        for (int i = 15; i >= 0; --i) {
+            R[i] = run;
+            run.x *= al[i].x;
+            run.y *= al[i].y;
+        }
+        float2 P = eA;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int t = 16 * tq + i;
+            P.x *= al[i].x;
+            P.y *= al[i].y;
+            uint8_t *qp = QK + telem(16384, t, cA);
+            uint8_t *kp = QK + telem(16384, 64 + t, cA);
+            float2 qv = ld_bf2(qp), kv = ld_bf2(kp);
+            if (t >= valid) qv = kv = make_float2(0.f, 0.f);
+            st_bf2(qp, qv.x * P.x, qv.y * P.y);
+            st_bf2(kp, kv.x * P.x, kv.y * P.y);
+            st_bf2(KI + telem(8192, t, cA), kv.x * (eB.x * R[i].x), kv.y * (eB.y * R[i].y));
+        }
+    }    return safe ? 1 : 0;
+}
+
+// ---------------------------------------------------------------- TMEM epilogues
+// D1 (M=128: rows 0..63 = Q~ K-^T, rows 64..127 = K~ K-^T) -> A (bf16, j <= i) into AQK and
+// L (fp32, times beta_i, j < i) into LT. Thread: TMEM lane r, columns [32 half, 32 half + 32).
+__device__ __forceinline__ void extract_al(uint32_t taddr, uint8_t *AQK, float *LT,
+                                           const float *s_beta, int r, int half) {
+    float v[32];
+    tmem_ld32(taddr, v);
+    tmem_wait_ld();
+    if (r < 64) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = (32 * half + e <= r) ? v[e] : 0.f;
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8)
+            st_chunk(AQK + tchunk(8192, r, 32 * half + 8 * q8), v + 8 * q8);
+    } else {
+        const int i = r - 64;
+        const float b = s_beta[i];
+        float4 *dst = reinterpret_cast<float4 *>(LT + i * LT_LD + 32 * half);
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+            const int j = 32 * half + 4 * e4;
+            dst[e4] = make_float4(j + 0 < i ? b * v[4 * e4 + 0] : 0.f,
+                                  j + 1 < i ? b * v[4 * e4 + 1] : 0.f,
+                                  j + 2 < i ? b * v[4 * e4 + 2] : 0.f,
+                                  j + 3 < i ? b * v[4 * e4 + 3] : 0.f);
+        }
+    }
+}
+
+// An M=64 accumulator (row 16*quad + lane in lanes 0..15 of each quadrant) -> bf16 tile rows,
+// NCOLS columns starting at column col0 of both the TMEM region (taddr) and the tile.
+template <int NCOLS>
+__device__ __forceinline__ void rows64_to_tile(uint32_t taddr, uint8_t *tile, uint32_t bs,
+                                               int col0, int quad, int lane) {
+#pragma unroll
+    for (int part = 0; part < NCOLS / 32; ++part) {
+        float v[32];
+        tmem_ld32(taddr + 32 * part, v);
+        tmem_wait_ld();
+        if (lane < 16) {
+            const int row = 16 * quad + lane;
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8)
+                st_chunk(tile + tchunk(bs, row, col0 + 32 * part + 8 * q8), v + 8 * q8);
+        }
+    }
+}
+
+// S <- diag(gamma) S in TMEM for this thread's lane (gamma) and NCOLS columns at taddr.
+template <int NCOLS>
+__device__ __forceinline__ void scale_tmem_row(uint32_t taddr, float gm) {
+#pragma unroll
+    for (int part = 0; part < NCOLS / 32; ++part) {
+        float v[32];
+        tmem_ld32(taddr + 32 * part, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] *= gm;
+        tmem_st32(taddr + 32 * part, v);
+    }
+    tmem_wait_st();
+}
+
+}  // namespace chunk
+
+// 3-D TMA map over [T][H][inner] with a box of (box_inner, 1, 64 tokens); false on failure.
+bool make_token_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint32_t esize,
+                    uint64_t inner, uint64_t H, uint64_t T, uint32_t box_inner, bool swizzle);
+
+}  // namespace kda

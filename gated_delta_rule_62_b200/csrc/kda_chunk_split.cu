@@ -1,0 +1,646 @@
+// Split-role chunked prefill for workloads with few (sequence, head) pairs.
+//
+// The chunk algebra is that of kda_chunk.cu. Its key-side half -- gating, the intra-chunk
+// products A and L, T' = (I + L)^-1 diag(beta), W = T' K~ -- does not depend on the state and
+// can run for any chunk at any time; only U = T'V - W S, O = Q~ S + A U and the state update
+// form the sequential chain. With few heads a fused kernel leaves most SMs idle while each
+// head's CTA serialises both halves. Here one persistent cooperative launch fills the GPU:
+//
+//   consumer CTAs (one per head): the state chain. Per chunk: U = T'V - W S and O = Q~ S
+//     (one MMA batch), U to bf16, O += A U and S += K-^T U (one batch), then the outputs and
+//     S <- diag(gamma) S. The fp32 state stays in TMEM for the whole sequence.
+//   producer CTAs (all other SMs): the key-side half for chunks ahead, chunk-major order,
+//     written as ready-to-use shared-memory images (Q~, K- or K^, W, A, T' tiles, gamma,
+//     path flag) into a ring of RING slots per head in the workspace (L2 resident).
+//
+// Hand-off: a producer fills slot (head, c % RING) with generic stores, then releases
+// filled[slot] = c + 1; the consumer acquires it, copies the image into shared memory with a
+// bulk copy, and releases consumed[head] = c + 1 once the copy has landed; the producer
+// acquires consumed[head] >= c - RING + 1 before reusing the slot. Producer items are
+// ordered by chunk, and every producer works through its items in order, so the item a
+// consumer waits for never waits on anything later: no cycle. Every spin and mbarrier wait is
+// bounded; on timeout the status word is set and the CTA stops. The launch is cooperative,
+// so all CTAs are resident together or the launch fails.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "kda_chunk_common.cuh"
+
+namespace kda {
+namespace {
+
+using namespace sm100;
+using namespace chunk;
+
+constexpr int RING = 4;
+// Slot image (bytes): Q~ 64-row tile (8 KB blocks), K- (or K^), W, A, T', gamma[128], meta.
+constexpr uint32_t SL_Q = 0, SL_KI = 16384, SL_W = 32768, SL_A = 49152, SL_T = 57344;
+constexpr uint32_t SL_G = 65536, SL_META = 65536 + 512, SLOT = 66560;
+static_assert(SLOT % 1024 == 0 && SLOT == 4 * 16384 + 1024, "slot layout");
+
+struct SplitParams {
+    const int32_t *cu_seqlens;
+    const float *beta;
+    const float *s0;
+    float *sT;
+    __nv_bfloat16 *out;
+    int32_t *status;
+    uint8_t *ring;       // [heads][RING][SLOT]
+    int32_t *filled;     // [heads][RING]
+    int32_t *consumed;   // [heads]
+    int32_t H, heads, max_chunks;
+    uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ int ld_acquire(const int32_t *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(int32_t *p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Bounded spin until *p >= target; false on timeout.
+__device__ __forceinline__ bool wait_flag_ge(const int32_t *p, int target, uint64_t timeout_ns) {
+    if (ld_acquire(p) >= target) return true;
+    const uint64_t deadline = globaltimer_ns() + timeout_ns;
+    while (true) {
+        __nanosleep(100);
+        if (ld_acquire(p) >= target) return true;
+        if (globaltimer_ns() > deadline) return false;
+    }
+}
+// Bulk (untiled) copy global -> shared, completing on `bar` (16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// ---------------------------------------------------------------- consumer (state chain)
+namespace cons {
+constexpr uint32_t STAGE0 = 0, STAGE1 = SLOT;
+constexpr uint32_t V0 = 2 * SLOT, V1 = V0 + 16384;
+constexpr uint32_t S = V1 + 16384;   // S [c][d] bf16 128 x 128, blocks 16 KB
+constexpr uint32_t U = S + 32768;    // U [j][d] bf16 64 x 128, blocks 8 KB
+constexpr uint32_t MISC = U + 16384; // barriers, flags
+constexpr uint32_t BYTES = MISC + 256;
+constexpr uint32_t TM_S = 0, TM_U = 128, TM_O = 256, TM_COLS = 512;
+}  // namespace cons
+
+__device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t *sm, int hd) {
+    using namespace cons;
+    constexpr uint32_t I_M64 = idesc_bf16_f32(64, 128, false, 0, 1);      // T'V, Q~S, AU
+    constexpr uint32_t I_M64N = idesc_bf16_f32(64, 128, true, 0, 1);      // -W S
+    constexpr uint32_t I_S = idesc_bf16_f32(128, 128, false, 1, 1);       // K-^T U
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);  // in0, in1, mma
+    uint32_t *s_flags = reinterpret_cast<uint32_t *>(sm + MISC + 64);  // abort, tmem
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+    const int H = p.H, n = hd / H, h = hd % H;
+    const int c_me = 32 * quad + lane;
+    const int64_t bos = p.cu_seqlens[n], eos = p.cu_seqlens[n + 1];
+    const int nchunks = (int)((eos - bos + C - 1) / C);
+    const size_t state_off = ((size_t)n * H + h) * (size_t)(D * D);
+
+    if (tid == 0) {
+        s_flags[0] = 0;
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_init(&bars[2], 1);
+        fence_mbarrier_init();
+        prefetch_tmap(tm_v);
+    }
+    if (warp == 0) {
+        tmem_alloc(&s_flags[1], TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_flags[1];
+
+    // thread 0: bring chunk c's image and V into stage c & 1 (block: wait for the producer)
+    int requested = 0;  // chunks requested so far (thread 0)
+    auto request = [&](int c, bool block) -> bool {
+        int32_t *fl = p.filled + hd * RING + (c % RING);
+        if (block) {
+            if (!wait_flag_ge(fl, c + 1, p.timeout_ns)) {
+                s_flags[0] = 1;
+                atomicOr(p.status, 1);
+                return false;
+            }
+        } else if (ld_acquire(fl) < c + 1) {
+            return false;
+        }
+        fence_proxy_async_global();
+        fence_proxy_async_smem();
+        const int b = c & 1;
+        uint8_t *dst = sm + (b ? STAGE1 : STAGE0);
+        const uint8_t *src = p.ring + ((size_t)hd * RING + (c % RING)) * SLOT;
+        mbar_arrive_expect_tx(&bars[b], SLOT + 16384);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) bulk_g2s(dst + 16384 * k, src + 16384 * k, 16384, &bars[b]);
+        bulk_g2s(dst + 65536, src + 65536, 1024, &bars[b]);
+        const int64_t t0 = bos + (int64_t)c * C;
+        tma_load_3d(sm + (b ? V1 : V0), tm_v, &bars[b], 0, h, (int32_t)t0);
+        tma_load_3d(sm + (b ? V1 : V0) + 8192, tm_v, &bars[b], 64, h, (int32_t)t0);
+        requested = c + 1;
+        return true;
+    };
+    auto poll_next = [&](int c) {  // thread 0, non-blocking
+        if (c + 1 < nchunks && requested == c + 1) request(c + 1, false);
+    };
+
+    // initial state -> TMEM (lane c, columns d) and its bf16 tile; empty sequences copy it out
+    {
+        const size_t row = state_off + (size_t)c_me * D + 64 * half;
+        const float *src = p.s0 ? p.s0 + row : nullptr;
+        float *dst = p.sT ? p.sT + row : nullptr;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            float v[32];
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+                float4 f = src ? *reinterpret_cast<const float4 *>(src + 32 * part + e)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[e] = f.x; v[e + 1] = f.y; v[e + 2] = f.z; v[e + 3] = f.w;
+            }
+            if (nchunks == 0) {
+                if (dst) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4 *>(dst + 32 * part + e) =
+                            make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                }
+            } else {
+                const int col = 64 * half + 32 * part;
+                tmem_st32(tmem + lane_base + TM_S + col, v);
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8)
+                    st_chunk(sm + S + tchunk(16384, c_me, col + 8 * q8), v + 8 * q8);
+            }
+        }
+        tmem_wait_st();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    uint32_t ph_in[2] = {0, 0}, ph_mma = 0;
+    auto wait_bar = [&](uint64_t *bar, uint32_t &ph) {
+        const bool ok = mbar_wait_bounded(bar, ph, p.timeout_ns);
+        ph ^= 1u;
+        if (!ok) {
+            s_flags[0] = 1;
+            atomicOr(p.status, 1);
+        }
+    };
+
+    int inflight = 0;  // thread 0: stage copies requested but not yet waited on
+    for (int c = 0; c < nchunks; ++c) {
+        const int b = c & 1;
+        const int64_t t0 = bos + (int64_t)c * C;
+        const int valid = (int)(eos - t0 < C ? eos - t0 : C);
+        const bool has_next = c + 1 < nchunks;
+        if (tid == 0 && requested <= c) request(c, true);
+        __syncthreads();
+        if (s_flags[0]) break;
+        wait_bar(&bars[b], ph_in[b]);
+        uint8_t *stage = sm + (b ? STAGE1 : STAGE0);
+        const uint32_t st_base = sb + (b ? STAGE1 : STAGE0);
+        if (tid == 0) {
+            fence_proxy_async_global();
+            st_release(p.consumed + hd, c + 1);  // the image is in shared memory: slot reusable
+            poll_next(c);
+        }
+        const float *gam = reinterpret_cast<const float *>(stage + SL_G);
+        const bool safe = *reinterpret_cast<const int32_t *>(stage + SL_META) != 0;
+        if (safe) {  // exact path: S <- diag(gamma) S ahead of S += K^^T U
+            scale_tmem_row<64>(tmem + lane_base + TM_S + 64 * half, gam[c_me]);
+            tc_fence_before();
+        }
+        __syncthreads();
+        if (s_flags[0]) break;
+
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t vb = sb + (b ? V1 : V0);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)  // U = T' V
+                mma_bf16_ss(tmem + TM_U, desc_k(st_base + SL_T, 8192, kk), desc_mn(vb, 8192, kk),
+                            I_M64, kk > 0);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 8; ++kk)  // U -= W S
+                mma_bf16_ss(tmem + TM_U, desc_k(st_base + SL_W, 8192, kk),
+                            desc_mn(sb + S, 16384, kk), I_M64N, 1);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 8; ++kk)  // O = Q~ S
+                mma_bf16_ss(tmem + TM_O, desc_k(st_base + SL_Q, 8192, kk),
+                            desc_mn(sb + S, 16384, kk), I_M64, kk > 0);
+            mma_commit(&bars[2]);
+            poll_next(c);
+        }
+        wait_bar(&bars[2], ph_mma);
+        tc_fence_after();
+
+        rows64_to_tile<64>(tmem + lane_base + TM_U + 64 * half, sm + U, 8192, 64 * half, quad, lane);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (s_flags[0]) break;
+
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)  // O += A U
+                mma_bf16_ss(tmem + TM_O, desc_k(st_base + SL_A, 8192, kk),
+                            desc_mn(sb + U, 8192, kk), I_M64, 1);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)  // S += K-^T U  (K^^T U on the exact path)
+                mma_bf16_ss(tmem + TM_S, desc_mn(st_base + SL_KI, 8192, kk),
+                            desc_mn(sb + U, 8192, kk), I_S, 1);
+            mma_commit(&bars[2]);
+            poll_next(c);
+        }
+        wait_bar(&bars[2], ph_mma);
+        tc_fence_after();
+
+        {
+            float v[32];
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int col = 64 * half + 32 * part;
+                tmem_ld32(tmem + lane_base + TM_O + col, v);
+                tmem_wait_ld();
+                const int i = 16 * quad + lane;
+                if (lane < 16 && i < valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(t0 + i) * H + h) * D + col);
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8)
+                        dst[q8] = make_uint4(pack2(v[8 * q8], v[8 * q8 + 1]),
+                                             pack2(v[8 * q8 + 2], v[8 * q8 + 3]),
+                                             pack2(v[8 * q8 + 4], v[8 * q8 + 5]),
+                                             pack2(v[8 * q8 + 6], v[8 * q8 + 7]));
+                }
+            }
+            const float gm = safe ? 1.f : gam[c_me];
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int col = 64 * half + 32 * part;
+                const uint32_t ta = tmem + lane_base + TM_S + col;
+                tmem_ld32(ta, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] *= gm;
+                if (!safe) tmem_st32(ta, v);
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8)
+                    st_chunk(sm + S + tchunk(16384, c_me, col + 8 * q8), v + 8 * q8);
+                if (!has_next && p.sT) {
+                    float *dst = p.sT + state_off + (size_t)c_me * D + col;
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4 *>(dst + e) =
+                            make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                }
+            }
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        (void)inflight;
+    }
+
+    // teardown: let requested copies and issued MMAs land before freeing TMEM
+    if (s_flags[0] && tid == 0) {
+        for (int c = 0; c < 2; ++c) mbar_wait_bounded(&bars[c], ph_in[c], p.timeout_ns);
+        mma_commit(&bars[2]);
+        mbar_wait_bounded(&bars[2], ph_mma, p.timeout_ns);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- producer (key-side half)
+namespace prod {
+constexpr uint32_t QK0 = 0, QK1 = 32768;       // raw q/k -> Q~/K~ (128-row tiles, 16 KB blocks)
+constexpr uint32_t LA0 = 65536, LA1 = 98304;   // raw log_alpha fp32
+constexpr uint32_t KI = 131072;                // K- / K^ [j][c] 64 x 128
+constexpr uint32_t W = KI + 16384;             // W [i][c] 64 x 128
+constexpr uint32_t AQK = W + 16384;            // A [i][j]
+constexpr uint32_t TT = AQK + 8192;            // T' [i][j]
+constexpr uint32_t LT = TT + 8192;             // L -> T fp32 [64][LT_LD]
+constexpr uint32_t PB = LT + 64 * LT_LD * 4;   // 32 x PB_LD fp32
+constexpr uint32_t MISC = PB + 32 * PB_LD * 4; // beta, gamma, psum, flags, barriers
+constexpr uint32_t BYTES = MISC + 64 * 4 + 128 * 4 + 4 * 128 * 4 + 64 + 64;
+constexpr uint32_t TM_D1 = 0, TM_W = 128, TM_COLS = 256;
+}  // namespace prod
+
+__device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_la,
+                         const SplitParams &p, uint8_t *sm, int pid, int nprod) {
+    using namespace prod;
+    constexpr uint32_t I_D1 = idesc_bf16_f32(128, 64);
+    constexpr uint32_t I_W = idesc_bf16_f32(64, 128, false, 0, 1);
+    float *s_beta = reinterpret_cast<float *>(sm + MISC);
+    float *s_gamma = s_beta + 64;
+    float *s_psum = s_gamma + 128;
+    uint32_t *s_flags = reinterpret_cast<uint32_t *>(s_psum + 512);  // abort, tmem
+    uint64_t *bars = reinterpret_cast<uint64_t *>(s_flags + 16);     // in0, in1, mma
+    float *LTp = reinterpret_cast<float *>(sm + LT);
+    float *PBp = reinterpret_cast<float *>(sm + PB);
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+    const int H = p.H;
+    const int64_t total = (int64_t)p.max_chunks * p.heads;
+
+    if (tid == 0) {
+        s_flags[0] = 0;
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_init(&bars[2], 1);
+        fence_mbarrier_init();
+        prefetch_tmap(tm_q);
+        prefetch_tmap(tm_k);
+        prefetch_tmap(tm_la);
+    }
+    if (warp == 0) {
+        tmem_alloc(&s_flags[1], TM_COLS);
+        tmem_relinquish();
+    }
+    for (int e = tid; e < 8192 / 16; e += NT)  // strictly upper 16x16 blocks of T' stay zero
+        reinterpret_cast<uint4 *>(sm + TT)[e] = make_uint4(0u, 0u, 0u, 0u);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_flags[1];
+
+    // item i -> chunk c = i / heads of head hd = i % heads; empty when c is past that sequence
+    auto item_valid = [&](int64_t i, int &c, int &hd, int64_t &t0, int &valid) -> bool {
+        c = (int)(i / p.heads);
+        hd = (int)(i % p.heads);
+        const int n = hd / H;
+        const int64_t bos = p.cu_seqlens[n], eos = p.cu_seqlens[n + 1];
+        t0 = bos + (int64_t)c * C;
+        if (t0 >= eos) return false;
+        valid = (int)(eos - t0 < C ? eos - t0 : C);
+        return true;
+    };
+    auto next_item = [&](int64_t i) -> int64_t {
+        int c, hd, valid;
+        int64_t t0;
+        for (; i < total; i += nprod)
+            if (item_valid(i, c, hd, t0, valid)) return i;
+        return total;
+    };
+    auto issue_inputs = [&](int64_t i, int b) {  // thread 0
+        int c, hd, valid;
+        int64_t t0;
+        item_valid(i, c, hd, t0, valid);
+        const int h = hd % H;
+        uint8_t *qk = sm + (b ? QK1 : QK0);
+        fence_proxy_async_smem();  // the stage's previous contents were read by generic loads
+        mbar_arrive_expect_tx(&bars[b], 32768 + 32768);
+        tma_load_3d(qk, tm_q, &bars[b], 0, h, (int32_t)t0);
+        tma_load_3d(qk + 8192, tm_k, &bars[b], 0, h, (int32_t)t0);
+        tma_load_3d(qk + 16384, tm_q, &bars[b], 64, h, (int32_t)t0);
+        tma_load_3d(qk + 24576, tm_k, &bars[b], 64, h, (int32_t)t0);
+        tma_load_3d(sm + (b ? LA1 : LA0), tm_la, &bars[b], 0, h, (int32_t)t0);
+    };
+    auto load_beta = [&](int64_t i) -> float {  // tid < C
+        int c, hd, valid;
+        int64_t t0;
+        if (i >= total || !item_valid(i, c, hd, t0, valid) || tid >= valid) return 0.f;
+        return p.beta[(size_t)(t0 + tid) * H + hd % H];
+    };
+
+    uint32_t ph_in[2] = {0, 0}, ph_mma = 0;
+    bool pending[2] = {false, false};
+    auto wait_bar = [&](uint64_t *bar, uint32_t &ph) {
+        const bool ok = mbar_wait_bounded(bar, ph, p.timeout_ns);
+        ph ^= 1u;
+        if (!ok) {
+            s_flags[0] = 1;
+            atomicOr(p.status, 1);
+        }
+    };
+
+    int64_t item = next_item(pid);
+    if (item < total) {
+        if (tid == 0) issue_inputs(item, 0);
+        pending[0] = true;
+    }
+    float beta_next = (tid < C) ? load_beta(item) : 0.f;
+    int b = 0;
+    while (item < total) {
+        int c, hd, valid;
+        int64_t t0;
+        item_valid(item, c, hd, t0, valid);
+        const int64_t nxt = next_item(item + nprod);
+        if (tid < C) s_beta[tid] = beta_next;
+        wait_bar(&bars[b], ph_in[b]);
+        pending[b] = false;
+        if (nxt < total) {
+            if (tid == 0) issue_inputs(nxt, b ^ 1);  // the other stage's last user is done
+            pending[b ^ 1] = true;
+        }
+        if (tid < C) beta_next = load_beta(nxt);
+        uint8_t *qk = sm + (b ? QK1 : QK0);
+        float *la = reinterpret_cast<float *>(sm + (b ? LA1 : LA0));
+
+        const int gate = gate_chunk(qk, sm + KI, sm + AQK, la, LTp, s_beta, s_gamma, s_psum,
+                                    s_flags, valid, tid);
+        if (gate < 0) break;
+        const bool safe = gate == 1;
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        if (tid == 0) {
+            tc_fence_after();
+            if (!safe) {
+#pragma unroll
+                for (uint32_t kk = 0; kk < 8; ++kk)
+                    mma_bf16_ss(tmem + TM_D1, desc_k(smem_u32(qk), 16384, kk),
+                                desc_k(sb + KI, 8192, kk), I_D1, kk > 0);
+            }
+            mma_commit(&bars[2]);
+        }
+        wait_bar(&bars[2], ph_mma);
+        tc_fence_after();
+        if (!safe) extract_al(tmem + lane_base + TM_D1 + 32 * half, sm + AQK, LTp, s_beta, 32 * quad + lane, half);
+        tc_fence_before();
+        __syncthreads();
+        if (s_flags[0]) break;
+
+        invert_unit_lower(LTp, PBp, sm + TT, s_beta, tid);
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)  // W = T' K~
+                mma_bf16_ss(tmem + TM_W, desc_k(sb + TT, 8192, kk),
+                            desc_mn(smem_u32(qk) + 8192, 16384, kk), I_W, kk > 0);
+            mma_commit(&bars[2]);
+        }
+        wait_bar(&bars[2], ph_mma);
+        tc_fence_after();
+        rows64_to_tile<64>(tmem + lane_base + TM_W + 64 * half, sm + W, 8192, 64 * half, quad, lane);
+        if (tid == 0 && c >= RING) {  // the slot's previous chunk must have been taken
+            if (!wait_flag_ge(p.consumed + hd, c - RING + 1, p.timeout_ns)) {
+                s_flags[0] = 1;
+                atomicOr(p.status, 1);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (s_flags[0]) break;
+
+        // copy the image out: Q~ (rows 0..63 of both 16 KB blocks), K-, W, A, T', gamma, meta
+        uint8_t *slot = p.ring + ((size_t)hd * RING + (c % RING)) * SLOT;
+        for (int e = tid; e < SLOT / 16; e += NT) {
+            const uint32_t off = e * 16;
+            uint4 val;
+            if (off < 16384) {
+                val = *reinterpret_cast<const uint4 *>(qk + (off < 8192 ? off : off + 8192));
+            } else if (off < SL_G) {
+                val = *reinterpret_cast<const uint4 *>(sm + KI + (off - SL_KI));  // K-, W, A, T' are contiguous
+            } else if (off < SL_META) {
+                val = *reinterpret_cast<const uint4 *>(reinterpret_cast<const uint8_t *>(s_gamma) + (off - SL_G));
+            } else {
+                val = make_uint4(off == SL_META ? (safe ? 1u : 0u) : 0u, 0u, 0u, 0u);
+            }
+            *reinterpret_cast<uint4 *>(slot + off) = val;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            st_release(p.filled + hd * RING + (c % RING), c + 1);
+        }
+        item = nxt;
+        b ^= 1;
+    }
+
+    if (s_flags[0] && tid == 0) {
+        for (int k = 0; k < 2; ++k)
+            if (pending[k]) mbar_wait_bounded(&bars[k], ph_in[k], p.timeout_ns);
+        mma_commit(&bars[2]);
+        mbar_wait_bounded(&bars[2], ph_mma, p.timeout_ns);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TM_COLS);
+    }
+}
+
+constexpr uint32_t SPLIT_SMEM = (cons::BYTES > prod::BYTES ? cons::BYTES : prod::BYTES) + 1024;
+
+__global__ void __launch_bounds__(NT, 1)
+split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
+             const SplitParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+    if ((int)blockIdx.x < p.heads)
+        consumer(&tm_v, p, sm, blockIdx.x);
+    else
+        producer(&tm_q, &tm_k, &tm_la, p, sm, blockIdx.x - p.heads, gridDim.x - p.heads);
+}
+
+// Zeroes the status word and the ring flags.
+__global__ void split_init_kernel(int32_t *status, int32_t *flags, int nflags) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nflags; i += gridDim.x * blockDim.x)
+        flags[i] = 0;
+}
+
+int sm_count() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+size_t flags_bytes(int64_t heads) { return ((size_t)heads * (RING + 1) * 4 + 1023) / 1024 * 1024; }
+
+}  // namespace
+
+bool split_eligible(int64_t heads, kda_dtype_t dtype, int32_t dk, int32_t dv) {
+    return dtype == KDA_BF16 && dk == D && dv == D && heads > 0 && heads * 4 <= sm_count();
+}
+
+size_t split_workspace_bytes(int64_t heads) {
+    return 1024 + flags_bytes(heads) + (size_t)heads * RING * SLOT;
+}
+
+cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *workspace,
+                                 cudaStream_t stream, uint64_t timeout_ns) {
+    const int64_t heads = (int64_t)p.num_seqs * p.H;
+    const int sms = sm_count();
+    int per_sm = 0;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)SPLIT_SMEM);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, split_kernel, NT, SPLIT_SMEM);
+    if (e != cudaSuccess) return e;
+    const int grid = per_sm * sms;
+    if (per_sm < 1 || grid <= heads) return cudaErrorInvalidConfiguration;
+
+    CUtensorMap mq, mk, mv, mla;
+    const uint64_t T = (uint64_t)p.total_tokens, H = (uint64_t)p.H;
+    if (!make_token_map(&mq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, H, T, 64, true) ||
+        !make_token_map(&mk, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, H, T, 64, true) ||
+        !make_token_map(&mv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, H, T, 64, true) ||
+        !make_token_map(&mla, p.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, H, T, D, false))
+        return cudaErrorInvalidValue;
+
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int32_t *status = reinterpret_cast<int32_t *>(ws);
+    int32_t *flags = reinterpret_cast<int32_t *>(ws + 1024);
+    const int nflags = (int)(heads * (RING + 1));
+    split_init_kernel<<<(nflags + 255) / 256, 256, 0, stream>>>(status, flags, nflags);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    SplitParams sp;
+    sp.cu_seqlens = p.cu_seqlens;
+    sp.beta = p.beta;
+    sp.s0 = p.initial_state;
+    sp.sT = p.final_state;
+    sp.out = static_cast<__nv_bfloat16 *>(p.out);
+    sp.status = status;
+    sp.filled = flags;
+    sp.consumed = flags + heads * RING;
+    sp.ring = ws + 1024 + flags_bytes(heads);
+    sp.H = p.H;
+    sp.heads = (int32_t)heads;
+    sp.max_chunks = max_chunks;
+    sp.timeout_ns = timeout_ns;
+    void *args[] = {&mq, &mk, &mv, &mla, &sp};
+    return cudaLaunchCooperativeKernel((const void *)split_kernel, dim3(grid), dim3(NT), args,
+                                       SPLIT_SMEM, stream);
+}
+
+}  // namespace kda

@@ -71,9 +71,13 @@ typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
 /* Supported head sizes: d_k, d_v in {32, 64, 128}. */
 
 /*
- * Bytes of device workspace kda_prefill needs for this problem (>= 256; a
- * multiple of 256). Pure host function; never fails (returns 0 only for
- * arguments kda_prefill would reject).
+ * Bytes of device workspace that let kda_prefill take its fastest path for this
+ * problem (a multiple of 256). Problems with few (sequence, head) pairs get room
+ * for the split-role kernel's ring of chunk images (about 260 KiB per pair); any
+ * workspace of at least 256 + 4 * num_seqs bytes (rounded up to 256) is accepted,
+ * and a smaller one than returned here selects the single-role kernel. Host
+ * function: queries the current device's SM count; returns 0 only for
+ * arguments kda_prefill would reject.
  */
 KDA_API size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H,
                                   int32_t d_k, int32_t d_v, kda_dtype_t dtype);
@@ -92,21 +96,25 @@ KDA_API size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens
  *   out         [total_tokens, H, d_v]  dtype  (written)
  *   final_state [num_seqs, H, d_k, d_v] fp32, or NULL if not wanted (written;
  *               may alias initial_state)
- *   workspace   >= kda_prefill_workspace_size(...) bytes of device memory,
- *               256-byte aligned; contents on entry are ignored.
+ *   workspace   device memory, 256-byte aligned, contents on entry ignored: at
+ *               least 256 + 4 * num_seqs bytes rounded up to 256, and
+ *               kda_prefill_workspace_size(...) bytes for the fastest path.
  *
  * cu_seqlens must start at 0, be non-decreasing and end at total_tokens.
  * Zero-length sequences are allowed (their final state is their initial state).
  * A dense [B, T] batch is cu_seqlens = {0, T, 2T, ..., B*T}.
  *
  * Tokens are processed in chunks of 64 per sequence: bf16 inputs with
- * d_k = d_v = 128 run on the tensor-core chunk kernel; every other supported
+ * d_k = d_v = 128 run on the tensor-core chunk kernels (with few (sequence,
+ * head) pairs and a full-size workspace, a split-role kernel in which some
+ * thread blocks run the per-head state chains and the others prepare the
+ * state-independent half of upcoming chunks); every other supported
  * combination runs the token-serial fp32 kernel (see kda_prefill_recurrent).
  * The result does not depend on that choice beyond rounding.
  *
  * Status: KDA_ERR_INVALID_ARGUMENT for a NULL required pointer, H <= 0,
  * num_seqs < 0, an unsupported d_k/d_v, bad cu_seqlens_host, or a workspace
- * smaller than required; KDA_ERR_CUDA if a launch fails.
+ * smaller than the minimum; KDA_ERR_CUDA if a launch fails.
  */
 KDA_API kda_status_t kda_prefill(const void *q, const void *k, const void *v,
                          const float *log_alpha, const float *beta,

@@ -166,3 +166,25 @@ def test_prefill_1m_first_window_and_final_state():
         bound = float(np.exp(ld) * nb)
         assert bound < 1e-6 * scale, bound
         assert_close(fs[0, h], ls[0, i], TOL["bf16"] + bound / scale, scale, f"1M final state head {h}")
+
+
+@pytest.mark.parametrize("lens,H", [((8192,), 32), ((700, 0, 130, 64, 1), 6), ((1000,), 2)])
+def test_split_role_and_fused_kernels_agree_with_oracle(lens, H):
+    """Few-head problems run the split-role kernel when the workspace holds its ring; with only
+    the minimum workspace they run the fused kernel. Both must match the oracle."""
+    wl = W.custom(lens, H, 128, 128, "bf16", seed=len(lens) * 10 + H, init_state="normal")
+    inp = W.make_inputs(wl, DEV)
+    N = len(lens)
+    full = torch.empty(K.workspace_size(N, wl.total_tokens, H, 128, 128, torch.bfloat16),
+                       dtype=torch.uint8, device=DEV)
+    minimal = torch.empty(256 + (4 * N + 255) // 256 * 256, dtype=torch.uint8, device=DEV)
+    assert full.numel() > minimal.numel()
+    heads = list(range(H)) if H <= 6 else [0, 13, 31]
+    ref_o, ref_s = oracle_forward(inp, heads=heads)
+    scale = vmax(inp)
+    for ws in (full, minimal):
+        out, fs = K.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                            inp["initial_state"], inp["cu_seqlens"], inp["cu_seqlens_dev"], workspace=ws)
+        assert K.read_device_status(ws) == K.KDA_OK
+        assert_close(out[:, heads], ref_o, TOL["bf16"], scale, f"out ws={ws.numel()}")
+        assert_close(fs[:, heads], ref_s, TOL["bf16"], scale, f"state ws={ws.numel()}")
