@@ -149,6 +149,7 @@ kda_status_t kda_prefill(const void *q, const void *k, const void *v, const floa
     }
     const int64_t heads = (int64_t)num_seqs * H;
     if (kda::chunk_supported(p) && max_chunks >= 2 && kda::split_eligible(heads, dtype, d_k, d_v) &&
+        kda::split_eligible_seqs(num_seqs) &&
         workspace_bytes >= kda::split_workspace_bytes(heads)) {
         // few heads: consumer CTAs run the state chains, producer CTAs fill the other SMs
         e = kda::launch_prefill_split(p, max_chunks, workspace, s, kda::kWaitTimeoutNs);

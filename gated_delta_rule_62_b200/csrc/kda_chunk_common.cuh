@@ -187,11 +187,12 @@ static __device__ void invert_unit_lower(float *LT, float *PB, uint8_t *TT, cons
 // Out: QK holds Q~ and K~ in place, KI holds K- (factored path) or K^ (exact path), s_gamma =
 // e^(g_{C-1}); the exact path also writes A into AQK and beta-scaled L into LT (zeros elsewhere).
 // Thread mapping: channel pair (cA, cA + 1), token quarter tq (tokens 16 tq .. 16 tq + 15).
+// If KH is not null it also receives K^ = k e^(g_{C-1} - g) on both paths.
 // Returns 1 for the exact path, 0 for the factored path, -1 if *s_abort was set.
 __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK, float *LA,
                                           float *LT, const float *s_beta, float *s_gamma,
                                           float *s_psum, const uint32_t *s_abort, int valid,
-                                          int tid) {
+                                          int tid, uint8_t *KH = nullptr) {
     const int tq = tid >> 6, cA = 2 * (tid & 63);
     const int warp = tid >> 5, lane = tid & 31;
     // ---- gates: log_alpha of 16 tokens x 2 channels into registers, quarter totals
@@ -277,8 +278,8 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
 #pragma unroll
         for (int i = 0; i < 16; ++i) al[i] = make_float2(__expf(la[i].x), __expf(la[i].y));
         const float2 eA = make_float2(__expf(goff.x), __expf(goff.y));
-        const float2 eB = safe ? make_float2(__expf(gC.x - goff.x - tot.x), __expf(gC.y - goff.y - tot.y))
-                               : make_float2(__expf(-goff.x - tot.x), __expf(-goff.y - tot.y));
+        const float2 eH = make_float2(__expf(gC.x - goff.x - tot.x), __expf(gC.y - goff.y - tot.y));
+        const float2 eB = safe ? eH : make_float2(__expf(-goff.x - tot.x), __expf(-goff.y - tot.y));
         float2 R[16];
         float2 run = make_float2(1.f, 1.f);
 #pragma unroll
@@ -300,6 +301,7 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
             st_bf2(qp, qv.x * P.x, qv.y * P.y);
             st_bf2(kp, kv.x * P.x, kv.y * P.y);
             st_bf2(KI + telem(8192, t, cA), kv.x * (eB.x * R[i].x), kv.y * (eB.y * R[i].y));
+            if (KH) st_bf2(KH + telem(8192, t, cA), kv.x * (eH.x * R[i].x), kv.y * (eH.y * R[i].y));
         }
     }    return safe ? 1 : 0;
 }

@@ -33,7 +33,7 @@ namespace {
 using namespace sm100;
 using namespace chunk;
 
-constexpr int RING = 4;
+constexpr int RING = 8;
 // Slot image (bytes): Q~ 64-row tile (8 KB blocks), K- (or K^), W, A, T', gamma[128], meta.
 constexpr uint32_t SL_Q = 0, SL_KI = 16384, SL_W = 32768, SL_A = 49152, SL_T = 57344;
 constexpr uint32_t SL_G = 65536, SL_META = 65536 + 512, SLOT = 66560;
@@ -83,6 +83,19 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
+// Bulk (untiled) copy shared -> global, tracked by this thread's bulk async-group.
+__device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until the committed bulk stores have finished reading shared memory / are complete.
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ---------------------------------------------------------------- consumer (state chain)
 namespace cons {
 constexpr uint32_t STAGE0 = 0, STAGE1 = SLOT;
@@ -91,7 +104,7 @@ constexpr uint32_t S = V1 + 16384;   // S [c][d] bf16 128 x 128, blocks 16 KB
 constexpr uint32_t U = S + 32768;    // U [j][d] bf16 64 x 128, blocks 8 KB
 constexpr uint32_t MISC = U + 16384; // barriers, flags
 constexpr uint32_t BYTES = MISC + 256;
-constexpr uint32_t TM_S = 0, TM_U = 128, TM_O = 256, TM_COLS = 512;
+constexpr uint32_t TM_S = 0, TM_U = 128, TM_O0 = 256, TM_O1 = 384, TM_COLS = 512;
 }  // namespace cons
 
 __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t *sm, int hd) {
@@ -99,7 +112,7 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
     constexpr uint32_t I_M64 = idesc_bf16_f32(64, 128, false, 0, 1);      // T'V, Q~S, AU
     constexpr uint32_t I_M64N = idesc_bf16_f32(64, 128, true, 0, 1);      // -W S
     constexpr uint32_t I_S = idesc_bf16_f32(128, 128, false, 1, 1);       // K-^T U
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);  // in0, in1, mma
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);  // in0, in1, u, s, o
     uint32_t *s_flags = reinterpret_cast<uint32_t *>(sm + MISC + 64);  // abort, tmem
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -113,9 +126,7 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
 
     if (tid == 0) {
         s_flags[0] = 0;
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
-        mbar_init(&bars[2], 1);
+        for (int k = 0; k < 5; ++k) mbar_init(&bars[k], 1);
         fence_mbarrier_init();
         prefetch_tmap(tm_v);
     }
@@ -195,7 +206,7 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
     tc_fence_before();
     __syncthreads();
 
-    uint32_t ph_in[2] = {0, 0}, ph_mma = 0;
+    uint32_t ph_in[2] = {0, 0}, ph_u = 0, ph_s = 0, ph_o = 0;
     auto wait_bar = [&](uint64_t *bar, uint32_t &ph) {
         const bool ok = mbar_wait_bounded(bar, ph, p.timeout_ns);
         ph ^= 1u;
@@ -204,13 +215,32 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
             atomicOr(p.status, 1);
         }
     };
+    // O of chunk cc (TMEM, M=64 rows, columns [64 half, 64 half + 64)) -> bf16 outputs
+    auto store_o = [&](int cc, uint32_t tm_o) {
+        const int64_t tc = bos + (int64_t)cc * C;
+        const int vc = (int)(eos - tc < C ? eos - tc : C);
+        float v[32];
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int col = 64 * half + 32 * part;
+            tmem_ld32(tmem + lane_base + tm_o + col, v);
+            tmem_wait_ld();
+            const int i = 16 * quad + lane;
+            if (lane < 16 && i < vc) {
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(tc + i) * H + h) * D + col);
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8)
+                    dst[q8] = make_uint4(pack2(v[8 * q8], v[8 * q8 + 1]), pack2(v[8 * q8 + 2], v[8 * q8 + 3]),
+                                         pack2(v[8 * q8 + 4], v[8 * q8 + 5]), pack2(v[8 * q8 + 6], v[8 * q8 + 7]));
+            }
+        }
+    };
 
     int inflight = 0;  // thread 0: stage copies requested but not yet waited on
     for (int c = 0; c < nchunks; ++c) {
         const int b = c & 1;
-        const int64_t t0 = bos + (int64_t)c * C;
-        const int valid = (int)(eos - t0 < C ? eos - t0 : C);
         const bool has_next = c + 1 < nchunks;
+        const uint32_t tm_o = b ? TM_O1 : TM_O0;
         if (tid == 0 && requested <= c) request(c, true);
         __syncthreads();
         if (s_flags[0]) break;
@@ -220,16 +250,11 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
         if (tid == 0) {
             fence_proxy_async_global();
             st_release(p.consumed + hd, c + 1);  // the image is in shared memory: slot reusable
-            poll_next(c);
+            // The other stage is free once the previous chunk's last MMA (O += A U) is done:
+            // for c = 0 it never held anything; otherwise it was requested at the end of c - 1.
+            if (c == 0) poll_next(c);
         }
         const float *gam = reinterpret_cast<const float *>(stage + SL_G);
-        const bool safe = *reinterpret_cast<const int32_t *>(stage + SL_META) != 0;
-        if (safe) {  // exact path: S <- diag(gamma) S ahead of S += K^^T U
-            scale_tmem_row<64>(tmem + lane_base + TM_S + 64 * half, gam[c_me]);
-            tc_fence_before();
-        }
-        __syncthreads();
-        if (s_flags[0]) break;
 
         if (tid == 0) {
             tc_fence_after();
@@ -242,14 +267,21 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
             for (uint32_t kk = 0; kk < 8; ++kk)  // U -= W S
                 mma_bf16_ss(tmem + TM_U, desc_k(st_base + SL_W, 8192, kk),
                             desc_mn(sb + S, 16384, kk), I_M64N, 1);
-#pragma unroll
-            for (uint32_t kk = 0; kk < 8; ++kk)  // O = Q~ S
-                mma_bf16_ss(tmem + TM_O, desc_k(st_base + SL_Q, 8192, kk),
-                            desc_mn(sb + S, 16384, kk), I_M64, kk > 0);
             mma_commit(&bars[2]);
-            poll_next(c);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 8; ++kk)  // O = Q~ S  (completes behind the U batch)
+                mma_bf16_ss(tmem + tm_o, desc_k(st_base + SL_Q, 8192, kk),
+                            desc_mn(sb + S, 16384, kk), I_M64, kk > 0);
         }
-        wait_bar(&bars[2], ph_mma);
+        // While the U batch runs (it reads only shared memory and writes U, O):
+        // S <- diag(gamma) S in TMEM, ahead of S += K^^T U with K^ = k e^(g_{C-1} - g);
+        // and the previous chunk's outputs from the other O buffer.
+        scale_tmem_row<64>(tmem + lane_base + TM_S + 64 * half, gam[c_me]);
+        if (c > 0) {
+            if (tid == 0) poll_next(c);
+            store_o(c - 1, b ? TM_O0 : TM_O1);  // its MMAs were waited on at the end of c - 1
+        }
+        wait_bar(&bars[2], ph_u);
         tc_fence_after();
 
         rows64_to_tile<64>(tmem + lane_base + TM_U + 64 * half, sm + U, 8192, 64 * half, quad, lane);
@@ -261,71 +293,55 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)  // O += A U
-                mma_bf16_ss(tmem + TM_O, desc_k(st_base + SL_A, 8192, kk),
-                            desc_mn(sb + U, 8192, kk), I_M64, 1);
-#pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)  // S += K-^T U  (K^^T U on the exact path)
+            for (uint32_t kk = 0; kk < 4; ++kk)  // S += K^^T U   (S already scaled by gamma)
                 mma_bf16_ss(tmem + TM_S, desc_mn(st_base + SL_KI, 8192, kk),
                             desc_mn(sb + U, 8192, kk), I_S, 1);
-            mma_commit(&bars[2]);
+            mma_commit(&bars[3]);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)  // O += A U
+                mma_bf16_ss(tmem + tm_o, desc_k(st_base + SL_A, 8192, kk),
+                            desc_mn(sb + U, 8192, kk), I_M64, 1);
+            mma_commit(&bars[4]);
             poll_next(c);
         }
-        wait_bar(&bars[2], ph_mma);
+        wait_bar(&bars[3], ph_s);
         tc_fence_after();
 
-        {
+        // the next state's bf16 tile (and the final state after the last chunk)
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int col = 64 * half + 32 * part;
             float v[32];
+            tmem_ld32(tmem + lane_base + TM_S + col, v);
+            tmem_wait_ld();
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int col = 64 * half + 32 * part;
-                tmem_ld32(tmem + lane_base + TM_O + col, v);
-                tmem_wait_ld();
-                const int i = 16 * quad + lane;
-                if (lane < 16 && i < valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(t0 + i) * H + h) * D + col);
+            for (int q8 = 0; q8 < 4; ++q8)
+                st_chunk(sm + S + tchunk(16384, c_me, col + 8 * q8), v + 8 * q8);
+            if (!has_next && p.sT) {
+                float *dst = p.sT + state_off + (size_t)c_me * D + col;
 #pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8)
-                        dst[q8] = make_uint4(pack2(v[8 * q8], v[8 * q8 + 1]),
-                                             pack2(v[8 * q8 + 2], v[8 * q8 + 3]),
-                                             pack2(v[8 * q8 + 4], v[8 * q8 + 5]),
-                                             pack2(v[8 * q8 + 6], v[8 * q8 + 7]));
-                }
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4 *>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
             }
-            const float gm = safe ? 1.f : gam[c_me];
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int col = 64 * half + 32 * part;
-                const uint32_t ta = tmem + lane_base + TM_S + col;
-                tmem_ld32(ta, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] *= gm;
-                if (!safe) tmem_st32(ta, v);
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8)
-                    st_chunk(sm + S + tchunk(16384, c_me, col + 8 * q8), v + 8 * q8);
-                if (!has_next && p.sT) {
-                    float *dst = p.sT + state_off + (size_t)c_me * D + col;
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4 *>(dst + e) =
-                            make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                }
-            }
-            tmem_wait_st();
         }
+        // this chunk's last MMA (O += A U): after it, its stage may take chunk c + 2 and
+        // the other stage chunk c + 1's image can be requested with a whole chunk to land
+        wait_bar(&bars[4], ph_o);
+        tc_fence_after();
+        if (tid == 0) poll_next(c);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         (void)inflight;
     }
+    if (nchunks > 0 && !s_flags[0])  // outputs of the last chunk
+        store_o(nchunks - 1, ((nchunks - 1) & 1) ? TM_O1 : TM_O0);
 
     // teardown: let requested copies and issued MMAs land before freeing TMEM
     if (s_flags[0] && tid == 0) {
         for (int c = 0; c < 2; ++c) mbar_wait_bounded(&bars[c], ph_in[c], p.timeout_ns);
         mma_commit(&bars[2]);
-        mbar_wait_bounded(&bars[2], ph_mma, p.timeout_ns);
+        mbar_wait_bounded(&bars[2], ph_u, p.timeout_ns);
     }
     tc_fence_before();
     __syncthreads();
@@ -346,7 +362,8 @@ constexpr uint32_t TT = AQK + 8192;            // T' [i][j]
 constexpr uint32_t LT = TT + 8192;             // L -> T fp32 [64][LT_LD]
 constexpr uint32_t PB = LT + 64 * LT_LD * 4;   // 32 x PB_LD fp32
 constexpr uint32_t MISC = PB + 32 * PB_LD * 4; // beta, gamma, psum, flags, barriers
-constexpr uint32_t BYTES = MISC + 64 * 4 + 128 * 4 + 4 * 128 * 4 + 64 + 64;
+constexpr uint32_t KH = (MISC + 64 * 4 + 128 * 4 + 4 * 128 * 4 + 64 + 64 + 1023) / 1024 * 1024;  // K^ [j][c]
+constexpr uint32_t BYTES = KH + 16384;
 constexpr uint32_t TM_D1 = 0, TM_W = 128, TM_COLS = 256;
 }  // namespace prod
 
@@ -367,7 +384,14 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     const int quad = warp & 3, half = warp >> 2;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
     const int H = p.H;
-    const int64_t total = (int64_t)p.max_chunks * p.heads;
+    // Static assignment: producer pid serves head hd = pid % heads, making chunks j, j + cnt, ...
+    // (j = pid / heads, cnt = number of producers of that head), so it only ever waits on its
+    // own head's consumer.
+    const int hd = pid % p.heads, pj = pid / p.heads;
+    const int pcnt = (nprod - 1 - hd) / p.heads + 1;
+    const int h = hd % H;
+    const int64_t bos = p.cu_seqlens[hd / H], eos = p.cu_seqlens[hd / H + 1];
+    const int nch = (int)((eos - bos + C - 1) / C);
 
     if (tid == 0) {
         s_flags[0] = 0;
@@ -390,29 +414,8 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     tc_fence_after();
     const uint32_t tmem = s_flags[1];
 
-    // item i -> chunk c = i / heads of head hd = i % heads; empty when c is past that sequence
-    auto item_valid = [&](int64_t i, int &c, int &hd, int64_t &t0, int &valid) -> bool {
-        c = (int)(i / p.heads);
-        hd = (int)(i % p.heads);
-        const int n = hd / H;
-        const int64_t bos = p.cu_seqlens[n], eos = p.cu_seqlens[n + 1];
-        t0 = bos + (int64_t)c * C;
-        if (t0 >= eos) return false;
-        valid = (int)(eos - t0 < C ? eos - t0 : C);
-        return true;
-    };
-    auto next_item = [&](int64_t i) -> int64_t {
-        int c, hd, valid;
-        int64_t t0;
-        for (; i < total; i += nprod)
-            if (item_valid(i, c, hd, t0, valid)) return i;
-        return total;
-    };
-    auto issue_inputs = [&](int64_t i, int b) {  // thread 0
-        int c, hd, valid;
-        int64_t t0;
-        item_valid(i, c, hd, t0, valid);
-        const int h = hd % H;
+    auto issue_inputs = [&](int c, int b) {  // thread 0
+        const int64_t t0 = bos + (int64_t)c * C;
         uint8_t *qk = sm + (b ? QK1 : QK0);
         fence_proxy_async_smem();  // the stage's previous contents were read by generic loads
         mbar_arrive_expect_tx(&bars[b], 32768 + 32768);
@@ -422,11 +425,23 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         tma_load_3d(qk + 24576, tm_k, &bars[b], 64, h, (int32_t)t0);
         tma_load_3d(sm + (b ? LA1 : LA0), tm_la, &bars[b], 0, h, (int32_t)t0);
     };
-    auto load_beta = [&](int64_t i) -> float {  // tid < C
-        int c, hd, valid;
-        int64_t t0;
-        if (i >= total || !item_valid(i, c, hd, t0, valid) || tid >= valid) return 0.f;
-        return p.beta[(size_t)(t0 + tid) * H + hd % H];
+    auto load_beta = [&](int c) -> float {  // tid < C
+        const int64_t t0 = bos + (int64_t)c * C;
+        if (c >= nch || t0 + tid >= eos) return 0.f;
+        return p.beta[(size_t)(t0 + tid) * H + h];
+    };
+    // thread 0: publish a filled slot once its bulk stores are complete (deferred so that the
+    // completion wait overlaps the next item's work)
+    int32_t *rel_flag = nullptr;
+    int rel_val = 0;
+    auto release = [&]() {
+        if (rel_flag) {
+            bulk_wait_all();
+            fence_proxy_async_global();
+            __threadfence();
+            st_release(rel_flag, rel_val);
+            rel_flag = nullptr;
+        }
     };
 
     uint32_t ph_in[2] = {0, 0}, ph_mma = 0;
@@ -440,22 +455,22 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         }
     };
 
-    int64_t item = next_item(pid);
-    if (item < total) {
+    int item = pj;  // chunk index
+    if (item < nch) {
         if (tid == 0) issue_inputs(item, 0);
         pending[0] = true;
     }
     float beta_next = (tid < C) ? load_beta(item) : 0.f;
     int b = 0;
-    while (item < total) {
-        int c, hd, valid;
-        int64_t t0;
-        item_valid(item, c, hd, t0, valid);
-        const int64_t nxt = next_item(item + nprod);
+    while (item < nch) {
+        const int c = item;
+        const int64_t t0 = bos + (int64_t)c * C;
+        const int valid = (int)(eos - t0 < C ? eos - t0 : C);
+        const int nxt = item + pcnt;
         if (tid < C) s_beta[tid] = beta_next;
         wait_bar(&bars[b], ph_in[b]);
         pending[b] = false;
-        if (nxt < total) {
+        if (nxt < nch) {
             if (tid == 0) issue_inputs(nxt, b ^ 1);  // the other stage's last user is done
             pending[b ^ 1] = true;
         }
@@ -464,7 +479,8 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         float *la = reinterpret_cast<float *>(sm + (b ? LA1 : LA0));
 
         const int gate = gate_chunk(qk, sm + KI, sm + AQK, la, LTp, s_beta, s_gamma, s_psum,
-                                    s_flags, valid, tid);
+                                    s_flags, valid, tid, sm + KH);
+        if (tid == 0) release();  // the previous item's image
         if (gate < 0) break;
         const bool safe = gate == 1;
         fence_proxy_async_smem();
@@ -508,36 +524,34 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                 atomicOr(p.status, 1);
             }
         }
+        fence_proxy_async_smem();  // A, K^, W were written by generic stores; the copy-out is async
         tc_fence_before();
         __syncthreads();
         if (s_flags[0]) break;
 
-        // copy the image out: Q~ (rows 0..63 of both 16 KB blocks), K-, W, A, T', gamma, meta
-        uint8_t *slot = p.ring + ((size_t)hd * RING + (c % RING)) * SLOT;
-        for (int e = tid; e < SLOT / 16; e += NT) {
-            const uint32_t off = e * 16;
-            uint4 val;
-            if (off < 16384) {
-                val = *reinterpret_cast<const uint4 *>(qk + (off < 8192 ? off : off + 8192));
-            } else if (off < SL_G) {
-                val = *reinterpret_cast<const uint4 *>(sm + KI + (off - SL_KI));  // K-, W, A, T' are contiguous
-            } else if (off < SL_META) {
-                val = *reinterpret_cast<const uint4 *>(reinterpret_cast<const uint8_t *>(s_gamma) + (off - SL_G));
-            } else {
-                val = make_uint4(off == SL_META ? (safe ? 1u : 0u) : 0u, 0u, 0u, 0u);
-            }
-            *reinterpret_cast<uint4 *>(slot + off) = val;
+        // copy the image out with bulk stores: Q~ (rows 0..63 of both 16 KB blocks), K^, then
+        // W, A, T' (contiguous), gamma; published at the next item (see release)
+        if (tid == 0) {
+            uint8_t *slot = p.ring + ((size_t)hd * RING + (c % RING)) * SLOT;
+            fence_proxy_async_smem();
+            bulk_s2g(slot + SL_Q, qk, 8192);
+            bulk_s2g(slot + SL_Q + 8192, qk + 16384, 8192);
+            bulk_s2g(slot + SL_KI, sm + KH, 16384);
+            bulk_s2g(slot + SL_W, sm + W, SL_G - SL_W);
+            bulk_s2g(slot + SL_G, s_gamma, 512);
+            bulk_commit();
+            bulk_wait_read();  // shared memory may be rewritten by the next item
+            rel_flag = p.filled + hd * RING + (c % RING);
+            rel_val = c + 1;
         }
         __syncthreads();
-        if (tid == 0) {
-            __threadfence();
-            st_release(p.filled + hd * RING + (c % RING), c + 1);
-        }
         item = nxt;
         b ^= 1;
     }
 
+    if (tid == 0 && !s_flags[0]) release();
     if (s_flags[0] && tid == 0) {
+        bulk_wait_all();
         for (int k = 0; k < 2; ++k)
             if (pending[k]) mbar_wait_bounded(&bars[k], ph_in[k], p.timeout_ns);
         mma_commit(&bars[2]);
@@ -586,6 +600,8 @@ size_t flags_bytes(int64_t heads) { return ((size_t)heads * (RING + 1) * 4 + 102
 bool split_eligible(int64_t heads, kda_dtype_t dtype, int32_t dk, int32_t dv) {
     return dtype == KDA_BF16 && dk == D && dv == D && heads > 0 && heads * 4 <= sm_count();
 }
+
+bool split_eligible_seqs(int32_t num_seqs) { return num_seqs >= 1; }
 
 size_t split_workspace_bytes(int64_t heads) {
     return 1024 + flags_bytes(heads) + (size_t)heads * RING * SLOT;

@@ -47,6 +47,7 @@ cudaError_t launch_bounded_wait_probe(void *workspace, uint64_t timeout_ns, cuda
 // Split-role chunk kernel (consumers run the state chain, producers the key-side half) for
 // workloads with few (sequence, head) pairs; it needs a larger workspace (a ring of chunk images).
 bool split_eligible(int64_t heads, kda_dtype_t dtype, int32_t dk, int32_t dv);
+bool split_eligible_seqs(int32_t num_seqs);
 size_t split_workspace_bytes(int64_t heads);
 cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *workspace,
                                  cudaStream_t stream, uint64_t timeout_ns);
