@@ -40,6 +40,13 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t base, uint32_t bs, uint32_t
     return smem_desc_sw128(base + kk * 2048, bs, 1024);
 }
 
+// The same descriptors from a precomputed step-0 descriptor: only the start-address field
+// (address / 16, low 14 bits; shared addresses stay below 256 KB, so no carry) moves.
+__device__ __forceinline__ uint64_t desc_k_at(uint64_t d0, uint32_t bs, uint32_t kk) {
+    return d0 + (((kk >> 2) * bs + (kk & 3) * 32) >> 4);
+}
+__device__ __forceinline__ uint64_t desc_mn_at(uint64_t d0, uint32_t kk) { return d0 + kk * 128; }
+
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t *>(&h);

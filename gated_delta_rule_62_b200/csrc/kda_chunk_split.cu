@@ -167,8 +167,12 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
         requested = c + 1;
         return true;
     };
-    auto poll_next = [&](int c) {  // thread 0, non-blocking
-        if (c + 1 < nchunks && requested == c + 1) request(c + 1, false);
+    // thread 0, non-blocking: request every chunk whose stage is free (the chunk two back has
+    // finished all its MMAs: `done` chunks have) and whose image the producer has published
+    int done = 0;
+    auto poll_ahead = [&]() {
+        while (requested < nchunks && requested < done + 2)
+            if (!request(requested, false)) break;
     };
 
     // initial state -> TMEM (lane c, columns d) and its bf16 tile; empty sequences copy it out
@@ -252,33 +256,32 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
             st_release(p.consumed + hd, c + 1);  // the image is in shared memory: slot reusable
             // The other stage is free once the previous chunk's last MMA (O += A U) is done:
             // for c = 0 it never held anything; otherwise it was requested at the end of c - 1.
-            if (c == 0) poll_next(c);
+            poll_ahead();
         }
         const float *gam = reinterpret_cast<const float *>(stage + SL_G);
 
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t vb = sb + (b ? V1 : V0);
+            const uint64_t dT = desc_k(st_base + SL_T, 8192, 0), dW = desc_k(st_base + SL_W, 8192, 0);
+            const uint64_t dQ = desc_k(st_base + SL_Q, 8192, 0), dS = desc_mn(sb + S, 16384, 0);
+            const uint64_t dV = desc_mn(sb + (b ? V1 : V0), 8192, 0);
 #pragma unroll
             for (uint32_t kk = 0; kk < 4; ++kk)  // U = T' V
-                mma_bf16_ss(tmem + TM_U, desc_k(st_base + SL_T, 8192, kk), desc_mn(vb, 8192, kk),
-                            I_M64, kk > 0);
+                mma_bf16_ss(tmem + TM_U, desc_k_at(dT, 8192, kk), desc_mn_at(dV, kk), I_M64, kk > 0);
 #pragma unroll
             for (uint32_t kk = 0; kk < 8; ++kk)  // U -= W S
-                mma_bf16_ss(tmem + TM_U, desc_k(st_base + SL_W, 8192, kk),
-                            desc_mn(sb + S, 16384, kk), I_M64N, 1);
+                mma_bf16_ss(tmem + TM_U, desc_k_at(dW, 8192, kk), desc_mn_at(dS, kk), I_M64N, 1);
             mma_commit(&bars[2]);
 #pragma unroll
             for (uint32_t kk = 0; kk < 8; ++kk)  // O = Q~ S  (completes behind the U batch)
-                mma_bf16_ss(tmem + tm_o, desc_k(st_base + SL_Q, 8192, kk),
-                            desc_mn(sb + S, 16384, kk), I_M64, kk > 0);
+                mma_bf16_ss(tmem + tm_o, desc_k_at(dQ, 8192, kk), desc_mn_at(dS, kk), I_M64, kk > 0);
         }
         // While the U batch runs (it reads only shared memory and writes U, O):
         // S <- diag(gamma) S in TMEM, ahead of S += K^^T U with K^ = k e^(g_{C-1} - g);
         // and the previous chunk's outputs from the other O buffer.
         scale_tmem_row<64>(tmem + lane_base + TM_S + 64 * half, gam[c_me]);
         if (c > 0) {
-            if (tid == 0) poll_next(c);
+            if (tid == 0) poll_ahead();
             store_o(c - 1, b ? TM_O0 : TM_O1);  // its MMAs were waited on at the end of c - 1
         }
         wait_bar(&bars[2], ph_u);
@@ -292,17 +295,17 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
 
         if (tid == 0) {
             tc_fence_after();
+            const uint64_t dK = desc_mn(st_base + SL_KI, 8192, 0), dU = desc_mn(sb + U, 8192, 0);
+            const uint64_t dA = desc_k(st_base + SL_A, 8192, 0);
 #pragma unroll
             for (uint32_t kk = 0; kk < 4; ++kk)  // S += K^^T U   (S already scaled by gamma)
-                mma_bf16_ss(tmem + TM_S, desc_mn(st_base + SL_KI, 8192, kk),
-                            desc_mn(sb + U, 8192, kk), I_S, 1);
+                mma_bf16_ss(tmem + TM_S, desc_mn_at(dK, kk), desc_mn_at(dU, kk), I_S, 1);
             mma_commit(&bars[3]);
 #pragma unroll
             for (uint32_t kk = 0; kk < 4; ++kk)  // O += A U
-                mma_bf16_ss(tmem + tm_o, desc_k(st_base + SL_A, 8192, kk),
-                            desc_mn(sb + U, 8192, kk), I_M64, 1);
+                mma_bf16_ss(tmem + tm_o, desc_k_at(dA, 8192, kk), desc_mn_at(dU, kk), I_M64, 1);
             mma_commit(&bars[4]);
-            poll_next(c);
+            poll_ahead();
         }
         wait_bar(&bars[3], ph_s);
         tc_fence_after();
@@ -328,7 +331,10 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
         // the other stage chunk c + 1's image can be requested with a whole chunk to land
         wait_bar(&bars[4], ph_o);
         tc_fence_after();
-        if (tid == 0) poll_next(c);
+        if (tid == 0) {
+            done = c + 1;
+            poll_ahead();  // usually chunk c + 2 into this chunk's stage: a whole chunk to land
+        }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
