@@ -346,12 +346,16 @@ __device__ __forceinline__ void extract_al(uint32_t taddr, uint8_t *AQK, float *
 // NCOLS columns starting at column col0 of both the TMEM region (taddr) and the tile.
 template <int NCOLS>
 __device__ __forceinline__ void rows64_to_tile(uint32_t taddr, uint8_t *tile, uint32_t bs,
-                                               int col0, int quad, int lane) {
+                                               int col0, int quad, int lane, float scale = 1.f) {
 #pragma unroll
     for (int part = 0; part < NCOLS / 32; ++part) {
         float v[32];
         tmem_ld32(taddr + 32 * part, v);
         tmem_wait_ld();
+        if (scale != 1.f) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] *= scale;
+        }
         if (lane < 16) {
             const int row = 16 * quad + lane;
 #pragma unroll

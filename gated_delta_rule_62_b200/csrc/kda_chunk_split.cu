@@ -34,10 +34,17 @@ using namespace sm100;
 using namespace chunk;
 
 constexpr int RING = 8;
-// Slot image (bytes): Q~ 64-row tile (8 KB blocks), K- (or K^), W, A, T', gamma[128], meta.
-constexpr uint32_t SL_Q = 0, SL_KI = 16384, SL_W = 32768, SL_A = 49152, SL_T = 57344;
-constexpr uint32_t SL_G = 65536, SL_META = 65536 + 512, SLOT = 66560;
-static_assert(SLOT % 1024 == 0 && SLOT == 4 * 16384 + 1024, "slot layout");
+// Chunk image (bytes), the same in a ring slot and in a consumer stage:
+//   [0, 8K)      T' [i][j]                     \ with the zero block: [T'; 0] (K-major, 128 rows)
+//   [8K, 16K)    zero block (consumer only)     |
+//   [16K, 24K)   A [i][j]                      / with the zero block: [0; A] (K-major, 128 rows)
+//   [24K, 56K)   [-W; Q~] (K-major, 128 rows, two 64-column blocks of 16 KB: rows 0..63 = -W,
+//                rows 64..127 = Q~)
+//   [56K, 72K)   K^ [j][c] (an MN-major A operand for K^^T U)
+//   [72K, 72K + 512) gamma[128]
+constexpr uint32_t SL_T = 0, SL_Z = 8192, SL_A = 16384, SL_WQ = 24576, SL_KH = 57344;
+constexpr uint32_t SL_G = 73728, SLOT = 74752;
+static_assert(SLOT % 1024 == 0, "slot layout");
 
 struct SplitParams {
     const int32_t *cu_seqlens;
@@ -99,27 +106,27 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 // ---------------------------------------------------------------- consumer (state chain)
 namespace cons {
 constexpr uint32_t STAGE0 = 0, STAGE1 = SLOT;
-constexpr uint32_t V0 = 2 * SLOT, V1 = V0 + 16384;
+constexpr uint32_t V0 = 2 * SLOT, V1 = V0 + 16384;  // V [j][d]; after the first batch, U [j][d]
 constexpr uint32_t S = V1 + 16384;   // S [c][d] bf16 128 x 128, blocks 16 KB
-constexpr uint32_t U = S + 32768;    // U [j][d] bf16 64 x 128, blocks 8 KB
-constexpr uint32_t MISC = U + 16384; // barriers, flags
+constexpr uint32_t MISC = S + 32768; // barriers, flags
 constexpr uint32_t BYTES = MISC + 256;
-constexpr uint32_t TM_S = 0, TM_U = 128, TM_O0 = 256, TM_O1 = 384, TM_COLS = 512;
+// TMEM: the fp32 state (lane = key channel) and two accumulators D (rows 0..63 = U,
+// rows 64..127 = O; lane = row), used by alternate chunks.
+constexpr uint32_t TM_S = 0, TM_D0 = 128, TM_D1 = 256, TM_COLS = 512;
 }  // namespace cons
 
 __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t *sm, int hd) {
     using namespace cons;
-    constexpr uint32_t I_M64 = idesc_bf16_f32(64, 128, false, 0, 1);      // T'V, Q~S, AU
-    constexpr uint32_t I_M64N = idesc_bf16_f32(64, 128, true, 0, 1);      // -W S
-    constexpr uint32_t I_S = idesc_bf16_f32(128, 128, false, 1, 1);       // K-^T U
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);  // in0, in1, u, s, o
-    uint32_t *s_flags = reinterpret_cast<uint32_t *>(sm + MISC + 64);  // abort, tmem
+    constexpr uint32_t I_D = idesc_bf16_f32(128, 128, false, 0, 1);  // [T';0]V + [-W;Q~]S, [0;A]U
+    constexpr uint32_t I_S = idesc_bf16_f32(128, 128, false, 1, 1);  // K^^T U
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);         // in0, in1, u, s, o
+    uint32_t *s_flags = reinterpret_cast<uint32_t *>(sm + MISC + 64); // abort, tmem
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
     const int H = p.H, n = hd / H, h = hd % H;
-    const int c_me = 32 * quad + lane;
+    const int c_me = 32 * quad + lane;  // TMEM lane of this thread
     const int64_t bos = p.cu_seqlens[n], eos = p.cu_seqlens[n + 1];
     const int nchunks = (int)((eos - bos + C - 1) / C);
     const size_t state_off = ((size_t)n * H + h) * (size_t)(D * D);
@@ -134,13 +141,20 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
         tmem_alloc(&s_flags[1], TM_COLS);
         tmem_relinquish();
     }
+    for (int e = tid; e < 8192 / 16; e += NT) {  // the zero blocks of both stages
+        reinterpret_cast<uint4 *>(sm + STAGE0 + SL_Z)[e] = make_uint4(0u, 0u, 0u, 0u);
+        reinterpret_cast<uint4 *>(sm + STAGE1 + SL_Z)[e] = make_uint4(0u, 0u, 0u, 0u);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_flags[1];
 
-    // thread 0: bring chunk c's image and V into stage c & 1 (block: wait for the producer)
-    int requested = 0;  // chunks requested so far (thread 0)
+    // Flag thread (lane 31 of warp 0: it never stores outputs, so its release stores do not wait
+    // behind output stores in flight): brings chunk c's image and V into stage c & 1 (block:
+    // wait for the producer) and publishes what has been consumed.
+    constexpr int FT = 31;
+    int requested = 0;  // chunks requested so far (flag thread)
     auto request = [&](int c, bool block) -> bool {
         int32_t *fl = p.filled + hd * RING + (c % RING);
         if (block) {
@@ -157,17 +171,16 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
         const int b = c & 1;
         uint8_t *dst = sm + (b ? STAGE1 : STAGE0);
         const uint8_t *src = p.ring + ((size_t)hd * RING + (c % RING)) * SLOT;
-        mbar_arrive_expect_tx(&bars[b], SLOT + 16384);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) bulk_g2s(dst + 16384 * k, src + 16384 * k, 16384, &bars[b]);
-        bulk_g2s(dst + 65536, src + 65536, 1024, &bars[b]);
+        mbar_arrive_expect_tx(&bars[b], 8192 + (SL_G + 512 - SL_A) + 16384);
+        bulk_g2s(dst + SL_T, src + SL_T, 8192, &bars[b]);
+        bulk_g2s(dst + SL_A, src + SL_A, SL_G + 512 - SL_A, &bars[b]);
         const int64_t t0 = bos + (int64_t)c * C;
         tma_load_3d(sm + (b ? V1 : V0), tm_v, &bars[b], 0, h, (int32_t)t0);
         tma_load_3d(sm + (b ? V1 : V0) + 8192, tm_v, &bars[b], 64, h, (int32_t)t0);
         requested = c + 1;
         return true;
     };
-    // thread 0, non-blocking: request every chunk whose stage is free (the chunk two back has
+    // flag thread, non-blocking: request every chunk whose stage is free (the chunk two back has
     // finished all its MMAs: `done` chunks have) and whose image the producer has published
     int done = 0;
     auto poll_ahead = [&]() {
@@ -219,18 +232,18 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
             atomicOr(p.status, 1);
         }
     };
-    // O of chunk cc (TMEM, M=64 rows, columns [64 half, 64 half + 64)) -> bf16 outputs
-    auto store_o = [&](int cc, uint32_t tm_o) {
+    // O of chunk cc: D rows 64..127 (lanes 64..127, quadrants 2 and 3) -> bf16 outputs
+    auto store_o = [&](int cc, uint32_t tm_d) {
         const int64_t tc = bos + (int64_t)cc * C;
         const int vc = (int)(eos - tc < C ? eos - tc : C);
+        const int i = c_me - 64;
         float v[32];
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
             const int col = 64 * half + 32 * part;
-            tmem_ld32(tmem + lane_base + tm_o + col, v);
+            tmem_ld32(tmem + lane_base + tm_d + col, v);
             tmem_wait_ld();
-            const int i = 16 * quad + lane;
-            if (lane < 16 && i < vc) {
+            if (i < vc) {
                 uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(tc + i) * H + h) * D + col);
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8)
@@ -240,54 +253,56 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
         }
     };
 
-    int inflight = 0;  // thread 0: stage copies requested but not yet waited on
     for (int c = 0; c < nchunks; ++c) {
         const int b = c & 1;
         const bool has_next = c + 1 < nchunks;
-        const uint32_t tm_o = b ? TM_O1 : TM_O0;
-        if (tid == 0 && requested <= c) request(c, true);
+        const uint32_t tm_d = b ? TM_D1 : TM_D0;
+        if (tid == FT && requested <= c) request(c, true);
         __syncthreads();
         if (s_flags[0]) break;
         wait_bar(&bars[b], ph_in[b]);
         uint8_t *stage = sm + (b ? STAGE1 : STAGE0);
         const uint32_t st_base = sb + (b ? STAGE1 : STAGE0);
-        if (tid == 0) {
+        const uint32_t vb = sb + (b ? V1 : V0);
+        if (tid == FT) {
             fence_proxy_async_global();
             st_release(p.consumed + hd, c + 1);  // the image is in shared memory: slot reusable
-            // The other stage is free once the previous chunk's last MMA (O += A U) is done:
-            // for c = 0 it never held anything; otherwise it was requested at the end of c - 1.
             poll_ahead();
         }
         const float *gam = reinterpret_cast<const float *>(stage + SL_G);
 
         if (tid == 0) {
             tc_fence_after();
-            const uint64_t dT = desc_k(st_base + SL_T, 8192, 0), dW = desc_k(st_base + SL_W, 8192, 0);
-            const uint64_t dQ = desc_k(st_base + SL_Q, 8192, 0), dS = desc_mn(sb + S, 16384, 0);
-            const uint64_t dV = desc_mn(sb + (b ? V1 : V0), 8192, 0);
+            const uint64_t dTZ = desc_k(st_base + SL_T, 16384, 0), dWQ = desc_k(st_base + SL_WQ, 16384, 0);
+            const uint64_t dV = desc_mn(vb, 8192, 0), dS = desc_mn(sb + S, 16384, 0);
 #pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)  // U = T' V
-                mma_bf16_ss(tmem + TM_U, desc_k_at(dT, 8192, kk), desc_mn_at(dV, kk), I_M64, kk > 0);
+            for (uint32_t kk = 0; kk < 4; ++kk)  // [U; O] = [T'; 0] V ...
+                mma_bf16_ss(tmem + tm_d, desc_k_at(dTZ, 16384, kk), desc_mn_at(dV, kk), I_D, kk > 0);
 #pragma unroll
-            for (uint32_t kk = 0; kk < 8; ++kk)  // U -= W S
-                mma_bf16_ss(tmem + TM_U, desc_k_at(dW, 8192, kk), desc_mn_at(dS, kk), I_M64N, 1);
+            for (uint32_t kk = 0; kk < 8; ++kk)  // ... + [-W; Q~] S
+                mma_bf16_ss(tmem + tm_d, desc_k_at(dWQ, 16384, kk), desc_mn_at(dS, kk), I_D, 1);
             mma_commit(&bars[2]);
-#pragma unroll
-            for (uint32_t kk = 0; kk < 8; ++kk)  // O = Q~ S  (completes behind the U batch)
-                mma_bf16_ss(tmem + tm_o, desc_k_at(dQ, 8192, kk), desc_mn_at(dS, kk), I_M64, kk > 0);
         }
-        // While the U batch runs (it reads only shared memory and writes U, O):
-        // S <- diag(gamma) S in TMEM, ahead of S += K^^T U with K^ = k e^(g_{C-1} - g);
-        // and the previous chunk's outputs from the other O buffer.
+        // While the batch runs (it reads only shared memory and writes D): S <- diag(gamma) S in
+        // TMEM ahead of S += K^^T U, and (rows 64..127) the previous chunk's outputs.
         scale_tmem_row<64>(tmem + lane_base + TM_S + 64 * half, gam[c_me]);
-        if (c > 0) {
-            if (tid == 0) poll_ahead();
-            store_o(c - 1, b ? TM_O0 : TM_O1);  // its MMAs were waited on at the end of c - 1
-        }
+        if (c > 0 && quad >= 2) store_o(c - 1, b ? TM_D0 : TM_D1);
         wait_bar(&bars[2], ph_u);
         tc_fence_after();
 
-        rows64_to_tile<64>(tmem + lane_base + TM_U + 64 * half, sm + U, 8192, 64 * half, quad, lane);
+        // U (D rows 0..63) -> bf16 [j][d] into this stage's V buffer (V is consumed)
+        if (quad < 2) {
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int col = 64 * half + 32 * part;
+                float v[32];
+                tmem_ld32(tmem + lane_base + tm_d + col, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8)
+                    st_chunk(sm + (b ? V1 : V0) + tchunk(8192, c_me, col + 8 * q8), v + 8 * q8);
+            }
+        }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -295,17 +310,16 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
 
         if (tid == 0) {
             tc_fence_after();
-            const uint64_t dK = desc_mn(st_base + SL_KI, 8192, 0), dU = desc_mn(sb + U, 8192, 0);
-            const uint64_t dA = desc_k(st_base + SL_A, 8192, 0);
+            const uint64_t dK = desc_mn(st_base + SL_KH, 8192, 0), dU = desc_mn(vb, 8192, 0);
+            const uint64_t dAZ = desc_k(st_base + SL_Z, 16384, 0);
 #pragma unroll
             for (uint32_t kk = 0; kk < 4; ++kk)  // S += K^^T U   (S already scaled by gamma)
                 mma_bf16_ss(tmem + TM_S, desc_mn_at(dK, kk), desc_mn_at(dU, kk), I_S, 1);
             mma_commit(&bars[3]);
 #pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)  // O += A U
-                mma_bf16_ss(tmem + tm_o, desc_k_at(dA, 8192, kk), desc_mn_at(dU, kk), I_M64, 1);
+            for (uint32_t kk = 0; kk < 4; ++kk)  // [U; O] += [0; A] U
+                mma_bf16_ss(tmem + tm_d, desc_k_at(dAZ, 16384, kk), desc_mn_at(dU, kk), I_D, 1);
             mma_commit(&bars[4]);
-            poll_ahead();
         }
         wait_bar(&bars[3], ph_s);
         tc_fence_after();
@@ -327,25 +341,26 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
                     *reinterpret_cast<float4 *>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
             }
         }
-        // this chunk's last MMA (O += A U): after it, its stage may take chunk c + 2 and
-        // the other stage chunk c + 1's image can be requested with a whole chunk to land
+        // this chunk's last MMA ([0; A] U): after it, its stage may take chunk c + 2
         wait_bar(&bars[4], ph_o);
         tc_fence_after();
-        if (tid == 0) {
+        if (tid == FT) {
             done = c + 1;
-            poll_ahead();  // usually chunk c + 2 into this chunk's stage: a whole chunk to land
+            poll_ahead();
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        (void)inflight;
     }
-    if (nchunks > 0 && !s_flags[0])  // outputs of the last chunk
-        store_o(nchunks - 1, ((nchunks - 1) & 1) ? TM_O1 : TM_O0);
+    if (nchunks > 0 && !s_flags[0] && quad >= 2)  // outputs of the last chunk
+        store_o(nchunks - 1, ((nchunks - 1) & 1) ? TM_D1 : TM_D0);
 
     // teardown: let requested copies and issued MMAs land before freeing TMEM
+    if (s_flags[0] && tid == FT) {
+        for (int c = 0; c < 2; ++c)
+            if (requested > c) mbar_wait_bounded(&bars[c], ph_in[c], p.timeout_ns);
+    }
     if (s_flags[0] && tid == 0) {
-        for (int c = 0; c < 2; ++c) mbar_wait_bounded(&bars[c], ph_in[c], p.timeout_ns);
         mma_commit(&bars[2]);
         mbar_wait_bounded(&bars[2], ph_u, p.timeout_ns);
     }
@@ -523,7 +538,7 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         }
         wait_bar(&bars[2], ph_mma);
         tc_fence_after();
-        rows64_to_tile<64>(tmem + lane_base + TM_W + 64 * half, sm + W, 8192, 64 * half, quad, lane);
+        rows64_to_tile<64>(tmem + lane_base + TM_W + 64 * half, sm + W, 8192, 64 * half, quad, lane, -1.f);
         if (tid == 0 && c >= RING) {  // the slot's previous chunk must have been taken
             if (!wait_flag_ge(p.consumed + hd, c - RING + 1, p.timeout_ns)) {
                 s_flags[0] = 1;
@@ -535,15 +550,18 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         __syncthreads();
         if (s_flags[0]) break;
 
-        // copy the image out with bulk stores: Q~ (rows 0..63 of both 16 KB blocks), K^, then
-        // W, A, T' (contiguous), gamma; published at the next item (see release)
+        // copy the image out with bulk stores (layout at the top of this file); published at the
+        // next item (see release)
         if (tid == 0) {
             uint8_t *slot = p.ring + ((size_t)hd * RING + (c % RING)) * SLOT;
             fence_proxy_async_smem();
-            bulk_s2g(slot + SL_Q, qk, 8192);
-            bulk_s2g(slot + SL_Q + 8192, qk + 16384, 8192);
-            bulk_s2g(slot + SL_KI, sm + KH, 16384);
-            bulk_s2g(slot + SL_W, sm + W, SL_G - SL_W);
+            bulk_s2g(slot + SL_T, sm + TT, 8192);
+            bulk_s2g(slot + SL_A, sm + AQK, 8192);
+            bulk_s2g(slot + SL_WQ, sm + W, 8192);                  // -W, columns 0..63
+            bulk_s2g(slot + SL_WQ + 8192, qk, 8192);               // Q~, columns 0..63
+            bulk_s2g(slot + SL_WQ + 16384, sm + W + 8192, 8192);   // -W, columns 64..127
+            bulk_s2g(slot + SL_WQ + 24576, qk + 16384, 8192);      // Q~, columns 64..127
+            bulk_s2g(slot + SL_KH, sm + KH, 16384);
             bulk_s2g(slot + SL_G, s_gamma, 512);
             bulk_commit();
             bulk_wait_read();  // shared memory may be rewritten by the next item
