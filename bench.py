@@ -254,6 +254,34 @@ def bench_decode(args, K, stream, ws):
             "gpu_launches": nsteps}
 
 
+def bench_prefill_workload(wl, K, stream, steps, warmup, rank):
+    """Device-timed kda_prefill of one workload (inputs resident in HBM); returns a summary dict."""
+    inp = W.make_inputs(wl, "cuda", seed=wl.seed + 7919 * rank)
+    N, T, H = wl.num_seqs, wl.total_tokens, wl.H
+    out = torch.empty(T, H, wl.dv, dtype=wl.torch_dtype, device="cuda")
+    fs = torch.empty(N, H, wl.dk, wl.dv, dtype=torch.float32, device="cuda")
+    work = torch.empty(K.workspace_size(N, T, H, wl.dk, wl.dv, wl.torch_dtype), dtype=torch.uint8,
+                       device="cuda")
+
+    def step():
+        K.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["initial_state"],
+                  inp["cu_seqlens"], inp["cu_seqlens_dev"], out=out, final_state=fs, workspace=work,
+                  stream=stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ms = time_events(step, steps, stream)
+    th = T * H
+    pk = peaks()
+    del inp, out, fs, work
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "tokens": T, "heads": H, "sequences": N, "ms_per_step": ms,
+            "tokens_per_s": T / (ms * 1e-3),
+            "tc_frac": FLOP_PER_TOKEN_HEAD * th / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
+            "hbm_frac": PREFILL_BYTES_PER_TOKEN_HEAD * th / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+
+
 def run_ours(args, rank, local, ws):
     from gated_delta_rule_62_b200 import build
     from gated_delta_rule_62_b200 import kda as K
@@ -327,6 +355,10 @@ def run_ours(args, rank, local, ws):
     del host, dev
 
     dec = bench_decode(args, K, stream, ws) if not args.no_decode else None
+    extra = None
+    if not args.no_extra:
+        extra = [bench_prefill_workload(W.VARLEN_24, K, stream, 5, 3, rank),
+                 bench_prefill_workload(W.PREFILL_1M, K, stream, 3, 3, rank)]
 
     if rank != 0:
         return
@@ -353,6 +385,7 @@ def run_ours(args, rank, local, ws):
             "value": T * ws / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "decode": dec,
+        "other_prefill_workloads": extra,
         "gpu_launches": args.steps * kernels_per_step,
         "clocks": clocks,
         "cpu_baseline": cpu,
@@ -370,6 +403,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the varlen-24 and 1M-token prefill measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-tokens", type=int, default=2048)
