@@ -6,17 +6,19 @@
 // form the sequential chain. With few heads a fused kernel leaves most SMs idle while each
 // head's CTA serialises both halves. Here one persistent cooperative launch fills the GPU:
 //
-//   consumer CTAs (one per head): the state chain. Per chunk: U = T'V - W S and O = Q~ S
-//     (one MMA batch), U to bf16, O += A U and S += K-^T U (one batch), then the outputs and
-//     S <- diag(gamma) S. The fp32 state stays in TMEM for the whole sequence.
+//   consumer CTAs (one per head, or two per head with 64 value channels each when the SMs
+//     left over still give every head about three producers): the state chain. Per chunk:
+//     [U; O] = [T'; 0] V + [-W; Q~] S (one MMA batch), U to bf16, S += K^^T U and
+//     [U; O] += [0; A] U (a second batch), then the outputs and the state's bf16 copy. The fp32
+//     state (pre-scaled by gamma while the first batch runs) stays in TMEM for the whole sequence.
 //   producer CTAs (all other SMs): the key-side half for chunks ahead, chunk-major order,
 //     written as ready-to-use shared-memory images (Q~, K- or K^, W, A, T' tiles, gamma,
 //     path flag) into a ring of RING slots per head in the workspace (L2 resident).
 //
 // Hand-off: a producer fills slot (head, c % RING) with generic stores, then releases
 // filled[slot] = c + 1; the consumer acquires it, copies the image into shared memory with a
-// bulk copy, and releases consumed[head] = c + 1 once the copy has landed; the producer
-// acquires consumed[head] >= c - RING + 1 before reusing the slot. Producer items are
+// bulk copy, and releases consumed[consumer] = c + 1 once the copy has landed; the producer
+// acquires both consumers' counters >= c - RING + 1 before reusing the slot. Producer items are
 // ordered by chunk, and every producer works through its items in order, so the item a
 // consumer waits for never waits on anything later: no cycle. Every spin and mbarrier wait is
 // bounded; on timeout the status word is set and the CTA stops. The launch is cooperative,
@@ -55,8 +57,8 @@ struct SplitParams {
     int32_t *status;
     uint8_t *ring;       // [heads][RING][SLOT]
     int32_t *filled;     // [heads][RING]
-    int32_t *consumed;   // [heads]
-    int32_t H, heads, max_chunks;
+    int32_t *consumed;   // [heads][2]: one counter per consumer (the second unused with one)
+    int32_t H, heads, max_chunks, cph;
     uint64_t timeout_ns;
 };
 
@@ -104,21 +106,32 @@ __device__ __forceinline__ void bulk_wait_read() {
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ---------------------------------------------------------------- consumer (state chain)
-namespace cons {
-constexpr uint32_t STAGE0 = 0, STAGE1 = SLOT;
-constexpr uint32_t V0 = 2 * SLOT, V1 = V0 + 16384;  // V [j][d]; after the first batch, U [j][d]
-constexpr uint32_t S = V1 + 16384;   // S [c][d] bf16 128 x 128, blocks 16 KB
-constexpr uint32_t MISC = S + 32768; // barriers, flags
-constexpr uint32_t BYTES = MISC + 256;
-// TMEM: the fp32 state (lane = key channel) and two accumulators D (rows 0..63 = U,
-// rows 64..127 = O; lane = row), used by alternate chunks.
-constexpr uint32_t TM_S = 0, TM_D0 = 128, TM_D1 = 256, TM_COLS = 512;
-}  // namespace cons
+// CPH consumers per head, each owning DC = 128 / CPH value channels (columns of S are
+// independent: the chain of one column block never reads another's).
+template <int CPH>
+struct Cons {
+    static constexpr int DC = D / CPH;                            // value channels per consumer
+    static constexpr int NP = DC / 64;                            // 32-column parts per thread
+    static constexpr uint32_t STAGE0 = 0, STAGE1 = SLOT;
+    static constexpr uint32_t V0 = 2 * SLOT, V1 = V0 + 128 * DC;  // V [j][d]; after batch 1, U
+    static constexpr uint32_t S = V1 + 128 * DC;                  // S [c][d] bf16 128 x DC
+    static constexpr uint32_t MISC = S + 256 * DC;                // barriers, flags
+    static constexpr uint32_t BYTES = MISC + 256;
+    // TMEM: the fp32 state (lane = key channel) and two accumulators D (rows 0..63 = U,
+    // rows 64..127 = O; lane = row), used by alternate chunks.
+    static constexpr uint32_t TM_S = 0, TM_D0 = DC, TM_D1 = 2 * DC, TM_COLS = CPH == 1 ? 512 : 256;
+};
 
-__device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t *sm, int hd) {
-    using namespace cons;
-    constexpr uint32_t I_D = idesc_bf16_f32(128, 128, false, 0, 1);  // [T';0]V + [-W;Q~]S, [0;A]U
-    constexpr uint32_t I_S = idesc_bf16_f32(128, 128, false, 1, 1);  // K^^T U
+template <int CPH>
+__device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t *sm, int cid) {
+    using L = Cons<CPH>;
+    constexpr int DC = L::DC, NP = L::NP;
+    constexpr uint32_t STAGE0 = L::STAGE0, STAGE1 = L::STAGE1, V0 = L::V0, V1 = L::V1, S = L::S;
+    constexpr uint32_t MISC = L::MISC, TM_S = L::TM_S, TM_D0 = L::TM_D0, TM_D1 = L::TM_D1;
+    constexpr uint32_t TM_COLS = L::TM_COLS;
+    constexpr uint32_t I_D = idesc_bf16_f32(128, DC, false, 0, 1);  // [T';0]V + [-W;Q~]S, [0;A]U
+    constexpr uint32_t I_S = idesc_bf16_f32(128, DC, false, 1, 1);  // K^^T U
+    const int hd = cid / CPH, sub = cid % CPH, d0 = DC * sub;  // head, first value channel
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);         // in0, in1, u, s, o
     uint32_t *s_flags = reinterpret_cast<uint32_t *>(sm + MISC + 64); // abort, tmem
     const uint32_t sb = smem_u32(sm);
@@ -150,10 +163,11 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
     tc_fence_after();
     const uint32_t tmem = s_flags[1];
 
-    // Flag thread (lane 31 of warp 0: it never stores outputs, so its release stores do not wait
-    // behind output stores in flight): brings chunk c's image and V into stage c & 1 (block:
-    // wait for the producer) and publishes what has been consumed.
-    constexpr int FT = 31;
+    // Flag thread (lane 31 of warp 5: not the MMA-issuing warp, and it never stores outputs, so
+    // its fences and release stores neither stall MMA issue nor wait behind output stores):
+    // brings chunk c's image and V into stage c & 1 (block: wait for the producer) and
+    // publishes what has been consumed.
+    constexpr int FT = 5 * 32 + 31;
     int requested = 0;  // chunks requested so far (flag thread)
     auto request = [&](int c, bool block) -> bool {
         int32_t *fl = p.filled + hd * RING + (c % RING);
@@ -171,12 +185,13 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
         const int b = c & 1;
         uint8_t *dst = sm + (b ? STAGE1 : STAGE0);
         const uint8_t *src = p.ring + ((size_t)hd * RING + (c % RING)) * SLOT;
-        mbar_arrive_expect_tx(&bars[b], 8192 + (SL_G + 512 - SL_A) + 16384);
+        mbar_arrive_expect_tx(&bars[b], 8192 + (SL_G + 512 - SL_A) + 128 * DC);
         bulk_g2s(dst + SL_T, src + SL_T, 8192, &bars[b]);
         bulk_g2s(dst + SL_A, src + SL_A, SL_G + 512 - SL_A, &bars[b]);
         const int64_t t0 = bos + (int64_t)c * C;
-        tma_load_3d(sm + (b ? V1 : V0), tm_v, &bars[b], 0, h, (int32_t)t0);
-        tma_load_3d(sm + (b ? V1 : V0) + 8192, tm_v, &bars[b], 64, h, (int32_t)t0);
+#pragma unroll
+        for (int part = 0; part < NP; ++part)
+            tma_load_3d(sm + (b ? V1 : V0) + 8192 * part, tm_v, &bars[b], d0 + 64 * part, h, (int32_t)t0);
         requested = c + 1;
         return true;
     };
@@ -190,11 +205,11 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
 
     // initial state -> TMEM (lane c, columns d) and its bf16 tile; empty sequences copy it out
     {
-        const size_t row = state_off + (size_t)c_me * D + 64 * half;
+        const size_t row = state_off + (size_t)c_me * D + d0 + 32 * NP * half;
         const float *src = p.s0 ? p.s0 + row : nullptr;
         float *dst = p.sT ? p.sT + row : nullptr;
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
+        for (int part = 0; part < NP; ++part) {
             float v[32];
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
@@ -210,7 +225,7 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
                             make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
                 }
             } else {
-                const int col = 64 * half + 32 * part;
+                const int col = 32 * NP * half + 32 * part;
                 tmem_st32(tmem + lane_base + TM_S + col, v);
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8)
@@ -239,12 +254,12 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
         const int i = c_me - 64;
         float v[32];
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            const int col = 64 * half + 32 * part;
+        for (int part = 0; part < NP; ++part) {
+            const int col = 32 * NP * half + 32 * part;
             tmem_ld32(tmem + lane_base + tm_d + col, v);
             tmem_wait_ld();
             if (i < vc) {
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(tc + i) * H + h) * D + col);
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(tc + i) * H + h) * D + d0 + col);
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8)
                     dst[q8] = make_uint4(pack2(v[8 * q8], v[8 * q8 + 1]), pack2(v[8 * q8 + 2], v[8 * q8 + 3]),
@@ -266,15 +281,16 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
         const uint32_t vb = sb + (b ? V1 : V0);
         if (tid == FT) {
             fence_proxy_async_global();
-            st_release(p.consumed + hd, c + 1);  // the image is in shared memory: slot reusable
-            poll_ahead();
+            st_release(p.consumed + 2 * hd + sub, c + 1);  // the image is in shared memory: slot reusable
+            done = c;  // every MMA of chunk c - 1 was waited on at the end of its iteration
+            poll_ahead();  // usually chunk c + 1 into the other stage: a whole chunk to land
         }
         const float *gam = reinterpret_cast<const float *>(stage + SL_G);
 
         if (tid == 0) {
             tc_fence_after();
             const uint64_t dTZ = desc_k(st_base + SL_T, 16384, 0), dWQ = desc_k(st_base + SL_WQ, 16384, 0);
-            const uint64_t dV = desc_mn(vb, 8192, 0), dS = desc_mn(sb + S, 16384, 0);
+            const uint64_t dV = desc_mn(vb, 8192, 0), dS = desc_mn(sb + S, 16384, 0);  // one N block
 #pragma unroll
             for (uint32_t kk = 0; kk < 4; ++kk)  // [U; O] = [T'; 0] V ...
                 mma_bf16_ss(tmem + tm_d, desc_k_at(dTZ, 16384, kk), desc_mn_at(dV, kk), I_D, kk > 0);
@@ -284,8 +300,12 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
             mma_commit(&bars[2]);
         }
         // While the batch runs (it reads only shared memory and writes D): S <- diag(gamma) S in
-        // TMEM ahead of S += K^^T U, and (rows 64..127) the previous chunk's outputs.
-        scale_tmem_row<64>(tmem + lane_base + TM_S + 64 * half, gam[c_me]);
+        // TMEM ahead of S += K^^T U (warp 4 takes warp 0's columns: warp 0 issues the MMAs), and
+        // (rows 64..127) the previous chunk's outputs.
+        if (warp == 4)
+            scale_tmem_row<DC>(tmem + lane_base + TM_S, gam[c_me]);
+        else if (warp != 0)
+            scale_tmem_row<DC / 2>(tmem + lane_base + TM_S + (DC / 2) * half, gam[c_me]);
         if (c > 0 && quad >= 2) store_o(c - 1, b ? TM_D0 : TM_D1);
         wait_bar(&bars[2], ph_u);
         tc_fence_after();
@@ -293,8 +313,8 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
         // U (D rows 0..63) -> bf16 [j][d] into this stage's V buffer (V is consumed)
         if (quad < 2) {
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int col = 64 * half + 32 * part;
+            for (int part = 0; part < NP; ++part) {
+                const int col = 32 * NP * half + 32 * part;
                 float v[32];
                 tmem_ld32(tmem + lane_base + tm_d + col, v);
                 tmem_wait_ld();
@@ -326,8 +346,8 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
 
         // the next state's bf16 tile (and the final state after the last chunk)
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            const int col = 64 * half + 32 * part;
+        for (int part = 0; part < NP; ++part) {
+            const int col = 32 * NP * half + 32 * part;
             float v[32];
             tmem_ld32(tmem + lane_base + TM_S + col, v);
             tmem_wait_ld();
@@ -335,7 +355,7 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
             for (int q8 = 0; q8 < 4; ++q8)
                 st_chunk(sm + S + tchunk(16384, c_me, col + 8 * q8), v + 8 * q8);
             if (!has_next && p.sT) {
-                float *dst = p.sT + state_off + (size_t)c_me * D + col;
+                float *dst = p.sT + state_off + (size_t)c_me * D + d0 + col;
 #pragma unroll
                 for (int e = 0; e < 32; e += 4)
                     *reinterpret_cast<float4 *>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
@@ -344,10 +364,6 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
         // this chunk's last MMA ([0; A] U): after it, its stage may take chunk c + 2
         wait_bar(&bars[4], ph_o);
         tc_fence_after();
-        if (tid == FT) {
-            done = c + 1;
-            poll_ahead();
-        }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -451,8 +467,11 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         if (c >= nch || t0 + tid >= eos) return 0.f;
         return p.beta[(size_t)(t0 + tid) * H + h];
     };
-    // thread 0: publish a filled slot once its bulk stores are complete (deferred so that the
-    // completion wait overlaps the next item's work)
+    // Bulk-store thread (lane 31 of warp 7: not the MMA-issuing thread; warp 7 idles during the
+    // first stage of the inverse, where the publish goes): issues an image's bulk stores, waits
+    // for them to have read shared memory before the next item rewrites it (just before its
+    // gating), and publishes the slot once they are complete (during the next item's inverse).
+    constexpr int BT = NT - 1;
     int32_t *rel_flag = nullptr;
     int rel_val = 0;
     auto release = [&]() {
@@ -491,17 +510,20 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         if (tid < C) s_beta[tid] = beta_next;
         wait_bar(&bars[b], ph_in[b]);
         pending[b] = false;
-        if (nxt < nch) {
-            if (tid == 0) issue_inputs(nxt, b ^ 1);  // the other stage's last user is done
-            pending[b ^ 1] = true;
-        }
+
         if (tid < C) beta_next = load_beta(nxt);
         uint8_t *qk = sm + (b ? QK1 : QK0);
         float *la = reinterpret_cast<float *>(sm + (b ? LA1 : LA0));
 
+        if (tid == BT) bulk_wait_read();  // the previous image's sources are rewritten below
         const int gate = gate_chunk(qk, sm + KI, sm + AQK, la, LTp, s_beta, s_gamma, s_psum,
                                     s_flags, valid, tid, sm + KH);
-        if (tid == 0) release();  // the previous item's image
+        // The next item's inputs go to the other stage, whose Q~ the previous image's bulk
+        // stores read: gate_chunk's barriers come after the bulk-store thread's read wait.
+        if (nxt < nch && gate >= 0) {
+            if (tid == 0) issue_inputs(nxt, b ^ 1);
+            pending[b ^ 1] = true;
+        }
         if (gate < 0) break;
         const bool safe = gate == 1;
         fence_proxy_async_smem();
@@ -524,6 +546,7 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         __syncthreads();
         if (s_flags[0]) break;
 
+        if (tid == BT) release();  // the previous item's image (warp 7 idles in the inverse's stage 1)
         invert_unit_lower(LTp, PBp, sm + TT, s_beta, tid);
         fence_proxy_async_smem();
         __syncthreads();
@@ -539,8 +562,9 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         wait_bar(&bars[2], ph_mma);
         tc_fence_after();
         rows64_to_tile<64>(tmem + lane_base + TM_W + 64 * half, sm + W, 8192, 64 * half, quad, lane, -1.f);
-        if (tid == 0 && c >= RING) {  // the slot's previous chunk must have been taken
-            if (!wait_flag_ge(p.consumed + hd, c - RING + 1, p.timeout_ns)) {
+        if (tid == BT && c >= RING) {  // the slot's previous chunk must have been taken
+            if (!wait_flag_ge(p.consumed + 2 * hd, c - RING + 1, p.timeout_ns) ||
+                (p.cph == 2 && !wait_flag_ge(p.consumed + 2 * hd + 1, c - RING + 1, p.timeout_ns))) {
                 s_flags[0] = 1;
                 atomicOr(p.status, 1);
             }
@@ -552,7 +576,7 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 
         // copy the image out with bulk stores (layout at the top of this file); published at the
         // next item (see release)
-        if (tid == 0) {
+        if (tid == BT) {
             uint8_t *slot = p.ring + ((size_t)hd * RING + (c % RING)) * SLOT;
             fence_proxy_async_smem();
             bulk_s2g(slot + SL_T, sm + TT, 8192);
@@ -564,7 +588,6 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             bulk_s2g(slot + SL_KH, sm + KH, 16384);
             bulk_s2g(slot + SL_G, s_gamma, 512);
             bulk_commit();
-            bulk_wait_read();  // shared memory may be rewritten by the next item
             rel_flag = p.filled + hd * RING + (c % RING);
             rel_val = c + 1;
         }
@@ -573,9 +596,9 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         b ^= 1;
     }
 
-    if (tid == 0 && !s_flags[0]) release();
+    if (tid == BT && !s_flags[0]) release();
+    if (s_flags[0] && tid == BT) bulk_wait_all();
     if (s_flags[0] && tid == 0) {
-        bulk_wait_all();
         for (int k = 0; k < 2; ++k)
             if (pending[k]) mbar_wait_bounded(&bars[k], ph_in[k], p.timeout_ns);
         mma_commit(&bars[2]);
@@ -589,8 +612,12 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     }
 }
 
-constexpr uint32_t SPLIT_SMEM = (cons::BYTES > prod::BYTES ? cons::BYTES : prod::BYTES) + 1024;
+constexpr uint32_t max3(uint32_t a, uint32_t b, uint32_t c) {
+    return a > b ? (a > c ? a : c) : (b > c ? b : c);
+}
+constexpr uint32_t SPLIT_SMEM = max3(Cons<1>::BYTES, Cons<2>::BYTES, prod::BYTES) + 1024;
 
+template <int CPH>
 __global__ void __launch_bounds__(NT, 1)
 split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
@@ -598,10 +625,10 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-    if ((int)blockIdx.x < p.heads)
-        consumer(&tm_v, p, sm, blockIdx.x);
+    if ((int)blockIdx.x < CPH * p.heads)
+        consumer<CPH>(&tm_v, p, sm, blockIdx.x);
     else
-        producer(&tm_q, &tm_k, &tm_la, p, sm, blockIdx.x - p.heads, gridDim.x - p.heads);
+        producer(&tm_q, &tm_k, &tm_la, p, sm, blockIdx.x - CPH * p.heads, gridDim.x - CPH * p.heads);
 }
 
 // Zeroes the status word and the ring flags.
@@ -617,7 +644,7 @@ int sm_count() {
     return sms;
 }
 
-size_t flags_bytes(int64_t heads) { return ((size_t)heads * (RING + 1) * 4 + 1023) / 1024 * 1024; }
+size_t flags_bytes(int64_t heads) { return ((size_t)heads * (RING + 2) * 4 + 1023) / 1024 * 1024; }
 
 }  // namespace
 
@@ -635,18 +662,26 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
                                  cudaStream_t stream, uint64_t timeout_ns) {
     const int64_t heads = (int64_t)p.num_seqs * p.H;
     const int sms = sm_count();
+    // Two consumers per head halve the chain's per-chunk work, but take SMs from the producers;
+    // worth it only while every head still gets about three producers (a producer's item costs
+    // about two and a half consumer chunks).
+    const int cph = heads * 5 <= sms ? 2 : 1;
+    const void *fn = cph == 2 ? (const void *)split_kernel<2> : (const void *)split_kernel<1>;
     int per_sm = 0;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute(split_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)SPLIT_SMEM);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(split_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)SPLIT_SMEM);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, split_kernel, NT, SPLIT_SMEM);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, NT, SPLIT_SMEM);
     if (e != cudaSuccess) return e;
     const int grid = per_sm * sms;
-    if (per_sm < 1 || grid <= heads) return cudaErrorInvalidConfiguration;
+    if (per_sm < 1 || grid < (cph + 1) * heads) return cudaErrorInvalidConfiguration;
 
     CUtensorMap mq, mk, mv, mla;
     const uint64_t T = (uint64_t)p.total_tokens, H = (uint64_t)p.H;
@@ -659,7 +694,7 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int32_t *status = reinterpret_cast<int32_t *>(ws);
     int32_t *flags = reinterpret_cast<int32_t *>(ws + 1024);
-    const int nflags = (int)(heads * (RING + 1));
+    const int nflags = (int)(heads * (RING + 2));
     split_init_kernel<<<(nflags + 255) / 256, 256, 0, stream>>>(status, flags, nflags);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -677,10 +712,10 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
     sp.H = p.H;
     sp.heads = (int32_t)heads;
     sp.max_chunks = max_chunks;
+    sp.cph = cph;
     sp.timeout_ns = timeout_ns;
     void *args[] = {&mq, &mk, &mv, &mla, &sp};
-    return cudaLaunchCooperativeKernel((const void *)split_kernel, dim3(grid), dim3(NT), args,
-                                       SPLIT_SMEM, stream);
+    return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(NT), args, SPLIT_SMEM, stream);
 }
 
 }  // namespace kda
