@@ -19,6 +19,23 @@ constexpr int D = 128;   // d_k = d_v
 constexpr int NT = 256;  // compute threads per CTA
 constexpr float kFastLimit = 60.f;  // max in-chunk decay exponent for the factored path
 
+// Barrier over the NT compute threads (warps 0 .. NT/32 - 1) only: hardware barrier 1, so a
+// CTA may run further warps (a control warp) that never join it.
+__device__ __forceinline__ void sync_compute() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
+// The same barrier, returning whether any compute thread passed a non-zero `pred`.
+__device__ __forceinline__ int sync_compute_or(int pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, 1, %2, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "n"(NT)
+        : "memory");
+    return (int)r;
+}
+
 // ---------------------------------------------------------------- tile addressing
 // bf16 tiles use the 128-byte swizzle: 128-byte rows of 64 elements, 8-row groups
 // 1024 bytes apart, 16-byte chunk index XOR (row % 8); 64-column blocks `bs` bytes apart.
@@ -129,7 +146,8 @@ __device__ __forceinline__ void frag_to_tt(uint8_t *TT, int r0, int c0, const fl
 // strictly upper 16x16 blocks must already be zero). Blocks of 16: the diagonal blocks by
 // forward substitution, then the block inverse [[A,0],[B,C]]^-1 = [[A^-1,0],[-C^-1 B A^-1,
 // C^-1]] at 16 and then at 32, on the tensor cores (tf32 mma.sync). LT keeps the fp32 blocks
-// later stages need. Called by all NT threads; ends with the TT stores issued (no barrier).
+// later stages need. Called by the NT compute threads (synchronised among themselves with
+// sync_compute); ends with the TT stores issued (no barrier).
 static __device__ void invert_unit_lower(float *LT, float *PB, uint8_t *TT, const float *beta, int tid) {
     const int warp = tid >> 5, lane = tid & 31;
     if (warp < 4 && lane < 16) {
@@ -157,7 +175,7 @@ static __device__ void invert_unit_lower(float *LT, float *PB, uint8_t *TT, cons
             st_bf(TT + telem(8192, b0 + i, b0 + lane), x[i] * bl);
         }
     }
-    __syncthreads();
+    sync_compute();
     if (warp < 2) {
         // warp 0: T10 = -T11 (L10 T00); warp 1: T32 = -T33 (L32 T22)
         const int r0 = warp ? 48 : 16, c0 = warp ? 32 : 0;
@@ -171,7 +189,7 @@ static __device__ void invert_unit_lower(float *LT, float *PB, uint8_t *TT, cons
         warp_store16(LT + r0 * LT_LD + c0, LT_LD, acc2, -1.f);
         frag_to_tt(TT, r0, c0, acc2, -1.f, beta);
     }
-    __syncthreads();
+    sync_compute();
     // rows 32..63 x cols 0..31: P = L[32:64, 0:32] T[0:32, 0:32];  T[32:64, 0:32] = -T[32:64, 32:64] P
     const int rt = (warp >> 1) & 1, ct = warp & 1;
     if (warp < 4) {
@@ -179,7 +197,7 @@ static __device__ void invert_unit_lower(float *LT, float *PB, uint8_t *TT, cons
         warp_mm16(acc, LT + (32 + 16 * rt) * LT_LD, LT_LD, LT + 16 * ct, LT_LD, 32);
         warp_store16(PB + (16 * rt) * PB_LD + 16 * ct, PB_LD, acc, 1.f);
     }
-    __syncthreads();
+    sync_compute();
     if (warp < 4) {
         float acc[2][4] = {};
         warp_mm16(acc, LT + (32 + 16 * rt) * LT_LD + 32, LT_LD, PB + 16 * ct, PB_LD, 32);
@@ -189,17 +207,23 @@ static __device__ void invert_unit_lower(float *LT, float *PB, uint8_t *TT, cons
 
 
 // ---------------------------------------------------------------- gating of one chunk
-// All NT threads. In: QK holds raw q (rows 0..63) and k (rows 64..127) as a K-major tile with
+// The NT compute threads (synchronised among themselves with sync_compute). In: QK holds raw
+// q (rows 0..63) and k (rows 64..127) as a K-major tile with
 // 16 KB blocks, LA the chunk's raw log_alpha [t][c] fp32, s_beta the chunk's beta (0 past `valid`).
 // Out: QK holds Q~ and K~ in place, KI holds K- (factored path) or K^ (exact path), s_gamma =
 // e^(g_{C-1}); the exact path also writes A into AQK and beta-scaled L into LT (zeros elsewhere).
 // Thread mapping: channel pair (cA, cA + 1), token quarter tq (tokens 16 tq .. 16 tq + 15).
-// If KH is not null it also receives K^ = k e^(g_{C-1} - g) on both paths.
-// Returns 1 for the exact path, 0 for the factored path, -1 if *s_abort was set.
+// If KH is not null it also receives K^ = k e^(g_{C-1} - g) on both paths. If src_free is not
+// null, the writes to KI, KH and AQK first wait (bounded by timeout_ns) for that mbarrier's
+// phase with parity src_parity: another thread may still be reading those tiles.
+// Returns 1 for the exact path, 0 for the factored path, -1 if *s_abort was set or the wait
+// timed out (which sets *s_abort).
 __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK, float *LA,
                                           float *LT, const float *s_beta, float *s_gamma,
-                                          float *s_psum, const uint32_t *s_abort, int valid,
-                                          int tid, uint8_t *KH = nullptr) {
+                                          float *s_psum, uint32_t *s_abort, int valid,
+                                          int tid, uint8_t *KH = nullptr,
+                                          uint64_t *src_free = nullptr, uint32_t src_parity = 0,
+                                          uint64_t timeout_ns = 0) {
     const int tq = tid >> 6, cA = 2 * (tid & 63);
     const int warp = tid >> 5, lane = tid & 31;
     // ---- gates: log_alpha of 16 tokens x 2 channels into registers, quarter totals
@@ -219,8 +243,12 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
     // down the exact path; otherwise the whole chunk decays by at most e^kFastLimit.
     // (NaN gates also take the exact path: the comparisons are false for NaN.)
     const int unsafe = !(-tot.x <= 0.25f * kFastLimit) || !(-tot.y <= 0.25f * kFastLimit);
-    const bool safe = __syncthreads_or(unsafe) != 0;
+    const bool safe = sync_compute_or(unsafe) != 0;
     if (*s_abort) return -1;
+    if (src_free && !mbar_wait_bounded(src_free, src_parity, timeout_ns)) {
+        *s_abort = 1;
+        return -1;
+    }
     float2 goff = make_float2(0.f, 0.f), gC = make_float2(0.f, 0.f);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -250,7 +278,7 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
             st_bf(AQK + telem(8192, i, j), 0.f);
             LT[i * LT_LD + j] = 0.f;
         }
-        __syncthreads();
+        sync_compute();
         for (int e = warp; e < 64 * 64; e += NT / 32) {
             const int i = e >> 6, j = e & 63;
             if (j > i || i >= valid) continue;
@@ -273,7 +301,7 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
                 if (j < i) LT[i * LT_LD + j] = s_beta[i] * l;
             }
         }
-        __syncthreads();  // raw q, k are read above and overwritten below
+        sync_compute();  // raw q, k are read above and overwritten below
     }
 
     // ---- gated operands. With alpha = e^log_alpha, prefix products P_i and suffix
@@ -385,5 +413,8 @@ __device__ __forceinline__ void scale_tmem_row(uint32_t taddr, float gm) {
 // 3-D TMA map over [T][H][inner] with a box of (box_inner, 1, 64 tokens); false on failure.
 bool make_token_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint32_t esize,
                     uint64_t inner, uint64_t H, uint64_t T, uint32_t box_inner, bool swizzle);
+// 2-D TMA map over `rows` 128-byte rows (64 bf16 each, copied verbatim: no swizzle) with a box of
+// box_rows rows; false on failure.
+bool make_rows_map(CUtensorMap *m, void *base, uint64_t rows, uint32_t box_rows);
 
 }  // namespace kda

@@ -1,28 +1,33 @@
 // Split-role chunked prefill for workloads with few (sequence, head) pairs.
 //
-// The chunk algebra is that of kda_chunk.cu. Its key-side half -- gating, the intra-chunk
-// products A and L, T' = (I + L)^-1 diag(beta), W = T' K~ -- does not depend on the state and
-// can run for any chunk at any time; only U = T'V - W S, O = Q~ S + A U and the state update
-// form the sequential chain. With few heads a fused kernel leaves most SMs idle while each
-// head's CTA serialises both halves. Here one persistent cooperative launch fills the GPU:
+// The chunk algebra is that of kda_chunk.cu, regrouped so that the sequential state chain
+// holds a single dependent MMA batch per chunk. With U = T'V - W S (T'V written U~):
 //
+//   S_next = diag(gamma) S + K^^T U = S + M S + K^^T U~,   M = diag(gamma - 1) - K^^T W,
+//   O      = Q~ S + A U             = P S + A U~,          P = Q~ - A W.
+//
+// M, P and U~ depend only on the chunk's own q, k, v, gates and beta, so they are computed
+// off the chain. One persistent cooperative launch fills the GPU:
+//
+//   producer CTAs (most SMs): for chunks ahead of the chain, chunk-major order: the gating,
+//     A and L, T' = (I + L)^-1 diag(beta), W = T' K~, then U~ and -A W in one M=128 MMA
+//     ([T'; 0] V + [0; A] (-W)) and -K^^T W in another, and from those U~, P and M as
+//     ready-to-use shared-memory images (bf16) in a ring of RING slots per head in the
+//     workspace (L2 resident).
 //   consumer CTAs (one per head, or two per head with 64 value channels each when the SMs
-//     left over still give every head about three producers): the state chain. Per chunk:
-//     [U; O] = [T'; 0] V + [-W; Q~] S (one MMA batch), U to bf16, S += K^^T U and
-//     [U; O] += [0; A] U (a second batch), then the outputs and the state's bf16 copy. The fp32
-//     state (pre-scaled by gamma while the first batch runs) stays in TMEM for the whole sequence.
-//   producer CTAs (all other SMs): the key-side half for chunks ahead, chunk-major order,
-//     written as ready-to-use shared-memory images (Q~, K- or K^, W, A, T' tiles, gamma,
-//     path flag) into a ring of RING slots per head in the workspace (L2 resident).
+//     left over still give every head about three producers): the chain. Per chunk:
+//     S += M S_b + K^^T U~ (S_b = the state's bf16 copy), O = P S_b + A U~ behind it, then
+//     the new state's bf16 copy; the outputs leave while the next chunk's batch runs. The fp32
+//     state stays in TMEM for the whole sequence.
 //
-// Hand-off: a producer fills slot (head, c % RING) with generic stores, then releases
-// filled[slot] = c + 1; the consumer acquires it, copies the image into shared memory with a
-// bulk copy, and releases consumed[consumer] = c + 1 once the copy has landed; the producer
-// acquires both consumers' counters >= c - RING + 1 before reusing the slot. Producer items are
-// ordered by chunk, and every producer works through its items in order, so the item a
-// consumer waits for never waits on anything later: no cycle. Every spin and mbarrier wait is
-// bounded; on timeout the status word is set and the CTA stops. The launch is cooperative,
-// so all CTAs are resident together or the launch fails.
+// Hand-off: a producer fills slot (head, c % RING) with bulk stores, then releases
+// filled[slot] = c + 1; a consumer acquires it, copies the image into shared memory with a
+// bulk copy, and releases its consumed counter = c + 1 once the copy has landed; the producer
+// acquires the head's consumers' counters >= c - RING + 1 before reusing the slot. Producer
+// items are ordered by chunk, and every producer works through its items in order, so the
+// item a consumer waits for never waits on anything later: no cycle. Every spin and mbarrier
+// wait is bounded; on timeout the status word is set and the CTA stops. The launch is
+// cooperative, so all CTAs are resident together or the launch fails.
 #include <cuda.h>
 
 #include <mutex>
@@ -36,17 +41,20 @@ using namespace sm100;
 using namespace chunk;
 
 constexpr int RING = 8;
-// Chunk image (bytes), the same in a ring slot and in a consumer stage:
-//   [0, 8K)      T' [i][j]                     \ with the zero block: [T'; 0] (K-major, 128 rows)
-//   [8K, 16K)    zero block (consumer only)     |
-//   [16K, 24K)   A [i][j]                      / with the zero block: [0; A] (K-major, 128 rows)
-//   [24K, 56K)   [-W; Q~] (K-major, 128 rows, two 64-column blocks of 16 KB: rows 0..63 = -W,
-//                rows 64..127 = Q~)
-//   [56K, 72K)   K^ [j][c] (an MN-major A operand for K^^T U)
-//   [72K, 72K + 512) gamma[128]
-constexpr uint32_t SL_T = 0, SL_Z = 8192, SL_A = 16384, SL_WQ = 24576, SL_KH = 57344;
-constexpr uint32_t SL_G = 73728, SLOT = 74752;
+// Chunk image (bytes), the same in a ring slot and in a consumer stage (bf16, 128-byte
+// swizzled tiles):
+//   [0, 32K)     M [c][c'] (K-major A operand, 128 rows, 64-column blocks of 16 KB)
+//   [32K, 48K)   K^ [j][c] (MN-major A operand of K^^T U~, blocks of 8 KB)
+//   [48K, 64K)   U~ [j][d] (MN-major B operand, blocks of 8 KB)
+//   [64K, 80K)   P [i][c] (K-major A operand, 64 rows, blocks of 8 KB)
+//   [80K, 88K)   A [i][j] (K-major A operand, 64 rows)
+constexpr uint32_t SL_M = 0, SL_KH = 32768, SL_U = 49152, SL_P = 65536, SL_A = 81920;
+constexpr uint32_t SLOT = 90112;
 static_assert(SLOT % 1024 == 0, "slot layout");
+// The ring moves with tiled TMA over a [rows][64] bf16 view (128-byte rows copied verbatim):
+// an image is SLOT_ROWS rows, loaded in RL_BOX-row boxes and stored in 8 KB pieces.
+constexpr uint32_t SLOT_ROWS = SLOT / 128, RL_BOX = 176, RS_BOX = 64;
+static_assert(SLOT_ROWS % RL_BOX == 0, "ring load boxes");
 
 struct SplitParams {
     const int32_t *cu_seqlens;
@@ -83,304 +91,278 @@ __device__ __forceinline__ bool wait_flag_ge(const int32_t *p, int target, uint6
         if (globaltimer_ns() > deadline) return false;
     }
 }
-// Bulk (untiled) copy global -> shared, completing on `bar` (16-byte aligned, size % 16 == 0).
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// Bulk (untiled) copy shared -> global, tracked by this thread's bulk async-group.
-__device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
-                 "r"(smem_u32(src)), "r"(bytes)
-                 : "memory");
-}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Waits until the committed bulk stores have finished reading shared memory / are complete.
+// Waits until the committed TMA stores have finished reading shared memory / are complete.
 __device__ __forceinline__ void bulk_wait_read() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Every split CTA runs the NT compute threads (warps 0..7) plus two control warps: lane 0 of
+// warp 8 issues the tensor-core MMAs (and, in a producer, the TMA loads and stores and the
+// hand-off flags); lane 0 of warp 9 brings a consumer its chunk images. None of their waits
+// stalls a compute warp. (Ten warps leave at most three per SM sub-partition, so they cost no
+// more registers per thread than nine.)
+constexpr int NTS = NT + 64;
+constexpr int CTL = NT;       // the MMA / control thread
+constexpr int LDR = NT + 32;  // the consumer's loader thread
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_volatile(const uint32_t *p) {
+    return *reinterpret_cast<const volatile uint32_t *>(p);
+}
 
 // ---------------------------------------------------------------- consumer (state chain)
 // CPH consumers per head, each owning DC = 128 / CPH value channels (columns of S are
 // independent: the chain of one column block never reads another's).
 template <int CPH>
 struct Cons {
-    static constexpr int DC = D / CPH;                            // value channels per consumer
-    static constexpr int NP = DC / 64;                            // 32-column parts per thread
+    static constexpr int DC = D / CPH;                  // value channels per consumer
+    static constexpr int NP = DC / 64;                  // 32-column parts per thread
     static constexpr uint32_t STAGE0 = 0, STAGE1 = SLOT;
-    static constexpr uint32_t V0 = 2 * SLOT, V1 = V0 + 128 * DC;  // V [j][d]; after batch 1, U
-    static constexpr uint32_t S = V1 + 128 * DC;                  // S [c][d] bf16 128 x DC
-    static constexpr uint32_t MISC = S + 256 * DC;                // barriers, flags
+    static constexpr uint32_t S = 2 * SLOT;             // S_b [c][d] bf16 128 x DC
+    static constexpr uint32_t MISC = S + 256 * DC;      // barriers, flags
     static constexpr uint32_t BYTES = MISC + 256;
-    // TMEM: the fp32 state (lane = key channel) and two accumulators D (rows 0..63 = U,
-    // rows 64..127 = O; lane = row), used by alternate chunks.
-    static constexpr uint32_t TM_S = 0, TM_D0 = DC, TM_D1 = 2 * DC, TM_COLS = CPH == 1 ? 512 : 256;
+    // TMEM: the fp32 state (lane = key channel, column = value channel) and two M=64 output
+    // accumulators (row i in lane i % 16 + 32 (i / 16)), used by alternate chunks.
+    static constexpr uint32_t TM_S = 0, TM_O0 = DC, TM_O1 = 2 * DC, TM_COLS = CPH == 1 ? 512 : 256;
 };
 
+// Consumer roles, per chunk c (stage b = c & 1). Loader: once chunk c - 2's MMAs have completed
+// (o[b]) and the producer has published chunk c, copy its image into stage b (full[b]); publish
+// consumption as the copies land. MMA thread: wait for the image and for the compute threads'
+// "S_b ready", then issue S += M S_b + K^^T U~ (commit s), O = P S_b (commit sr), O += A U~
+// (commit o[b]). Compute threads: the outputs of chunk c - 1 (after o), the new state into
+// registers (after s), its bf16 copy S_b (after sr), then arrive on "S_b ready". No CTA-wide
+// barrier inside the loop.
 template <int CPH>
-__device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t *sm, int cid) {
+__device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t *sm, int cid) {
     using L = Cons<CPH>;
     constexpr int DC = L::DC, NP = L::NP;
-    constexpr uint32_t STAGE0 = L::STAGE0, STAGE1 = L::STAGE1, V0 = L::V0, V1 = L::V1, S = L::S;
-    constexpr uint32_t MISC = L::MISC, TM_S = L::TM_S, TM_D0 = L::TM_D0, TM_D1 = L::TM_D1;
-    constexpr uint32_t TM_COLS = L::TM_COLS;
-    constexpr uint32_t I_D = idesc_bf16_f32(128, DC, false, 0, 1);  // [T';0]V + [-W;Q~]S, [0;A]U
-    constexpr uint32_t I_S = idesc_bf16_f32(128, DC, false, 1, 1);  // K^^T U
+    constexpr uint32_t STAGE0 = L::STAGE0, STAGE1 = L::STAGE1, S = L::S, MISC = L::MISC;
+    constexpr uint32_t TM_S = L::TM_S, TM_O0 = L::TM_O0, TM_O1 = L::TM_O1, TM_COLS = L::TM_COLS;
+    constexpr uint32_t I_C = idesc_bf16_f32(128, DC, false, 0, 1);  // M S_b
+    constexpr uint32_t I_K = idesc_bf16_f32(128, DC, false, 1, 1);  // K^^T U~
+    constexpr uint32_t I_O = idesc_bf16_f32(64, DC, false, 0, 1);   // P S_b, A U~
     const int hd = cid / CPH, sub = cid % CPH, d0 = DC * sub;  // head, first value channel
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);         // in0, in1, u, s, o
+    // full0, full1, s, sr, o0, o1, ready, teardown
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);
     uint32_t *s_flags = reinterpret_cast<uint32_t *>(sm + MISC + 64); // abort, tmem
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
+    const int quad = warp & 3, half = (warp >> 2) & 1;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
     const int H = p.H, n = hd / H, h = hd % H;
     const int c_me = 32 * quad + lane;  // TMEM lane of this thread
     const int64_t bos = p.cu_seqlens[n], eos = p.cu_seqlens[n + 1];
     const int nchunks = (int)((eos - bos + C - 1) / C);
     const size_t state_off = ((size_t)n * H + h) * (size_t)(D * D);
+    const int col0 = (DC / 2) * half;  // this thread's first column of S and O
 
     if (tid == 0) {
         s_flags[0] = 0;
-        for (int k = 0; k < 5; ++k) mbar_init(&bars[k], 1);
+        for (int k = 0; k < 8; ++k) mbar_init(&bars[k], k == 6 ? NT : 1);
         fence_mbarrier_init();
-        prefetch_tmap(tm_v);
     }
     if (warp == 0) {
         tmem_alloc(&s_flags[1], TM_COLS);
         tmem_relinquish();
     }
-    for (int e = tid; e < 8192 / 16; e += NT) {  // the zero blocks of both stages
-        reinterpret_cast<uint4 *>(sm + STAGE0 + SL_Z)[e] = make_uint4(0u, 0u, 0u, 0u);
-        reinterpret_cast<uint4 *>(sm + STAGE1 + SL_Z)[e] = make_uint4(0u, 0u, 0u, 0u);
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_flags[1];
-
-    // Flag thread (lane 31 of warp 5: not the MMA-issuing warp, and it never stores outputs, so
-    // its fences and release stores neither stall MMA issue nor wait behind output stores):
-    // brings chunk c's image and V into stage c & 1 (block: wait for the producer) and
-    // publishes what has been consumed.
-    constexpr int FT = 5 * 32 + 31;
-    int requested = 0;  // chunks requested so far (flag thread)
-    auto request = [&](int c, bool block) -> bool {
-        int32_t *fl = p.filled + hd * RING + (c % RING);
-        if (block) {
-            if (!wait_flag_ge(fl, c + 1, p.timeout_ns)) {
-                s_flags[0] = 1;
-                atomicOr(p.status, 1);
-                return false;
-            }
-        } else if (ld_acquire(fl) < c + 1) {
-            return false;
-        }
-        fence_proxy_async_global();
-        fence_proxy_async_smem();
-        const int b = c & 1;
-        uint8_t *dst = sm + (b ? STAGE1 : STAGE0);
-        const uint8_t *src = p.ring + ((size_t)hd * RING + (c % RING)) * SLOT;
-        mbar_arrive_expect_tx(&bars[b], 8192 + (SL_G + 512 - SL_A) + 128 * DC);
-        bulk_g2s(dst + SL_T, src + SL_T, 8192, &bars[b]);
-        bulk_g2s(dst + SL_A, src + SL_A, SL_G + 512 - SL_A, &bars[b]);
-        const int64_t t0 = bos + (int64_t)c * C;
-#pragma unroll
-        for (int part = 0; part < NP; ++part)
-            tma_load_3d(sm + (b ? V1 : V0) + 8192 * part, tm_v, &bars[b], d0 + 64 * part, h, (int32_t)t0);
-        requested = c + 1;
-        return true;
-    };
-    // flag thread, non-blocking: request every chunk whose stage is free (the chunk two back has
-    // finished all its MMAs: `done` chunks have) and whose image the producer has published
-    int done = 0;
-    auto poll_ahead = [&]() {
-        while (requested < nchunks && requested < done + 2)
-            if (!request(requested, false)) break;
+    auto fail = [&]() {
+        s_flags[0] = 1;
+        atomicOr(p.status, 1);
     };
 
-    // initial state -> TMEM (lane c, columns d) and its bf16 tile; empty sequences copy it out
-    {
-        const size_t row = state_off + (size_t)c_me * D + d0 + 32 * NP * half;
-        const float *src = p.s0 ? p.s0 + row : nullptr;
-        float *dst = p.sT ? p.sT + row : nullptr;
-#pragma unroll
-        for (int part = 0; part < NP; ++part) {
-            float v[32];
-#pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-                float4 f = src ? *reinterpret_cast<const float4 *>(src + 32 * part + e)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-                v[e] = f.x; v[e + 1] = f.y; v[e + 2] = f.z; v[e + 3] = f.w;
+    if (tid == LDR) {
+        // ------------------------------------------------ loader thread
+        // Chunk c goes to stage c & 1 once chunk c - 2's MMAs have completed; the consumed
+        // counter follows the copies as they land.
+        uint32_t ph_full[2] = {0, 0}, ph_o[2] = {0, 0};
+        int requested = 0, landed = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1;
+            if (ld_volatile(&s_flags[0])) break;
+            if (c >= 2) {
+                if (!mbar_wait_bounded(&bars[4 + b], ph_o[b], p.timeout_ns)) { fail(); break; }
+                ph_o[b] ^= 1u;
             }
-            if (nchunks == 0) {
-                if (dst) {
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4 *>(dst + 32 * part + e) =
-                            make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                }
-            } else {
-                const int col = 32 * NP * half + 32 * part;
-                tmem_st32(tmem + lane_base + TM_S + col, v);
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8)
-                    st_chunk(sm + S + tchunk(16384, c_me, col + 8 * q8), v + 8 * q8);
-            }
-        }
-        tmem_wait_st();
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    uint32_t ph_in[2] = {0, 0}, ph_u = 0, ph_s = 0, ph_o = 0;
-    auto wait_bar = [&](uint64_t *bar, uint32_t &ph) {
-        const bool ok = mbar_wait_bounded(bar, ph, p.timeout_ns);
-        ph ^= 1u;
-        if (!ok) {
-            s_flags[0] = 1;
-            atomicOr(p.status, 1);
-        }
-    };
-    // O of chunk cc: D rows 64..127 (lanes 64..127, quadrants 2 and 3) -> bf16 outputs
-    auto store_o = [&](int cc, uint32_t tm_d) {
-        const int64_t tc = bos + (int64_t)cc * C;
-        const int vc = (int)(eos - tc < C ? eos - tc : C);
-        const int i = c_me - 64;
-        float v[32];
-#pragma unroll
-        for (int part = 0; part < NP; ++part) {
-            const int col = 32 * NP * half + 32 * part;
-            tmem_ld32(tmem + lane_base + tm_d + col, v);
-            tmem_wait_ld();
-            if (i < vc) {
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(tc + i) * H + h) * D + d0 + col);
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8)
-                    dst[q8] = make_uint4(pack2(v[8 * q8], v[8 * q8 + 1]), pack2(v[8 * q8 + 2], v[8 * q8 + 3]),
-                                         pack2(v[8 * q8 + 4], v[8 * q8 + 5]), pack2(v[8 * q8 + 6], v[8 * q8 + 7]));
-            }
-        }
-    };
-
-    for (int c = 0; c < nchunks; ++c) {
-        const int b = c & 1;
-        const bool has_next = c + 1 < nchunks;
-        const uint32_t tm_d = b ? TM_D1 : TM_D0;
-        if (tid == FT && requested <= c) request(c, true);
-        __syncthreads();
-        if (s_flags[0]) break;
-        wait_bar(&bars[b], ph_in[b]);
-        uint8_t *stage = sm + (b ? STAGE1 : STAGE0);
-        const uint32_t st_base = sb + (b ? STAGE1 : STAGE0);
-        const uint32_t vb = sb + (b ? V1 : V0);
-        if (tid == FT) {
+            if (!wait_flag_ge(p.filled + hd * RING + (c % RING), c + 1, p.timeout_ns)) { fail(); break; }
             fence_proxy_async_global();
-            st_release(p.consumed + 2 * hd + sub, c + 1);  // the image is in shared memory: slot reusable
-            done = c;  // every MMA of chunk c - 1 was waited on at the end of its iteration
-            poll_ahead();  // usually chunk c + 1 into the other stage: a whole chunk to land
+            const int32_t row0 = (int32_t)(((uint32_t)hd * RING + (uint32_t)(c % RING)) * SLOT_ROWS);
+            uint8_t *dst = sm + (b ? STAGE1 : STAGE0);
+            mbar_arrive_expect_tx(&bars[b], SLOT);
+#pragma unroll
+            for (uint32_t k = 0; k < SLOT_ROWS / RL_BOX; ++k)
+                tma_load_2d(dst + k * RL_BOX * 128, tm_rl, &bars[b], 0, row0 + (int32_t)(k * RL_BOX));
+            requested = c + 1;
+            if (c >= 1) {  // chunk c - 1's image is in shared memory: its slot may be refilled
+                if (!mbar_wait_bounded(&bars[b ^ 1], ph_full[b ^ 1], p.timeout_ns)) { fail(); break; }
+                ph_full[b ^ 1] ^= 1u;
+                landed = c;
+                fence_proxy_async_global();
+                st_release(p.consumed + 2 * hd + sub, c);
+            }
         }
-        const float *gam = reinterpret_cast<const float *>(stage + SL_G);
-
-        if (tid == 0) {
+        for (int c = landed; c < requested; ++c) {  // the copies still in flight land
+            if (!mbar_wait_bounded(&bars[c & 1], ph_full[c & 1], p.timeout_ns)) { fail(); break; }
+            ph_full[c & 1] ^= 1u;
+            fence_proxy_async_global();
+            st_release(p.consumed + 2 * hd + sub, c + 1);
+        }
+    } else if (tid == CTL) {
+        // ------------------------------------------------ MMA thread
+        uint32_t ph_full[2] = {0, 0}, ph_ready = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1;
+            if (ld_volatile(&s_flags[0])) break;
+            if (!mbar_wait_bounded(&bars[b], ph_full[b], p.timeout_ns)) { fail(); break; }
+            ph_full[b] ^= 1u;
+            if (!mbar_wait_bounded(&bars[6], ph_ready, p.timeout_ns)) { fail(); break; }
+            ph_ready ^= 1u;
             tc_fence_after();
-            const uint64_t dTZ = desc_k(st_base + SL_T, 16384, 0), dWQ = desc_k(st_base + SL_WQ, 16384, 0);
-            const uint64_t dV = desc_mn(vb, 8192, 0), dS = desc_mn(sb + S, 16384, 0);  // one N block
+            const uint32_t st = sb + (b ? STAGE1 : STAGE0);
+            const uint32_t tm_o = b ? TM_O1 : TM_O0;
+            const uint64_t dM = desc_k(st + SL_M, 16384, 0), dS = desc_mn(sb + S, 16384, 0);
+            const uint64_t dK = desc_mn(st + SL_KH, 8192, 0);
+            const uint64_t dU = desc_mn(st + SL_U + 8192 * (d0 / 64), 8192, 0);
+            const uint64_t dP = desc_k(st + SL_P, 8192, 0), dA = desc_k(st + SL_A, 8192, 0);
 #pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)  // [U; O] = [T'; 0] V ...
-                mma_bf16_ss(tmem + tm_d, desc_k_at(dTZ, 16384, kk), desc_mn_at(dV, kk), I_D, kk > 0);
+            for (uint32_t kk = 0; kk < 8; ++kk)  // S += M S_b ...
+                mma_bf16_ss(tmem + TM_S, desc_k_at(dM, 16384, kk), desc_mn_at(dS, kk), I_C, 1);
 #pragma unroll
-            for (uint32_t kk = 0; kk < 8; ++kk)  // ... + [-W; Q~] S
-                mma_bf16_ss(tmem + tm_d, desc_k_at(dWQ, 16384, kk), desc_mn_at(dS, kk), I_D, 1);
+            for (uint32_t kk = 0; kk < 4; ++kk)  // ... + K^^T U~
+                mma_bf16_ss(tmem + TM_S, desc_mn_at(dK, kk), desc_mn_at(dU, kk), I_K, 1);
             mma_commit(&bars[2]);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 8; ++kk)  // O = P S_b ...
+                mma_bf16_ss(tmem + tm_o, desc_k_at(dP, 8192, kk), desc_mn_at(dS, kk), I_O, kk > 0);
+            mma_commit(&bars[3]);                // S_b has been read
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)  // ... + A U~
+                mma_bf16_ss(tmem + tm_o, desc_k_at(dA, 8192, kk), desc_mn_at(dU, kk), I_O, 1);
+            mma_commit(&bars[4 + b]);            // O and the stage are done
         }
-        // While the batch runs (it reads only shared memory and writes D): S <- diag(gamma) S in
-        // TMEM ahead of S += K^^T U (warp 4 takes warp 0's columns: warp 0 issues the MMAs), and
-        // (rows 64..127) the previous chunk's outputs.
-        if (warp == 4)
-            scale_tmem_row<DC>(tmem + lane_base + TM_S, gam[c_me]);
-        else if (warp != 0)
-            scale_tmem_row<DC / 2>(tmem + lane_base + TM_S + (DC / 2) * half, gam[c_me]);
-        if (c > 0 && quad >= 2) store_o(c - 1, b ? TM_D0 : TM_D1);
-        wait_bar(&bars[2], ph_u);
-        tc_fence_after();
-
-        // U (D rows 0..63) -> bf16 [j][d] into this stage's V buffer (V is consumed)
-        if (quad < 2) {
+        // teardown: every issued MMA completes before TMEM is freed
+        mma_commit(&bars[7]);
+        mbar_wait_bounded(&bars[7], 0, p.timeout_ns);
+    } else if (tid < NT) {
+        // ------------------------------------------------ compute threads
+        // initial state -> TMEM (lane c, columns d) and S_b; empty sequences copy it out
+        {
+            const size_t row = state_off + (size_t)c_me * D + d0 + col0;
+            const float *src = p.s0 ? p.s0 + row : nullptr;
+            float *dst = p.sT ? p.sT + row : nullptr;
 #pragma unroll
             for (int part = 0; part < NP; ++part) {
-                const int col = 32 * NP * half + 32 * part;
                 float v[32];
-                tmem_ld32(tmem + lane_base + tm_d + col, v);
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    float4 f = src ? *reinterpret_cast<const float4 *>(src + 32 * part + e)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[e] = f.x; v[e + 1] = f.y; v[e + 2] = f.z; v[e + 3] = f.w;
+                }
+                if (nchunks == 0) {
+                    if (dst) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4)
+                            *reinterpret_cast<float4 *>(dst + 32 * part + e) =
+                                make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                    }
+                } else {
+                    const int col = col0 + 32 * part;
+                    tmem_st32(tmem + lane_base + TM_S + col, v);
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8)
+                        st_chunk(sm + S + tchunk(16384, c_me, col + 8 * q8), v + 8 * q8);
+                }
+            }
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bars[6]);  // S_b ready for chunk 0
+
+        uint32_t ph_s = 0, ph_sr = 0, ph_o[2] = {0, 0};
+        auto wait_bar = [&](uint64_t *bar, uint32_t &ph) -> bool {
+            const bool ok = mbar_wait_bounded(bar, ph, p.timeout_ns);
+            ph ^= 1u;
+            if (!ok) fail();
+            return ok;
+        };
+        // O of chunk cc (M=64 accumulator at tm_o) -> bf16 outputs; rows in lanes 0..15 of each
+        // quadrant
+        auto store_o = [&](int cc, uint32_t tm_o) {
+            const int64_t tc = bos + (int64_t)cc * C;
+            const int vc = (int)(eos - tc < C ? eos - tc : C);
+            const int i = 16 * quad + lane;
+#pragma unroll
+            for (int part = 0; part < NP; ++part) {
+                const int col = col0 + 32 * part;
+                float v[32];
+                tmem_ld32(tmem + lane_base + tm_o + col, v);
                 tmem_wait_ld();
+                if (lane < 16 && i < vc) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(tc + i) * H + h) * D + d0 + col);
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8)
+                        dst[q8] = make_uint4(pack2(v[8 * q8], v[8 * q8 + 1]), pack2(v[8 * q8 + 2], v[8 * q8 + 3]),
+                                             pack2(v[8 * q8 + 4], v[8 * q8 + 5]), pack2(v[8 * q8 + 6], v[8 * q8 + 7]));
+                }
+            }
+        };
+
+        int c = 0;
+        for (; c < nchunks; ++c) {
+            const int b = c & 1;
+            if (ld_volatile(&s_flags[0])) break;
+            if (c > 0) {  // the previous chunk's outputs while this chunk's batch runs
+                if (!wait_bar(&bars[4 + (b ^ 1)], ph_o[b ^ 1])) break;
+                tc_fence_after();
+                store_o(c - 1, b ? TM_O0 : TM_O1);
+            }
+            // the new state -> registers (and the final state after the last chunk)
+            if (!wait_bar(&bars[2], ph_s)) break;
+            tc_fence_after();
+            float v[NP][32];
+#pragma unroll
+            for (int part = 0; part < NP; ++part) tmem_ld32(tmem + lane_base + TM_S + col0 + 32 * part, v[part]);
+            tmem_wait_ld();
+            if (c + 1 == nchunks && p.sT) {
+#pragma unroll
+                for (int part = 0; part < NP; ++part) {
+                    float *dst = p.sT + state_off + (size_t)c_me * D + d0 + col0 + 32 * part;
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4 *>(dst + e) =
+                            make_float4(v[part][e], v[part][e + 1], v[part][e + 2], v[part][e + 3]);
+                }
+            }
+            // its bf16 copy, once P S_b has read the old one
+            if (!wait_bar(&bars[3], ph_sr)) break;
+#pragma unroll
+            for (int part = 0; part < NP; ++part)
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8)
-                    st_chunk(sm + (b ? V1 : V0) + tchunk(8192, c_me, col + 8 * q8), v + 8 * q8);
+                    st_chunk(sm + S + tchunk(16384, c_me, col0 + 32 * part + 8 * q8), v[part] + 8 * q8);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[6]);  // S_b ready for chunk c + 1
+        }
+        if (c == nchunks && nchunks > 0) {  // outputs of the last chunk
+            const int bl = (nchunks - 1) & 1;
+            if (wait_bar(&bars[4 + bl], ph_o[bl])) {
+                tc_fence_after();
+                store_o(nchunks - 1, bl ? TM_O1 : TM_O0);
             }
         }
-        fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
-        if (s_flags[0]) break;
-
-        if (tid == 0) {
-            tc_fence_after();
-            const uint64_t dK = desc_mn(st_base + SL_KH, 8192, 0), dU = desc_mn(vb, 8192, 0);
-            const uint64_t dAZ = desc_k(st_base + SL_Z, 16384, 0);
-#pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)  // S += K^^T U   (S already scaled by gamma)
-                mma_bf16_ss(tmem + TM_S, desc_mn_at(dK, kk), desc_mn_at(dU, kk), I_S, 1);
-            mma_commit(&bars[3]);
-#pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)  // [U; O] += [0; A] U
-                mma_bf16_ss(tmem + tm_d, desc_k_at(dAZ, 16384, kk), desc_mn_at(dU, kk), I_D, 1);
-            mma_commit(&bars[4]);
-        }
-        wait_bar(&bars[3], ph_s);
-        tc_fence_after();
-
-        // the next state's bf16 tile (and the final state after the last chunk)
-#pragma unroll
-        for (int part = 0; part < NP; ++part) {
-            const int col = 32 * NP * half + 32 * part;
-            float v[32];
-            tmem_ld32(tmem + lane_base + TM_S + col, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8)
-                st_chunk(sm + S + tchunk(16384, c_me, col + 8 * q8), v + 8 * q8);
-            if (!has_next && p.sT) {
-                float *dst = p.sT + state_off + (size_t)c_me * D + d0 + col;
-#pragma unroll
-                for (int e = 0; e < 32; e += 4)
-                    *reinterpret_cast<float4 *>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-            }
-        }
-        // this chunk's last MMA ([0; A] U): after it, its stage may take chunk c + 2
-        wait_bar(&bars[4], ph_o);
-        tc_fence_after();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
     }
-    if (nchunks > 0 && !s_flags[0] && quad >= 2)  // outputs of the last chunk
-        store_o(nchunks - 1, ((nchunks - 1) & 1) ? TM_D1 : TM_D0);
-
-    // teardown: let requested copies and issued MMAs land before freeing TMEM
-    if (s_flags[0] && tid == FT) {
-        for (int c = 0; c < 2; ++c)
-            if (requested > c) mbar_wait_bounded(&bars[c], ph_in[c], p.timeout_ns);
-    }
-    if (s_flags[0] && tid == 0) {
-        mma_commit(&bars[2]);
-        mbar_wait_bounded(&bars[2], ph_u, p.timeout_ns);
-    }
-    tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
@@ -390,40 +372,50 @@ __device__ void consumer(const CUtensorMap *tm_v, const SplitParams &p, uint8_t 
 
 // ---------------------------------------------------------------- producer (key-side half)
 namespace prod {
-constexpr uint32_t QK0 = 0, QK1 = 32768;       // raw q/k -> Q~/K~ (128-row tiles, 16 KB blocks)
-constexpr uint32_t LA0 = 65536, LA1 = 98304;   // raw log_alpha fp32
-constexpr uint32_t KI = 131072;                // K- / K^ [j][c] 64 x 128
-constexpr uint32_t W = KI + 16384;             // W [i][c] 64 x 128
-constexpr uint32_t AQK = W + 16384;            // A [i][j]
-constexpr uint32_t TT = AQK + 8192;            // T' [i][j]
-constexpr uint32_t LT = TT + 8192;             // L -> T fp32 [64][LT_LD]
+constexpr uint32_t QK0 = 0, QK1 = 32768;  // raw q/k -> Q~/K~ -> P over Q~ (128-row tiles, 16 KB blocks)
+constexpr uint32_t LA = 65536;            // raw log_alpha fp32 [t][c]
+constexpr uint32_t VB = LA + 32768;       // V [j][d] -> U~
+constexpr uint32_t KI = VB + 16384;       // K- [j][c]; with WN after it: M [c][c'] (2 x 16 KB)
+constexpr uint32_t WN = KI + 16384;       // -W [j][c]
+constexpr uint32_t KH = WN + 16384;       // K^ [j][c]
+constexpr uint32_t TT = KH + 16384;       // T' [i][j]   \  [T'; 0] and [0; A]: 128-row
+constexpr uint32_t ZB = TT + 8192;        // zero block   |  K-major operands
+constexpr uint32_t AQK = ZB + 8192;       // A [i][j]    /
+constexpr uint32_t LT = AQK + 8192;       // L -> T fp32 [64][LT_LD]
 constexpr uint32_t PB = LT + 64 * LT_LD * 4;   // 32 x PB_LD fp32
 constexpr uint32_t MISC = PB + 32 * PB_LD * 4; // beta, gamma, psum, flags, barriers
-constexpr uint32_t KH = (MISC + 64 * 4 + 128 * 4 + 4 * 128 * 4 + 64 + 64 + 1023) / 1024 * 1024;  // K^ [j][c]
-constexpr uint32_t BYTES = KH + 16384;
-constexpr uint32_t TM_D1 = 0, TM_W = 128, TM_COLS = 256;
+constexpr uint32_t BYTES = MISC + 64 * 4 + 128 * 4 + 4 * 128 * 4 + 64 + 64;
+// TMEM: D1 = [Q~; K~] K-^T (M=128, 64 columns), W (M=64), D3 = [U~; -A W], D4 = -K^^T W
+constexpr uint32_t TM_D1 = 0, TM_W = 128, TM_D3 = 256, TM_D4 = 384, TM_COLS = 512;
 }  // namespace prod
 
-__device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_la,
-                         const SplitParams &p, uint8_t *sm, int pid, int nprod) {
+// Producer roles: the compute threads run the gating, the TMEM epilogues and the inverse; the
+// control thread issues the TMA loads, the MMAs and the image's bulk stores, waits for a free
+// ring slot and publishes the image. The phases of one item are separated by CTA barriers.
+__device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
+                         const CUtensorMap *tm_la, const CUtensorMap *tm_rs, const SplitParams &p,
+                         uint8_t *sm, int pid, int nprod) {
     using namespace prod;
     constexpr uint32_t I_D1 = idesc_bf16_f32(128, 64);
     constexpr uint32_t I_W = idesc_bf16_f32(64, 128, false, 0, 1);
+    constexpr uint32_t I_3 = idesc_bf16_f32(128, 128, false, 0, 1);
+    constexpr uint32_t I_4 = idesc_bf16_f32(128, 128, false, 1, 1);
     float *s_beta = reinterpret_cast<float *>(sm + MISC);
     float *s_gamma = s_beta + 64;
     float *s_psum = s_gamma + 128;
-    uint32_t *s_flags = reinterpret_cast<uint32_t *>(s_psum + 512);  // abort, tmem
-    uint64_t *bars = reinterpret_cast<uint64_t *>(s_flags + 16);     // in0, in1, mma
+    uint32_t *s_flags = reinterpret_cast<uint32_t *>(s_psum + 512);  // abort, tmem, gate
+    uint64_t *bars = reinterpret_cast<uint64_t *>(s_flags + 16);     // qk0, qk1, la, v, mma, src
     float *LTp = reinterpret_cast<float *>(sm + LT);
     float *PBp = reinterpret_cast<float *>(sm + PB);
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
+    const int quad = warp & 3, half = (warp >> 2) & 1;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+    const bool compute = tid < NT, ctl = tid == CTL;
     const int H = p.H;
     // Static assignment: producer pid serves head hd = pid % heads, making chunks j, j + cnt, ...
     // (j = pid / heads, cnt = number of producers of that head), so it only ever waits on its
-    // own head's consumer.
+    // own head's consumers.
     const int hd = pid % p.heads, pj = pid / p.heads;
     const int pcnt = (nprod - 1 - hd) / p.heads + 1;
     const int h = hd % H;
@@ -432,46 +424,61 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 
     if (tid == 0) {
         s_flags[0] = 0;
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
-        mbar_init(&bars[2], 1);
+        for (int k = 0; k < 6; ++k) mbar_init(&bars[k], 1);
         fence_mbarrier_init();
         prefetch_tmap(tm_q);
         prefetch_tmap(tm_k);
+        prefetch_tmap(tm_v);
         prefetch_tmap(tm_la);
+        prefetch_tmap(tm_rs);
     }
     if (warp == 0) {
         tmem_alloc(&s_flags[1], TM_COLS);
         tmem_relinquish();
     }
-    for (int e = tid; e < 8192 / 16; e += NT)  // strictly upper 16x16 blocks of T' stay zero
+    for (int e = tid; e < 16384 / 16; e += NTS)  // T' (its strictly upper 16x16 blocks) and ZB stay zero
         reinterpret_cast<uint4 *>(sm + TT)[e] = make_uint4(0u, 0u, 0u, 0u);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_flags[1];
+    auto fail = [&]() {
+        s_flags[0] = 1;
+        atomicOr(p.status, 1);
+    };
 
-    auto issue_inputs = [&](int c, int b) {  // thread 0
+    // control thread; each buffer's previous contents were read by generic loads or bulk stores
+    // that have completed (see the call sites)
+    auto issue_qk = [&](int c, int b) {
         const int64_t t0 = bos + (int64_t)c * C;
         uint8_t *qk = sm + (b ? QK1 : QK0);
-        fence_proxy_async_smem();  // the stage's previous contents were read by generic loads
-        mbar_arrive_expect_tx(&bars[b], 32768 + 32768);
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&bars[b], 32768);
         tma_load_3d(qk, tm_q, &bars[b], 0, h, (int32_t)t0);
         tma_load_3d(qk + 8192, tm_k, &bars[b], 0, h, (int32_t)t0);
         tma_load_3d(qk + 16384, tm_q, &bars[b], 64, h, (int32_t)t0);
         tma_load_3d(qk + 24576, tm_k, &bars[b], 64, h, (int32_t)t0);
-        tma_load_3d(sm + (b ? LA1 : LA0), tm_la, &bars[b], 0, h, (int32_t)t0);
+    };
+    auto issue_la = [&](int c) {
+        const int64_t t0 = bos + (int64_t)c * C;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&bars[2], 32768);
+        tma_load_3d(sm + LA, tm_la, &bars[2], 0, h, (int32_t)t0);
+    };
+    auto issue_v = [&](int c) {
+        const int64_t t0 = bos + (int64_t)c * C;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&bars[3], 16384);
+        tma_load_3d(sm + VB, tm_v, &bars[3], 0, h, (int32_t)t0);
+        tma_load_3d(sm + VB + 8192, tm_v, &bars[3], 64, h, (int32_t)t0);
     };
     auto load_beta = [&](int c) -> float {  // tid < C
         const int64_t t0 = bos + (int64_t)c * C;
         if (c >= nch || t0 + tid >= eos) return 0.f;
         return p.beta[(size_t)(t0 + tid) * H + h];
     };
-    // Bulk-store thread (lane 31 of warp 7: not the MMA-issuing thread; warp 7 idles during the
-    // first stage of the inverse, where the publish goes): issues an image's bulk stores, waits
-    // for them to have read shared memory before the next item rewrites it (just before its
-    // gating), and publishes the slot once they are complete (during the next item's inverse).
-    constexpr int BT = NT - 1;
+    // the previous image, published once its bulk stores are complete (control thread, during
+    // the next item's gating)
     int32_t *rel_flag = nullptr;
     int rel_val = 0;
     auto release = [&]() {
@@ -484,21 +491,21 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         }
     };
 
-    uint32_t ph_in[2] = {0, 0}, ph_mma = 0;
-    bool pending[2] = {false, false};
+    uint32_t ph_qk[2] = {0, 0}, ph_la = 0, ph_v = 0, ph_mma = 0, ph_src = 0;
+    bool pend_qk[2] = {false, false}, pend_la = false, pend_v = false;
     auto wait_bar = [&](uint64_t *bar, uint32_t &ph) {
         const bool ok = mbar_wait_bounded(bar, ph, p.timeout_ns);
         ph ^= 1u;
-        if (!ok) {
-            s_flags[0] = 1;
-            atomicOr(p.status, 1);
-        }
+        if (!ok) fail();
     };
 
     int item = pj;  // chunk index
     if (item < nch) {
-        if (tid == 0) issue_inputs(item, 0);
-        pending[0] = true;
+        if (ctl) {
+            issue_qk(item, 0);
+            issue_la(item);
+        }
+        pend_qk[0] = pend_la = true;
     }
     float beta_next = (tid < C) ? load_beta(item) : 0.f;
     int b = 0;
@@ -507,29 +514,38 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         const int64_t t0 = bos + (int64_t)c * C;
         const int valid = (int)(eos - t0 < C ? eos - t0 : C);
         const int nxt = item + pcnt;
+        uint8_t *qk = sm + (b ? QK1 : QK0);
         if (tid < C) s_beta[tid] = beta_next;
-        wait_bar(&bars[b], ph_in[b]);
-        pending[b] = false;
+        if (ctl) {  // the previous image's sources (K-, K^, A, ...) are rewritten by the gating
+            bulk_wait_read();
+            mbar_arrive(&bars[5]);
+        }
+        wait_bar(&bars[b], ph_qk[b]);
+        wait_bar(&bars[2], ph_la);
+        pend_qk[b] = pend_la = false;
 
         if (tid < C) beta_next = load_beta(nxt);
-        uint8_t *qk = sm + (b ? QK1 : QK0);
-        float *la = reinterpret_cast<float *>(sm + (b ? LA1 : LA0));
-
-        if (tid == BT) bulk_wait_read();  // the previous image's sources are rewritten below
-        const int gate = gate_chunk(qk, sm + KI, sm + AQK, la, LTp, s_beta, s_gamma, s_psum,
-                                    s_flags, valid, tid, sm + KH);
-        // The next item's inputs go to the other stage, whose Q~ the previous image's bulk
-        // stores read: gate_chunk's barriers come after the bulk-store thread's read wait.
-        if (nxt < nch && gate >= 0) {
-            if (tid == 0) issue_inputs(nxt, b ^ 1);
-            pending[b ^ 1] = true;
+        if (ctl) release();  // the previous item's image, while the compute threads gate
+        if (compute) {
+            const int gate = gate_chunk(qk, sm + KI, sm + AQK, reinterpret_cast<float *>(sm + LA), LTp,
+                                        s_beta, s_gamma, s_psum, s_flags, valid, tid, sm + KH,
+                                        &bars[5], ph_src, p.timeout_ns);
+            if (gate < 0) atomicOr(p.status, 1);
+            if (tid == 0) s_flags[2] = (uint32_t)(gate + 1);
+            fence_proxy_async_smem();
         }
-        if (gate < 0) break;
+        ph_src ^= 1u;
+        const bool stop = __syncthreads_or(ld_volatile(&s_flags[0]) != 0) != 0;
+        const int gate = (int)s_flags[2] - 1;
+        if (gate < 0 || stop) break;
         const bool safe = gate == 1;
-        fence_proxy_async_smem();
-        __syncthreads();
-
-        if (tid == 0) {
+        if (ctl) {
+            // V of this chunk; q/k and log_alpha of the next one (the gating is done with them)
+            issue_v(c);
+            if (nxt < nch) {
+                issue_qk(nxt, b ^ 1);
+                issue_la(nxt);
+            }
             tc_fence_after();
             if (!safe) {
 #pragma unroll
@@ -537,72 +553,142 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                     mma_bf16_ss(tmem + TM_D1, desc_k(smem_u32(qk), 16384, kk),
                                 desc_k(sb + KI, 8192, kk), I_D1, kk > 0);
             }
-            mma_commit(&bars[2]);
+            mma_commit(&bars[4]);
         }
-        wait_bar(&bars[2], ph_mma);
+        pend_v = true;
+        if (nxt < nch) pend_qk[b ^ 1] = pend_la = true;
+        wait_bar(&bars[4], ph_mma);
         tc_fence_after();
-        if (!safe) extract_al(tmem + lane_base + TM_D1 + 32 * half, sm + AQK, LTp, s_beta, 32 * quad + lane, half);
+        if (compute && !safe) extract_al(tmem + lane_base + TM_D1 + 32 * half, sm + AQK, LTp, s_beta, 32 * quad + lane, half);
         tc_fence_before();
-        __syncthreads();
-        if (s_flags[0]) break;
+        if (__syncthreads_or(ld_volatile(&s_flags[0]) != 0)) break;
 
-        if (tid == BT) release();  // the previous item's image (warp 7 idles in the inverse's stage 1)
-        invert_unit_lower(LTp, PBp, sm + TT, s_beta, tid);
-        fence_proxy_async_smem();
+        if (compute) {
+            invert_unit_lower(LTp, PBp, sm + TT, s_beta, tid);
+            fence_proxy_async_smem();
+        }
         __syncthreads();
 
-        if (tid == 0) {
+        if (ctl) {
             tc_fence_after();
 #pragma unroll
             for (uint32_t kk = 0; kk < 4; ++kk)  // W = T' K~
                 mma_bf16_ss(tmem + TM_W, desc_k(sb + TT, 8192, kk),
                             desc_mn(smem_u32(qk) + 8192, 16384, kk), I_W, kk > 0);
-            mma_commit(&bars[2]);
+            mma_commit(&bars[4]);
         }
-        wait_bar(&bars[2], ph_mma);
+        wait_bar(&bars[4], ph_mma);
         tc_fence_after();
-        rows64_to_tile<64>(tmem + lane_base + TM_W + 64 * half, sm + W, 8192, 64 * half, quad, lane, -1.f);
-        if (tid == BT && c >= RING) {  // the slot's previous chunk must have been taken
-            if (!wait_flag_ge(p.consumed + 2 * hd, c - RING + 1, p.timeout_ns) ||
-                (p.cph == 2 && !wait_flag_ge(p.consumed + 2 * hd + 1, c - RING + 1, p.timeout_ns))) {
-                s_flags[0] = 1;
-                atomicOr(p.status, 1);
-            }
+        if (compute) {
+            rows64_to_tile<64>(tmem + lane_base + TM_W + 64 * half, sm + WN, 8192, 64 * half, quad, lane, -1.f);
+            fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();  // A, K^, W were written by generic stores; the copy-out is async
         tc_fence_before();
         __syncthreads();
-        if (s_flags[0]) break;
+
+        // D3 = [T'; 0] V + [0; A] (-W) = [U~; -A W] and D4 = K^^T (-W)
+        if (ctl) {
+            if (!mbar_wait_bounded(&bars[3], ph_v, p.timeout_ns)) fail();
+            tc_fence_after();
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tmem + TM_D3, desc_k(sb + TT, 16384, kk), desc_mn(sb + VB, 8192, kk), I_3, kk > 0);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tmem + TM_D3, desc_k(sb + ZB, 16384, kk), desc_mn(sb + WN, 8192, kk), I_3, 1);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tmem + TM_D4, desc_mn(sb + KH, 8192, kk), desc_mn(sb + WN, 8192, kk), I_4, kk > 0);
+            mma_commit(&bars[4]);
+        }
+        ph_v ^= 1u;
+        pend_v = false;
+        wait_bar(&bars[4], ph_mma);
+        tc_fence_after();
+        if (compute) {
+            const int r = 32 * quad + lane;  // TMEM lane
+            // D3 rows 0..63: U~ [j][d] over V; rows 64..127: P = Q~ - A W over Q~
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int col = 64 * half + 32 * part;
+                float v[32];
+                tmem_ld32(tmem + lane_base + TM_D3 + col, v);
+                tmem_wait_ld();
+                if (r < 64) {
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8)
+                        st_chunk(sm + VB + tchunk(8192, r, col + 8 * q8), v + 8 * q8);
+                } else {
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        uint8_t *qp = qk + tchunk(16384, r - 64, col + 8 * q8);
+                        const uint4 raw = *reinterpret_cast<const uint4 *>(qp);
+                        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
+                            v[8 * q8 + 2 * e] += f.x;
+                            v[8 * q8 + 2 * e + 1] += f.y;
+                        }
+                        st_chunk(qp, v + 8 * q8);
+                    }
+                }
+            }
+            // D4 -> M = diag(gamma - 1) - K^^T W [c][c'] over K- and -W
+            const float gm1 = s_gamma[r] - 1.f;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int col = 64 * half + 32 * part;
+                float v[32];
+                tmem_ld32(tmem + lane_base + TM_D4 + col, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    if (col + e == r) v[e] += gm1;
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8)
+                    st_chunk(sm + KI + tchunk(16384, r, col + 8 * q8), v + 8 * q8);
+            }
+            fence_proxy_async_smem();  // written by generic stores; the copy-out is async
+        }
+        if (ctl && c >= RING) {  // the slot's previous chunk must have been taken
+            if (!wait_flag_ge(p.consumed + 2 * hd, c - RING + 1, p.timeout_ns) ||
+                (p.cph == 2 && !wait_flag_ge(p.consumed + 2 * hd + 1, c - RING + 1, p.timeout_ns)))
+                fail();
+        }
+        tc_fence_before();
+        if (__syncthreads_or(ld_volatile(&s_flags[0]) != 0)) break;
 
         // copy the image out with bulk stores (layout at the top of this file); published at the
         // next item (see release)
-        if (tid == BT) {
-            uint8_t *slot = p.ring + ((size_t)hd * RING + (c % RING)) * SLOT;
-            fence_proxy_async_smem();
-            bulk_s2g(slot + SL_T, sm + TT, 8192);
-            bulk_s2g(slot + SL_A, sm + AQK, 8192);
-            bulk_s2g(slot + SL_WQ, sm + W, 8192);                  // -W, columns 0..63
-            bulk_s2g(slot + SL_WQ + 8192, qk, 8192);               // Q~, columns 0..63
-            bulk_s2g(slot + SL_WQ + 16384, sm + W + 8192, 8192);   // -W, columns 64..127
-            bulk_s2g(slot + SL_WQ + 24576, qk + 16384, 8192);      // Q~, columns 64..127
-            bulk_s2g(slot + SL_KH, sm + KH, 16384);
-            bulk_s2g(slot + SL_G, s_gamma, 512);
+        if (ctl) {
+            const int32_t row0 = (int32_t)(((uint32_t)hd * RING + (uint32_t)(c % RING)) * SLOT_ROWS);
+            // 8 KB pieces (RS_BOX rows): source, image offset
+            const uint8_t *src[11] = {sm + KI, sm + KI + 8192, sm + KI + 16384, sm + KI + 24576,
+                                      sm + KH, sm + KH + 8192, sm + VB, sm + VB + 8192,
+                                      qk, qk + 16384,  // P, columns 0..63 and 64..127
+                                      sm + AQK};
+            const uint32_t off[11] = {SL_M, SL_M + 8192, SL_M + 16384, SL_M + 24576, SL_KH, SL_KH + 8192,
+                                      SL_U, SL_U + 8192, SL_P, SL_P + 8192, SL_A};
+#pragma unroll
+            for (int k = 0; k < 11; ++k) tma_store_2d(tm_rs, src[k], 0, row0 + (int32_t)(off[k] / 128));
             bulk_commit();
             rel_flag = p.filled + hd * RING + (c % RING);
             rel_val = c + 1;
         }
-        __syncthreads();
         item = nxt;
         b ^= 1;
     }
 
-    if (tid == BT && !s_flags[0]) release();
-    if (s_flags[0] && tid == BT) bulk_wait_all();
-    if (s_flags[0] && tid == 0) {
+    if (ctl) {
+        if (!s_flags[0]) release();
+        bulk_wait_all();
         for (int k = 0; k < 2; ++k)
-            if (pending[k]) mbar_wait_bounded(&bars[k], ph_in[k], p.timeout_ns);
-        mma_commit(&bars[2]);
-        mbar_wait_bounded(&bars[2], ph_mma, p.timeout_ns);
+            if (pend_qk[k]) mbar_wait_bounded(&bars[k], ph_qk[k], p.timeout_ns);
+        if (pend_la) mbar_wait_bounded(&bars[2], ph_la, p.timeout_ns);
+        if (pend_v) mbar_wait_bounded(&bars[3], ph_v, p.timeout_ns);
+        mma_commit(&bars[4]);
+        mbar_wait_bounded(&bars[4], ph_mma, p.timeout_ns);
     }
     tc_fence_before();
     __syncthreads();
@@ -618,17 +704,19 @@ constexpr uint32_t max3(uint32_t a, uint32_t b, uint32_t c) {
 constexpr uint32_t SPLIT_SMEM = max3(Cons<1>::BYTES, Cons<2>::BYTES, prod::BYTES) + 1024;
 
 template <int CPH>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NTS, 1)
 split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
+             const __grid_constant__ CUtensorMap tm_rl, const __grid_constant__ CUtensorMap tm_rs,
              const SplitParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
     if ((int)blockIdx.x < CPH * p.heads)
-        consumer<CPH>(&tm_v, p, sm, blockIdx.x);
+        consumer<CPH>(&tm_rl, p, sm, blockIdx.x);
     else
-        producer(&tm_q, &tm_k, &tm_la, p, sm, blockIdx.x - CPH * p.heads, gridDim.x - CPH * p.heads);
+        producer(&tm_q, &tm_k, &tm_v, &tm_la, &tm_rs, p, sm, blockIdx.x - CPH * p.heads,
+                 gridDim.x - CPH * p.heads);
 }
 
 // Zeroes the status word and the ring flags.
@@ -678,12 +766,12 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
                                             (int)SPLIT_SMEM);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, NT, SPLIT_SMEM);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, NTS, SPLIT_SMEM);
     if (e != cudaSuccess) return e;
     const int grid = per_sm * sms;
     if (per_sm < 1 || grid < (cph + 1) * heads) return cudaErrorInvalidConfiguration;
 
-    CUtensorMap mq, mk, mv, mla;
+    CUtensorMap mq, mk, mv, mla, mrl, mrs;
     const uint64_t T = (uint64_t)p.total_tokens, H = (uint64_t)p.H;
     if (!make_token_map(&mq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, H, T, 64, true) ||
         !make_token_map(&mk, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, H, T, 64, true) ||
@@ -692,6 +780,10 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
         return cudaErrorInvalidValue;
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint8_t *ring = ws + 1024 + flags_bytes(heads);
+    const uint64_t ring_rows = (uint64_t)heads * RING * SLOT_ROWS;
+    if (!make_rows_map(&mrl, ring, ring_rows, RL_BOX) || !make_rows_map(&mrs, ring, ring_rows, RS_BOX))
+        return cudaErrorInvalidValue;
     int32_t *status = reinterpret_cast<int32_t *>(ws);
     int32_t *flags = reinterpret_cast<int32_t *>(ws + 1024);
     const int nflags = (int)(heads * (RING + 2));
@@ -708,14 +800,14 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
     sp.status = status;
     sp.filled = flags;
     sp.consumed = flags + heads * RING;
-    sp.ring = ws + 1024 + flags_bytes(heads);
+    sp.ring = ring;
     sp.H = p.H;
     sp.heads = (int32_t)heads;
     sp.max_chunks = max_chunks;
     sp.cph = cph;
     sp.timeout_ns = timeout_ns;
-    void *args[] = {&mq, &mk, &mv, &mla, &sp};
-    return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(NT), args, SPLIT_SMEM, stream);
+    void *args[] = {&mq, &mk, &mv, &mla, &mrl, &mrs, &sp};
+    return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(NTS), args, SPLIT_SMEM, stream);
 }
 
 }  // namespace kda
