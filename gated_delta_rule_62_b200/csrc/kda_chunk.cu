@@ -509,9 +509,9 @@ bool make_token_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, ui
 bool make_rows_map(CUtensorMap *m, void *base, uint64_t rows, uint32_t box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[2] = {64, rows};
-    cuuint64_t strides[1] = {128};
-    cuuint32_t box[2] = {64, box_rows};
+    cuuint64_t dims[2] = {256, rows};
+    cuuint64_t strides[1] = {512};
+    cuuint32_t box[2] = {256, box_rows};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,

@@ -413,7 +413,7 @@ __device__ __forceinline__ void scale_tmem_row(uint32_t taddr, float gm) {
 // 3-D TMA map over [T][H][inner] with a box of (box_inner, 1, 64 tokens); false on failure.
 bool make_token_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint32_t esize,
                     uint64_t inner, uint64_t H, uint64_t T, uint32_t box_inner, bool swizzle);
-// 2-D TMA map over `rows` 128-byte rows (64 bf16 each, copied verbatim: no swizzle) with a box of
+// 2-D TMA map over `rows` 512-byte rows (256 bf16 each, copied verbatim: no swizzle) with a box of
 // box_rows rows; false on failure.
 bool make_rows_map(CUtensorMap *m, void *base, uint64_t rows, uint32_t box_rows);
 

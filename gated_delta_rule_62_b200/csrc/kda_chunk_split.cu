@@ -51,10 +51,10 @@ constexpr int RING = 8;
 constexpr uint32_t SL_M = 0, SL_KH = 32768, SL_U = 49152, SL_P = 65536, SL_A = 81920;
 constexpr uint32_t SLOT = 90112;
 static_assert(SLOT % 1024 == 0, "slot layout");
-// The ring moves with tiled TMA over a [rows][64] bf16 view (128-byte rows copied verbatim):
-// an image is SLOT_ROWS rows, loaded in RL_BOX-row boxes and stored in 8 KB pieces.
-constexpr uint32_t SLOT_ROWS = SLOT / 128, RL_BOX = 176, RS_BOX = 64;
-static_assert(SLOT_ROWS % RL_BOX == 0, "ring load boxes");
+// The ring moves with tiled TMA over a [rows][256] bf16 view (512-byte rows copied verbatim):
+// an image is SLOT_ROWS rows, loaded as one box and stored in 8 KB pieces of RS_BOX rows.
+constexpr uint32_t ROW_BYTES = 512, SLOT_ROWS = SLOT / ROW_BYTES, RL_BOX = SLOT_ROWS, RS_BOX = 8192 / ROW_BYTES;
+static_assert(SLOT % ROW_BYTES == 0 && RL_BOX <= 256, "ring load box");
 
 struct SplitParams {
     const int32_t *cu_seqlens;
@@ -130,9 +130,9 @@ struct Cons {
     static constexpr uint32_t TM_S = 0, TM_O0 = DC, TM_O1 = 2 * DC, TM_COLS = CPH == 1 ? 512 : 256;
 };
 
-// Consumer roles, per chunk c (stage b = c & 1). Loader: once chunk c - 2's MMAs have completed
-// (o[b]) and the producer has published chunk c, copy its image into stage b (full[b]); publish
-// consumption as the copies land. MMA thread: wait for the image and for the compute threads'
+// Consumer roles, per chunk c (stage b = c & 1). Loader: once the producer has published chunk c
+// and chunk c - 2's MMAs have completed (o[b]), copy its image into stage b (full[b]); publish
+// consumption of chunk c - 2 at that point. MMA thread: wait for the image and for the compute threads'
 // "S_b ready", then issue S += M S_b + K^^T U~ (commit s), O = P S_b (commit sr), O += A U~
 // (commit o[b]). Compute threads: the outputs of chunk c - 1 (after o), the new state into
 // registers (after s), its bf16 copy S_b (after sr), then arrive on "S_b ready". No CTA-wide
@@ -181,40 +181,33 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
 
     if (tid == LDR) {
         // ------------------------------------------------ loader thread
-        // Chunk c goes to stage c & 1 once chunk c - 2's MMAs have completed; the consumed
-        // counter follows the copies as they land.
-        uint32_t ph_full[2] = {0, 0}, ph_o[2] = {0, 0};
-        int requested = 0, landed = 0;
+        // Chunk c goes to stage c & 1 once the producer has published it (acquired ahead, so
+        // the acquire's latency overlaps the wait) and chunk c - 2's MMAs have completed (o[b]);
+        // that completion also means chunk c - 2's image had landed: its slot may be refilled.
+        uint32_t ph_o[2] = {0, 0};
+        int requested = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
             if (ld_volatile(&s_flags[0])) break;
+            if (!wait_flag_ge(p.filled + hd * RING + (c % RING), c + 1, p.timeout_ns)) { fail(); break; }
+            fence_proxy_async_global();
             if (c >= 2) {
                 if (!mbar_wait_bounded(&bars[4 + b], ph_o[b], p.timeout_ns)) { fail(); break; }
                 ph_o[b] ^= 1u;
+                st_release(p.consumed + 2 * hd + sub, c - 1);
             }
-            if (!wait_flag_ge(p.filled + hd * RING + (c % RING), c + 1, p.timeout_ns)) { fail(); break; }
-            fence_proxy_async_global();
             const int32_t row0 = (int32_t)(((uint32_t)hd * RING + (uint32_t)(c % RING)) * SLOT_ROWS);
             uint8_t *dst = sm + (b ? STAGE1 : STAGE0);
             mbar_arrive_expect_tx(&bars[b], SLOT);
 #pragma unroll
             for (uint32_t k = 0; k < SLOT_ROWS / RL_BOX; ++k)
-                tma_load_2d(dst + k * RL_BOX * 128, tm_rl, &bars[b], 0, row0 + (int32_t)(k * RL_BOX));
+                tma_load_2d(dst + k * RL_BOX * ROW_BYTES, tm_rl, &bars[b], 0, row0 + (int32_t)(k * RL_BOX));
             requested = c + 1;
-            if (c >= 1) {  // chunk c - 1's image is in shared memory: its slot may be refilled
-                if (!mbar_wait_bounded(&bars[b ^ 1], ph_full[b ^ 1], p.timeout_ns)) { fail(); break; }
-                ph_full[b ^ 1] ^= 1u;
-                landed = c;
-                fence_proxy_async_global();
-                st_release(p.consumed + 2 * hd + sub, c);
-            }
         }
-        for (int c = landed; c < requested; ++c) {  // the copies still in flight land
-            if (!mbar_wait_bounded(&bars[c & 1], ph_full[c & 1], p.timeout_ns)) { fail(); break; }
-            ph_full[c & 1] ^= 1u;
-            fence_proxy_async_global();
-            st_release(p.consumed + 2 * hd + sub, c + 1);
-        }
+        // the last images land before the CTA exits (the MMA thread may have stopped early)
+        for (int c = requested - 2 < 0 ? 0 : requested - 2; c < requested; ++c)
+            if (!mbar_wait_bounded(&bars[c & 1], (uint32_t)(c >> 1) & 1u, p.timeout_ns)) fail();
+        if (requested == nchunks) st_release(p.consumed + 2 * hd + sub, nchunks);
     } else if (tid == CTL) {
         // ------------------------------------------------ MMA thread
         uint32_t ph_full[2] = {0, 0}, ph_ready = 0;
@@ -671,7 +664,7 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             const uint32_t off[11] = {SL_M, SL_M + 8192, SL_M + 16384, SL_M + 24576, SL_KH, SL_KH + 8192,
                                       SL_U, SL_U + 8192, SL_P, SL_P + 8192, SL_A};
 #pragma unroll
-            for (int k = 0; k < 11; ++k) tma_store_2d(tm_rs, src[k], 0, row0 + (int32_t)(off[k] / 128));
+            for (int k = 0; k < 11; ++k) tma_store_2d(tm_rs, src[k], 0, row0 + (int32_t)(off[k] / ROW_BYTES));
             bulk_commit();
             rel_flag = p.filled + hd * RING + (c % RING);
             rel_val = c + 1;

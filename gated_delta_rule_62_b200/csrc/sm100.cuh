@@ -51,15 +51,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
-// Bounded wait: spins until the phase with `parity` completes or `timeout_ns` have passed
-// (measured on %globaltimer, read only once the phase is found incomplete). Returns false on
-// timeout.
+// try_wait with a suspend-time hint: a thread whose phase is incomplete is parked by the hardware
+// (waking when the phase completes or after about `hint_ns`) instead of spinning, so waiting warps
+// leave their sub-partition's issue slots to the warps that do work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return done != 0;
+}
+
+// Bounded wait: until the phase with `parity` completes or `timeout_ns` have passed (measured on
+// %globaltimer, read only once the phase is found incomplete): a few plain tries, then tries that
+// park the thread for at most 1 ms each. Returns false on timeout.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   uint64_t timeout_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+    for (int i = 0; i < 16; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
     const uint64_t deadline = globaltimer_ns() + timeout_ns;
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
         if (globaltimer_ns() > deadline) return false;
     }
 }
