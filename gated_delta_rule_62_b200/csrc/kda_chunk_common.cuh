@@ -375,11 +375,13 @@ __device__ __forceinline__ void extract_al(uint32_t taddr, uint8_t *AQK, float *
 template <int NCOLS>
 __device__ __forceinline__ void rows64_to_tile(uint32_t taddr, uint8_t *tile, uint32_t bs,
                                                int col0, int quad, int lane, float scale = 1.f) {
+    float vv[NCOLS / 32][32];  // every 32-column load in flight before one wait
+#pragma unroll
+    for (int part = 0; part < NCOLS / 32; ++part) tmem_ld32(taddr + 32 * part, vv[part]);
+    tmem_wait_ld();
 #pragma unroll
     for (int part = 0; part < NCOLS / 32; ++part) {
-        float v[32];
-        tmem_ld32(taddr + 32 * part, v);
-        tmem_wait_ld();
+        float *v = vv[part];
         if (scale != 1.f) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] *= scale;

@@ -293,13 +293,15 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
         auto store_o = [&](int cc, uint32_t tm_o) {
             const int64_t tc = bos + (int64_t)cc * C;
             const int vc = (int)(eos - tc < C ? eos - tc : C);
-            const int i = 16 * quad + lane;
+                const int i = 16 * quad + lane;
+            float vv[NP][32];
+#pragma unroll
+            for (int part = 0; part < NP; ++part) tmem_ld32(tmem + lane_base + tm_o + col0 + 32 * part, vv[part]);
+            tmem_wait_ld();
 #pragma unroll
             for (int part = 0; part < NP; ++part) {
                 const int col = col0 + 32 * part;
-                float v[32];
-                tmem_ld32(tmem + lane_base + tm_o + col, v);
-                tmem_wait_ld();
+                const float *v = vv[part];
                 if (lane < 16 && i < vc) {
                     uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(tc + i) * H + h) * D + d0 + col);
 #pragma unroll
@@ -600,13 +602,16 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         tc_fence_after();
         if (compute) {
             const int r = 32 * quad + lane;  // TMEM lane
-            // D3 rows 0..63: U~ [j][d] over V; rows 64..127: P = Q~ - A W over Q~
+            // D3 rows 0..63: U~ [j][d] over V; rows 64..127: P = Q~ - A W over Q~ (both 32-column
+            // loads in flight before one wait)
+            float vv[2][32];
+            tmem_ld32(tmem + lane_base + TM_D3 + 64 * half, vv[0]);
+            tmem_ld32(tmem + lane_base + TM_D3 + 64 * half + 32, vv[1]);
+            tmem_wait_ld();
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
                 const int col = 64 * half + 32 * part;
-                float v[32];
-                tmem_ld32(tmem + lane_base + TM_D3 + col, v);
-                tmem_wait_ld();
+                float *v = vv[part];
                 if (r < 64) {
 #pragma unroll
                     for (int q8 = 0; q8 < 4; ++q8)
@@ -629,12 +634,13 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             }
             // D4 -> M = diag(gamma - 1) - K^^T W [c][c'] over K- and -W
             const float gm1 = s_gamma[r] - 1.f;
+            tmem_ld32(tmem + lane_base + TM_D4 + 64 * half, vv[0]);
+            tmem_ld32(tmem + lane_base + TM_D4 + 64 * half + 32, vv[1]);
+            tmem_wait_ld();
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
                 const int col = 64 * half + 32 * part;
-                float v[32];
-                tmem_ld32(tmem + lane_base + TM_D4 + col, v);
-                tmem_wait_ld();
+                float *v = vv[part];
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
                     if (col + e == r) v[e] += gm1;
