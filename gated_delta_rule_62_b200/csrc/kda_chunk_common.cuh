@@ -323,22 +323,32 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
             run.x *= al[i].x;
             run.y *= al[i].y;
         }
+        // Token t = 16 tq + i: with i known at compile time, t & 7 = i & 7 and t >> 3 = 2 tq + i / 8,
+        // so telem(bs, t, cA) = base_bs + (i / 8) 1024 + (i & 7) 128 + ((cx ^ (i & 7)) << 4):
+        // one XOR per token instead of a full swizzle per tile.
+        const uint32_t cx = (uint32_t)(cA & 63) >> 3;
+        const uint32_t row0 = (uint32_t)(2 * tq) * 1024 + (uint32_t)(cA & 7) * 2;
+        uint8_t *const q0 = QK + (uint32_t)(cA >> 6) * 16384 + row0;  // K~ rows: + 8 row groups
+        uint8_t *const i0 = KI + (uint32_t)(cA >> 6) * 8192 + row0;
+        uint8_t *const h0 = KH ? KH + (uint32_t)(cA >> 6) * 8192 + row0 : nullptr;
         float2 P = eA;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int t = 16 * tq + i;
             P.x *= al[i].x;
             P.y *= al[i].y;
-            uint8_t *qp = QK + telem(16384, t, cA);
-            uint8_t *kp = QK + telem(16384, 64 + t, cA);
+            const uint32_t off = (uint32_t)(i >> 3) * 1024 + (uint32_t)(i & 7) * 128 + ((cx ^ (uint32_t)(i & 7)) << 4);
+            uint8_t *qp = q0 + off;
+            uint8_t *kp = q0 + 8192 + off;
             float2 qv = ld_bf2(qp), kv = ld_bf2(kp);
             if (t >= valid) qv = kv = make_float2(0.f, 0.f);
             st_bf2(qp, qv.x * P.x, qv.y * P.y);
             st_bf2(kp, kv.x * P.x, kv.y * P.y);
-            st_bf2(KI + telem(8192, t, cA), kv.x * (eB.x * R[i].x), kv.y * (eB.y * R[i].y));
-            if (KH) st_bf2(KH + telem(8192, t, cA), kv.x * (eH.x * R[i].x), kv.y * (eH.y * R[i].y));
+            st_bf2(i0 + off, kv.x * (eB.x * R[i].x), kv.y * (eB.y * R[i].y));
+            if (KH) st_bf2(h0 + off, kv.x * (eH.x * R[i].x), kv.y * (eH.y * R[i].y));
         }
-    }    return safe ? 1 : 0;
+    }
+    return safe ? 1 : 0;
 }
 
 // ---------------------------------------------------------------- TMEM epilogues

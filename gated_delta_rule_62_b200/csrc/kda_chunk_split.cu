@@ -14,11 +14,9 @@
 //     ([T'; 0] V + [0; A] (-W)) and -K^^T W in another, and from those U~, P and M as
 //     ready-to-use shared-memory images (bf16) in a ring of RING slots per head in the
 //     workspace (L2 resident).
-//   consumer CTAs (one per head, or two per head with 64 value channels each when the SMs
-//     left over still give every head about three producers): the chain. Per chunk:
-//     S += M S_b + K^^T U~ (S_b = the state's bf16 copy), O = P S_b + A U~ behind it, then
-//     the new state's bf16 copy; the outputs leave while the next chunk's batch runs. The fp32
-//     state stays in TMEM for the whole sequence.
+//   consumer CTAs (one per head): the chain. Per chunk: S += M S_b + K^^T U~ (S_b = the
+//     state's bf16 copy, fed from tensor memory), O = P S_b + A U~ behind it; the outputs leave
+//     while the next chunk's chain runs. The fp32 state stays in TMEM for the whole sequence.
 //
 // Hand-off: a producer fills slot (head, c % RING) with bulk stores, then releases
 // filled[slot] = c + 1; a consumer acquires it, copies the image into shared memory with a
@@ -65,8 +63,9 @@ struct SplitParams {
     int32_t *status;
     uint8_t *ring;       // [heads][RING][SLOT]
     int32_t *filled;     // [heads][RING]
-    int32_t *consumed;   // [heads][2]: one counter per consumer (the second unused with one)
-    int32_t H, heads, max_chunks, cph;
+    int32_t *consumed;   // [heads]
+    int32_t *next_item;  // producers' work counter (items k = chunk * heads + head, chunk-major)
+    int32_t H, heads, max_chunks;
     uint64_t timeout_ns;
 };
 
@@ -115,55 +114,50 @@ __device__ __forceinline__ uint32_t ld_volatile(const uint32_t *p) {
 }
 
 // ---------------------------------------------------------------- consumer (state chain)
-// CPH consumers per head, each owning DC = 128 / CPH value channels (columns of S are
-// independent: the chain of one column block never reads another's).
-template <int CPH>
-struct Cons {
-    static constexpr int DC = D / CPH;                  // value channels per consumer
-    static constexpr int NP = DC / 64;                  // 32-column parts per thread
-    static constexpr uint32_t STAGE0 = 0, STAGE1 = SLOT;
-    static constexpr uint32_t S = 2 * SLOT;             // S_b [c][d] bf16 128 x DC
-    static constexpr uint32_t MISC = S + 256 * DC;      // barriers, flags
-    static constexpr uint32_t BYTES = MISC + 256;
-    // TMEM: the fp32 state (lane = key channel, column = value channel) and two M=64 output
-    // accumulators (row i in lane i % 16 + 32 (i / 16)), used by alternate chunks.
-    static constexpr uint32_t TM_S = 0, TM_O0 = DC, TM_O1 = 2 * DC, TM_COLS = CPH == 1 ? 512 : 256;
-};
+// One consumer per head. The state is kept transposed, S^T [d][c] (lane = value channel d), so its
+// bf16 copy can feed the chain's MMA as an A operand straight from tensor memory:
+//   S^T += S_b^T M^T + U~^T K^   (A = S_b^T in TMEM, B = M as stored; A = U~, B = K^ MN-major)
+//   O    = P S_b + A U~          (M = 64 tokens; B = S_b^T [d][c], a K-major tile in shared memory)
+// so the next chunk's chain waits neither for the output MMA nor for a shared-memory store.
+namespace cons {
+constexpr uint32_t STAGE0 = 0, STAGE1 = SLOT;
+constexpr uint32_t SBT = 2 * SLOT;         // S_b^T [d][c] bf16 128 x 128 (64-column blocks of 16 KB)
+constexpr uint32_t MISC = SBT + 32768;     // barriers, flags
+constexpr uint32_t BYTES = MISC + 256;
+// TMEM: S^T fp32 (128 columns), two bf16 copies S_b^T (64 columns each, used by alternate chunks),
+// two M=64 output accumulators (row i in lane i % 16 + 32 (i / 16); 128 columns each).
+constexpr uint32_t TM_S = 0, TM_SB0 = 128, TM_SB1 = 192, TM_O0 = 256, TM_O1 = 384, TM_COLS = 512;
+}  // namespace cons
 
 // Consumer roles, per chunk c (stage b = c & 1). Loader: once the producer has published chunk c
 // and chunk c - 2's MMAs have completed (o[b]), copy its image into stage b (full[b]); publish
-// consumption of chunk c - 2 at that point. MMA thread: wait for the image and for the compute threads'
-// "S_b ready", then issue S += M S_b + K^^T U~ (commit s), O = P S_b (commit sr), O += A U~
-// (commit o[b]). Compute threads: the outputs of chunk c - 1 (after o), the new state into
-// registers (after s), its bf16 copy S_b (after sr), then arrive on "S_b ready". No CTA-wide
-// barrier inside the loop.
-template <int CPH>
-__device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t *sm, int cid) {
-    using L = Cons<CPH>;
-    constexpr int DC = L::DC, NP = L::NP;
-    constexpr uint32_t STAGE0 = L::STAGE0, STAGE1 = L::STAGE1, S = L::S, MISC = L::MISC;
-    constexpr uint32_t TM_S = L::TM_S, TM_O0 = L::TM_O0, TM_O1 = L::TM_O1, TM_COLS = L::TM_COLS;
-    constexpr uint32_t I_C = idesc_bf16_f32(128, DC, false, 0, 1);  // M S_b
-    constexpr uint32_t I_K = idesc_bf16_f32(128, DC, false, 1, 1);  // K^^T U~
-    constexpr uint32_t I_O = idesc_bf16_f32(64, DC, false, 0, 1);   // P S_b, A U~
-    const int hd = cid / CPH, sub = cid % CPH, d0 = DC * sub;  // head, first value channel
-    // full0, full1, s, sr, o0, o1, ready, teardown
+// consumption of chunk c - 2 at that point. MMA thread: wait for the image and for S_b^T(c) in TMEM,
+// issue the chain (commit s); wait for S_b^T(c) in shared memory and for the output warps to have
+// read accumulator b (chunk c - 2), issue O = P S_b (commit sr) and O += A U~ (commit o[b]). State
+// warps 0..3 (lane = value channel): after s, the new state's bf16 copy into TMEM ("tmem ready": the
+// critical path), after sr into shared memory ("smem ready"). Output warps 4..7: after o[b], the
+// outputs ("o free"). No CTA-wide barrier inside the loop.
+__device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t *sm, int hd) {
+    using namespace cons;
+    constexpr uint32_t I_C = idesc_bf16_f32(128, 128, false, 0, 0);   // S_b^T M^T (A in TMEM)
+    constexpr uint32_t I_K = idesc_bf16_f32(128, 128, false, 1, 1);   // U~^T K^
+    constexpr uint32_t I_P = idesc_bf16_f32(64, 128, false, 0, 0);    // P S_b
+    constexpr uint32_t I_A = idesc_bf16_f32(64, 128, false, 0, 1);    // A U~
+    // full0, full1, s, sr, o0, o1, tmem ready, smem ready, o free 0, o free 1, teardown
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);
-    uint32_t *s_flags = reinterpret_cast<uint32_t *>(sm + MISC + 64); // abort, tmem
+    uint32_t *s_flags = reinterpret_cast<uint32_t *>(sm + MISC + 96); // abort, tmem
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = (warp >> 2) & 1;
+    const int quad = warp & 3;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
     const int H = p.H, n = hd / H, h = hd % H;
-    const int c_me = 32 * quad + lane;  // TMEM lane of this thread
     const int64_t bos = p.cu_seqlens[n], eos = p.cu_seqlens[n + 1];
     const int nchunks = (int)((eos - bos + C - 1) / C);
     const size_t state_off = ((size_t)n * H + h) * (size_t)(D * D);
-    const int col0 = (DC / 2) * half;  // this thread's first column of S and O
 
     if (tid == 0) {
         s_flags[0] = 0;
-        for (int k = 0; k < 8; ++k) mbar_init(&bars[k], k == 6 ? NT : 1);
+        for (int k = 0; k < 11; ++k) mbar_init(&bars[k], (k >= 6 && k <= 9) ? NT / 2 : 1);
         fence_mbarrier_init();
     }
     if (warp == 0) {
@@ -194,7 +188,7 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
             if (c >= 2) {
                 if (!mbar_wait_bounded(&bars[4 + b], ph_o[b], p.timeout_ns)) { fail(); break; }
                 ph_o[b] ^= 1u;
-                st_release(p.consumed + 2 * hd + sub, c - 1);
+                st_release(p.consumed + hd, c - 1);
             }
             const int32_t row0 = (int32_t)(((uint32_t)hd * RING + (uint32_t)(c % RING)) * SLOT_ROWS);
             uint8_t *dst = sm + (b ? STAGE1 : STAGE0);
@@ -207,154 +201,172 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
         // the last images land before the CTA exits (the MMA thread may have stopped early)
         for (int c = requested - 2 < 0 ? 0 : requested - 2; c < requested; ++c)
             if (!mbar_wait_bounded(&bars[c & 1], (uint32_t)(c >> 1) & 1u, p.timeout_ns)) fail();
-        if (requested == nchunks) st_release(p.consumed + 2 * hd + sub, nchunks);
+        if (requested == nchunks) st_release(p.consumed + hd, nchunks);
     } else if (tid == CTL) {
         // ------------------------------------------------ MMA thread
-        uint32_t ph_full[2] = {0, 0}, ph_ready = 0;
+        uint32_t ph_full[2] = {0, 0}, ph_t = 0, ph_s = 0, ph_free[2] = {0, 0};
+        const uint64_t dSBT = desc_k(sb + SBT, 16384, 0);
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
             if (ld_volatile(&s_flags[0])) break;
             if (!mbar_wait_bounded(&bars[b], ph_full[b], p.timeout_ns)) { fail(); break; }
             ph_full[b] ^= 1u;
-            if (!mbar_wait_bounded(&bars[6], ph_ready, p.timeout_ns)) { fail(); break; }
-            ph_ready ^= 1u;
+            if (!mbar_wait_bounded(&bars[6], ph_t, p.timeout_ns)) { fail(); break; }
+            ph_t ^= 1u;
             tc_fence_after();
             const uint32_t st = sb + (b ? STAGE1 : STAGE0);
-            const uint32_t tm_o = b ? TM_O1 : TM_O0;
-            const uint64_t dM = desc_k(st + SL_M, 16384, 0), dS = desc_mn(sb + S, 16384, 0);
-            const uint64_t dK = desc_mn(st + SL_KH, 8192, 0);
-            const uint64_t dU = desc_mn(st + SL_U + 8192 * (d0 / 64), 8192, 0);
+            const uint32_t tm_sb = tmem + (b ? TM_SB1 : TM_SB0);
+            const uint32_t tm_o = tmem + (b ? TM_O1 : TM_O0);
+            const uint64_t dM = desc_k(st + SL_M, 16384, 0), dK = desc_mn(st + SL_KH, 8192, 0);
+            const uint64_t dU = desc_mn(st + SL_U, 8192, 0);
             const uint64_t dP = desc_k(st + SL_P, 8192, 0), dA = desc_k(st + SL_A, 8192, 0);
 #pragma unroll
-            for (uint32_t kk = 0; kk < 8; ++kk)  // S += M S_b ...
-                mma_bf16_ss(tmem + TM_S, desc_k_at(dM, 16384, kk), desc_mn_at(dS, kk), I_C, 1);
+            for (uint32_t kk = 0; kk < 8; ++kk)  // S^T += S_b^T M^T ...
+                mma_bf16_ts(tmem + TM_S, tm_sb + 8 * kk, desc_k_at(dM, 16384, kk), I_C, 1);
 #pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)  // ... + K^^T U~
-                mma_bf16_ss(tmem + TM_S, desc_mn_at(dK, kk), desc_mn_at(dU, kk), I_K, 1);
+            for (uint32_t kk = 0; kk < 4; ++kk)  // ... + U~^T K^
+                mma_bf16_ss(tmem + TM_S, desc_mn_at(dU, kk), desc_mn_at(dK, kk), I_K, 1);
             mma_commit(&bars[2]);
+            if (!mbar_wait_bounded(&bars[7], ph_s, p.timeout_ns)) { fail(); break; }
+            ph_s ^= 1u;
+            if (c >= 2) {  // the output warps have read this accumulator's previous chunk
+                if (!mbar_wait_bounded(&bars[8 + b], ph_free[b], p.timeout_ns)) { fail(); break; }
+                ph_free[b] ^= 1u;
+            }
+            tc_fence_after();
 #pragma unroll
             for (uint32_t kk = 0; kk < 8; ++kk)  // O = P S_b ...
-                mma_bf16_ss(tmem + tm_o, desc_k_at(dP, 8192, kk), desc_mn_at(dS, kk), I_O, kk > 0);
-            mma_commit(&bars[3]);                // S_b has been read
+                mma_bf16_ss(tm_o, desc_k_at(dP, 8192, kk), desc_k_at(dSBT, 16384, kk), I_P, kk > 0);
+            mma_commit(&bars[3]);                // S_b^T in shared memory has been read
 #pragma unroll
             for (uint32_t kk = 0; kk < 4; ++kk)  // ... + A U~
-                mma_bf16_ss(tmem + tm_o, desc_k_at(dA, 8192, kk), desc_mn_at(dU, kk), I_O, 1);
+                mma_bf16_ss(tm_o, desc_k_at(dA, 8192, kk), desc_mn_at(dU, kk), I_A, 1);
             mma_commit(&bars[4 + b]);            // O and the stage are done
         }
         // teardown: every issued MMA completes before TMEM is freed
-        mma_commit(&bars[7]);
-        mbar_wait_bounded(&bars[7], 0, p.timeout_ns);
-    } else if (tid < NT) {
-        // ------------------------------------------------ compute threads
-        // initial state -> TMEM (lane c, columns d) and S_b; empty sequences copy it out
-        {
-            const size_t row = state_off + (size_t)c_me * D + d0 + col0;
-            const float *src = p.s0 ? p.s0 + row : nullptr;
-            float *dst = p.sT ? p.sT + row : nullptr;
-#pragma unroll
-            for (int part = 0; part < NP; ++part) {
-                float v[32];
-#pragma unroll
-                for (int e = 0; e < 32; e += 4) {
-                    float4 f = src ? *reinterpret_cast<const float4 *>(src + 32 * part + e)
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-                    v[e] = f.x; v[e + 1] = f.y; v[e + 2] = f.z; v[e + 3] = f.w;
-                }
-                if (nchunks == 0) {
-                    if (dst) {
-#pragma unroll
-                        for (int e = 0; e < 32; e += 4)
-                            *reinterpret_cast<float4 *>(dst + 32 * part + e) =
-                                make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                    }
-                } else {
-                    const int col = col0 + 32 * part;
-                    tmem_st32(tmem + lane_base + TM_S + col, v);
-#pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8)
-                        st_chunk(sm + S + tchunk(16384, c_me, col + 8 * q8), v + 8 * q8);
-                }
-            }
-            tmem_wait_st();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(&bars[6]);  // S_b ready for chunk 0
-
-        uint32_t ph_s = 0, ph_sr = 0, ph_o[2] = {0, 0};
+        mma_commit(&bars[10]);
+        mbar_wait_bounded(&bars[10], 0, p.timeout_ns);
+    } else if (warp < 4) {
+        // ------------------------------------------------ state warps (lane = value channel d)
+        // per chunk: the new state -> its bf16 copy in TMEM (the next chain's A operand: the
+        // critical path), then, once P S_b has read the old one, into shared memory
+        const int d_me = tid;  // 0..127
         auto wait_bar = [&](uint64_t *bar, uint32_t &ph) -> bool {
             const bool ok = mbar_wait_bounded(bar, ph, p.timeout_ns);
             ph ^= 1u;
             if (!ok) fail();
             return ok;
         };
-        // O of chunk cc (M=64 accumulator at tm_o) -> bf16 outputs; rows in lanes 0..15 of each
-        // quadrant
-        auto store_o = [&](int cc, uint32_t tm_o) {
-            const int64_t tc = bos + (int64_t)cc * C;
-            const int vc = (int)(eos - tc < C ? eos - tc : C);
-                const int i = 16 * quad + lane;
-            float vv[NP][32];
+        uint32_t w[2][32];  // this thread's row of S_b^T, bf16 pairs (c, c + 1)
+        // S^T row d, columns [64 h, 64 h + 64) in v -> packed w[h] -> TMEM copy at tm_sb
+        auto pack_store = [&](const float (&v)[2][32], int hh, uint32_t tm_sb) {
 #pragma unroll
-            for (int part = 0; part < NP; ++part) tmem_ld32(tmem + lane_base + tm_o + col0 + 32 * part, vv[part]);
-            tmem_wait_ld();
+            for (int e = 0; e < 32; ++e) w[hh][e] = pack2(v[e >> 4][2 * (e & 15)], v[e >> 4][2 * (e & 15) + 1]);
+            float f[32];
 #pragma unroll
-            for (int part = 0; part < NP; ++part) {
-                const int col = col0 + 32 * part;
-                const float *v = vv[part];
-                if (lane < 16 && i < vc) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(tc + i) * H + h) * D + d0 + col);
-#pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8)
-                        dst[q8] = make_uint4(pack2(v[8 * q8], v[8 * q8 + 1]), pack2(v[8 * q8 + 2], v[8 * q8 + 3]),
-                                             pack2(v[8 * q8 + 4], v[8 * q8 + 5]), pack2(v[8 * q8 + 6], v[8 * q8 + 7]));
-                }
-            }
+            for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(w[hh][e]);
+            tmem_st32(tmem + lane_base + tm_sb + 32 * hh, f);
         };
-
-        int c = 0;
-        for (; c < nchunks; ++c) {
-            const int b = c & 1;
-            if (ld_volatile(&s_flags[0])) break;
-            if (c > 0) {  // the previous chunk's outputs while this chunk's batch runs
-                if (!wait_bar(&bars[4 + (b ^ 1)], ph_o[b ^ 1])) break;
-                tc_fence_after();
-                store_o(c - 1, b ? TM_O0 : TM_O1);
+        auto to_smem = [&]() {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int q8 = 0; q8 < 8; ++q8)
+                    *reinterpret_cast<uint4 *>(sm + SBT + tchunk(16384, d_me, 64 * hh + 8 * q8)) =
+                        make_uint4(w[hh][4 * q8], w[hh][4 * q8 + 1], w[hh][4 * q8 + 2], w[hh][4 * q8 + 3]);
+            fence_proxy_async_smem();
+            mbar_arrive(&bars[7]);
+        };
+        // initial state S[c][d] -> S^T in TMEM and both bf16 copies; empty sequences copy it out
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float v[2][32];
+            const float *src = p.s0 ? p.s0 + state_off + (size_t)(64 * hh) * D + d_me : nullptr;
+#pragma unroll
+            for (int e = 0; e < 64; ++e) v[e >> 5][e & 31] = src ? src[(size_t)e * D] : 0.f;
+            if (nchunks == 0) {
+                if (p.sT) {
+                    float *dst = p.sT + state_off + (size_t)(64 * hh) * D + d_me;
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) dst[(size_t)e * D] = v[e >> 5][e & 31];
+                }
+            } else {
+                tmem_st32(tmem + lane_base + TM_S + 64 * hh, v[0]);
+                tmem_st32(tmem + lane_base + TM_S + 64 * hh + 32, v[1]);
+                pack_store(v, hh, TM_SB0);
             }
-            // the new state -> registers (and the final state after the last chunk)
+        }
+        if (nchunks > 0) {
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars[6]);
+            to_smem();
+        }
+        uint32_t ph_s = 0, ph_sr = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1;
+            const bool last = c + 1 == nchunks;
+            if (ld_volatile(&s_flags[0])) break;
             if (!wait_bar(&bars[2], ph_s)) break;
             tc_fence_after();
-            float v[NP][32];
 #pragma unroll
-            for (int part = 0; part < NP; ++part) tmem_ld32(tmem + lane_base + TM_S + col0 + 32 * part, v[part]);
-            tmem_wait_ld();
-            if (c + 1 == nchunks && p.sT) {
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[2][32];
+                tmem_ld32(tmem + lane_base + TM_S + 64 * hh, v[0]);
+                tmem_ld32(tmem + lane_base + TM_S + 64 * hh + 32, v[1]);
+                tmem_wait_ld();
+                if (!last) {
+                    pack_store(v, hh, b ? TM_SB0 : TM_SB1);  // the next chunk's copy
+                } else if (p.sT) {
+                    float *dst = p.sT + state_off + (size_t)(64 * hh) * D + d_me;
 #pragma unroll
-                for (int part = 0; part < NP; ++part) {
-                    float *dst = p.sT + state_off + (size_t)c_me * D + d0 + col0 + 32 * part;
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4 *>(dst + e) =
-                            make_float4(v[part][e], v[part][e + 1], v[part][e + 2], v[part][e + 3]);
+                    for (int e = 0; e < 64; ++e) dst[(size_t)e * D] = v[e >> 5][e & 31];
                 }
             }
-            // its bf16 copy, once P S_b has read the old one
-            if (!wait_bar(&bars[3], ph_sr)) break;
-#pragma unroll
-            for (int part = 0; part < NP; ++part)
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8)
-                    st_chunk(sm + S + tchunk(16384, c_me, col0 + 32 * part + 8 * q8), v[part] + 8 * q8);
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bars[6]);  // S_b ready for chunk c + 1
-        }
-        if (c == nchunks && nchunks > 0) {  // outputs of the last chunk
-            const int bl = (nchunks - 1) & 1;
-            if (wait_bar(&bars[4 + bl], ph_o[bl])) {
-                tc_fence_after();
-                store_o(nchunks - 1, bl ? TM_O1 : TM_O0);
+            if (!last) {
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bars[6]);
             }
+            if (!wait_bar(&bars[3], ph_sr)) break;
+            if (!last) to_smem();
+        }
+        tc_fence_before();
+    } else if (tid < NT) {
+        // ------------------------------------------------ output warps
+        // O of chunk c (M=64 accumulator: row i in lane i % 16 + 32 (i / 16)) -> bf16 outputs
+        const int i = 16 * quad + lane;
+        uint32_t ph_o[2] = {0, 0};
+        for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1;
+            if (ld_volatile(&s_flags[0])) break;
+            const bool ok = mbar_wait_bounded(&bars[4 + b], ph_o[b], p.timeout_ns);
+            ph_o[b] ^= 1u;
+            if (!ok) { fail(); break; }
+            tc_fence_after();
+            const int64_t tc = bos + (int64_t)c * C;
+            const int vc = (int)(eos - tc < C ? eos - tc : C);
+            const uint32_t tm_o = b ? TM_O1 : TM_O0;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float vv[2][32];
+                tmem_ld32(tmem + lane_base + tm_o + 64 * hh, vv[0]);
+                tmem_ld32(tmem + lane_base + tm_o + 64 * hh + 32, vv[1]);
+                tmem_wait_ld();
+                if (lane < 16 && i < vc) {
+#pragma unroll
+                    for (int part = 0; part < 2; ++part) {
+                        const float *v = vv[part];
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(tc + i) * H + h) * D + 64 * hh + 32 * part);
+#pragma unroll
+                        for (int q8 = 0; q8 < 4; ++q8)
+                            dst[q8] = make_uint4(pack2(v[8 * q8], v[8 * q8 + 1]), pack2(v[8 * q8 + 2], v[8 * q8 + 3]),
+                                                 pack2(v[8 * q8 + 4], v[8 * q8 + 5]), pack2(v[8 * q8 + 6], v[8 * q8 + 7]));
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bars[8 + b]);  // this accumulator may take chunk c + 2
         }
         tc_fence_before();
     }
@@ -408,14 +420,36 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
     const bool compute = tid < NT, ctl = tid == CTL;
     const int H = p.H;
-    // Static assignment: producer pid serves head hd = pid % heads, making chunks j, j + cnt, ...
-    // (j = pid / heads, cnt = number of producers of that head), so it only ever waits on its
-    // own head's consumers.
-    const int hd = pid % p.heads, pj = pid / p.heads;
-    const int pcnt = (nprod - 1 - hd) / p.heads + 1;
-    const int h = hd % H;
-    const int64_t bos = p.cu_seqlens[hd / H], eos = p.cu_seqlens[hd / H + 1];
-    const int nch = (int)((eos - bos + C - 1) / C);
+    // Dynamic assignment: items k = chunk * heads + head are claimed from one counter in that
+    // (chunk-major) order, so every head advances at the producers' common rate. A producer's
+    // item only waits on consumption of earlier chunks of its head, whose items were claimed
+    // earlier and are finished by producers that never wait on anything later: no cycle.
+    (void)pid;
+    (void)nprod;
+    struct Item {
+        int hd, c, h;
+        int64_t bos, eos;
+    };
+    auto decode = [&](int k) -> Item {
+        Item it;
+        it.hd = k % p.heads;
+        it.c = k / p.heads;
+        it.h = it.hd % H;
+        it.bos = p.cu_seqlens[it.hd / H];
+        it.eos = p.cu_seqlens[it.hd / H + 1];
+        return it;
+    };
+    // control thread: the next item with a chunk to make, or -1 when none is left
+    auto claim = [&]() -> int {
+        while (true) {
+            const int k = atomicAdd(p.next_item, 1);
+            const int c = k / p.heads, hdk = k % p.heads;
+            if (c >= p.max_chunks) return -1;
+            const int64_t len = p.cu_seqlens[hdk / H + 1] - p.cu_seqlens[hdk / H];
+            if ((int64_t)c * C < len) return k;
+        }
+    };
+    int *s_items = reinterpret_cast<int *>(s_flags + 4);  // first two items; then the one after next
 
     if (tid == 0) {
         s_flags[0] = 0;
@@ -444,8 +478,10 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 
     // control thread; each buffer's previous contents were read by generic loads or bulk stores
     // that have completed (see the call sites)
-    auto issue_qk = [&](int c, int b) {
-        const int64_t t0 = bos + (int64_t)c * C;
+    auto issue_qk = [&](int k, int b) {
+        const Item it = decode(k);
+        const int h = it.h;
+        const int64_t t0 = it.bos + (int64_t)it.c * C;
         uint8_t *qk = sm + (b ? QK1 : QK0);
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&bars[b], 32768);
@@ -454,23 +490,29 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         tma_load_3d(qk + 16384, tm_q, &bars[b], 64, h, (int32_t)t0);
         tma_load_3d(qk + 24576, tm_k, &bars[b], 64, h, (int32_t)t0);
     };
-    auto issue_la = [&](int c) {
-        const int64_t t0 = bos + (int64_t)c * C;
+    auto issue_la = [&](int k) {
+        const Item it = decode(k);
+        const int h = it.h;
+        const int64_t t0 = it.bos + (int64_t)it.c * C;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&bars[2], 32768);
         tma_load_3d(sm + LA, tm_la, &bars[2], 0, h, (int32_t)t0);
     };
-    auto issue_v = [&](int c) {
-        const int64_t t0 = bos + (int64_t)c * C;
+    auto issue_v = [&](int k) {
+        const Item it = decode(k);
+        const int h = it.h;
+        const int64_t t0 = it.bos + (int64_t)it.c * C;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&bars[3], 16384);
         tma_load_3d(sm + VB, tm_v, &bars[3], 0, h, (int32_t)t0);
         tma_load_3d(sm + VB + 8192, tm_v, &bars[3], 64, h, (int32_t)t0);
     };
-    auto load_beta = [&](int c) -> float {  // tid < C
-        const int64_t t0 = bos + (int64_t)c * C;
-        if (c >= nch || t0 + tid >= eos) return 0.f;
-        return p.beta[(size_t)(t0 + tid) * H + h];
+    auto load_beta = [&](int k) -> float {  // tid < C
+        if (k < 0) return 0.f;
+        const Item it = decode(k);
+        const int64_t t0 = it.bos + (int64_t)it.c * C;
+        if (t0 + tid >= it.eos) return 0.f;
+        return p.beta[(size_t)(t0 + tid) * H + it.h];
     };
     // the previous image, published once its bulk stores are complete (control thread, during
     // the next item's gating)
@@ -494,21 +536,24 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         if (!ok) fail();
     };
 
-    int item = pj;  // chunk index
-    if (item < nch) {
-        if (ctl) {
-            issue_qk(item, 0);
-            issue_la(item);
+    if (ctl) {
+        s_items[0] = claim();
+        s_items[1] = s_items[0] >= 0 ? claim() : -1;
+        if (s_items[0] >= 0) {
+            issue_qk(s_items[0], 0);
+            issue_la(s_items[0]);
         }
-        pend_qk[0] = pend_la = true;
     }
+    __syncthreads();
+    int item = s_items[0], nxt = s_items[1];
+    if (item >= 0) pend_qk[0] = pend_la = true;
     float beta_next = (tid < C) ? load_beta(item) : 0.f;
     int b = 0;
-    while (item < nch) {
-        const int c = item;
-        const int64_t t0 = bos + (int64_t)c * C;
-        const int valid = (int)(eos - t0 < C ? eos - t0 : C);
-        const int nxt = item + pcnt;
+    while (item >= 0) {
+        const Item it = decode(item);
+        const int hd = it.hd, c = it.c;
+        const int64_t t0 = it.bos + (int64_t)c * C;
+        const int valid = (int)(it.eos - t0 < C ? it.eos - t0 : C);
         uint8_t *qk = sm + (b ? QK1 : QK0);
         if (tid < C) s_beta[tid] = beta_next;
         if (ctl) {  // the previous image's sources (K-, K^, A, ...) are rewritten by the gating
@@ -535,9 +580,10 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         if (gate < 0 || stop) break;
         const bool safe = gate == 1;
         if (ctl) {
-            // V of this chunk; q/k and log_alpha of the next one (the gating is done with them)
-            issue_v(c);
-            if (nxt < nch) {
+            // V of this chunk; q/k and log_alpha of the next one (the gating is done with them);
+            // then claim the item after the next one (read by all after the following barriers)
+            issue_v(item);
+            if (nxt >= 0) {
                 issue_qk(nxt, b ^ 1);
                 issue_la(nxt);
             }
@@ -549,9 +595,10 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                                 desc_k(sb + KI, 8192, kk), I_D1, kk > 0);
             }
             mma_commit(&bars[4]);
+            s_items[2] = nxt >= 0 ? claim() : -1;
         }
         pend_v = true;
-        if (nxt < nch) pend_qk[b ^ 1] = pend_la = true;
+        if (nxt >= 0) pend_qk[b ^ 1] = pend_la = true;
         wait_bar(&bars[4], ph_mma);
         tc_fence_after();
         if (compute && !safe) extract_al(tmem + lane_base + TM_D1 + 32 * half, sm + AQK, LTp, s_beta, 32 * quad + lane, half);
@@ -651,9 +698,7 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             fence_proxy_async_smem();  // written by generic stores; the copy-out is async
         }
         if (ctl && c >= RING) {  // the slot's previous chunk must have been taken
-            if (!wait_flag_ge(p.consumed + 2 * hd, c - RING + 1, p.timeout_ns) ||
-                (p.cph == 2 && !wait_flag_ge(p.consumed + 2 * hd + 1, c - RING + 1, p.timeout_ns)))
-                fail();
+            if (!wait_flag_ge(p.consumed + hd, c - RING + 1, p.timeout_ns)) fail();
         }
         tc_fence_before();
         if (__syncthreads_or(ld_volatile(&s_flags[0]) != 0)) break;
@@ -676,6 +721,7 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             rel_val = c + 1;
         }
         item = nxt;
+        nxt = s_items[2];
         b ^= 1;
     }
 
@@ -697,12 +743,8 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     }
 }
 
-constexpr uint32_t max3(uint32_t a, uint32_t b, uint32_t c) {
-    return a > b ? (a > c ? a : c) : (b > c ? b : c);
-}
-constexpr uint32_t SPLIT_SMEM = max3(Cons<1>::BYTES, Cons<2>::BYTES, prod::BYTES) + 1024;
+constexpr uint32_t SPLIT_SMEM = (cons::BYTES > prod::BYTES ? cons::BYTES : prod::BYTES) + 1024;
 
-template <int CPH>
 __global__ void __launch_bounds__(NTS, 1)
 split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
@@ -711,11 +753,10 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-    if ((int)blockIdx.x < CPH * p.heads)
-        consumer<CPH>(&tm_rl, p, sm, blockIdx.x);
+    if ((int)blockIdx.x < p.heads)
+        consumer(&tm_rl, p, sm, blockIdx.x);
     else
-        producer(&tm_q, &tm_k, &tm_v, &tm_la, &tm_rs, p, sm, blockIdx.x - CPH * p.heads,
-                 gridDim.x - CPH * p.heads);
+        producer(&tm_q, &tm_k, &tm_v, &tm_la, &tm_rs, p, sm, blockIdx.x - p.heads, gridDim.x - p.heads);
 }
 
 // Zeroes the status word and the ring flags.
@@ -749,26 +790,18 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
                                  cudaStream_t stream, uint64_t timeout_ns) {
     const int64_t heads = (int64_t)p.num_seqs * p.H;
     const int sms = sm_count();
-    // Two consumers per head halve the chain's per-chunk work, but take SMs from the producers;
-    // worth it only while every head still gets about three producers (a producer's item costs
-    // about two and a half consumer chunks).
-    const int cph = heads * 5 <= sms ? 2 : 1;
-    const void *fn = cph == 2 ? (const void *)split_kernel<2> : (const void *)split_kernel<1>;
     int per_sm = 0;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(split_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute(split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)SPLIT_SMEM);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(split_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            (int)SPLIT_SMEM);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, NTS, SPLIT_SMEM);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, split_kernel, NTS, SPLIT_SMEM);
     if (e != cudaSuccess) return e;
     const int grid = per_sm * sms;
-    if (per_sm < 1 || grid < (cph + 1) * heads) return cudaErrorInvalidConfiguration;
+    if (per_sm < 1 || grid < 2 * heads) return cudaErrorInvalidConfiguration;
 
     CUtensorMap mq, mk, mv, mla, mrl, mrs;
     const uint64_t T = (uint64_t)p.total_tokens, H = (uint64_t)p.H;
@@ -799,14 +832,15 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
     sp.status = status;
     sp.filled = flags;
     sp.consumed = flags + heads * RING;
+    sp.next_item = flags + heads * (RING + 1);
     sp.ring = ring;
     sp.H = p.H;
     sp.heads = (int32_t)heads;
     sp.max_chunks = max_chunks;
-    sp.cph = cph;
     sp.timeout_ns = timeout_ns;
     void *args[] = {&mq, &mk, &mv, &mla, &mrl, &mrs, &sp};
-    return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(NTS), args, SPLIT_SMEM, stream);
+    return cudaLaunchCooperativeKernel((const void *)split_kernel, dim3(grid), dim3(NTS), args,
+                                       SPLIT_SMEM, stream);
 }
 
 }  // namespace kda
