@@ -580,8 +580,7 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         if (gate < 0 || stop) break;
         const bool safe = gate == 1;
         if (ctl) {
-            // V of this chunk; q/k and log_alpha of the next one (the gating is done with them);
-            // then claim the item after the next one (read by all after the following barriers)
+            // V of this chunk; q/k and log_alpha of the next one (the gating is done with them)
             issue_v(item);
             if (nxt >= 0) {
                 issue_qk(nxt, b ^ 1);
@@ -595,7 +594,6 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                                 desc_k(sb + KI, 8192, kk), I_D1, kk > 0);
             }
             mma_commit(&bars[4]);
-            s_items[2] = nxt >= 0 ? claim() : -1;
         }
         pend_v = true;
         if (nxt >= 0) pend_qk[b ^ 1] = pend_la = true;
@@ -605,6 +603,9 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         tc_fence_before();
         if (__syncthreads_or(ld_volatile(&s_flags[0]) != 0)) break;
 
+        // the item after the next one, claimed while the compute threads invert (the atomic's
+        // latency stays off their path); read by all after the following barriers
+        if (ctl) s_items[2] = nxt >= 0 ? claim() : -1;
         if (compute) {
             invert_unit_lower(LTp, PBp, sm + TT, s_beta, tid);
             fence_proxy_async_smem();
