@@ -580,12 +580,6 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         if (gate < 0 || stop) break;
         const bool safe = gate == 1;
         if (ctl) {
-            // V of this chunk; q/k and log_alpha of the next one (the gating is done with them)
-            issue_v(item);
-            if (nxt >= 0) {
-                issue_qk(nxt, b ^ 1);
-                issue_la(nxt);
-            }
             tc_fence_after();
             if (!safe) {
 #pragma unroll
@@ -594,6 +588,12 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                                 desc_k(sb + KI, 8192, kk), I_D1, kk > 0);
             }
             mma_commit(&bars[4]);
+            // V of this chunk; q/k and log_alpha of the next one (the gating is done with them)
+            issue_v(item);
+            if (nxt >= 0) {
+                issue_qk(nxt, b ^ 1);
+                issue_la(nxt);
+            }
         }
         pend_v = true;
         if (nxt >= 0) pend_qk[b ^ 1] = pend_la = true;
