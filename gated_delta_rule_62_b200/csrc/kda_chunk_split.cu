@@ -601,7 +601,9 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         tc_fence_after();
         if (compute && !safe) extract_al(tmem + lane_base + TM_D1 + 32 * half, sm + AQK, LTp, s_beta, 32 * quad + lane, half);
         tc_fence_before();
-        if (__syncthreads_or(ld_volatile(&s_flags[0]) != 0)) break;
+        // L and A to the inverse: a barrier of the compute threads only (the control thread is
+        // still issuing the prefetches); the CTA-wide stop check follows the inverse
+        if (compute) sync_compute();
 
         // the item after the next one, claimed while the compute threads invert (the atomic's
         // latency stays off their path); read by all after the following barriers
@@ -610,7 +612,7 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             invert_unit_lower(LTp, PBp, sm + TT, s_beta, tid);
             fence_proxy_async_smem();
         }
-        __syncthreads();
+        if (__syncthreads_or(ld_volatile(&s_flags[0]) != 0)) break;
 
         if (ctl) {
             tc_fence_after();
