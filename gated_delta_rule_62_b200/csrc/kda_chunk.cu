@@ -100,8 +100,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     constexpr int SCOLS = DS / 2;  // TMEM columns of S / U / O per thread (two threads per lane)
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
+    // 1024-byte aligned (128-byte swizzled tiles); offsetting the shared array itself keeps the
+    // accesses in the shared state space (an integer round trip would make them generic)
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float *s_beta = reinterpret_cast<float *>(sm + SM::MISC);  // [64]
     float *s_gamma = s_beta + 64;                               // [128]
     float *s_psum = s_gamma + 128;                              // [4][128]

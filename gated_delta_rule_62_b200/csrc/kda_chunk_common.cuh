@@ -148,7 +148,8 @@ __device__ __forceinline__ void frag_to_tt(uint8_t *TT, int r0, int c0, const fl
 // C^-1]] at 16 and then at 32, on the tensor cores (tf32 mma.sync). LT keeps the fp32 blocks
 // later stages need. Called by the NT compute threads (synchronised among themselves with
 // sync_compute); ends with the TT stores issued (no barrier).
-static __device__ void invert_unit_lower(float *LT, float *PB, uint8_t *TT, const float *beta, int tid) {
+static __device__ __forceinline__ void invert_unit_lower(float *LT, float *PB, uint8_t *TT, const float *beta,
+                                                         int tid) {
     const int warp = tid >> 5, lane = tid & 31;
     if (warp < 4 && lane < 16) {
         const int b0 = 16 * warp;

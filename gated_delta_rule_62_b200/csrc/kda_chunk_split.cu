@@ -754,8 +754,9 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
              const __grid_constant__ CUtensorMap tm_rl, const __grid_constant__ CUtensorMap tm_rs,
              const SplitParams p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
+    // 1024-byte aligned (128-byte swizzled tiles); offsetting the shared array itself keeps the
+    // accesses in the shared state space (an integer round trip would make them generic)
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     if ((int)blockIdx.x < p.heads)
         consumer(&tm_rl, p, sm, blockIdx.x);
     else
