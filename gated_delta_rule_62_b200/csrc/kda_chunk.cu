@@ -56,7 +56,7 @@ struct Smem {
     static constexpr uint32_t LT = LA + 32768;              // L -> T fp32 [64][LT_LD]
     static constexpr uint32_t PB = LT + 64 * LT_LD * 4;     // 32 x PB_LD fp32
     static constexpr uint32_t MISC = PB + 32 * PB_LD * 4;   // beta, gamma, psum, flags, barriers
-    static constexpr uint32_t MISC_BYTES = 64 * 4 + 128 * 4 + 4 * 128 * 4 + 64 + 64;
+    static constexpr uint32_t MISC_BYTES = 64 * 4 + 128 * 4 + 8 * 128 * 4 + 64 + 64;
     static constexpr uint32_t BYTES = MISC + MISC_BYTES + 1024;  // + alignment slack
 };
 
@@ -105,8 +105,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float *s_beta = reinterpret_cast<float *>(sm + SM::MISC);  // [64]
     float *s_gamma = s_beta + 64;                               // [128]
-    float *s_psum = s_gamma + 128;                              // [4][128]
-    uint32_t *s_flags = reinterpret_cast<uint32_t *>(s_psum + 512);  // abort, exact path, tmem
+    float *s_psum = s_gamma + 128;                              // [8][128]
+    uint32_t *s_flags = reinterpret_cast<uint32_t *>(s_psum + 1024);  // abort, exact path, tmem
     uint64_t *bars = reinterpret_cast<uint64_t *>(s_flags + 16);     // qk, la, v, mma
     uint64_t *bar_qk = bars, *bar_la = bars + 1, *bar_v = bars + 2, *bar_mma = bars + 3;
     float *LA = reinterpret_cast<float *>(sm + SM::LA);

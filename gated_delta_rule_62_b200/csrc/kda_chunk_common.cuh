@@ -213,7 +213,8 @@ static __device__ __forceinline__ void invert_unit_lower(float *LT, float *PB, u
 // 16 KB blocks, LA the chunk's raw log_alpha [t][c] fp32, s_beta the chunk's beta (0 past `valid`).
 // Out: QK holds Q~ and K~ in place, KI holds K- (factored path) or K^ (exact path), s_gamma =
 // e^(g_{C-1}); the exact path also writes A into AQK and beta-scaled L into LT (zeros elsewhere).
-// Thread mapping: channel pair (cA, cA + 1), token quarter tq (tokens 16 tq .. 16 tq + 15).
+// Thread mapping: channels 4 lane .. 4 lane + 3, token octet = warp (tokens 8 warp .. 8 warp + 7);
+// s_psum holds [8][D] floats.
 // If KH is not null it also receives K^ = k e^(g_{C-1} - g) on both paths. If src_free is not
 // null, the writes to KI, KH and AQK first wait (bounded by timeout_ns) for that mbarrier's
 // phase with parity src_parity: another thread may still be reading those tiles.
@@ -225,53 +226,63 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
                                           int tid, uint8_t *KH = nullptr,
                                           uint64_t *src_free = nullptr, uint32_t src_parity = 0,
                                           uint64_t timeout_ns = 0) {
-    const int tq = tid >> 6, cA = 2 * (tid & 63);
     const int warp = tid >> 5, lane = tid & 31;
-    // ---- gates: log_alpha of 16 tokens x 2 channels into registers, quarter totals
-    float2 la[16];
-    float2 tot = make_float2(0.f, 0.f);
+    const int to = warp, c4 = 4 * lane;  // token octet 8 to .. 8 to + 7, channels c4 .. c4 + 3
+    // ---- gates: log_alpha of 8 tokens x 4 channels into registers, octet totals
+    float4 la[8];
+    float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int t = 16 * tq + i;
-        la[i] = (t < valid) ? *reinterpret_cast<const float2 *>(LA + t * D + cA)
-                            : make_float2(0.f, 0.f);
+    for (int i = 0; i < 8; ++i) {
+        const int t = 8 * to + i;
+        la[i] = (t < valid) ? *reinterpret_cast<const float4 *>(LA + t * D + c4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
         tot.x += la[i].x;
         tot.y += la[i].y;
+        tot.z += la[i].z;
+        tot.w += la[i].w;
     }
-    s_psum[tq * D + cA] = tot.x;
-    s_psum[tq * D + cA + 1] = tot.y;
-    // A quarter decaying by more than e^(kFastLimit/4) in some channel sends the chunk
-    // down the exact path; otherwise the whole chunk decays by at most e^kFastLimit.
+    *reinterpret_cast<float4 *>(s_psum + to * D + c4) = tot;
+    // An octet decaying by more than e^(kFastLimit/8) in some channel sends the chunk down the
+    // exact path; otherwise the whole chunk decays by at most e^kFastLimit.
     // (NaN gates also take the exact path: the comparisons are false for NaN.)
-    const int unsafe = !(-tot.x <= 0.25f * kFastLimit) || !(-tot.y <= 0.25f * kFastLimit);
+    const float lim = 0.125f * kFastLimit;
+    const int unsafe = !(-tot.x <= lim) || !(-tot.y <= lim) || !(-tot.z <= lim) || !(-tot.w <= lim);
     const bool safe = sync_compute_or(unsafe) != 0;
     if (*s_abort) return -1;
     if (src_free && !mbar_wait_bounded(src_free, src_parity, timeout_ns)) {
         *s_abort = 1;
         return -1;
     }
-    float2 goff = make_float2(0.f, 0.f), gC = make_float2(0.f, 0.f);
+    float4 goff = make_float4(0.f, 0.f, 0.f, 0.f), gC = goff;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float a = s_psum[q * D + cA], b = s_psum[q * D + cA + 1];
-        if (q < tq) { goff.x += a; goff.y += b; }
-        gC.x += a;
-        gC.y += b;
+    for (int o = 0; o < 8; ++o) {
+        const float4 a = *reinterpret_cast<const float4 *>(s_psum + o * D + c4);
+        if (o < to) {
+            goff.x += a.x;
+            goff.y += a.y;
+            goff.z += a.z;
+            goff.w += a.w;
+        }
+        gC.x += a.x;
+        gC.y += a.y;
+        gC.z += a.z;
+        gC.w += a.w;
     }
-    if (tq == 0) {
-        s_gamma[cA] = __expf(gC.x);
-        s_gamma[cA + 1] = __expf(gC.y);
-    }
+    if (to == 0)
+        *reinterpret_cast<float4 *>(s_gamma + c4) =
+            make_float4(__expf(gC.x), __expf(gC.y), __expf(gC.z), __expf(gC.w));
 
     if (safe) {
         // Exact path: A and L pairwise from raw q, k and the full g (no factored exponentials).
         {
-            float2 g = goff;
+            float4 g = goff;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
+            for (int i = 0; i < 8; ++i) {
                 g.x += la[i].x;
                 g.y += la[i].y;
-                *reinterpret_cast<float2 *>(LA + (16 * tq + i) * D + cA) = g;
+                g.z += la[i].z;
+                g.w += la[i].w;
+                *reinterpret_cast<float4 *>(LA + (8 * to + i) * D + c4) = g;
             }
         }
         for (int e = tid; e < 64 * 64; e += NT) {
@@ -306,47 +317,64 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
     }
 
     // ---- gated operands. With alpha = e^log_alpha, prefix products P_i and suffix
-    // products R_i (within the quarter): e^g_i = e^goff P_i; e^-g_i = e^(-goff-tot) R_i;
+    // products R_i (within the octet): e^g_i = e^goff P_i; e^-g_i = e^(-goff-tot) R_i;
     // e^(g_C - g_i) = e^(g_C-goff-tot) R_i. Q~, K~ overwrite q, k in place; the KI tile
     // gets K- (fast path) or K^ (exact path).
     {
-        float2 al[16];
+        float4 al[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) al[i] = make_float2(__expf(la[i].x), __expf(la[i].y));
-        const float2 eA = make_float2(__expf(goff.x), __expf(goff.y));
-        const float2 eH = make_float2(__expf(gC.x - goff.x - tot.x), __expf(gC.y - goff.y - tot.y));
-        const float2 eB = safe ? eH : make_float2(__expf(-goff.x - tot.x), __expf(-goff.y - tot.y));
-        float2 R[16];
-        float2 run = make_float2(1.f, 1.f);
+        for (int i = 0; i < 8; ++i)
+            al[i] = make_float4(__expf(la[i].x), __expf(la[i].y), __expf(la[i].z), __expf(la[i].w));
+        const float4 eA = make_float4(__expf(goff.x), __expf(goff.y), __expf(goff.z), __expf(goff.w));
+        const float4 eH = make_float4(__expf(gC.x - goff.x - tot.x), __expf(gC.y - goff.y - tot.y),
+                                      __expf(gC.z - goff.z - tot.z), __expf(gC.w - goff.w - tot.w));
+        const float4 eB = safe ? eH
+                               : make_float4(__expf(-goff.x - tot.x), __expf(-goff.y - tot.y),
+                                             __expf(-goff.z - tot.z), __expf(-goff.w - tot.w));
+        float4 R[8];
+        float4 run = make_float4(1.f, 1.f, 1.f, 1.f);
 #pragma unroll
-        for (int i = 15; i >= 0; --i) {
+        for (int i = 7; i >= 0; --i) {
             R[i] = run;
             run.x *= al[i].x;
             run.y *= al[i].y;
+            run.z *= al[i].z;
+            run.w *= al[i].w;
         }
-        // Token t = 16 tq + i: with i known at compile time, t & 7 = i & 7 and t >> 3 = 2 tq + i / 8,
-        // so telem(bs, t, cA) = base_bs + (i / 8) 1024 + (i & 7) 128 + ((cx ^ (i & 7)) << 4):
-        // one XOR per token instead of a full swizzle per tile.
-        const uint32_t cx = (uint32_t)(cA & 63) >> 3;
-        const uint32_t row0 = (uint32_t)(2 * tq) * 1024 + (uint32_t)(cA & 7) * 2;
-        uint8_t *const q0 = QK + (uint32_t)(cA >> 6) * 16384 + row0;  // K~ rows: + 8 row groups
-        uint8_t *const i0 = KI + (uint32_t)(cA >> 6) * 8192 + row0;
-        uint8_t *const h0 = KH ? KH + (uint32_t)(cA >> 6) * 8192 + row0 : nullptr;
-        float2 P = eA;
+        // Token t = 8 to + i: t >> 3 = to and t & 7 = i (known at compile time), so
+        // telem(bs, t, c4) = base_bs + to 1024 + i 128 + ((cx ^ i) << 4) + (c4 & 7) 2; K~ rows
+        // (64 + t) sit 8 row groups further. Four channels = one 8-byte access.
+        const uint32_t cx = (uint32_t)(c4 & 63) >> 3;
+        const uint32_t row0 = (uint32_t)to * 1024 + (uint32_t)(c4 & 7) * 2;
+        uint8_t *const q0 = QK + (uint32_t)(c4 >> 6) * 16384 + row0;
+        uint8_t *const i0 = KI + (uint32_t)(c4 >> 6) * 8192 + row0;
+        uint8_t *const h0 = KH ? KH + (uint32_t)(c4 >> 6) * 8192 + row0 : nullptr;
+        auto unpack4 = [](uint2 u) {
+            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+            const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+            return make_float4(a.x, a.y, b.x, b.y);
+        };
+        auto pack4 = [](float a, float b, float c, float d) { return make_uint2(pack2(a, b), pack2(c, d)); };
+        float4 P = eA;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int t = 16 * tq + i;
+        for (int i = 0; i < 8; ++i) {
+            const int t = 8 * to + i;
             P.x *= al[i].x;
             P.y *= al[i].y;
-            const uint32_t off = (uint32_t)(i >> 3) * 1024 + (uint32_t)(i & 7) * 128 + ((cx ^ (uint32_t)(i & 7)) << 4);
-            uint8_t *qp = q0 + off;
-            uint8_t *kp = q0 + 8192 + off;
-            float2 qv = ld_bf2(qp), kv = ld_bf2(kp);
-            if (t >= valid) qv = kv = make_float2(0.f, 0.f);
-            st_bf2(qp, qv.x * P.x, qv.y * P.y);
-            st_bf2(kp, kv.x * P.x, kv.y * P.y);
-            st_bf2(i0 + off, kv.x * (eB.x * R[i].x), kv.y * (eB.y * R[i].y));
-            if (KH) st_bf2(h0 + off, kv.x * (eH.x * R[i].x), kv.y * (eH.y * R[i].y));
+            P.z *= al[i].z;
+            P.w *= al[i].w;
+            const uint32_t off = (uint32_t)i * 128 + ((cx ^ (uint32_t)i) << 4);
+            uint2 *qp = reinterpret_cast<uint2 *>(q0 + off);
+            uint2 *kp = reinterpret_cast<uint2 *>(q0 + 8192 + off);
+            float4 qv = unpack4(*qp), kv = unpack4(*kp);
+            if (t >= valid) qv = kv = make_float4(0.f, 0.f, 0.f, 0.f);
+            *qp = pack4(qv.x * P.x, qv.y * P.y, qv.z * P.z, qv.w * P.w);
+            *kp = pack4(kv.x * P.x, kv.y * P.y, kv.z * P.z, kv.w * P.w);
+            *reinterpret_cast<uint2 *>(i0 + off) =
+                pack4(kv.x * (eB.x * R[i].x), kv.y * (eB.y * R[i].y), kv.z * (eB.z * R[i].z), kv.w * (eB.w * R[i].w));
+            if (KH)
+                *reinterpret_cast<uint2 *>(h0 + off) =
+                    pack4(kv.x * (eH.x * R[i].x), kv.y * (eH.y * R[i].y), kv.z * (eH.z * R[i].z), kv.w * (eH.w * R[i].w));
         }
     }
     return safe ? 1 : 0;

@@ -391,7 +391,7 @@ constexpr uint32_t AQK = ZB + 8192;       // A [i][j]    /
 constexpr uint32_t LT = AQK + 8192;       // L -> T fp32 [64][LT_LD]
 constexpr uint32_t PB = LT + 64 * LT_LD * 4;   // 32 x PB_LD fp32
 constexpr uint32_t MISC = PB + 32 * PB_LD * 4; // beta, gamma, psum, flags, barriers
-constexpr uint32_t BYTES = MISC + 64 * 4 + 128 * 4 + 4 * 128 * 4 + 64 + 64;
+constexpr uint32_t BYTES = MISC + 64 * 4 + 128 * 4 + 8 * 128 * 4 + 64 + 64;
 // TMEM: D1 = [Q~; K~] K-^T (M=128, 64 columns), W (M=64), D3 = [U~; -A W], D4 = -K^^T W
 constexpr uint32_t TM_D1 = 0, TM_W = 128, TM_D3 = 256, TM_D4 = 384, TM_COLS = 512;
 }  // namespace prod
@@ -410,7 +410,7 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     float *s_beta = reinterpret_cast<float *>(sm + MISC);
     float *s_gamma = s_beta + 64;
     float *s_psum = s_gamma + 128;
-    uint32_t *s_flags = reinterpret_cast<uint32_t *>(s_psum + 512);  // abort, tmem, gate
+    uint32_t *s_flags = reinterpret_cast<uint32_t *>(s_psum + 1024);  // abort, tmem, gate
     uint64_t *bars = reinterpret_cast<uint64_t *>(s_flags + 16);     // qk0, qk1, la, v, mma, src
     float *LTp = reinterpret_cast<float *>(sm + LT);
     float *PBp = reinterpret_cast<float *>(sm + PB);
