@@ -45,8 +45,8 @@ FLOP_PER_TOKEN_HEAD = 180224
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
 # dram__bytes_read.sum + dram__bytes_write.sum of one split_kernel launch on the headline workload,
 # from one ncu capture; reported only while the kernel's sources are the ones it was taken on.
-SPLIT_TRAFFIC_BYTES = 336.796416e6 + 58.295296e6
-SPLIT_TRAFFIC_SOURCES_SHA256 = "7283eb3cd2f47f9e861eba22aa5f8710354c45cde78690ecf95cdd03e0cd4afa"
+SPLIT_TRAFFIC_BYTES = 336.77824e6 + 57.831168e6
+SPLIT_TRAFFIC_SOURCES_SHA256 = "ad76fc8b96f411c8e64351c7abf0317f80067a5e31cf1b36c101f9c877711a8c"
 
 
 def measured_traffic():
