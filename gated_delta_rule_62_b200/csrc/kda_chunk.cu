@@ -157,6 +157,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         tma_load_3d(sm + SM::QK + 24576, &tm_k, bar_qk, 64, h, (int32_t)t0);
     };
     auto issue_la = [&](int64_t t0) {
+        fence_proxy_async_smem();  // the previous contents were read by generic loads
         mbar_arrive_expect_tx(bar_la, 32768);
         tma_load_3d(sm + SM::LA, &tm_la, bar_la, 0, h, (int32_t)t0);
     };
@@ -254,7 +255,6 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         __syncthreads();
 
         if (tid == 0) {
-            if (has_next) issue_la(t0 + C);
             tc_fence_after();
             if (!safe) {
 #pragma unroll
@@ -269,6 +269,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                                 desc_mn(sb + SM::S, 16384, kk), I_UT, kk > 0);
             }
             mma_commit(bar_mma);
+            if (has_next) issue_la(t0 + C);  // the gating is done with log_alpha
         }
         la_pending = has_next;
         wait_bar(bar_mma, ph_mma);
@@ -360,12 +361,16 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
         // ---- outputs (O: M=64 rows) and the next state (S *= gamma on the fast path)
         {
-            float v[32];
+            constexpr int NPART = SCOLS / 32;
+            float vv[NPART][32];  // every 32-column load in flight before one wait
 #pragma unroll
-            for (int part = 0; part < SCOLS / 32; ++part) {
+            for (int part = 0; part < NPART; ++part)
+                tmem_ld32(tmem + lane_base + TM::O + half * SCOLS + 32 * part, vv[part]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int part = 0; part < NPART; ++part) {
                 const int col = half * SCOLS + 32 * part;
-                tmem_ld32(tmem + lane_base + TM::O + col, v);
-                tmem_wait_ld();
+                const float *v = vv[part];
                 const int i = 16 * quad + lane;
                 if (lane < 16 && i < valid) {
                     uint4 *dst = reinterpret_cast<uint4 *>(
@@ -380,14 +385,17 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             }
             const float gm = safe ? 1.f : s_gamma[c_me];
 #pragma unroll
-            for (int part = 0; part < SCOLS / 32; ++part) {
+            for (int part = 0; part < NPART; ++part)
+                tmem_ld32(tmem + lane_base + TM::S + half * SCOLS + 32 * part, vv[part]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int part = 0; part < NPART; ++part) {
                 const int col = half * SCOLS + 32 * part;
                 const uint32_t ta = tmem + lane_base + TM::S + col;
-                tmem_ld32(ta, v);
-                tmem_wait_ld();
+                float *v = vv[part];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) v[e] *= gm;
-                if (!safe) tmem_st32(ta, v);
+                if (!safe) tmem_st32(ta, vv[part]);
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8)
                     st_chunk(sm + SM::S + tchunk(16384, c_me, col + 8 * q8), v + 8 * q8);
