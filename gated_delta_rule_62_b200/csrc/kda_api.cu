@@ -37,8 +37,6 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 constexpr size_t kStatusBytes = 256;
 
-size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
 // Checks shared by the prefill entry points. On success returns KDA_OK.
 kda_status_t check_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
                            const float *beta, const float *initial_state,
@@ -96,6 +94,41 @@ kda::Problem make_problem(const void *q, const void *k, const void *v, const flo
     return p;
 }
 
+// Workspace check and kernel choice shared by kda_prefill and kda_prefill_slots.
+kda_status_t run_prefill(kda::Problem &p, const int32_t *cu_seqlens_host, void *workspace,
+                         size_t workspace_bytes, cudaStream_t s, const char *who) {
+    // Any workspace of the minimum size is accepted; a larger one (as sized by
+    // kda_prefill_workspace_size) lets few-head problems use the split-role kernel.
+    const size_t need = kda::chunk_workspace_bytes(p.num_seqs);
+    if (!workspace || workspace_bytes < need)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "workspace %p of %zu bytes < required %zu",
+                    workspace, workspace_bytes, need);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "workspace is not 256-byte aligned");
+    cudaError_t e;
+    int32_t max_chunks = 0;
+    for (int32_t n = 0; n < p.num_seqs; ++n) {
+        const int32_t c = (cu_seqlens_host[n + 1] - cu_seqlens_host[n] + 63) / 64;
+        max_chunks = c > max_chunks ? c : max_chunks;
+    }
+    const int64_t heads = (int64_t)p.num_seqs * p.H;
+    if (kda::chunk_supported(p) && max_chunks >= 2 && kda::split_eligible(heads, p.dtype, p.dk, p.dv) &&
+        kda::split_eligible_seqs(p.num_seqs) &&
+        workspace_bytes >= kda::split_workspace_bytes(heads)) {
+        // few heads: consumer CTAs run the state chains, producer CTAs fill the other SMs
+        e = kda::launch_prefill_split(p, max_chunks, workspace, s, kda::kWaitTimeoutNs);
+    } else if (kda::chunk_supported(p)) {
+        // the planning kernel clears the status word
+        e = kda::launch_prefill_chunk(p, workspace, s, kda::kWaitTimeoutNs);
+    } else {
+        e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
+        p.slots.status = static_cast<int32_t *>(workspace);
+        if (e == cudaSuccess) e = kda::launch_prefill_recurrent(p, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, who);
+    return ok();
+}
+
 }  // namespace
 
 namespace kda {
@@ -130,38 +163,39 @@ kda_status_t kda_prefill(const void *q, const void *k, const void *v, const floa
                                     cu_seqlens_host, num_seqs, total_tokens, H, d_k, d_v, dtype,
                                     out, final_state);
     if (st != KDA_OK || num_seqs == 0) return st;
-    // Any workspace of the minimum size is accepted; a larger one (as sized by
-    // kda_prefill_workspace_size) lets few-head problems use the split-role kernel.
-    const size_t need = kda::chunk_workspace_bytes(num_seqs);
-    if (!workspace || workspace_bytes < need)
-        return fail(KDA_ERR_INVALID_ARGUMENT, "workspace %p of %zu bytes < required %zu",
-                    workspace, workspace_bytes, need);
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-        return fail(KDA_ERR_INVALID_ARGUMENT, "workspace is not 256-byte aligned");
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     kda::Problem p = make_problem(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev,
                                   num_seqs, total_tokens, H, d_k, d_v, dtype, out, final_state);
-    cudaError_t e;
-    int32_t max_chunks = 0;
-    for (int32_t n = 0; n < num_seqs; ++n) {
-        const int32_t c = (cu_seqlens_host[n + 1] - cu_seqlens_host[n] + 63) / 64;
-        max_chunks = c > max_chunks ? c : max_chunks;
-    }
-    const int64_t heads = (int64_t)num_seqs * H;
-    if (kda::chunk_supported(p) && max_chunks >= 2 && kda::split_eligible(heads, dtype, d_k, d_v) &&
-        kda::split_eligible_seqs(num_seqs) &&
-        workspace_bytes >= kda::split_workspace_bytes(heads)) {
-        // few heads: consumer CTAs run the state chains, producer CTAs fill the other SMs
-        e = kda::launch_prefill_split(p, max_chunks, workspace, s, kda::kWaitTimeoutNs);
-    } else if (kda::chunk_supported(p)) {
-        // the planning kernel clears the status word
-        e = kda::launch_prefill_chunk(p, workspace, s, kda::kWaitTimeoutNs);
-    } else {
-        e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
-        if (e == cudaSuccess) e = kda::launch_prefill_recurrent(p, s);
-    }
-    if (e != cudaSuccess) return cuda_fail(e, "kda_prefill: launch");
-    return ok();
+    return run_prefill(p, cu_seqlens_host, workspace, workspace_bytes,
+                       reinterpret_cast<cudaStream_t>(stream), "kda_prefill: launch");
+}
+
+kda_status_t kda_prefill_slots(const void *q, const void *k, const void *v, const float *log_alpha,
+                               const float *beta, float *state_pool, int64_t pool_slots,
+                               const int32_t *init_slot_dev, const int32_t *final_slot_dev,
+                               const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                               int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
+                               int32_t d_v, kda_dtype_t dtype, void *out, void *workspace,
+                               size_t workspace_bytes, kda_stream_t stream) {
+    if (pool_slots < 0 || pool_slots > INT32_MAX)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "pool_slots=%lld outside [0, 2^31)", (long long)pool_slots);
+    if (pool_slots > 0 && !state_pool)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "state_pool is NULL with pool_slots=%lld",
+                    (long long)pool_slots);
+    kda_status_t st = check_prefill(q, k, v, log_alpha, beta, state_pool, cu_seqlens_dev,
+                                    cu_seqlens_host, num_seqs, total_tokens, H, d_k, d_v, dtype,
+                                    out, state_pool);
+    if (st != KDA_OK || num_seqs == 0) return st;
+    if (!init_slot_dev || !final_slot_dev)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "init_slot_dev and final_slot_dev are required");
+    if (state_pool && out == (void *)state_pool)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "out must not alias the state pool");
+    kda::Problem p = make_problem(q, k, v, log_alpha, beta, state_pool, cu_seqlens_dev, num_seqs,
+                                  total_tokens, H, d_k, d_v, dtype, out, state_pool);
+    p.slots.init_slot = init_slot_dev;
+    p.slots.final_slot = final_slot_dev;
+    p.slots.slots = pool_slots;
+    return run_prefill(p, cu_seqlens_host, workspace, workspace_bytes,
+                       reinterpret_cast<cudaStream_t>(stream), "kda_prefill_slots: launch");
 }
 
 kda_status_t kda_prefill_recurrent(const void *q, const void *k, const void *v,
@@ -213,6 +247,51 @@ kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const 
     return ok();
 }
 
+kda_status_t kda_decode_step_slots(const void *q, const void *k, const void *v,
+                                   const float *log_alpha, const float *beta, float *state_pool,
+                                   int64_t pool_slots, const int32_t *slot_dev, int32_t num_seqs,
+                                   int32_t H, int32_t d_k, int32_t d_v, kda_dtype_t dtype,
+                                   void *out, void *workspace, size_t workspace_bytes,
+                                   kda_stream_t stream) {
+    if (pool_slots < 0 || pool_slots > INT32_MAX)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "pool_slots=%lld outside [0, 2^31)", (long long)pool_slots);
+    if (dtype != KDA_F32 && dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "dtype %d is not KDA_F32 or KDA_BF16", (int)dtype);
+    if (H <= 0) return fail(KDA_ERR_INVALID_ARGUMENT, "H=%d <= 0", H);
+    if (!supported_d(d_k) || !supported_d(d_v))
+        return fail(KDA_ERR_INVALID_ARGUMENT, "d_k=%d, d_v=%d: each must be 32, 64 or 128", d_k, d_v);
+    if (num_seqs < 0) return fail(KDA_ERR_INVALID_ARGUMENT, "num_seqs=%d < 0", num_seqs);
+    if ((int64_t)num_seqs * H > INT32_MAX)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "num_seqs * H exceeds 2^31 - 1");
+    if (num_seqs == 0) return ok();
+    if (!q || !k || !v || !log_alpha || !beta || !out || !slot_dev)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "q, k, v, log_alpha, beta, slot_dev and out are required");
+    if (pool_slots > 0 && !state_pool)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "state_pool is NULL with pool_slots=%lld",
+                    (long long)pool_slots);
+    if (!workspace || workspace_bytes < kStatusBytes ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "a 256-byte aligned workspace of >= %zu bytes is required",
+                    kStatusBytes);
+    const void *ptrs[] = {q, k, v, log_alpha, state_pool, out};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned16(ptr))
+            return fail(KDA_ERR_INVALID_ARGUMENT, "tensor pointer %p is not 16-byte aligned", ptr);
+    if (out == q || out == k || out == v || (state_pool && out == (void *)state_pool))
+        return fail(KDA_ERR_INVALID_ARGUMENT, "out must not alias an input or the state pool");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    kda::DecodeProblem p;
+    p.q = q; p.k = k; p.v = v; p.log_alpha = log_alpha; p.beta = beta; p.state = state_pool;
+    p.num_seqs = num_seqs; p.H = H; p.dk = d_k; p.dv = d_v; p.dtype = dtype; p.out = out;
+    p.slots.init_slot = p.slots.final_slot = slot_dev;
+    p.slots.slots = pool_slots;
+    p.slots.status = static_cast<int32_t *>(workspace);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
+    if (e == cudaSuccess) e = kda::launch_decode(p, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step_slots: launch");
+    return ok();
+}
+
 const char *kda_status_string(kda_status_t s) {
     switch (s) {
         case KDA_OK: return "KDA_OK";
@@ -234,6 +313,9 @@ kda_status_t kda_read_device_status(const void *workspace, kda_stream_t stream) 
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "kda_read_device_status");
     if (word == 0) return ok();
+    if (word & kda::kStatusBadSlot)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "device status word 0x%x: a state slot was outside "
+                    "[-1, pool_slots)", (unsigned)word);
     return fail(KDA_ERR_TIMEOUT, "device status word 0x%x: a bounded on-device wait gave up",
                 (unsigned)word);
 }

@@ -76,12 +76,13 @@ struct ChunkParams {
     const int32_t *cu_seqlens;
     const int32_t *order;  // sequences, longest first
     const float *beta;
-    const float *s0;
-    float *sT;
+    const float *s0;  // initial states, or the state pool
+    float *sT;        // final states, or the state pool
     __nv_bfloat16 *out;
     int32_t *status;
     int32_t H;
     uint64_t timeout_ns;
+    StateSlots ss;
 };
 
 template <int DS>
@@ -125,7 +126,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const int d0 = split * DS;  // first value channel of this CTA
     const int64_t bos = p.cu_seqlens[n], eos = p.cu_seqlens[n + 1];
     const int nchunks = (int)((eos - bos + C - 1) / C);
-    const size_t state_off = ((size_t)n * H + h) * (size_t)(D * D);
+    const float *s0b = init_state_block(p.s0, n, H, h, (size_t)D * D, p.ss);
+    float *sTb = final_state_block(p.sT, n, H, h, (size_t)D * D, p.ss);
     const int c_me = 32 * quad + lane;  // key channel = TMEM lane of this thread
 
     if (tid == 0) {
@@ -183,9 +185,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
     // Initial state -> S (TMEM fp32, lane c, columns d) and its bf16 tile [c][d].
     {
-        const size_t row = state_off + (size_t)c_me * D + d0 + half * SCOLS;
-        const float *src = p.s0 ? p.s0 + row : nullptr;
-        float *dst = p.sT ? p.sT + row : nullptr;
+        const size_t row = (size_t)c_me * D + d0 + half * SCOLS;
+        const float *src = s0b ? s0b + row : nullptr;
+        float *dst = sTb ? sTb + row : nullptr;
 #pragma unroll
         for (int part = 0; part < SCOLS / 32; ++part) {
             float v[32];
@@ -399,8 +401,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8)
                     st_chunk(sm + SM::S + tchunk(16384, c_me, col + 8 * q8), v + 8 * q8);
-                if (!has_next && p.sT) {
-                    float *dst = p.sT + state_off + (size_t)c_me * D + d0 + col;
+                if (!has_next && sTb) {
+                    float *dst = sTb + (size_t)c_me * D + d0 + col;
 #pragma unroll
                     for (int e = 0; e < 32; e += 4)
                         *reinterpret_cast<float4 *>(dst + e) =
@@ -573,6 +575,8 @@ cudaError_t launch_prefill_chunk(const Problem &p, void *workspace, cudaStream_t
     cp.sT = p.final_state;
     cp.out = static_cast<__nv_bfloat16 *>(p.out);
     cp.status = status;
+    cp.ss = p.slots;
+    cp.ss.status = status;
     cp.H = p.H;
     cp.timeout_ns = timeout_ns;
     const unsigned grid = (unsigned)(heads * nsplit);

@@ -57,10 +57,11 @@ static_assert(SLOT % ROW_BYTES == 0 && RL_BOX <= 256, "ring load box");
 struct SplitParams {
     const int32_t *cu_seqlens;
     const float *beta;
-    const float *s0;
-    float *sT;
+    const float *s0;  // initial states, or the state pool
+    float *sT;        // final states, or the state pool
     __nv_bfloat16 *out;
     int32_t *status;
+    StateSlots ss;
     uint8_t *ring;       // [heads][RING][SLOT]
     int32_t *filled;     // [heads][RING]
     int32_t *consumed;   // [heads]
@@ -153,7 +154,8 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
     const int H = p.H, n = hd / H, h = hd % H;
     const int64_t bos = p.cu_seqlens[n], eos = p.cu_seqlens[n + 1];
     const int nchunks = (int)((eos - bos + C - 1) / C);
-    const size_t state_off = ((size_t)n * H + h) * (size_t)(D * D);
+    const float *s0b = init_state_block(p.s0, n, H, h, (size_t)D * D, p.ss);
+    float *sTb = final_state_block(p.sT, n, H, h, (size_t)D * D, p.ss);
 
     if (tid == 0) {
         s_flags[0] = 0;
@@ -281,12 +283,12 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             float v[2][32];
-            const float *src = p.s0 ? p.s0 + state_off + (size_t)(64 * hh) * D + d_me : nullptr;
+            const float *src = s0b ? s0b + (size_t)(64 * hh) * D + d_me : nullptr;
 #pragma unroll
             for (int e = 0; e < 64; ++e) v[e >> 5][e & 31] = src ? src[(size_t)e * D] : 0.f;
             if (nchunks == 0) {
-                if (p.sT) {
-                    float *dst = p.sT + state_off + (size_t)(64 * hh) * D + d_me;
+                if (sTb) {
+                    float *dst = sTb + (size_t)(64 * hh) * D + d_me;
 #pragma unroll
                     for (int e = 0; e < 64; ++e) dst[(size_t)e * D] = v[e >> 5][e & 31];
                 }
@@ -317,8 +319,8 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
                 tmem_wait_ld();
                 if (!last) {
                     pack_store(v, hh, b ? TM_SB0 : TM_SB1);  // the next chunk's copy
-                } else if (p.sT) {
-                    float *dst = p.sT + state_off + (size_t)(64 * hh) * D + d_me;
+                } else if (sTb) {
+                    float *dst = sTb + (size_t)(64 * hh) * D + d_me;
 #pragma unroll
                     for (int e = 0; e < 64; ++e) dst[(size_t)e * D] = v[e >> 5][e & 31];
                 }
@@ -832,6 +834,8 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
     sp.beta = p.beta;
     sp.s0 = p.initial_state;
     sp.sT = p.final_state;
+    sp.ss = p.slots;
+    sp.ss.status = status;
     sp.out = static_cast<__nv_bfloat16 *>(p.out);
     sp.status = status;
     sp.filled = flags;

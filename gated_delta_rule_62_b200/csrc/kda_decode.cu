@@ -30,7 +30,7 @@ template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
 decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta,
-              float *__restrict__ state, Tin *__restrict__ out) {
+              float *__restrict__ state, Tin *__restrict__ out, int H, const StateSlots ss) {
     using Sh = DecodeShape<DK, DV>;
     constexpr int CG = Sh::CG, NT = Sh::NT, R = Sh::R, RPT = Sh::RPT;
     __shared__ float s_k[DK], s_q[DK], s_a[DK];
@@ -41,12 +41,15 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     const size_t head = blockIdx.x;  // n * H + h
     const int tid = threadIdx.x;
     const int cg = tid % CG, rg = tid / CG;
-    float4 *S4 = reinterpret_cast<float4 *>(state + head * (size_t)(DK * DV));
+    // this head's state: entry `head`, or its sequence's slot of the pool (none: zeros, not stored)
+    float *blk = final_state_block(state, (int)(head / H), H, (int)(head % H), (size_t)(DK * DV), ss);
+    float4 *S4 = reinterpret_cast<float4 *>(blk);
 
     // Issue the state loads first: they are the only long-latency traffic.
     float4 s[RPT];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) s[i] = __ldcs(&S4[(size_t)(rg + i * R) * CG + cg]);
+    for (int i = 0; i < RPT; ++i)
+        s[i] = blk ? __ldcs(&S4[(size_t)(rg + i * R) * CG + cg]) : make_float4(0.f, 0.f, 0.f, 0.f);
 
     for (int c = tid; c < DK; c += NT) {
         s_k[c] = to_f32(k[head * DK + c]);
@@ -93,7 +96,7 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
         const float kc = s_k[rg + i * R];
         s[i].x = fmaf(kc, u4.x, s[i].x); s[i].y = fmaf(kc, u4.y, s[i].y);
         s[i].z = fmaf(kc, u4.z, s[i].z); s[i].w = fmaf(kc, u4.w, s[i].w);
-        __stcs(&S4[(size_t)(rg + i * R) * CG + cg], s[i]);
+        if (blk) __stcs(&S4[(size_t)(rg + i * R) * CG + cg], s[i]);
     }
 }
 
@@ -102,7 +105,7 @@ cudaError_t launch3(const DecodeProblem &p, cudaStream_t stream) {
     const unsigned blocks = (unsigned)p.num_seqs * (unsigned)p.H;
     decode_kernel<Tin, DK, DV><<<blocks, DecodeShape<DK, DV>::NT, 0, stream>>>(
         (const Tin *)p.q, (const Tin *)p.k, (const Tin *)p.v, p.log_alpha, p.beta, p.state,
-        (Tin *)p.out);
+        (Tin *)p.out, p.H, p.slots);
     return cudaGetLastError();
 }
 

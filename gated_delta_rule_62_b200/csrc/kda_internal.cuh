@@ -19,18 +19,52 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// ---- where a sequence's states live ------------------------------------------------------
+// Entry n of initial_state / final_state ([N, H, d_k, d_v]); or, with slot tables, slot
+// init_slot[n] / final_slot[n] of one pool ([slots, H, d_k, d_v]), -1 meaning none. A slot outside
+// [-1, slots) counts as -1 and sets kStatusBadSlot in the device status word.
+constexpr int32_t kStatusTimeout = 1, kStatusBadSlot = 2;
+struct StateSlots {
+    const int32_t *init_slot = nullptr, *final_slot = nullptr;  // device tables (or null)
+    int64_t slots = 0;
+    int32_t *status = nullptr;  // device status word (may be null)
+};
+__device__ __forceinline__ int64_t state_slot(const int32_t *tab, int n, const StateSlots &ss) {
+    if (!tab) return n;
+    const int32_t s = tab[n];
+    if (s < -1 || (int64_t)s >= ss.slots) {
+        if (ss.status) atomicOr(ss.status, kStatusBadSlot);
+        return -1;
+    }
+    return s;
+}
+// Head h's [d_k, d_v] block of sequence n's initial / final state, or null for none.
+__device__ __forceinline__ const float *init_state_block(const float *base, int n, int H, int h,
+                                                         size_t elems, const StateSlots &ss) {
+    if (!base) return nullptr;
+    const int64_t s = state_slot(ss.init_slot, n, ss);
+    return s < 0 ? nullptr : base + ((size_t)s * H + h) * elems;
+}
+__device__ __forceinline__ float *final_state_block(float *base, int n, int H, int h, size_t elems,
+                                                    const StateSlots &ss) {
+    if (!base) return nullptr;
+    const int64_t s = state_slot(ss.final_slot, n, ss);
+    return s < 0 ? nullptr : base + ((size_t)s * H + h) * elems;
+}
+
 // ---- problem description passed from the API layer to the launchers --------------------
 struct Problem {
     const void *q, *k, *v;
     const float *log_alpha, *beta;
-    const float *initial_state;
+    const float *initial_state;  // or the state pool (with slots)
     const int32_t *cu_seqlens;  // device
     int32_t num_seqs;
     int64_t total_tokens;
     int32_t H, dk, dv;
     kda_dtype_t dtype;
     void *out;
-    float *final_state;
+    float *final_state;          // or the state pool (with slots)
+    StateSlots slots;
 };
 
 // Each launcher enqueues its kernel(s) on `stream` and returns the launch's cudaError_t.
@@ -61,10 +95,11 @@ constexpr uint64_t kWaitTimeoutNs = 4000000000ull;
 struct DecodeProblem {
     const void *q, *k, *v;
     const float *log_alpha, *beta;
-    float *state;
+    float *state;  // or the state pool (slots.init_slot == slots.final_slot: the slot table)
     int32_t num_seqs, H, dk, dv;
     kda_dtype_t dtype;
     void *out;
+    StateSlots slots;
 };
 cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream);
 

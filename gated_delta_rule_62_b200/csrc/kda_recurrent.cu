@@ -23,8 +23,8 @@ template <typename Tin, int DK>
 __global__ void __launch_bounds__(128)
 recurrent_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                  const float *__restrict__ log_alpha, const float *__restrict__ beta,
-                 const float *__restrict__ s0, const int32_t *__restrict__ cu_seqlens, int H,
-                 int dv, Tin *__restrict__ out, float *__restrict__ sT) {
+                 const float *s0, const int32_t *__restrict__ cu_seqlens, int H,
+                 int dv, Tin *__restrict__ out, float *sT, const StateSlots ss) {
     constexpr int R = DK / 32;  // key rows per lane
     const int n = blockIdx.x, h = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -32,12 +32,12 @@ recurrent_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin
     const int64_t bos = cu_seqlens[n], eos = cu_seqlens[n + 1];
 
     float S[R][kCols];
-    const size_t sbase = ((size_t)n * H + h) * (size_t)DK * dv;
+    const float *src = init_state_block(s0, n, H, h, (size_t)DK * dv, ss);
 #pragma unroll
     for (int m = 0; m < R; ++m)
 #pragma unroll
         for (int j = 0; j < kCols; ++j)
-            S[m][j] = s0 ? s0[sbase + (size_t)(lane + 32 * m) * dv + col0 + j] : 0.f;
+            S[m][j] = src ? src[(size_t)(lane + 32 * m) * dv + col0 + j] : 0.f;
 
     // Software pipeline: the next token's operands are loaded while this one computes.
     float kc[R], qc[R], lc[R], vj[kCols], bt = 0.f;
@@ -99,12 +99,13 @@ recurrent_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin
         for (int j = 0; j < kCols; ++j) vj[j] = nv[j];
         bt = nb;
     }
-    if (sT) {
+    float *dst = final_state_block(sT, n, H, h, (size_t)DK * dv, ss);
+    if (dst) {
 #pragma unroll
         for (int m = 0; m < R; ++m)
 #pragma unroll
             for (int j = 0; j < kCols; ++j)
-                sT[sbase + (size_t)(lane + 32 * m) * dv + col0 + j] = S[m][j];
+                dst[(size_t)(lane + 32 * m) * dv + col0 + j] = S[m][j];
     }
 }
 
@@ -114,7 +115,7 @@ cudaError_t launch_typed(const Problem &p, cudaStream_t stream) {
     auto args = [&](auto kern) {
         kern<<<grid, 128, 0, stream>>>((const Tin *)p.q, (const Tin *)p.k, (const Tin *)p.v,
                                        p.log_alpha, p.beta, p.initial_state, p.cu_seqlens, p.H,
-                                       p.dv, (Tin *)p.out, p.final_state);
+                                       p.dv, (Tin *)p.out, p.final_state, p.slots);
     };
     switch (p.dk) {
         case 32: args(recurrent_kernel<Tin, 32>); break;

@@ -42,6 +42,10 @@ SIGNATURES = {
     "kda_selftest_bounded_wait": (_i32, [_vp, _sz, ctypes.c_uint64, _vp]),
     "kda_prefill_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                                    _i32, _i32, _vp, _vp, _vp]),
+    "kda_prefill_slots": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _i32, _i64,
+                                 _i32, _i32, _i32, _i32, _vp, _vp, _sz, _vp]),
+    "kda_decode_step_slots": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _i32,
+                                     _i32, _vp, _vp, _sz, _vp]),
 }
 
 
@@ -201,6 +205,87 @@ def decode_step(q, k, v, log_alpha, beta, state, out=None, stream=None):
     _check(lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
                                  _ptr(state), N, H, dk, dv, _dtype_code(dtype), _ptr(out), None, 0,
                                  _stream(stream)), "kda_decode_step")
+    return out
+
+
+def prefill_slots(q, k, v, log_alpha, beta, state_pool, init_slot, final_slot, cu_seqlens=None,
+                  cu_seqlens_dev=None, out=None, workspace=None, stream=None):
+    """Chunked prefill with the states in a pool of slots (``kda_prefill_slots``).
+
+    q, k, log_alpha [T, H, d_k]; v [T, H, d_v]; beta [T, H]; state_pool [P, H, d_k, d_v] fp32
+    (read and written); init_slot, final_slot: int32 device tensors [N] (-1: zeros / not stored).
+    cu_seqlens: host int32 offsets [N + 1] (default: one sequence). Returns out.
+    """
+    dtype = q.dtype
+    _need(q, "q", ndim=3)
+    Ttot, H, dk = q.shape
+    dv = v.shape[-1]
+    _need(k, "k", dtype, 3)
+    _need(v, "v", dtype, 3)
+    _need(log_alpha, "log_alpha", torch.float32, 3)
+    _need(beta, "beta", torch.float32, 2)
+    if k.shape != q.shape or log_alpha.shape != q.shape or v.shape[:2] != (Ttot, H) or beta.shape != (Ttot, H):
+        raise ValueError("inconsistent shapes among q, k, v, log_alpha, beta")
+    _need(state_pool, "state_pool", torch.float32, 4)
+    P = state_pool.shape[0]
+    if tuple(state_pool.shape[1:]) != (H, dk, dv):
+        raise ValueError(f"state_pool must be [P, {H}, {dk}, {dv}]")
+    if cu_seqlens is None:
+        cu_seqlens = torch.tensor([0, Ttot], dtype=torch.int32)
+    cu_host = torch.as_tensor(cu_seqlens, dtype=torch.int32).cpu().contiguous()
+    N = cu_host.numel() - 1
+    if cu_seqlens_dev is None:
+        cu_seqlens_dev = cu_host.to(q.device, non_blocking=False)
+    _need(cu_seqlens_dev, "cu_seqlens_dev", torch.int32, 1)
+    for t, name in ((init_slot, "init_slot"), (final_slot, "final_slot")):
+        _need(t, name, torch.int32, 1)
+        if t.numel() != N:
+            raise ValueError(f"{name} must have {N} entries")
+    if out is None:
+        out = torch.empty(Ttot, H, dv, dtype=dtype, device=q.device)
+    _need(out, "out", dtype, 3)
+    if workspace is None:
+        workspace = torch.empty(workspace_size(N, Ttot, H, dk, dv, dtype), dtype=torch.uint8,
+                                device=q.device)
+    _need(workspace, "workspace", torch.uint8, 1)
+    _check(lib().kda_prefill_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                   _ptr(state_pool), P, _ptr(init_slot), _ptr(final_slot),
+                                   _ptr(cu_seqlens_dev), ctypes.c_void_p(cu_host.data_ptr()), N,
+                                   Ttot, H, dk, dv, _dtype_code(dtype), _ptr(out), _ptr(workspace),
+                                   workspace.numel(), _stream(stream)), "kda_prefill_slots")
+    return out
+
+
+def decode_step_slots(q, k, v, log_alpha, beta, state_pool, slot, out=None, workspace=None,
+                      stream=None):
+    """One decode token per sequence on pooled states (``kda_decode_step_slots``).
+
+    state_pool [P, H, d_k, d_v] fp32, updated in place at slot[n] (int32 device [N]; -1: a zero
+    state that is not stored). Returns out [N, H, d_v].
+    """
+    dtype = q.dtype
+    _need(q, "q", ndim=3)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    _need(k, "k", dtype, 3)
+    _need(v, "v", dtype, 3)
+    _need(log_alpha, "log_alpha", torch.float32, 3)
+    _need(beta, "beta", torch.float32, 2)
+    _need(state_pool, "state_pool", torch.float32, 4)
+    _need(slot, "slot", torch.int32, 1)
+    if k.shape != q.shape or log_alpha.shape != q.shape or tuple(state_pool.shape[1:]) != (H, dk, dv) \
+            or slot.numel() != N:
+        raise ValueError("inconsistent shapes among q, k, log_alpha, state_pool, slot")
+    if out is None:
+        out = torch.empty(N, H, dv, dtype=dtype, device=q.device)
+    _need(out, "out", dtype, 3)
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace", torch.uint8, 1)
+    _check(lib().kda_decode_step_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                       _ptr(state_pool), state_pool.shape[0], _ptr(slot), N, H, dk,
+                                       dv, _dtype_code(dtype), _ptr(out), _ptr(workspace),
+                                       workspace.numel(), _stream(stream)), "kda_decode_step_slots")
     return out
 
 

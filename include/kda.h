@@ -164,6 +164,58 @@ KDA_API kda_status_t kda_decode_step(const void *q, const void *k, const void *v
                              void *out, void *workspace, size_t workspace_bytes,
                              kda_stream_t stream);
 
+/*
+ * kda_prefill with the states held in a pool of slots instead of one state per
+ * sequence: the prefill cache of "Kimi K3 -- the architecture and
+ * infrastructure, explained" (shivam2003.com), section "Serving
+ * infrastructure: supernodes and the prefill cache" keeps computed states and
+ * restores them so that a returning request pays only for its new suffix; a
+ * pool addressed by slot lets one call resume many requests from cached states
+ * (several may start from the same slot) and store their new states, without
+ * gathering them into a dense array first.
+ *
+ *   state_pool      [pool_slots, H, d_k, d_v] fp32: read and written
+ *   init_slot_dev   [num_seqs] int32 (device): sequence n starts from slot
+ *                   init_slot_dev[n], or from zeros if it is -1
+ *   final_slot_dev  [num_seqs] int32 (device): sequence n's final state goes to
+ *                   slot final_slot_dev[n], or nowhere if it is -1
+ *
+ * A slot may be both read and written by the same sequence (in-place resume).
+ * A slot written by one sequence must not be read or written by another
+ * sequence of the same call (the result would be unspecified). Slot values
+ * outside [-1, pool_slots) are treated as -1 and recorded in the device status
+ * word, for which kda_read_device_status then returns KDA_ERR_INVALID_ARGUMENT.
+ * state_pool may be NULL only if pool_slots == 0 (then every slot must be -1).
+ * Everything else (workspace, kernels, status) is as kda_prefill; the results
+ * equal kda_prefill's with the states gathered and scattered by slot.
+ */
+KDA_API kda_status_t kda_prefill_slots(const void *q, const void *k, const void *v,
+                                       const float *log_alpha, const float *beta,
+                                       float *state_pool, int64_t pool_slots,
+                                       const int32_t *init_slot_dev, const int32_t *final_slot_dev,
+                                       const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                                       int32_t num_seqs, int64_t total_tokens, int32_t H,
+                                       int32_t d_k, int32_t d_v, kda_dtype_t dtype, void *out,
+                                       void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * kda_decode_step on states held in a pool of slots (the same prefill cache):
+ * sequence n's state is slot slot_dev[n] of state_pool ([pool_slots, H, d_k,
+ * d_v] fp32), read and written in place; slot -1 means a zero state that is
+ * not stored. Two sequences must not name the same slot. Out-of-range slots
+ * are treated as -1 and recorded in the device status word at the start of
+ * `workspace` (required here: at least 256 bytes, 256-byte aligned), which
+ * kda_read_device_status reports as KDA_ERR_INVALID_ARGUMENT. Other arguments
+ * and status as kda_decode_step.
+ */
+KDA_API kda_status_t kda_decode_step_slots(const void *q, const void *k, const void *v,
+                                           const float *log_alpha, const float *beta,
+                                           float *state_pool, int64_t pool_slots,
+                                           const int32_t *slot_dev, int32_t num_seqs, int32_t H,
+                                           int32_t d_k, int32_t d_v, kda_dtype_t dtype,
+                                           void *out, void *workspace, size_t workspace_bytes,
+                                           kda_stream_t stream);
+
 /* Static string naming a status code. Never NULL. */
 KDA_API const char *kda_status_string(kda_status_t status);
 
@@ -173,9 +225,11 @@ KDA_API const char *kda_last_error(void);
 
 /*
  * Reads the device status word that kda_prefill keeps at the start of its
- * workspace: KDA_OK, or KDA_ERR_TIMEOUT if a bounded on-device wait of the
- * last prefill that used this workspace gave up (its outputs are then
- * invalid). Synchronises `stream` (this is the only call that does).
+ * workspace: KDA_OK; KDA_ERR_TIMEOUT if a bounded on-device wait of the last
+ * prefill that used this workspace gave up (its outputs are then invalid); or
+ * KDA_ERR_INVALID_ARGUMENT if the last kda_prefill_slots /
+ * kda_decode_step_slots that used it met a slot outside [-1, pool_slots).
+ * Synchronises `stream` (this is the only call that does).
  */
 KDA_API kda_status_t kda_read_device_status(const void *workspace, kda_stream_t stream);
 

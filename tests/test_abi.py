@@ -123,3 +123,42 @@ def test_product_path_does_not_import_oracle():
         if fn.endswith(".py"):
             src = open(os.path.join(pkg, fn)).read()
             assert not re.search(r"^\s*(from|import)\s+oracle", src, re.M), fn
+
+
+def test_slot_entry_points_reject_bad_arguments():
+    L = K.lib()
+    fake = ctypes.c_void_p(0x10000)
+    out = ctypes.c_void_p(0x20000)
+    cu = (ctypes.c_int32 * 3)(0, 5, 9)
+    cuh = ctypes.cast(cu, ctypes.c_void_p)
+
+    def prefill_slots(pool=fake, slots=4, init=fake, fin=fake, ws=None, wsb=0):
+        rc = L.kda_prefill_slots(fake, fake, fake, fake, fake, pool, slots, init, fin, fake, cuh, 2,
+                                 9, 2, 32, 32, 0, out, ws, wsb, None)
+        return rc, L.kda_last_error().decode()
+
+    rc, msg = prefill_slots(pool=None)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "state_pool" in msg
+    rc, msg = prefill_slots(slots=-1)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "pool_slots" in msg
+    rc, msg = prefill_slots(init=None)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "init_slot_dev" in msg
+    rc, msg = prefill_slots()  # all else valid: the missing workspace is reported
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "workspace" in msg
+
+    def decode_slots(slot=fake, ws=None, wsb=0, pool=fake, slots=4):
+        rc = L.kda_decode_step_slots(fake, fake, fake, fake, fake, pool, slots, slot, 4, 2, 64, 64, 1,
+                                     out, ws, wsb, None)
+        return rc, L.kda_last_error().decode()
+
+    rc, msg = decode_slots(slot=None)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "slot_dev" in msg
+    rc, msg = decode_slots()
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "workspace" in msg
+    rc, msg = decode_slots(ws=ctypes.c_void_p(0x30010), wsb=256)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "256-byte aligned" in msg
+    rc, msg = decode_slots(pool=None)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "state_pool" in msg
+    # zero sequences: a no-op
+    assert L.kda_decode_step_slots(None, None, None, None, None, None, 0, None, 0, 2, 64, 64, 1, None,
+                                   None, 0, None) == K.KDA_OK
