@@ -45,8 +45,8 @@ FLOP_PER_TOKEN_HEAD = 180224
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
 # dram__bytes_read.sum + dram__bytes_write.sum of one split_kernel launch on the headline workload,
 # from one ncu capture; reported only while the kernel's sources are the ones it was taken on.
-SPLIT_TRAFFIC_BYTES = 336.77824e6 + 57.831168e6
-SPLIT_TRAFFIC_SOURCES_SHA256 = "ad76fc8b96f411c8e64351c7abf0317f80067a5e31cf1b36c101f9c877711a8c"
+SPLIT_TRAFFIC_BYTES = 336.771584e6 + 59.779840e6
+SPLIT_TRAFFIC_SOURCES_SHA256 = "5b2a693e41e6f3c6b9124eabe932e3b1425eeb43528fc67d2cfa66d03da1247c"
 
 
 def measured_traffic():
@@ -58,6 +58,12 @@ def measured_traffic():
     return SPLIT_TRAFFIC_BYTES if h.hexdigest() == SPLIT_TRAFFIC_SOURCES_SHA256 else None
 # Decode: state read + write (fp32) + q, k, v + log_alpha + beta + out.
 DECODE_BYTES_PER_TOKEN_HEAD = 2 * 128 * 128 * 4 + 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
+# Speculative decode, per (sequence, head) and draft token: verify reads the state once and per
+# token q, k, v (bf16), log_alpha, beta, writes out (bf16) and u (fp32); commit reads and writes the
+# state once and per accepted token reads k, log_alpha and u.
+DRAFT_TOKENS = 4
+VERIFY_STATE_BYTES, VERIFY_TOKEN_BYTES = 128 * 128 * 4, 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2 + 128 * 4
+COMMIT_STATE_BYTES, COMMIT_TOKEN_BYTES = 2 * 128 * 128 * 4, 128 * 2 + 128 * 4 + 128 * 4
 
 
 def peaks():
@@ -267,6 +273,76 @@ def bench_decode(args, K, stream, ws):
             "gpu_launches": nsteps}
 
 
+def bench_speculative(args, K, stream, ws, decode_ms):
+    """Speculative decode on the decode workload's states with DRAFT_TOKENS draft tokens per
+    sequence, all accepted: the verify and commit calls timed alone, and the steady-state step
+    (commit the previous draft while verifying the next, one pass over the states), compared with
+    as many single decode steps."""
+    wl = W.DECODE_256
+    inp = W.make_inputs(wl, "cuda", seed=wl.seed + 7919 * args.rank)
+    _, state = K.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], None,
+                         inp["cu_seqlens"], inp["cu_seqlens_dev"])
+    N, H, T, sets = wl.num_seqs, wl.H, DRAFT_TOKENS, 8
+    steps = W.make_decode_steps(wl, inp["_gen"], sets * T, "cuda")
+    del inp
+    # [sets * T, N, ...] -> per set [N, T, ...]
+    x = {n: t.reshape(sets, T, N, *t.shape[2:]).transpose(1, 2).contiguous() for n, t in steps.items()}
+    del steps
+    out = torch.empty(sets, N, T, H, wl.dv, dtype=torch.bfloat16, device="cuda")
+    u = torch.empty(sets, N, T, H, wl.dv, dtype=torch.float32, device="cuda")
+    acc = torch.full((N,), T, dtype=torch.int32, device="cuda")
+    work = torch.empty(256, dtype=torch.uint8, device="cuda")
+    i = [0]
+
+    def verify():
+        j = i[0] % sets
+        K.decode_verify(x["q"][j], x["k"][j], x["v"][j], x["log_alpha"][j], x["beta"][j], state,
+                        out=out[j], u_cache=u[j], workspace=work, stream=stream)
+        i[0] += 1
+
+    def commit():
+        j = i[0] % sets
+        K.decode_commit(x["k"][j], x["log_alpha"][j], u[j], state, acc, workspace=work, stream=stream)
+        i[0] += 1
+
+    def fused():  # steady state: commit the previous draft (all accepted) while verifying this one
+        j = i[0] % sets
+        jp = (j - 1) % sets
+        K.decode_commit_verify(x["k"][jp], x["log_alpha"][jp], u[jp], acc, x["q"][j], x["k"][j],
+                               x["v"][j], x["log_alpha"][j], x["beta"][j], state, out=out[j],
+                               u_cache=u[j], workspace=work, stream=stream)
+        i[0] += 1
+
+    nsteps = max(8, args.decode_steps // 4)
+    timed = {}
+    for name, fn in (("verify", verify), ("commit", commit), ("commit_verify", fused)):
+        i[0] = 0
+        for _ in range(sets):
+            fn()
+        torch.cuda.synchronize()
+        barrier(ws)
+        timed[name] = max_over_ranks(time_events(fn, nsteps, stream), ws)
+    pk = peaks()
+
+    def roof(state_b, tok_b, ms):
+        gbs = N * H * (state_b + T * tok_b) / (ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"]}
+
+    del x, out, u, state
+    torch.cuda.empty_cache()
+    ms = timed["commit_verify"]
+    return {"workload": f"{wl.name} states, {T} draft tokens per sequence, all accepted",
+            "draft_tokens": T, "steps": nsteps, "verify_ms": timed["verify"],
+            "commit_ms": timed["commit"], "ms_per_step": ms,
+            "tokens_per_s": N * T * ws / (ms * 1e-3),
+            "speedup_vs_single_steps": None if decode_ms is None else T * decode_ms / ms,
+            "roofline": roof(COMMIT_STATE_BYTES, VERIFY_TOKEN_BYTES + COMMIT_TOKEN_BYTES, ms),
+            "verify_roofline": roof(VERIFY_STATE_BYTES, VERIFY_TOKEN_BYTES, timed["verify"]),
+            "commit_roofline": roof(COMMIT_STATE_BYTES, COMMIT_TOKEN_BYTES, timed["commit"]),
+            "gpu_launches": 3 * nsteps}
+
+
 def bench_prefill_workload(wl, K, stream, steps, warmup, rank):
     """Device-timed kda_prefill of one workload (inputs resident in HBM); returns a summary dict."""
     inp = W.make_inputs(wl, "cuda", seed=wl.seed + 7919 * rank)
@@ -368,6 +444,7 @@ def run_ours(args, rank, local, ws):
     del host, dev
 
     dec = bench_decode(args, K, stream, ws) if not args.no_decode else None
+    spec = None if args.no_decode else bench_speculative(args, K, stream, ws, dec["ms_per_step"])
     extra = None
     if not args.no_extra:
         extra = [bench_prefill_workload(W.VARLEN_24, K, stream, 5, 3, rank),
@@ -399,6 +476,7 @@ def run_ours(args, rank, local, ws):
             "value": T * ws / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "decode": dec,
+        "speculative_decode": spec,
         "other_prefill_workloads": extra,
         "gpu_launches": args.steps * kernels_per_step,
         "clocks": clocks,

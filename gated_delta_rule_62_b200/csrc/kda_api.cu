@@ -292,6 +292,164 @@ kda_status_t kda_decode_step_slots(const void *q, const void *k, const void *v,
     return ok();
 }
 
+}  // extern "C"
+
+namespace {
+
+// Checks shared by kda_decode_verify and kda_decode_commit (shapes, pool, workspace).
+kda_status_t check_verify(const char *who, const float *state, int64_t pool_slots,
+                          const int32_t *slot_dev, int32_t num_seqs, int32_t T, int32_t H,
+                          int32_t d_k, int32_t d_v, kda_dtype_t dtype, const void *workspace,
+                          size_t workspace_bytes) {
+    if (dtype != KDA_F32 && dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: dtype %d is not KDA_F32 or KDA_BF16", who, (int)dtype);
+    if (H <= 0) return fail(KDA_ERR_INVALID_ARGUMENT, "%s: H=%d <= 0", who, H);
+    if (!supported_d(d_k) || !supported_d(d_v))
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: d_k=%d, d_v=%d: each must be 32, 64 or 128", who,
+                    d_k, d_v);
+    if (T < 1 || T > KDA_MAX_DRAFT_TOKENS)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: T=%d outside [1, %d]", who, T, KDA_MAX_DRAFT_TOKENS);
+    if (num_seqs < 0) return fail(KDA_ERR_INVALID_ARGUMENT, "%s: num_seqs=%d < 0", who, num_seqs);
+    if ((int64_t)num_seqs * T * H > INT32_MAX)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: num_seqs * T * H exceeds 2^31 - 1", who);
+    if (slot_dev && (pool_slots < 0 || pool_slots > INT32_MAX))
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: pool_slots=%lld outside [0, 2^31)", who,
+                    (long long)pool_slots);
+    if (num_seqs > 0 && !state && !(slot_dev && pool_slots == 0))
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: state is NULL", who);
+    if (!workspace || workspace_bytes < kStatusBytes ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(KDA_ERR_INVALID_ARGUMENT,
+                    "%s: a 256-byte aligned workspace of >= %zu bytes is required", who, kStatusBytes);
+    if (state && !aligned16(state))
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: state %p is not 16-byte aligned", who,
+                    (const void *)state);
+    return ok();
+}
+
+// Pointer checks of the draft to verify (kda_decode_verify, kda_decode_commit_verify).
+kda_status_t check_draft(const char *who, const void *q, const void *k, const void *v,
+                         const float *log_alpha, const float *beta, const float *state,
+                         const void *out, const float *u_cache) {
+    if (!q || !k || !v || !log_alpha || !beta || !out || !u_cache)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: q, k, v, log_alpha, beta, out and u_cache are "
+                    "required", who);
+    const void *ptrs[] = {q, k, v, log_alpha, out, u_cache};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr))
+            return fail(KDA_ERR_INVALID_ARGUMENT, "%s: tensor pointer %p is not 16-byte aligned", who, ptr);
+    const void *outs[] = {out, u_cache};
+    for (const void *o : outs)
+        if (o == q || o == k || o == v || o == (const void *)log_alpha || o == (const void *)state)
+            return fail(KDA_ERR_INVALID_ARGUMENT, "%s: out and u_cache must not alias an input or "
+                        "the state", who);
+    if (out == (const void *)u_cache)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: out aliases u_cache", who);
+    return ok();
+}
+
+// Pointer checks of the accepted tokens to commit (kda_decode_commit, kda_decode_commit_verify).
+kda_status_t check_accepted(const char *who, const void *k, const float *log_alpha,
+                            const float *u_cache, const int32_t *accepted_dev, const float *state) {
+    if (!k || !log_alpha || !u_cache || !accepted_dev)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: k, log_alpha, u_cache and accepted_dev are "
+                    "required", who);
+    if (!aligned16(k) || !aligned16(log_alpha) || !aligned16(u_cache))
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: k, log_alpha and u_cache must be 16-byte aligned",
+                    who);
+    if (state && (k == (const void *)state || log_alpha == state || u_cache == state))
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: an input aliases the state", who);
+    return ok();
+}
+
+kda_status_t launch_spec(const char *who, kda::VerifyProblem &p, int64_t pool_slots,
+                         const int32_t *slot_dev, void *workspace, cudaStream_t s) {
+    p.slots.init_slot = p.slots.final_slot = slot_dev;
+    p.slots.slots = pool_slots;
+    p.slots.status = static_cast<int32_t *>(workspace);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
+    if (e == cudaSuccess) e = kda::launch_verify(p, s);
+    if (e != cudaSuccess) return cuda_fail(e, who);
+    return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status_t kda_decode_verify(const void *q, const void *k, const void *v, const float *log_alpha,
+                               const float *beta, const float *state, int64_t pool_slots,
+                               const int32_t *slot_dev, int32_t num_seqs, int32_t T, int32_t H,
+                               int32_t d_k, int32_t d_v, kda_dtype_t dtype, void *out,
+                               float *u_cache, void *workspace, size_t workspace_bytes,
+                               kda_stream_t stream) {
+    const char *who = "kda_decode_verify";
+    kda_status_t st = check_verify(who, state, pool_slots, slot_dev, num_seqs, T, H, d_k, d_v, dtype,
+                                   workspace, workspace_bytes);
+    if (st != KDA_OK || num_seqs == 0) return st;
+    st = check_draft(who, q, k, v, log_alpha, beta, state, out, u_cache);
+    if (st != KDA_OK) return st;
+    kda::VerifyProblem p{};
+    p.q = q; p.k = k; p.v = v; p.log_alpha = log_alpha; p.beta = beta;
+    p.state = const_cast<float *>(state);  // only read without a commit
+    p.num_seqs = num_seqs; p.T = T; p.H = H; p.dk = d_k; p.dv = d_v; p.dtype = dtype;
+    p.out = out; p.u_cache = u_cache;
+    return launch_spec(who, p, pool_slots, slot_dev, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kda_status_t kda_decode_commit(const void *k, const float *log_alpha, const float *u_cache,
+                               float *state, int64_t pool_slots, const int32_t *slot_dev,
+                               const int32_t *accepted_dev, int32_t num_seqs, int32_t T, int32_t H,
+                               int32_t d_k, int32_t d_v, kda_dtype_t dtype, void *workspace,
+                               size_t workspace_bytes, kda_stream_t stream) {
+    const char *who = "kda_decode_commit";
+    kda_status_t st = check_verify(who, state, pool_slots, slot_dev, num_seqs, T, H, d_k, d_v, dtype,
+                                   workspace, workspace_bytes);
+    if (st != KDA_OK || num_seqs == 0) return st;
+    st = check_accepted(who, k, log_alpha, u_cache, accepted_dev, state);
+    if (st != KDA_OK) return st;
+    kda::VerifyProblem p{};
+    p.prev_k = k; p.prev_log_alpha = log_alpha; p.prev_u = u_cache; p.accepted = accepted_dev;
+    p.state = state;
+    p.num_seqs = num_seqs; p.T_prev = T; p.H = H; p.dk = d_k; p.dv = d_v; p.dtype = dtype;
+    return launch_spec(who, p, pool_slots, slot_dev, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kda_status_t kda_decode_commit_verify(const void *prev_k, const float *prev_log_alpha,
+                                      const float *prev_u, const int32_t *accepted_dev,
+                                      int32_t T_prev, const void *q, const void *k, const void *v,
+                                      const float *log_alpha, const float *beta, float *state,
+                                      int64_t pool_slots, const int32_t *slot_dev, int32_t num_seqs,
+                                      int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                      kda_dtype_t dtype, void *out, float *u_cache,
+                                      void *workspace, size_t workspace_bytes,
+                                      kda_stream_t stream) {
+    const char *who = "kda_decode_commit_verify";
+    kda_status_t st = check_verify(who, state, pool_slots, slot_dev, num_seqs, T, H, d_k, d_v, dtype,
+                                   workspace, workspace_bytes);
+    if (st != KDA_OK) return st;
+    if (T_prev < 1 || T_prev > KDA_MAX_DRAFT_TOKENS)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: T_prev=%d outside [1, %d]", who, T_prev,
+                    KDA_MAX_DRAFT_TOKENS);
+    if ((int64_t)num_seqs * T_prev * H > INT32_MAX)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: num_seqs * T_prev * H exceeds 2^31 - 1", who);
+    if (num_seqs == 0) return ok();
+    st = check_draft(who, q, k, v, log_alpha, beta, state, out, u_cache);
+    if (st == KDA_OK) st = check_accepted(who, prev_k, prev_log_alpha, prev_u, accepted_dev, state);
+    if (st != KDA_OK) return st;
+    if (u_cache == prev_u || out == (const void *)prev_u || out == prev_k || u_cache == prev_k ||
+        out == (const void *)prev_log_alpha || u_cache == prev_log_alpha)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "%s: out and u_cache must not alias the previous "
+                    "draft's k, log_alpha or u", who);
+    kda::VerifyProblem p{};
+    p.q = q; p.k = k; p.v = v; p.log_alpha = log_alpha; p.beta = beta;
+    p.prev_k = prev_k; p.prev_log_alpha = prev_log_alpha; p.prev_u = prev_u; p.accepted = accepted_dev;
+    p.state = state;
+    p.num_seqs = num_seqs; p.T = T; p.T_prev = T_prev; p.H = H; p.dk = d_k; p.dv = d_v;
+    p.dtype = dtype; p.out = out; p.u_cache = u_cache;
+    return launch_spec(who, p, pool_slots, slot_dev, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
 const char *kda_status_string(kda_status_t s) {
     switch (s) {
         case KDA_OK: return "KDA_OK";
@@ -313,9 +471,9 @@ kda_status_t kda_read_device_status(const void *workspace, kda_stream_t stream) 
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "kda_read_device_status");
     if (word == 0) return ok();
-    if (word & kda::kStatusBadSlot)
-        return fail(KDA_ERR_INVALID_ARGUMENT, "device status word 0x%x: a state slot was outside "
-                    "[-1, pool_slots)", (unsigned)word);
+    if (word & (kda::kStatusBadSlot | kda::kStatusBadAccept))
+        return fail(KDA_ERR_INVALID_ARGUMENT, "device status word 0x%x: a state slot outside "
+                    "[-1, pool_slots) or an accepted count outside [0, T]", (unsigned)word);
     return fail(KDA_ERR_TIMEOUT, "device status word 0x%x: a bounded on-device wait gave up",
                 (unsigned)word);
 }

@@ -23,7 +23,7 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // Entry n of initial_state / final_state ([N, H, d_k, d_v]); or, with slot tables, slot
 // init_slot[n] / final_slot[n] of one pool ([slots, H, d_k, d_v]), -1 meaning none. A slot outside
 // [-1, slots) counts as -1 and sets kStatusBadSlot in the device status word.
-constexpr int32_t kStatusTimeout = 1, kStatusBadSlot = 2;
+constexpr int32_t kStatusTimeout = 1, kStatusBadSlot = 2, kStatusBadAccept = 4;
 struct StateSlots {
     const int32_t *init_slot = nullptr, *final_slot = nullptr;  // device tables (or null)
     int64_t slots = 0;
@@ -102,5 +102,23 @@ struct DecodeProblem {
     StateSlots slots;
 };
 cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream);
+
+// Speculative decode: T draft tokens per sequence (rows n*T + t). With q set, the draft is
+// verified (out and u_cache written); with accepted set, state n is first advanced by accepted[n]
+// tokens of the previous draft (prev_k, prev_log_alpha, prev_u; rows n*T_prev + t) and stored.
+struct VerifyProblem {
+    const void *q, *k, *v;      // the draft to verify (q == null: commit only)
+    const float *log_alpha, *beta;
+    const void *prev_k;         // the accepted tokens to commit (accepted == null: none)
+    const float *prev_log_alpha, *prev_u;
+    const int32_t *accepted;    // device, [num_seqs]
+    float *state;               // [num_seqs, ...] or, with slots, the pool
+    int32_t num_seqs, T, T_prev, H, dk, dv;
+    kda_dtype_t dtype;
+    void *out;
+    float *u_cache;
+    StateSlots slots;
+};
+cudaError_t launch_verify(const VerifyProblem &p, cudaStream_t stream);
 
 }  // namespace kda

@@ -46,6 +46,13 @@ SIGNATURES = {
                                  _i32, _i32, _i32, _i32, _vp, _vp, _sz, _vp]),
     "kda_decode_step_slots": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _i32,
                                      _i32, _vp, _vp, _sz, _vp]),
+    "kda_decode_verify": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _i32,
+                                 _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "kda_decode_commit": (_i32, [_vp, _vp, _vp, _vp, _i64, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+                                 _i32, _vp, _sz, _vp]),
+    "kda_decode_commit_verify": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
+                                        _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz,
+                                        _vp]),
 }
 
 
@@ -287,6 +294,126 @@ def decode_step_slots(q, k, v, log_alpha, beta, state_pool, slot, out=None, work
                                        dv, _dtype_code(dtype), _ptr(out), _ptr(workspace),
                                        workspace.numel(), _stream(stream)), "kda_decode_step_slots")
     return out
+
+
+MAX_DRAFT_TOKENS = 16
+
+
+def _pool_args(state, slot, N, H, dk, dv):
+    _need(state, "state", torch.float32, 4)
+    if tuple(state.shape[1:]) != (H, dk, dv):
+        raise ValueError(f"state shape {tuple(state.shape)} does not end in {(H, dk, dv)}")
+    if slot is None:
+        if state.shape[0] != N:
+            raise ValueError(f"state holds {state.shape[0]} entries for {N} sequences")
+        return state.shape[0], None
+    _need(slot, "slot", torch.int32, 1)
+    if slot.numel() != N:
+        raise ValueError("slot must have one entry per sequence")
+    return state.shape[0], slot
+
+
+def decode_verify(q, k, v, log_alpha, beta, state, slot=None, out=None, u_cache=None,
+                  workspace=None, stream=None):
+    """Check T draft tokens per sequence in one pass (``kda_decode_verify``); states unchanged.
+
+    q, k [N, T, H, d_k]; v [N, T, H, d_v]; log_alpha [N, T, H, d_k] fp32; beta [N, T, H] fp32;
+    state [N, H, d_k, d_v] fp32, or a pool [P, ...] addressed by ``slot`` (int32 device [N]).
+    Returns (out, u_cache), both [N, T, H, d_v] (out in the input dtype, u_cache fp32).
+    """
+    dtype = q.dtype
+    _need(q, "q", ndim=4)
+    N, T, H, dk = q.shape
+    dv = v.shape[-1]
+    _need(k, "k", dtype, 4)
+    _need(v, "v", dtype, 4)
+    _need(log_alpha, "log_alpha", torch.float32, 4)
+    _need(beta, "beta", torch.float32, 3)
+    if k.shape != q.shape or log_alpha.shape != q.shape or tuple(v.shape[:3]) != (N, T, H) \
+            or tuple(beta.shape) != (N, T, H):
+        raise ValueError("inconsistent shapes among q, k, v, log_alpha, beta")
+    P, slot = _pool_args(state, slot, N, H, dk, dv)
+    if out is None:
+        out = torch.empty(N, T, H, dv, dtype=dtype, device=q.device)
+    if u_cache is None:
+        u_cache = torch.empty(N, T, H, dv, dtype=torch.float32, device=q.device)
+    _need(out, "out", dtype, 4)
+    _need(u_cache, "u_cache", torch.float32, 4)
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace", torch.uint8, 1)
+    _check(lib().kda_decode_verify(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                   _ptr(state), P, _ptr(slot), N, T, H, dk, dv, _dtype_code(dtype),
+                                   _ptr(out), _ptr(u_cache), _ptr(workspace), workspace.numel(),
+                                   _stream(stream)), "kda_decode_verify")
+    return out, u_cache
+
+
+def decode_commit(k, log_alpha, u_cache, state, accepted, slot=None, workspace=None, stream=None):
+    """Advance each state by its accepted draft tokens (``kda_decode_commit``), in place.
+
+    k, log_alpha, u_cache as given to / returned by :func:`decode_verify`; accepted int32 device
+    [N], each in [0, T].
+    """
+    _need(k, "k", ndim=4)
+    N, T, H, dk = k.shape
+    dv = u_cache.shape[-1]
+    _need(log_alpha, "log_alpha", torch.float32, 4)
+    _need(u_cache, "u_cache", torch.float32, 4)
+    _need(accepted, "accepted", torch.int32, 1)
+    if log_alpha.shape != k.shape or tuple(u_cache.shape[:3]) != (N, T, H) or accepted.numel() != N:
+        raise ValueError("inconsistent shapes among k, log_alpha, u_cache, accepted")
+    P, slot = _pool_args(state, slot, N, H, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=k.device)
+    _need(workspace, "workspace", torch.uint8, 1)
+    _check(lib().kda_decode_commit(_ptr(k), _ptr(log_alpha), _ptr(u_cache), _ptr(state), P,
+                                   _ptr(slot), _ptr(accepted), N, T, H, dk, dv,
+                                   _dtype_code(k.dtype), _ptr(workspace), workspace.numel(),
+                                   _stream(stream)), "kda_decode_commit")
+
+
+def decode_commit_verify(prev_k, prev_log_alpha, prev_u, accepted, q, k, v, log_alpha, beta, state,
+                         slot=None, out=None, u_cache=None, workspace=None, stream=None):
+    """Commit the previous draft's accepted tokens and verify the next draft in one pass over the
+    states (``kda_decode_commit_verify``). prev_* as the previous :func:`decode_verify` took and
+    returned them ([N, T_prev, H, ...]); the rest as :func:`decode_verify`. Returns (out, u_cache),
+    which must be new buffers (not prev_u)."""
+    _need(prev_k, "prev_k", q.dtype, 4)
+    _need(prev_log_alpha, "prev_log_alpha", torch.float32, 4)
+    _need(prev_u, "prev_u", torch.float32, 4)
+    _need(accepted, "accepted", torch.int32, 1)
+    _need(q, "q", ndim=4)
+    N, T, H, dk = q.shape
+    dv = v.shape[-1]
+    Tp = prev_k.shape[1]
+    if prev_log_alpha.shape != prev_k.shape or tuple(prev_k.shape) != (N, Tp, H, dk) \
+            or tuple(prev_u.shape) != (N, Tp, H, dv) or accepted.numel() != N:
+        raise ValueError("inconsistent shapes among prev_k, prev_log_alpha, prev_u, accepted")
+    _need(k, "k", q.dtype, 4)
+    _need(v, "v", q.dtype, 4)
+    _need(log_alpha, "log_alpha", torch.float32, 4)
+    _need(beta, "beta", torch.float32, 3)
+    if k.shape != q.shape or log_alpha.shape != q.shape or tuple(v.shape[:3]) != (N, T, H) \
+            or tuple(beta.shape) != (N, T, H):
+        raise ValueError("inconsistent shapes among q, k, v, log_alpha, beta")
+    P, slot = _pool_args(state, slot, N, H, dk, dv)
+    if out is None:
+        out = torch.empty(N, T, H, dv, dtype=q.dtype, device=q.device)
+    if u_cache is None:
+        u_cache = torch.empty(N, T, H, dv, dtype=torch.float32, device=q.device)
+    _need(out, "out", q.dtype, 4)
+    _need(u_cache, "u_cache", torch.float32, 4)
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=q.device)
+    _need(workspace, "workspace", torch.uint8, 1)
+    _check(lib().kda_decode_commit_verify(_ptr(prev_k), _ptr(prev_log_alpha), _ptr(prev_u),
+                                          _ptr(accepted), Tp, _ptr(q), _ptr(k), _ptr(v),
+                                          _ptr(log_alpha), _ptr(beta), _ptr(state), P, _ptr(slot), N,
+                                          T, H, dk, dv, _dtype_code(q.dtype), _ptr(out), _ptr(u_cache),
+                                          _ptr(workspace), workspace.numel(), _stream(stream)),
+           "kda_decode_commit_verify")
+    return out, u_cache
 
 
 def selftest_bounded_wait(workspace, timeout_ns: int, stream=None):

@@ -216,6 +216,92 @@ KDA_API kda_status_t kda_decode_step_slots(const void *q, const void *k, const v
                                            void *out, void *workspace, size_t workspace_bytes,
                                            kda_stream_t stream);
 
+/* Most draft tokens per sequence that kda_decode_verify / kda_decode_commit take. */
+#define KDA_MAX_DRAFT_TOKENS 16
+
+/*
+ * Speculative (multi-token) decode, verify half. The draft model proposes T
+ * tokens per sequence and the main model checks them all in one pass
+ * ("Optimization for Inference: 4-Bit and Speculative Decoding" in the Kimi K3
+ * article, EAGLE-3 with a multi-token-prediction draft layer). For each
+ * (sequence, head) this reads the state once, runs the T tokens through the
+ * recurrence, and leaves the state UNCHANGED; kda_decode_commit then advances
+ * it by however many tokens were accepted. Row n*T + t holds draft token t of
+ * sequence n:
+ *
+ *   q, k        [num_seqs*T, H, d_k]  dtype
+ *   v           [num_seqs*T, H, d_v]  dtype
+ *   log_alpha   [num_seqs*T, H, d_k]  fp32
+ *   beta        [num_seqs*T, H]       fp32
+ *   state       slot_dev == NULL: [num_seqs, H, d_k, d_v] fp32, sequence n's
+ *               state is entry n; otherwise a pool [pool_slots, H, d_k, d_v]
+ *               and sequence n's state is slot slot_dev[n] (-1: zeros). Only read.
+ *   out         [num_seqs*T, H, d_v]  dtype (written): token t's output, as if
+ *               tokens 0..t had been decoded one by one
+ *   u_cache     [num_seqs*T, H, d_v]  fp32 (written): token t's correction
+ *               u_t = beta_t (v_t - (Diag(alpha_t) S_{t-1})^T k_t), the value
+ *               written into the memory, so that
+ *               S_t = Diag(alpha_t) S_{t-1} + k_t u_t^T
+ *               ("How the delta rule actually works" in the same article)
+ *   workspace   required: >= 256 bytes, 256-byte aligned; its first word is
+ *               the device status word (out-of-range slots, as
+ *               kda_decode_step_slots)
+ *
+ * 1 <= T <= KDA_MAX_DRAFT_TOKENS. The outputs equal those of T calls of
+ * kda_decode_step on a copy of the states, bit for bit. Status as
+ * kda_decode_step_slots.
+ */
+KDA_API kda_status_t kda_decode_verify(const void *q, const void *k, const void *v,
+                                       const float *log_alpha, const float *beta,
+                                       const float *state, int64_t pool_slots,
+                                       const int32_t *slot_dev, int32_t num_seqs, int32_t T,
+                                       int32_t H, int32_t d_k, int32_t d_v, kda_dtype_t dtype,
+                                       void *out, float *u_cache, void *workspace,
+                                       size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * Speculative decode, commit half: advances sequence n's state in place by its
+ * first accepted_dev[n] draft tokens (0 <= accepted <= T; 0 leaves it as it
+ * is), using the k, log_alpha and u_cache of the kda_decode_verify call that
+ * checked them (same T, layouts, state / pool and slot_dev). Each state that
+ * moves is read once and written once; the result equals accepted_dev[n] calls
+ * of kda_decode_step, bit for bit. An accepted count outside [0, T] leaves the
+ * sequence untouched and is recorded in the device status word, which
+ * kda_read_device_status reports as KDA_ERR_INVALID_ARGUMENT; slot -1 stores
+ * nothing; two sequences must not name the same slot. Workspace and status as
+ * kda_decode_verify.
+ */
+KDA_API kda_status_t kda_decode_commit(const void *k, const float *log_alpha,
+                                       const float *u_cache, float *state, int64_t pool_slots,
+                                       const int32_t *slot_dev, const int32_t *accepted_dev,
+                                       int32_t num_seqs, int32_t T, int32_t H, int32_t d_k,
+                                       int32_t d_v, kda_dtype_t dtype, void *workspace,
+                                       size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * kda_decode_commit of the previous draft followed by kda_decode_verify of the
+ * next one, in one pass over the states: each state is read once, advanced by
+ * accepted_dev[n] tokens of the previous draft (prev_k, prev_log_alpha,
+ * prev_u: rows n*T_prev + t, as that draft's verify call took and returned
+ * them), stored if it moved, and the T new draft tokens are run from it. A
+ * speculative decode loop thus moves each state through HBM once per step,
+ * like a single kda_decode_step, however many tokens the step accepts. Results
+ * (out, u_cache, states) equal those of the two calls bit for bit; u_cache and
+ * out must not alias prev_k, prev_log_alpha or prev_u (use two buffers in turn).
+ * 1 <= T_prev <= KDA_MAX_DRAFT_TOKENS; two sequences must not name the same
+ * slot. Other arguments, workspace and status as the two calls.
+ */
+KDA_API kda_status_t kda_decode_commit_verify(const void *prev_k, const float *prev_log_alpha,
+                                              const float *prev_u, const int32_t *accepted_dev,
+                                              int32_t T_prev, const void *q, const void *k,
+                                              const void *v, const float *log_alpha,
+                                              const float *beta, float *state, int64_t pool_slots,
+                                              const int32_t *slot_dev, int32_t num_seqs, int32_t T,
+                                              int32_t H, int32_t d_k, int32_t d_v,
+                                              kda_dtype_t dtype, void *out, float *u_cache,
+                                              void *workspace, size_t workspace_bytes,
+                                              kda_stream_t stream);
+
 /* Static string naming a status code. Never NULL. */
 KDA_API const char *kda_status_string(kda_status_t status);
 
@@ -228,7 +314,9 @@ KDA_API const char *kda_last_error(void);
  * workspace: KDA_OK; KDA_ERR_TIMEOUT if a bounded on-device wait of the last
  * prefill that used this workspace gave up (its outputs are then invalid); or
  * KDA_ERR_INVALID_ARGUMENT if the last kda_prefill_slots /
- * kda_decode_step_slots that used it met a slot outside [-1, pool_slots).
+ * kda_decode_step_slots / kda_decode_verify / kda_decode_commit /
+ * kda_decode_commit_verify that used it
+ * met a slot outside [-1, pool_slots) or an accepted count outside [0, T].
  * Synchronises `stream` (this is the only call that does).
  */
 KDA_API kda_status_t kda_read_device_status(const void *workspace, kda_stream_t stream);

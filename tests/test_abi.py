@@ -162,3 +162,75 @@ def test_slot_entry_points_reject_bad_arguments():
     # zero sequences: a no-op
     assert L.kda_decode_step_slots(None, None, None, None, None, None, 0, None, 0, 2, 64, 64, 1, None,
                                    None, 0, None) == K.KDA_OK
+
+
+def test_speculative_entry_points_reject_bad_arguments():
+    L = K.lib()
+    fake = ctypes.c_void_p(0x10000)
+    ws = ctypes.c_void_p(0x40000)
+
+    def verify(T=4, state=fake, slot=None, slots=0, ws=ws, wsb=256, out=ctypes.c_void_p(0x20000),
+               u=ctypes.c_void_p(0x30000)):
+        rc = L.kda_decode_verify(fake, fake, fake, fake, fake, state, slots, slot, 3, T, 2, 64, 64, 1,
+                                 out, u, ws, wsb, None)
+        return rc, L.kda_last_error().decode()
+
+    for T in (0, K.MAX_DRAFT_TOKENS + 1):
+        rc, msg = verify(T=T)
+        assert rc == K.KDA_ERR_INVALID_ARGUMENT and "T=" in msg
+    rc, msg = verify(state=None)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "state" in msg
+    rc, msg = verify(slot=fake, slots=-2)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "pool_slots" in msg
+    rc, msg = verify(ws=None, wsb=0)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "workspace" in msg
+    rc, msg = verify(u=None)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "u_cache" in msg
+    rc, msg = verify(out=fake)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "alias" in msg
+    rc, msg = verify(u=ctypes.c_void_p(0x20000))
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "alias" in msg
+
+    def commit(acc=fake, T=4, state=ctypes.c_void_p(0x50000), u=ctypes.c_void_p(0x30000)):
+        rc = L.kda_decode_commit(fake, fake, u, state, 0, None, acc, 3, T, 2, 64, 64, 1, ws, 256, None)
+        return rc, L.kda_last_error().decode()
+
+    rc, msg = commit(acc=None)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "accepted_dev" in msg
+    rc, msg = commit(T=17)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "T=" in msg
+    rc, msg = commit(u=ctypes.c_void_p(0x50000))
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "aliases the state" in msg
+    # zero sequences: no-ops
+    assert L.kda_decode_verify(None, None, None, None, None, None, 0, None, 0, 4, 2, 64, 64, 1, None,
+                               None, ws, 256, None) == K.KDA_OK
+    assert L.kda_decode_commit(None, None, None, None, 0, None, None, 0, 4, 2, 64, 64, 1, ws, 256,
+                               None) == K.KDA_OK
+
+
+def test_max_draft_tokens_matches_header():
+    txt = open(os.path.join(ROOT, "include", "kda.h")).read()
+    assert int(re.search(r"#define KDA_MAX_DRAFT_TOKENS (\d+)", txt).group(1)) == K.MAX_DRAFT_TOKENS
+
+
+def test_commit_verify_rejects_bad_arguments():
+    L = K.lib()
+    fake = ctypes.c_void_p(0x10000)
+    ws = ctypes.c_void_p(0x40000)
+    out, u, pu = ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000), ctypes.c_void_p(0x60000)
+    state = ctypes.c_void_p(0x50000)
+
+    def cv(Tp=4, acc=fake, out=out, u=u, pu=pu, pk=fake):
+        rc = L.kda_decode_commit_verify(pk, fake, pu, acc, Tp, fake, fake, fake, fake, fake, state, 0,
+                                        None, 3, 4, 2, 64, 64, 1, out, u, ws, 256, None)
+        return rc, L.kda_last_error().decode()
+
+    for Tp in (0, K.MAX_DRAFT_TOKENS + 1):
+        rc, msg = cv(Tp=Tp)
+        assert rc == K.KDA_ERR_INVALID_ARGUMENT and "T_prev" in msg
+    rc, msg = cv(acc=None)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "accepted_dev" in msg
+    rc, msg = cv(u=pu)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "previous draft" in msg
+    rc, msg = cv(pk=out)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "previous draft" in msg
