@@ -143,11 +143,10 @@ static_assert(SpecSmem<32, 32>(3, 5).cu % 4 == 0 && SpecSmem<128, 128>(1, 16).cu
               SpecSmem<64, 64>(7, 3).cu % 4 == 0, "u rows must be 16-byte aligned");
 
 __device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
-__device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {  // bf16 -> fp32 is exact: a shift
     const uint2 r = *reinterpret_cast<const uint2 *>(p);
-    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.x));
-    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&r.y));
-    return make_float4(lo.x, lo.y, hi.x, hi.y);
+    return make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xffff0000u),
+                       __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xffff0000u));
 }
 // (x, y, z, w) -> pairs (x, x), (y, y), (z, z), (w, w) at dst[0..3]
 __device__ __forceinline__ void st_dup4(float2 *dst, float4 x) {
