@@ -83,17 +83,18 @@ class ClockSampler:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
+    def __init__(self, index, tag="", interval_ms=200):
         self.index = index
+        self.interval_ms = interval_ms
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks{tag}_rank{index}.csv")
 
     def __enter__(self):
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.interval_ms)],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except Exception:
@@ -113,7 +114,7 @@ class ClockSampler:
         if self.proc is None or not os.path.exists(self.path):
             return None
         rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
-        sm, mx, reasons = [], None, set()
+        sm, mx, reasons, pw = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
             r = [x.strip() for x in r]
@@ -122,6 +123,7 @@ class ClockSampler:
             try:
                 sm.append(float(r[1]))
                 mx = float(r[2])
+                pw.append(float(r[3]))
             except ValueError:
                 continue
             for n, v in zip(names, r[5:9]):
@@ -131,7 +133,7 @@ class ClockSampler:
             return None
         load = [s for s in sm if s > 0.5 * (mx or max(sm))] or sm
         return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "power_w": statistics.median(pw) if pw else None}
 
 
 def dist_setup(args):
@@ -343,9 +345,10 @@ def bench_speculative(args, K, stream, ws, decode_ms):
             "gpu_launches": 3 * nsteps}
 
 
-def bench_prefill_workload(wl, K, stream, steps, warmup, rank):
-    """Device-timed kda_prefill of one workload (inputs resident in HBM); returns a summary dict."""
-    inp = W.make_inputs(wl, "cuda", seed=wl.seed + 7919 * rank)
+def bench_prefill_workload(wl, K, stream, steps, warmup, rank, prologue=0):
+    """Device-timed kda_prefill of one workload (inputs resident in HBM); returns a summary dict.
+    With ``prologue`` flags: kda_prefill_prologue on the same draws before activation."""
+    inp = W.make_inputs(wl, "cuda", seed=wl.seed + 7919 * rank, raw=bool(prologue))
     N, T, H = wl.num_seqs, wl.total_tokens, wl.H
     out = torch.empty(T, H, wl.dv, dtype=wl.torch_dtype, device="cuda")
     fs = torch.empty(N, H, wl.dk, wl.dv, dtype=torch.float32, device="cuda")
@@ -355,20 +358,24 @@ def bench_prefill_workload(wl, K, stream, steps, warmup, rank):
     def step():
         K.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["initial_state"],
                   inp["cu_seqlens"], inp["cu_seqlens_dev"], out=out, final_state=fs, workspace=work,
-                  stream=stream)
+                  stream=stream, prologue=prologue, gate_scale=W.GATE_SCALE)
 
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
-    ms = time_events(step, steps, stream)
+    with ClockSampler(torch.cuda.current_device(), tag="_" + wl.name[:12], interval_ms=50) as clk:
+        ms = time_events(step, steps, stream)
     th = T * H
     pk = peaks()
     del inp, out, fs, work
     torch.cuda.empty_cache()
-    return {"workload": wl.name, "tokens": T, "heads": H, "sequences": N, "ms_per_step": ms,
+    name = wl.name + (" raw inputs, fused prologue (q/k L2 norm, gate -softplus, beta sigmoid)"
+                      if prologue else "")
+    return {"workload": name, "tokens": T, "heads": H, "sequences": N, "ms_per_step": ms,
             "tokens_per_s": T / (ms * 1e-3),
             "tc_frac": FLOP_PER_TOKEN_HEAD * th / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
-            "hbm_frac": PREFILL_BYTES_PER_TOKEN_HEAD * th / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+            "hbm_frac": PREFILL_BYTES_PER_TOKEN_HEAD * th / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+            "clocks": clk.summary()}
 
 
 def run_ours(args, rank, local, ws):
@@ -447,8 +454,9 @@ def run_ours(args, rank, local, ws):
     spec = None if args.no_decode else bench_speculative(args, K, stream, ws, dec["ms_per_step"])
     extra = None
     if not args.no_extra:
-        extra = [bench_prefill_workload(W.VARLEN_24, K, stream, 5, 3, rank),
-                 bench_prefill_workload(W.PREFILL_1M, K, stream, 3, 3, rank)]
+        extra = [bench_prefill_workload(W.VARLEN_24, K, stream, 10, 3, rank),
+                 bench_prefill_workload(W.PREFILL_1M, K, stream, 6, 3, rank),
+                 bench_prefill_workload(wl, K, stream, 20, 3, rank, prologue=K.PROLOGUE_ALL)]
 
     if rank != 0:
         return

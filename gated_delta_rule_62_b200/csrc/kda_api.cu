@@ -1,5 +1,6 @@
 // libkda C ABI: host-side validation, planning and dispatch to the kernels.
 // Every argument error is caught here, before anything is enqueued.
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -167,6 +168,32 @@ kda_status_t kda_prefill(const void *q, const void *k, const void *v, const floa
                                   num_seqs, total_tokens, H, d_k, d_v, dtype, out, final_state);
     return run_prefill(p, cu_seqlens_host, workspace, workspace_bytes,
                        reinterpret_cast<cudaStream_t>(stream), "kda_prefill: launch");
+}
+
+kda_status_t kda_prefill_prologue(const void *q, const void *k, const void *v,
+                                  const float *log_alpha, const float *beta,
+                                  const float *initial_state, const int32_t *cu_seqlens_dev,
+                                  const int32_t *cu_seqlens_host, int32_t num_seqs,
+                                  int64_t total_tokens, int32_t H, int32_t d_k, int32_t d_v,
+                                  kda_dtype_t dtype, void *out, float *final_state, void *workspace,
+                                  size_t workspace_bytes, uint32_t prologue_flags, float gate_scale,
+                                  kda_stream_t stream) {
+    constexpr uint32_t kAll =
+        KDA_PROLOGUE_QK_L2NORM | KDA_PROLOGUE_GATE_SOFTPLUS | KDA_PROLOGUE_BETA_SIGMOID;
+    if (prologue_flags & ~kAll)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "prologue_flags 0x%x has unknown bits", prologue_flags);
+    if ((prologue_flags & KDA_PROLOGUE_GATE_SOFTPLUS) && !(gate_scale > 0.f && gate_scale < INFINITY))
+        return fail(KDA_ERR_INVALID_ARGUMENT, "gate_scale=%g must be finite and > 0", (double)gate_scale);
+    kda_status_t st = check_prefill(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev,
+                                    cu_seqlens_host, num_seqs, total_tokens, H, d_k, d_v, dtype,
+                                    out, final_state);
+    if (st != KDA_OK || num_seqs == 0) return st;
+    kda::Problem p = make_problem(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev,
+                                  num_seqs, total_tokens, H, d_k, d_v, dtype, out, final_state);
+    p.pro.flags = prologue_flags;
+    p.pro.gate_scale = gate_scale;
+    return run_prefill(p, cu_seqlens_host, workspace, workspace_bytes,
+                       reinterpret_cast<cudaStream_t>(stream), "kda_prefill_prologue: launch");
 }
 
 kda_status_t kda_prefill_slots(const void *q, const void *k, const void *v, const float *log_alpha,

@@ -76,6 +76,7 @@ struct ChunkParams {
     const int32_t *cu_seqlens;
     const int32_t *order;  // sequences, longest first
     const float *beta;
+    Prologue pro;
     const float *s0;  // initial states, or the state pool
     float *sT;        // final states, or the state pool
     __nv_bfloat16 *out;
@@ -85,7 +86,7 @@ struct ChunkParams {
     StateSlots ss;
 };
 
-template <int DS>
+template <int DS, bool PRO>
 __global__ void __launch_bounds__(NT, 1)
 chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
@@ -229,8 +230,13 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     };
 
     // beta of the next chunk is loaded one chunk ahead (one value per thread < C)
+    const bool raw_beta = PRO && (p.pro.flags & KDA_PROLOGUE_BETA_SIGMOID) != 0;
+    auto load_beta = [&](int64_t t) {
+        const float b = p.beta[(size_t)t * H + h];
+        return raw_beta ? beta_from_raw(b) : b;
+    };
     float beta_next = 0.f;
-    if (nchunks > 0 && tid < C && bos + tid < eos) beta_next = p.beta[(size_t)(bos + tid) * H + h];
+    if (nchunks > 0 && tid < C && bos + tid < eos) beta_next = load_beta(bos + tid);
 
     for (int ci = 0; ci < nchunks; ++ci) {
         const int64_t t0 = bos + (int64_t)ci * C;
@@ -238,15 +244,15 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const bool has_next = ci + 1 < nchunks;
         if (tid < C) {
             s_beta[tid] = beta_next;
-            beta_next = (has_next && t0 + C + tid < eos) ? p.beta[(size_t)(t0 + C + tid) * H + h] : 0.f;
+            beta_next = (has_next && t0 + C + tid < eos) ? load_beta(t0 + C + tid) : 0.f;
         }
         wait_bar(bar_la, ph_la);
         wait_bar(bar_qk, ph_qk);
         la_pending = qk_pending = false;
 
         // ---- gates and gated operands (exact path: also A and L, and S <- diag(gamma) S)
-        const int gate = gate_chunk(sm + SM::QK, sm + SM::KI, sm + SM::AQK, LA, LT, s_beta, s_gamma,
-                                    s_psum, s_flags, valid, tid);
+        const int gate = gate_chunk<PRO>(sm + SM::QK, sm + SM::KI, sm + SM::AQK, LA, LT, s_beta, s_gamma,
+                                    s_psum, s_flags, valid, tid, nullptr, nullptr, 0, 0, p.pro);
         if (gate < 0) break;
         const bool safe = gate == 1;
         if (safe) {
@@ -463,18 +469,18 @@ __global__ void bounded_wait_probe(int32_t *status, uint64_t timeout_ns) {
         atomicOr(status, 1);
 }
 
-template <int DS>
+template <int DS, bool PRO>
 cudaError_t launch_ds(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                       const CUtensorMap &mla, const ChunkParams &cp, unsigned grid,
                       cudaStream_t stream) {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(chunk_kernel<DS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute(chunk_kernel<DS, PRO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)Smem<DS>::BYTES);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    chunk_kernel<DS><<<grid, NT, Smem<DS>::BYTES, stream>>>(mq, mk, mv, mla, cp);
+    chunk_kernel<DS, PRO><<<grid, NT, Smem<DS>::BYTES, stream>>>(mq, mk, mv, mla, cp);
     return cudaGetLastError();
 }
 
@@ -571,6 +577,7 @@ cudaError_t launch_prefill_chunk(const Problem &p, void *workspace, cudaStream_t
     cp.cu_seqlens = p.cu_seqlens;
     cp.order = order;
     cp.beta = p.beta;
+    cp.pro = p.pro;
     cp.s0 = p.initial_state;
     cp.sT = p.final_state;
     cp.out = static_cast<__nv_bfloat16 *>(p.out);
@@ -580,8 +587,11 @@ cudaError_t launch_prefill_chunk(const Problem &p, void *workspace, cudaStream_t
     cp.H = p.H;
     cp.timeout_ns = timeout_ns;
     const unsigned grid = (unsigned)(heads * nsplit);
-    return nsplit == 2 ? launch_ds<64>(mq, mk, mv, mla, cp, grid, stream)
-                       : launch_ds<128>(mq, mk, mv, mla, cp, grid, stream);
+    if (p.pro.flags)
+        return nsplit == 2 ? launch_ds<64, true>(mq, mk, mv, mla, cp, grid, stream)
+                           : launch_ds<128, true>(mq, mk, mv, mla, cp, grid, stream);
+    return nsplit == 2 ? launch_ds<64, false>(mq, mk, mv, mla, cp, grid, stream)
+                       : launch_ds<128, false>(mq, mk, mv, mla, cp, grid, stream);
 }
 
 }  // namespace kda

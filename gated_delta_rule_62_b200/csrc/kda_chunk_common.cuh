@@ -220,14 +220,42 @@ static __device__ __forceinline__ void invert_unit_lower(float *LT, float *PB, u
 // phase with parity src_parity: another thread may still be reading those tiles.
 // Returns 1 for the exact path, 0 for the factored path, -1 if *s_abort was set or the wait
 // timed out (which sets *s_abort).
+// PRO: the prologue (raw q, k rows and raw gates, per pro.flags) is compiled in; without it the
+// function is the plain gating.
+template <bool PRO = false>
 __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK, float *LA,
                                           float *LT, const float *s_beta, float *s_gamma,
                                           float *s_psum, uint32_t *s_abort, int valid,
                                           int tid, uint8_t *KH = nullptr,
                                           uint64_t *src_free = nullptr, uint32_t src_parity = 0,
-                                          uint64_t timeout_ns = 0) {
+                                          uint64_t timeout_ns = 0, const Prologue pro = Prologue()) {
     const int warp = tid >> 5, lane = tid & 31;
     const int to = warp, c4 = 4 * lane;  // token octet 8 to .. 8 to + 7, channels c4 .. c4 + 3
+    if (PRO && (pro.flags & KDA_PROLOGUE_QK_L2NORM)) {
+        // Raw q and k rows -> x / sqrt(x.x + eps), in place. A warp holds its 8 tokens' whole
+        // rows (lane: 4 channels), addressed as in the operand loop below.
+        const uint32_t cx = (uint32_t)(c4 & 63) >> 3;
+        uint8_t *const q0 = QK + (uint32_t)(c4 >> 6) * 16384 + (uint32_t)to * 1024 + (uint32_t)(c4 & 7) * 2;
+        auto widen = [](uint32_t u) { return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u)); };
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (8 * to + i >= valid) break;  // the same for the whole warp
+            const uint32_t off = (uint32_t)i * 128 + ((cx ^ (uint32_t)i) << 4);
+            uint2 *qp = reinterpret_cast<uint2 *>(q0 + off), *kp = reinterpret_cast<uint2 *>(q0 + 8192 + off);
+            const uint2 qu = *qp, ku = *kp;
+            const float2 qa = widen(qu.x), qb = widen(qu.y), ka = widen(ku.x), kb = widen(ku.y);
+            float sq = qa.x * qa.x + qa.y * qa.y + qb.x * qb.x + qb.y * qb.y;
+            float sk = ka.x * ka.x + ka.y * ka.y + kb.x * kb.x + kb.y * kb.y;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                sk += __shfl_xor_sync(0xffffffffu, sk, o);
+            }
+            const float rq = rsqrtf(sq + kL2NormEps), rk = rsqrtf(sk + kL2NormEps);
+            *qp = make_uint2(pack2(qa.x * rq, qa.y * rq), pack2(qb.x * rq, qb.y * rq));
+            *kp = make_uint2(pack2(ka.x * rk, ka.y * rk), pack2(kb.x * rk, kb.y * rk));
+        }
+    }
     // ---- gates: log_alpha of 8 tokens x 4 channels into registers, octet totals
     float4 la[8];
     float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -236,6 +264,11 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
         const int t = 8 * to + i;
         la[i] = (t < valid) ? *reinterpret_cast<const float4 *>(LA + t * D + c4)
                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (PRO && (pro.flags & KDA_PROLOGUE_GATE_SOFTPLUS) && t < valid) {
+            const float sc = pro.gate_scale;
+            la[i] = make_float4(gate_from_raw(la[i].x, sc), gate_from_raw(la[i].y, sc),
+                                gate_from_raw(la[i].z, sc), gate_from_raw(la[i].w, sc));
+        }
         tot.x += la[i].x;
         tot.y += la[i].y;
         tot.z += la[i].z;

@@ -57,6 +57,7 @@ static_assert(SLOT % ROW_BYTES == 0 && RL_BOX <= 256, "ring load box");
 struct SplitParams {
     const int32_t *cu_seqlens;
     const float *beta;
+    Prologue pro;
     const float *s0;  // initial states, or the state pool
     float *sT;        // final states, or the state pool
     __nv_bfloat16 *out;
@@ -401,6 +402,7 @@ constexpr uint32_t TM_D1 = 0, TM_W = 128, TM_D3 = 256, TM_D4 = 384, TM_COLS = 51
 // Producer roles: the compute threads run the gating, the TMEM epilogues and the inverse; the
 // control thread issues the TMA loads, the MMAs and the image's bulk stores, waits for a free
 // ring slot and publishes the image. The phases of one item are separated by CTA barriers.
+template <bool PRO>
 __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
                          const CUtensorMap *tm_la, const CUtensorMap *tm_rs, const SplitParams &p,
                          uint8_t *sm, int pid, int nprod) {
@@ -514,7 +516,8 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         const Item it = decode(k);
         const int64_t t0 = it.bos + (int64_t)it.c * C;
         if (t0 + tid >= it.eos) return 0.f;
-        return p.beta[(size_t)(t0 + tid) * H + it.h];
+        const float b = p.beta[(size_t)(t0 + tid) * H + it.h];
+        return (PRO && (p.pro.flags & KDA_PROLOGUE_BETA_SIGMOID)) ? beta_from_raw(b) : b;
     };
     // the previous image, published once its bulk stores are complete (control thread, during
     // the next item's gating)
@@ -569,9 +572,9 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         if (tid < C) beta_next = load_beta(nxt);
         if (ctl) release();  // the previous item's image, while the compute threads gate
         if (compute) {
-            const int gate = gate_chunk(qk, sm + KI, sm + AQK, reinterpret_cast<float *>(sm + LA), LTp,
+            const int gate = gate_chunk<PRO>(qk, sm + KI, sm + AQK, reinterpret_cast<float *>(sm + LA), LTp,
                                         s_beta, s_gamma, s_psum, s_flags, valid, tid, sm + KH,
-                                        &bars[5], ph_src, p.timeout_ns);
+                                        &bars[5], ph_src, p.timeout_ns, p.pro);
             if (gate < 0) atomicOr(p.status, 1);
             if (tid == 0) s_flags[2] = (uint32_t)(gate + 1);
             fence_proxy_async_smem();
@@ -750,6 +753,7 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 
 constexpr uint32_t SPLIT_SMEM = (cons::BYTES > prod::BYTES ? cons::BYTES : prod::BYTES) + 1024;
 
+template <bool PRO>
 __global__ void __launch_bounds__(NTS, 1)
 split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
@@ -762,7 +766,7 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     if ((int)blockIdx.x < p.heads)
         consumer(&tm_rl, p, sm, blockIdx.x);
     else
-        producer(&tm_q, &tm_k, &tm_v, &tm_la, &tm_rs, p, sm, blockIdx.x - p.heads, gridDim.x - p.heads);
+        producer<PRO>(&tm_q, &tm_k, &tm_v, &tm_la, &tm_rs, p, sm, blockIdx.x - p.heads, gridDim.x - p.heads);
 }
 
 // Zeroes the status word and the ring flags.
@@ -800,11 +804,15 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute(split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)SPLIT_SMEM);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)SPLIT_SMEM);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, split_kernel, NTS, SPLIT_SMEM);
+    const void *kern = p.pro.flags ? (const void *)split_kernel<true> : (const void *)split_kernel<false>;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NTS, SPLIT_SMEM);
     if (e != cudaSuccess) return e;
     const int grid = per_sm * sms;
     if (per_sm < 1 || grid < 2 * heads) return cudaErrorInvalidConfiguration;
@@ -832,6 +840,7 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
     SplitParams sp;
     sp.cu_seqlens = p.cu_seqlens;
     sp.beta = p.beta;
+    sp.pro = p.pro;
     sp.s0 = p.initial_state;
     sp.sT = p.final_state;
     sp.ss = p.slots;
@@ -847,7 +856,7 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
     sp.max_chunks = max_chunks;
     sp.timeout_ns = timeout_ns;
     void *args[] = {&mq, &mk, &mv, &mla, &mrl, &mrs, &sp};
-    return cudaLaunchCooperativeKernel((const void *)split_kernel, dim3(grid), dim3(NTS), args,
+    return cudaLaunchCooperativeKernel(kern, dim3(grid), dim3(NTS), args,
                                        SPLIT_SMEM, stream);
 }
 

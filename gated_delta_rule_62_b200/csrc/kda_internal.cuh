@@ -52,6 +52,20 @@ __device__ __forceinline__ float *final_state_block(float *base, int n, int H, i
     return s < 0 ? nullptr : base + ((size_t)s * H + h) * elems;
 }
 
+// ---- the KDA layer's elementwise prologue (kda_prefill_prologue) -------------------------
+// Raw q, k rows are L2-normalised, raw gates g give log alpha = -scale softplus(g), raw logits b
+// give beta = sigmoid(b), as the kernels load them.
+struct Prologue {
+    uint32_t flags = 0;
+    float gate_scale = 1.f;
+};
+constexpr float kL2NormEps = 1e-6f;
+// -scale softplus(g), softplus(g) = max(g, 0) + log(1 + e^-|g|) (no overflow for any g)
+__device__ __forceinline__ float gate_from_raw(float g, float scale) {
+    return -scale * (fmaxf(g, 0.f) + __logf(1.f + __expf(-fabsf(g))));
+}
+__device__ __forceinline__ float beta_from_raw(float b) { return 1.f / (1.f + __expf(-b)); }
+
 // ---- problem description passed from the API layer to the launchers --------------------
 struct Problem {
     const void *q, *k, *v;
@@ -65,6 +79,7 @@ struct Problem {
     void *out;
     float *final_state;          // or the state pool (with slots)
     StateSlots slots;
+    Prologue pro;
 };
 
 // Each launcher enqueues its kernel(s) on `stream` and returns the launch's cudaError_t.

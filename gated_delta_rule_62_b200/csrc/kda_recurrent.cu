@@ -24,7 +24,8 @@ __global__ void __launch_bounds__(128)
 recurrent_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                  const float *__restrict__ log_alpha, const float *__restrict__ beta,
                  const float *s0, const int32_t *__restrict__ cu_seqlens, int H,
-                 int dv, Tin *__restrict__ out, float *sT, const StateSlots ss) {
+                 int dv, Tin *__restrict__ out, float *sT, const StateSlots ss,
+                 const Prologue pro) {
     constexpr int R = DK / 32;  // key rows per lane
     const int n = blockIdx.x, h = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -59,6 +60,25 @@ recurrent_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin
         float nk[R], nq[R], nl[R], nv[kCols], nb = 0.f;
         if (t + 1 < eos) load(t + 1, nk, nq, nl, nv, nb);
 
+        // the prologue on this token's inputs (the next token's loads stay in flight)
+        if (pro.flags & KDA_PROLOGUE_GATE_SOFTPLUS) {
+#pragma unroll
+            for (int m = 0; m < R; ++m) lc[m] = gate_from_raw(lc[m], pro.gate_scale);
+        }
+        if (pro.flags & KDA_PROLOGUE_BETA_SIGMOID) bt = beta_from_raw(bt);
+        if (pro.flags & KDA_PROLOGUE_QK_L2NORM) {  // raw rows: x / sqrt(x.x + eps), lanes hold all d_k
+            float sk = 0.f, sq = 0.f;
+#pragma unroll
+            for (int m = 0; m < R; ++m) { sk = fmaf(kc[m], kc[m], sk); sq = fmaf(qc[m], qc[m], sq); }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            }
+            const float rk = rsqrtf(sk + kL2NormEps), rq = rsqrtf(sq + kL2NormEps);
+#pragma unroll
+            for (int m = 0; m < R; ++m) { kc[m] *= rk; qc[m] *= rq; }
+        }
         float pa[kCols], pb[kCols], kq = 0.f;
 #pragma unroll
         for (int j = 0; j < kCols; ++j) pa[j] = pb[j] = 0.f;
@@ -115,7 +135,7 @@ cudaError_t launch_typed(const Problem &p, cudaStream_t stream) {
     auto args = [&](auto kern) {
         kern<<<grid, 128, 0, stream>>>((const Tin *)p.q, (const Tin *)p.k, (const Tin *)p.v,
                                        p.log_alpha, p.beta, p.initial_state, p.cu_seqlens, p.H,
-                                       p.dv, (Tin *)p.out, p.final_state, p.slots);
+                                       p.dv, (Tin *)p.out, p.final_state, p.slots, p.pro);
     };
     switch (p.dk) {
         case 32: args(recurrent_kernel<Tin, 32>); break;

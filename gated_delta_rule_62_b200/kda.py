@@ -50,6 +50,9 @@ SIGNATURES = {
                                  _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
     "kda_decode_commit": (_i32, [_vp, _vp, _vp, _vp, _i64, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                  _i32, _vp, _sz, _vp]),
+    "kda_prefill_prologue": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
+                                    _i32, _i32, _vp, _vp, _vp, _sz, ctypes.c_uint32, ctypes.c_float,
+                                    _vp]),
     "kda_decode_commit_verify": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
                                         _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz,
                                         _vp]),
@@ -123,8 +126,11 @@ def workspace_size(num_seqs: int, total_tokens: int, H: int, dk: int, dv: int, d
 
 def prefill(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, cu_seqlens_dev=None,
             out=None, final_state=None, workspace=None, output_final_state=True,
-            algo: str = "auto", stream=None):
+            algo: str = "auto", stream=None, prologue: int = 0, gate_scale: float = 1.0):
     """Chunked KDA prefill over packed sequences (``kda_prefill``).
+
+    prologue: KDA_PROLOGUE_* flags (``kda_prefill_prologue``): q, k, log_alpha, beta hold the
+    layer's raw projections and are activated inside the kernels (gate_scale for the gate).
 
     q, k, log_alpha: [T, H, d_k] (or [B, T, H, d_k]); v: [T, H, d_v]; beta [T, H].
     cu_seqlens: host int32 offsets [N + 1] (default: one sequence, or B equal ones
@@ -174,14 +180,20 @@ def prefill(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, cu_se
               _ptr(cu_seqlens_dev), ctypes.c_void_p(cu_host.data_ptr()), N, Ttot, H, dk, dv, code,
               _ptr(out), _ptr(final_state)]
     if algo == "recurrent":
+        if prologue:
+            raise ValueError("the prologue runs through kda_prefill_prologue (algo='auto')")
         _check(L.kda_prefill_recurrent(*common, _stream(stream)), "kda_prefill_recurrent")
     elif algo == "auto":
         need = workspace_size(N, Ttot, H, dk, dv, dtype)
         if workspace is None:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         _need(workspace, "workspace", torch.uint8, 1)
-        _check(L.kda_prefill(*common, _ptr(workspace), workspace.numel(), _stream(stream)),
-               "kda_prefill")
+        if prologue:
+            _check(L.kda_prefill_prologue(*common, _ptr(workspace), workspace.numel(), int(prologue),
+                                          float(gate_scale), _stream(stream)), "kda_prefill_prologue")
+        else:
+            _check(L.kda_prefill(*common, _ptr(workspace), workspace.numel(), _stream(stream)),
+                   "kda_prefill")
     else:
         raise ValueError(f"unknown algo {algo!r}")
     if dense:
@@ -297,6 +309,8 @@ def decode_step_slots(q, k, v, log_alpha, beta, state_pool, slot, out=None, work
 
 
 MAX_DRAFT_TOKENS = 16
+PROLOGUE_QK_L2NORM, PROLOGUE_GATE_SOFTPLUS, PROLOGUE_BETA_SIGMOID = 1, 2, 4
+PROLOGUE_ALL = 7
 
 
 def _pool_args(state, slot, N, H, dk, dv):

@@ -106,14 +106,21 @@ def cu_seqlens_of(seqlens) -> np.ndarray:
     return out
 
 
+# log alpha = -softplus(g) * GATE_SCALE with g ~ N(0, 1) (the workloads' gate distribution)
+GATE_SCALE = 1.0 / 16.0
+
+
 def _l2n(x: torch.Tensor) -> torch.Tensor:
     # Input recipe, not method arithmetic: unit-norm keys/queries per token and head.
     return x / torch.linalg.vector_norm(x, dim=-1, keepdim=True).clamp_min(1e-30)
 
 
 def draw_tokens(gen: torch.Generator, ntok: int, H: int, dk: int, dv: int,
-                dtype: torch.dtype, device) -> dict:
-    """Draw ``ntok`` tokens of (q, k, v, beta, log_alpha) in blocks of _DRAW_BLOCK."""
+                dtype: torch.dtype, device, raw: bool = False) -> dict:
+    """Draw ``ntok`` tokens of (q, k, v, beta, log_alpha) in blocks of _DRAW_BLOCK.
+
+    ``raw``: the same draws before activation (q, k not normalised; ``log_alpha`` holds the
+    N(0, 1) gates and ``beta`` the N(0, 1) logits), the inputs of the fused-prologue prefill."""
     q = torch.empty(ntok, H, dk, dtype=dtype, device=device)
     k = torch.empty(ntok, H, dk, dtype=dtype, device=device)
     v = torch.empty(ntok, H, dv, dtype=dtype, device=device)
@@ -122,15 +129,18 @@ def draw_tokens(gen: torch.Generator, ntok: int, H: int, dk: int, dv: int,
     for s in range(0, ntok, _DRAW_BLOCK):
         n = min(_DRAW_BLOCK, ntok - s)
         f32 = dict(dtype=torch.float32, device=device, generator=gen)
-        q[s:s + n] = _l2n(torch.randn(n, H, dk, **f32)).to(dtype)
-        k[s:s + n] = _l2n(torch.randn(n, H, dk, **f32)).to(dtype)
+        act = (lambda x: x) if raw else _l2n
+        q[s:s + n] = act(torch.randn(n, H, dk, **f32)).to(dtype)
+        k[s:s + n] = act(torch.randn(n, H, dk, **f32)).to(dtype)
         v[s:s + n] = torch.randn(n, H, dv, **f32).to(dtype)
-        beta[s:s + n] = torch.sigmoid(torch.randn(n, H, **f32))
-        la[s:s + n] = -torch.nn.functional.softplus(torch.randn(n, H, dk, **f32)) / 16.0
+        b = torch.randn(n, H, **f32)
+        beta[s:s + n] = b if raw else torch.sigmoid(b)
+        g = torch.randn(n, H, dk, **f32)
+        la[s:s + n] = g if raw else -torch.nn.functional.softplus(g) * GATE_SCALE
     return {"q": q, "k": k, "v": v, "beta": beta, "log_alpha": la}
 
 
-def make_inputs(wl: Workload, device="cpu", seed: Optional[int] = None) -> dict:
+def make_inputs(wl: Workload, device="cpu", seed: Optional[int] = None, raw: bool = False) -> dict:
     """Prefill inputs of a workload: q, k, v, beta, log_alpha, initial_state, cu_seqlens.
 
     ``initial_state`` is None for a zero start. ``cu_seqlens`` is a CPU int32
@@ -140,7 +150,7 @@ def make_inputs(wl: Workload, device="cpu", seed: Optional[int] = None) -> dict:
     device = torch.device(device)
     gen = torch.Generator(device=device)
     gen.manual_seed(wl.seed if seed is None else seed)
-    d = draw_tokens(gen, wl.total_tokens, wl.H, wl.dk, wl.dv, wl.torch_dtype, device)
+    d = draw_tokens(gen, wl.total_tokens, wl.H, wl.dk, wl.dv, wl.torch_dtype, device, raw=raw)
     if wl.init_state == "normal":
         d["initial_state"] = 0.02 * torch.randn(wl.num_seqs, wl.H, wl.dk, wl.dv,
                                                 dtype=torch.float32, device=device, generator=gen)

@@ -164,6 +164,39 @@ KDA_API kda_status_t kda_decode_step(const void *q, const void *k, const void *v
                              void *out, void *workspace, size_t workspace_bytes,
                              kda_stream_t stream);
 
+/* Prologue flags for kda_prefill_prologue: which inputs hold the layer's raw projections. */
+#define KDA_PROLOGUE_QK_L2NORM 1u     /* q and k: each (token, head) row x becomes x / sqrt(x.x + 1e-6) */
+#define KDA_PROLOGUE_GATE_SOFTPLUS 2u /* log_alpha holds gates g: log alpha = -gate_scale * softplus(g) */
+#define KDA_PROLOGUE_BETA_SIGMOID 4u  /* beta holds logits b: beta = 1 / (1 + e^-b) */
+
+/*
+ * kda_prefill with the KDA layer's elementwise prologue fused into the
+ * kernels' input staging: with the flags above, q and k are L2-normalised per
+ * (token, head) row, the forgetting gate is log alpha = -gate_scale *
+ * softplus(g) per key channel and beta = sigmoid(b), each applied as the chunk
+ * kernels (and the token-serial kernel) load their inputs, so the activated
+ * tensors are never written to HBM. ("Kimi Delta Attention: the load-bearing
+ * choice" in the shivam2003.com Kimi K3 article: per-channel forgetting gates
+ * and a writing strength; the L2 normalisation of q and k keeps the delta
+ * rule's step within its stable range.) prologue_flags is any combination of
+ * KDA_PROLOGUE_* (0: exactly kda_prefill); gate_scale must be finite and > 0
+ * when KDA_PROLOGUE_GATE_SOFTPLUS is set. Tokens past a sequence's end are
+ * never read. Arguments, workspace, results and status otherwise as
+ * kda_prefill; the results equal kda_prefill's on the activated inputs up to
+ * rounding (the activated q and k are rounded to bf16 once more for bf16
+ * inputs).
+ */
+KDA_API kda_status_t kda_prefill_prologue(const void *q, const void *k, const void *v,
+                                          const float *log_alpha, const float *beta,
+                                          const float *initial_state,
+                                          const int32_t *cu_seqlens_dev,
+                                          const int32_t *cu_seqlens_host, int32_t num_seqs,
+                                          int64_t total_tokens, int32_t H, int32_t d_k,
+                                          int32_t d_v, kda_dtype_t dtype, void *out,
+                                          float *final_state, void *workspace,
+                                          size_t workspace_bytes, uint32_t prologue_flags,
+                                          float gate_scale, kda_stream_t stream);
+
 /*
  * kda_prefill with the states held in a pool of slots instead of one state per
  * sequence: the prefill cache of "Kimi K3 -- the architecture and

@@ -144,3 +144,43 @@ def forward_np(q, k, v, log_alpha, beta, initial_state=None):
             S[h] += beta[t, h] * np.outer(k[t, h], v[t, h] - pred)  # write the error only
             out[t, h] = S[h].T @ q[t, h]                     # read after the write
     return out, S
+
+
+# ---- the KDA layer's elementwise prologue (what kda_prefill_prologue fuses) ----------------
+# Sources: "Kimi Delta Attention: the load-bearing choice" (shivam2003.com Kimi K3 article):
+# per-key-channel forgetting gates alpha in (0, 1] and a writing strength beta; the synthetic
+# workloads draw q, k ~ N(0, 1) then L2-normalise them per token, log alpha = -softplus(g)/16 and
+# beta = sigmoid(b) with g, b ~ N(0, 1). The epsilon inside the norm is this library's reading.
+L2NORM_EPS = 1e-6
+QK_L2NORM, GATE_SOFTPLUS, BETA_SIGMOID = 1, 2, 4
+
+
+def l2_normalise(x):
+    """Rows along the last axis divided by sqrt(sum of squares + L2NORM_EPS), fp64."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + L2NORM_EPS)
+
+
+def softplus(x):
+    """log(1 + e^x), fp64, without overflow: max(x, 0) + log(1 + e^-|x|)."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x)))
+
+
+def sigmoid(x):
+    """1 / (1 + e^-x), fp64, without overflow."""
+    x = np.asarray(x, dtype=np.float64)
+    e = np.exp(-np.abs(x))
+    return np.where(x >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def prologue(q, k, log_alpha, beta, flags, gate_scale=1.0):
+    """The activated (q, k, log_alpha, beta) from raw ones, per ``flags`` (fp64 arrays)."""
+    q, k, la, b = (np.asarray(x, dtype=np.float64) for x in (q, k, log_alpha, beta))
+    if flags & QK_L2NORM:
+        q, k = l2_normalise(q), l2_normalise(k)
+    if flags & GATE_SOFTPLUS:
+        la = -gate_scale * softplus(la)
+    if flags & BETA_SIGMOID:
+        b = sigmoid(b)
+    return q, k, la, b

@@ -234,3 +234,32 @@ def test_commit_verify_rejects_bad_arguments():
     assert rc == K.KDA_ERR_INVALID_ARGUMENT and "previous draft" in msg
     rc, msg = cv(pk=out)
     assert rc == K.KDA_ERR_INVALID_ARGUMENT and "previous draft" in msg
+
+
+def test_prologue_entry_point_rejects_bad_arguments():
+    L = K.lib()
+    fake = ctypes.c_void_p(0x10000)
+    cu = (ctypes.c_int32 * 2)(0, 5)
+    cuh = ctypes.cast(cu, ctypes.c_void_p)
+
+    def call(flags, scale):
+        rc = L.kda_prefill_prologue(fake, fake, fake, fake, fake, None, fake, cuh, 1, 5, 2, 32, 32, 0,
+                                    ctypes.c_void_p(0x20000), None, None, 0, flags, scale, None)
+        return rc, L.kda_last_error().decode()
+
+    rc, msg = call(8, 1.0)
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "unknown bits" in msg
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        rc, msg = call(K.PROLOGUE_GATE_SOFTPLUS, bad)
+        assert rc == K.KDA_ERR_INVALID_ARGUMENT and "gate_scale" in msg
+    rc, msg = call(K.PROLOGUE_ALL, 1.0 / 16)  # valid up to the missing workspace
+    assert rc == K.KDA_ERR_INVALID_ARGUMENT and "workspace" in msg
+
+
+def test_prologue_flags_match_header():
+    txt = open(os.path.join(ROOT, "include", "kda.h")).read()
+    got = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define KDA_PROLOGUE_(\w+) (\d+)u", txt)}
+    assert got == {"QK_L2NORM": K.PROLOGUE_QK_L2NORM, "GATE_SOFTPLUS": K.PROLOGUE_GATE_SOFTPLUS,
+                   "BETA_SIGMOID": K.PROLOGUE_BETA_SIGMOID}
+    import oracle
+    assert (oracle.QK_L2NORM, oracle.GATE_SOFTPLUS, oracle.BETA_SIGMOID) == (1, 2, 4)
