@@ -203,3 +203,47 @@ def pin_key_channel_decay(fwd, seed=61):
 ALL_PINS = [pin_golden, pin_noop, pin_exact_recall, pin_orthonormal_recall, pin_pure_decay,
             pin_brute_force, pin_linearity, pin_value_permutation, pin_resume,
             pin_key_channel_decay]
+
+
+# ---- the prologue functions (q/k L2 normalisation, gate -softplus, beta sigmoid) -------------
+# Each pin takes an object with softplus(x), sigmoid(x), l2_normalise(x) and L2NORM_EPS, and
+# checks it against closed forms and identities that owe nothing to its code.
+def pin_softplus(f):
+    assert abs(float(f.softplus(0.0)) - math.log(2.0)) < 1e-15          # log(1 + 1)
+    assert abs(float(f.softplus(math.log(3.0))) - math.log(4.0)) < 1e-15  # log(1 + 3)
+    x = np.linspace(-40.0, 40.0, 801)
+    y = f.softplus(x)
+    # softplus(x) - softplus(-x) = log((1 + e^x) / (1 + e^-x)) = x
+    assert np.max(np.abs(y - f.softplus(-x) - x)) < 1e-12
+    assert np.all(y > 0) and np.all(np.diff(y) > 0)
+    assert float(f.softplus(800.0)) == 800.0 and float(f.softplus(-800.0)) == 0.0  # no overflow
+
+
+def pin_sigmoid(f):
+    assert float(f.sigmoid(0.0)) == 0.5
+    assert abs(float(f.sigmoid(math.log(3.0))) - 0.75) < 1e-15           # 3 / (1 + 3)
+    x = np.linspace(-40.0, 40.0, 801)
+    assert np.max(np.abs(f.sigmoid(x) + f.sigmoid(-x) - 1.0)) < 1e-15
+    assert float(f.sigmoid(800.0)) == 1.0 and float(f.sigmoid(-800.0)) == 0.0
+
+
+def pin_softplus_slope_is_sigmoid(f, h=1e-5):
+    x = np.linspace(-40.0, 40.0, 801)
+    d = (f.softplus(x + h) - f.softplus(x - h)) / (2 * h)
+    assert np.max(np.abs(d - f.sigmoid(x))) < 1e-8
+
+
+def pin_l2_normalise(f):
+    y = f.l2_normalise(np.array([[3.0, 4.0], [0.0, 0.0]]))
+    assert np.max(np.abs(y[0] - np.array([0.6, 0.8]))) < 1e-7   # eps / 25 relative
+    assert np.all(y[1] == 0.0)
+    x = _rng(3).standard_normal((7, 5, 128))
+    z = f.l2_normalise(x)
+    n = np.linalg.norm(x, axis=-1)
+    want = n / np.sqrt(n * n + f.L2NORM_EPS)
+    assert np.max(np.abs(np.linalg.norm(z, axis=-1) - want)) < 1e-12
+    # parallel to the input: z . x = |x|^2 / sqrt(|x|^2 + eps)
+    assert np.max(np.abs(np.sum(z * x, -1) - n * want)) < 1e-10
+
+
+PROLOGUE_PINS = [pin_softplus, pin_sigmoid, pin_softplus_slope_is_sigmoid, pin_l2_normalise]

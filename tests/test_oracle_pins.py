@@ -75,39 +75,9 @@ def test_window_bound_holds():
 
 
 # ---- the prologue functions, pinned to closed forms and identities ---------------------------
-def test_softplus_pins():
-    assert oracle.softplus(0.0) == pytest.approx(np.log(2.0), abs=1e-15)    # log(1 + 1)
-    assert oracle.softplus(np.log(3.0)) == pytest.approx(np.log(4.0), abs=1e-15)  # log(1 + 3)
-    x = np.linspace(-40.0, 40.0, 801)
-    # softplus(x) - softplus(-x) = log((1 + e^x) / (1 + e^-x)) = x
-    assert np.max(np.abs(oracle.softplus(x) - oracle.softplus(-x) - x)) < 1e-12
-    assert np.all(oracle.softplus(x) > 0) and np.all(np.diff(oracle.softplus(x)) > 0)
-    assert oracle.softplus(800.0) == 800.0 and oracle.softplus(-800.0) == 0.0  # no overflow
-
-
-def test_sigmoid_pins():
-    assert oracle.sigmoid(0.0) == 0.5
-    assert oracle.sigmoid(np.log(3.0)) == pytest.approx(0.75, abs=1e-15)    # 3 / (1 + 3)
-    x = np.linspace(-40.0, 40.0, 801)
-    assert np.max(np.abs(oracle.sigmoid(x) + oracle.sigmoid(-x) - 1.0)) < 1e-15
-    assert oracle.sigmoid(800.0) == 1.0 and oracle.sigmoid(-800.0) == 0.0
-    # d/dx softplus = sigmoid (central difference)
-    h = 1e-5
-    d = (oracle.softplus(x + h) - oracle.softplus(x - h)) / (2 * h)
-    assert np.max(np.abs(d - oracle.sigmoid(x))) < 1e-8
-
-
-def test_l2_normalise_pins():
-    y = oracle.l2_normalise(np.array([[3.0, 4.0], [0.0, 0.0]]))
-    assert y[0] == pytest.approx([0.6, 0.8], abs=1e-7)  # eps / 25 relative
-    assert np.all(y[1] == 0.0)
-    rng = np.random.default_rng(3)
-    x = rng.standard_normal((7, 5, 128))
-    z = oracle.l2_normalise(x)
-    n = np.linalg.norm(x, axis=-1)
-    assert np.max(np.abs(np.linalg.norm(z, axis=-1) - n / np.sqrt(n * n + oracle.L2NORM_EPS))) < 1e-12
-    # parallel to the input: z . x = |x|^2 / sqrt(|x|^2 + eps)
-    assert np.max(np.abs(np.sum(z * x, -1) - n * n / np.sqrt(n * n + oracle.L2NORM_EPS))) < 1e-10
+@pytest.mark.parametrize("pin", pins.PROLOGUE_PINS, ids=lambda f: f.__name__)
+def test_prologue_pin(pin):
+    pin(oracle)
 
 
 def test_prologue_flags_are_independent():
