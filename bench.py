@@ -10,7 +10,11 @@ I/O) of the 8192-token, 32-head, d=128 bf16 workload through ``kda_prefill``.
 with the step's inputs copied from pinned host memory and its outputs read back
 inside the timed region. The decode step (256 sequences x 32 heads, fp32 state
 of 512 MiB streamed once in and once out) is measured in the same run and
-reported under ``decode``. Inputs (404 MB prefill, 512 MiB decode state) are
+reported under ``decode``; speculative decode on the same states (verify 4 draft
+tokens, commit them, and the fused commit + verify step) under
+``speculative_decode``; the varlen-24 and 1M-token prefills and the headline
+prefill on raw inputs through the fused prologue under
+``other_prefill_workloads``. Inputs (404 MB prefill, 512 MiB decode state) are
 larger than L2, so no L2 flush is done between timed iterations.
 
 Multi-GPU (torchrun): every rank runs its own replica of the workload (sequences
