@@ -85,7 +85,8 @@ class ClockSampler:
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+         "clocks.mem,temperature.memory")
 
     def __init__(self, index, tag="", interval_ms=200):
         self.index = index
@@ -118,7 +119,7 @@ class ClockSampler:
         if self.proc is None or not os.path.exists(self.path):
             return None
         rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
-        sm, mx, reasons, pw = [], None, set(), []
+        sm, mx, reasons, pw, mem, mtemp = [], None, set(), [], [], []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
             r = [x.strip() for x in r]
@@ -133,11 +134,18 @@ class ClockSampler:
             for n, v in zip(names, r[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
+            for col, dst in ((9, mem), (10, mtemp)):  # may read N/A on some boards
+                try:
+                    dst.append(float(r[col]))
+                except (IndexError, ValueError):
+                    pass
         if not sm:
             return None
         load = [s for s in sm if s > 0.5 * (mx or max(sm))] or sm
         return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm), "power_w": statistics.median(pw) if pw else None}
+                "samples": len(sm), "power_w": statistics.median(pw) if pw else None,
+                "mem_mhz": statistics.median(mem) if mem else None,
+                "mem_temp_c": max(mtemp) if mtemp else None}
 
 
 def dist_setup(args):
@@ -411,6 +419,7 @@ def run_ours(args, rank, local, ws):
         torch.cuda.synchronize()
         ms = time_events(step, args.steps, stream)
         torch.cuda.synchronize()
+    kernels_per_step_measured = K.last_launch_count()  # this library's kernels in one step
     barrier(ws)
     ms = max_over_ranks(ms, ws)
     clocks = clk.summary()
@@ -510,7 +519,7 @@ def run_ours(args, rank, local, ws):
     cpu = None
     if ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(wl, seconds_target=args.cpu_seconds)
-    kernels_per_step = K.LAST_LAUNCH_COUNT if hasattr(K, "LAST_LAUNCH_COUNT") else 1
+    kernels_per_step = kernels_per_step_measured
     line = {
         "metric": METRIC, "value": T * ws / (ms * 1e-3), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,

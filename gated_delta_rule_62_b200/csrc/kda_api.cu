@@ -11,6 +11,7 @@
 namespace {
 
 thread_local std::string g_last_error;
+thread_local int32_t g_last_launches = 0;  // kernels enqueued by the thread's last successful call
 
 kda_status_t fail(kda_status_t st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
 kda_status_t fail(kda_status_t st, const char *fmt, ...) {
@@ -26,6 +27,12 @@ kda_status_t fail(kda_status_t st, const char *fmt, ...) {
 kda_status_t ok() {
     g_last_error.clear();
     return KDA_OK;
+}
+
+// Success after enqueuing `n` of this library's kernels (memsets and copies are not counted).
+kda_status_t launched(int32_t n) {
+    g_last_launches = n;
+    return ok();
 }
 
 kda_status_t cuda_fail(cudaError_t e, const char *where) {
@@ -127,7 +134,7 @@ kda_status_t run_prefill(kda::Problem &p, const int32_t *cu_seqlens_host, void *
         if (e == cudaSuccess) e = kda::launch_prefill_recurrent(p, s);
     }
     if (e != cudaSuccess) return cuda_fail(e, who);
-    return ok();
+    return launched(kda::chunk_supported(p) ? 2 : 1);  // init/plan + chunk kernel, or token-serial
 }
 
 }  // namespace
@@ -240,7 +247,7 @@ kda_status_t kda_prefill_recurrent(const void *q, const void *k, const void *v,
                                   num_seqs, total_tokens, H, d_k, d_v, dtype, out, final_state);
     cudaError_t e = kda::launch_prefill_recurrent(p, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kda_prefill_recurrent: launch");
-    return ok();
+    return launched(1);
 }
 
 kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -271,7 +278,7 @@ kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const 
     p.num_seqs = num_seqs; p.H = H; p.dk = d_k; p.dv = d_v; p.dtype = dtype; p.out = out;
     cudaError_t e = kda::launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step: launch");
-    return ok();
+    return launched(1);
 }
 
 kda_status_t kda_decode_step_slots(const void *q, const void *k, const void *v,
@@ -316,7 +323,7 @@ kda_status_t kda_decode_step_slots(const void *q, const void *k, const void *v,
     cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
     if (e == cudaSuccess) e = kda::launch_decode(p, s);
     if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step_slots: launch");
-    return ok();
+    return launched(1);
 }
 
 }  // extern "C"
@@ -397,7 +404,7 @@ kda_status_t launch_spec(const char *who, kda::VerifyProblem &p, int64_t pool_sl
     cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
     if (e == cudaSuccess) e = kda::launch_verify(p, s);
     if (e != cudaSuccess) return cuda_fail(e, who);
-    return ok();
+    return launched(1);
 }
 
 }  // namespace
@@ -516,9 +523,11 @@ kda_status_t kda_selftest_bounded_wait(void *workspace, size_t workspace_bytes,
     cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
     if (e == cudaSuccess) e = kda::launch_bounded_wait_probe(workspace, timeout_ns, s);
     if (e != cudaSuccess) return cuda_fail(e, "kda_selftest_bounded_wait: launch");
-    return ok();
+    return launched(1);
 }
 
 int32_t kda_version(void) { return 100; }
+
+int32_t kda_last_launch_count(void) { return g_last_launches; }
 
 }  // extern "C"

@@ -39,6 +39,7 @@ SIGNATURES = {
     "kda_last_error": (ctypes.c_char_p, []),
     "kda_read_device_status": (_i32, [_vp, _vp]),
     "kda_version": (_i32, []),
+    "kda_last_launch_count": (_i32, []),
     "kda_selftest_bounded_wait": (_i32, [_vp, _sz, ctypes.c_uint64, _vp]),
     "kda_prefill_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                                    _i32, _i32, _vp, _vp, _vp]),
@@ -428,6 +429,11 @@ def decode_commit_verify(prev_k, prev_log_alpha, prev_u, accepted, q, k, v, log_
                                           _ptr(workspace), workspace.numel(), _stream(stream)),
            "kda_decode_commit_verify")
     return out, u_cache
+
+
+def last_launch_count() -> int:
+    """Kernels enqueued by this thread's last successful library call (``kda_last_launch_count``)."""
+    return int(lib().kda_last_launch_count())
 
 
 def selftest_bounded_wait(workspace, timeout_ns: int, stream=None):

@@ -335,6 +335,15 @@ KDA_API kda_status_t kda_decode_commit_verify(const void *prev_k, const float *p
                                               void *workspace, size_t workspace_bytes,
                                               kda_stream_t stream);
 
+/*
+ * Number of this library's kernels that the calling thread's last successful
+ * prefill, decode or speculative-decode call enqueued (memsets and copies are
+ * not counted): 2 for the chunked prefill (a planning or initialisation kernel
+ * and the chunk kernel), 1 for the token-serial prefill, the decode step and
+ * each speculative-decode call. 0 before any such call. Diagnostic only.
+ */
+KDA_API int32_t kda_last_launch_count(void);
+
 /* Static string naming a status code. Never NULL. */
 KDA_API const char *kda_status_string(kda_status_t status);
 
