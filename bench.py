@@ -62,6 +62,24 @@ def measured_traffic():
     return SPLIT_TRAFFIC_BYTES if h.hexdigest() == SPLIT_TRAFFIC_SOURCES_SHA256 else None
 # Decode: state read + write (fp32) + q, k, v + log_alpha + beta + out.
 DECODE_BYTES_PER_TOKEN_HEAD = 2 * 128 * 128 * 4 + 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch of each decode-side kernel on the
+# decode workload (ncu, one capture each), reported while kda_decode.cu and kda_internal.cuh hash
+# to the sources they were taken on.
+DECODE_SIDE_TRAFFIC = {"decode": 547.409152e6 + 479.214336e6, "verify": 581.512192e6 + 10.139392e6,
+                       "commit": 602.596608e6 + 480.340992e6,
+                       "commit_verify": 802.48832e6 + 505.373952e6}
+DECODE_SIDE_SOURCES_SHA256 = "a0901424501414022377629fe654c9a9d34e9e5a922a5e5d3ae32419e8122e94"
+
+
+def decode_side_traffic(kernel):
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("kda_decode.cu", "kda_internal.cuh"):
+        with open(os.path.join(ROOT, "gated_delta_rule_62_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return DECODE_SIDE_TRAFFIC[kernel] if h.hexdigest() == DECODE_SIDE_SOURCES_SHA256 else None
+
+
 # Speculative decode, per (sequence, head) and draft token: verify reads the state once and per
 # token q, k, v (bf16), log_alpha, beta, writes out (bf16) and u (fp32); commit reads and writes the
 # state once and per accepted token reads k, log_alpha and u.
@@ -281,7 +299,7 @@ def bench_decode(args, K, stream, ws):
     return {"workload": wl.name, "steps": nsteps, "ms_per_step": ms,
             "tokens_per_s": wl.num_seqs * ws / (ms * 1e-3),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "frac": gbs / pk["hbm_gbs"], "traffic": decode_side_traffic("decode"),
                          "bytes_per_token_head": DECODE_BYTES_PER_TOKEN_HEAD,
                          "peak_source": pk["source"]},
             "gpu_launches": nsteps}
@@ -338,10 +356,11 @@ def bench_speculative(args, K, stream, ws, decode_ms):
         timed[name] = max_over_ranks(time_events(fn, nsteps, stream), ws)
     pk = peaks()
 
-    def roof(state_b, tok_b, ms):
+    def roof(state_b, tok_b, ms, kernel):
         gbs = N * H * (state_b + T * tok_b) / (ms * 1e-3) / 1e9
         return {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": gbs / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"]}
+                "frac": gbs / pk["hbm_gbs"], "traffic": decode_side_traffic(kernel),
+                "peak_source": pk["source"]}
 
     del x, out, u, state
     torch.cuda.empty_cache()
@@ -351,9 +370,10 @@ def bench_speculative(args, K, stream, ws, decode_ms):
             "commit_ms": timed["commit"], "ms_per_step": ms,
             "tokens_per_s": N * T * ws / (ms * 1e-3),
             "speedup_vs_single_steps": None if decode_ms is None else T * decode_ms / ms,
-            "roofline": roof(COMMIT_STATE_BYTES, VERIFY_TOKEN_BYTES + COMMIT_TOKEN_BYTES, ms),
-            "verify_roofline": roof(VERIFY_STATE_BYTES, VERIFY_TOKEN_BYTES, timed["verify"]),
-            "commit_roofline": roof(COMMIT_STATE_BYTES, COMMIT_TOKEN_BYTES, timed["commit"]),
+            "roofline": roof(COMMIT_STATE_BYTES, VERIFY_TOKEN_BYTES + COMMIT_TOKEN_BYTES, ms,
+                             "commit_verify"),
+            "verify_roofline": roof(VERIFY_STATE_BYTES, VERIFY_TOKEN_BYTES, timed["verify"], "verify"),
+            "commit_roofline": roof(COMMIT_STATE_BYTES, COMMIT_TOKEN_BYTES, timed["commit"], "commit"),
             "gpu_launches": 3 * nsteps}
 
 
