@@ -82,3 +82,20 @@ def test_prologue_strong_raw_gates_take_the_exact_path():
     scale = float(raw["v"].abs().max())
     assert_close(out, ref_o, TOL["bf16"], scale, "out")
     assert_close(fs, ref_s, TOL["bf16"], scale, "final state")
+
+
+def test_prologue_8k_full_size():
+    """The headline workload (8192 tokens x 32 heads, split-role kernel) on raw inputs."""
+    wl = W.PREFILL_8K
+    raw = W.make_inputs(wl, DEV, raw=True)
+    out, fs = K.prefill(raw["q"], raw["k"], raw["v"], raw["log_alpha"], raw["beta"], None,
+                        raw["cu_seqlens"], raw["cu_seqlens_dev"], prologue=K.PROLOGUE_ALL,
+                        gate_scale=W.GATE_SCALE)
+    torch.cuda.synchronize()
+    q, k, la, b = oracle.prologue(f64(raw["q"]), f64(raw["k"]), f64(raw["log_alpha"]), f64(raw["beta"]),
+                                  K.PROLOGUE_ALL, W.GATE_SCALE)
+    ref_o, ref_s = oracle.forward(q, k, f64(raw["v"]), la, b, None,
+                                  raw["cu_seqlens"].numpy().astype(np.int64))
+    scale = float(raw["v"].abs().max())
+    assert_close(out, ref_o, TOL["bf16"], scale, "out")
+    assert_close(fs, ref_s, TOL["bf16"], scale, "final state")

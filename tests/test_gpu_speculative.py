@@ -207,3 +207,44 @@ def test_speculative_loop_matches_oracle_on_accepted_tokens(use_slots):
         _, s_fin = oracle.forward(ctx["q"], ctx["k"], ctx["v"], ctx["log_alpha"], ctx["beta"],
                                   s_ref[n][None])
         assert_close(pool[rows[n]], s_fin[0], TOL[dtype], scale, f"final state seq {n}")
+
+
+def test_speculative_decode_256_full_size():
+    """The decode workload's 256 x 32 states (seeded by the GPU prefill), 4 draft tokens each:
+    verify, then the fused commit (a mix of accepted counts) + verify of a second draft."""
+    wl = W.DECODE_256
+    inp = W.make_inputs(wl, DEV)
+    _, state = K.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], None,
+                         inp["cu_seqlens"], inp["cu_seqlens_dev"])
+    N, H, T = wl.num_seqs, wl.H, 4
+    g = torch.Generator(device=DEV).manual_seed(99)
+    drafts = []
+    for _ in range(2):
+        st = W.make_decode_steps(wl, g, T, DEV)  # [T, N, ...] -> [N, T, ...]
+        drafts.append({n: t.transpose(0, 1).contiguous() for n, t in st.items()})
+    s0 = f64(state)
+    x = drafts[0]
+    out, u = K.decode_verify(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], state)
+    accepted = torch.arange(N, dtype=torch.int32, device=DEV) % (T + 1)
+    y = drafts[1]
+    out2, _ = K.decode_commit_verify(x["k"], x["log_alpha"], u, accepted, y["q"], y["k"], y["v"],
+                                     y["log_alpha"], y["beta"], state)
+    torch.cuda.synchronize()
+    scale = max(float(x["v"].abs().max()), float(y["v"].abs().max()))
+    cu = np.arange(N + 1, dtype=np.int64) * T
+    ref_o, _ = oracle.forward(*(f64(x[m]).reshape(N * T, *x[m].shape[2:]) for m in
+                                ("q", "k", "v", "log_alpha", "beta")), s0, cu)
+    assert_close(out.reshape(N * T, H, -1), ref_o, TOL["bf16"], scale, "verify out")
+    acc = accepted.cpu().numpy()
+    s1 = np.empty_like(s0)
+    for n in range(N):  # the states after each sequence's accepted prefix
+        if acc[n] == 0:
+            s1[n] = s0[n]
+        else:
+            _, s = oracle.forward(*(f64(x[m][n, :acc[n]]) for m in ("q", "k", "v", "log_alpha", "beta")),
+                                  s0[n][None])
+            s1[n] = s[0]
+    assert_close(state, s1, TOL["bf16"], scale, "committed states")
+    ref_o2, _ = oracle.forward(*(f64(y[m]).reshape(N * T, *y[m].shape[2:]) for m in
+                                 ("q", "k", "v", "log_alpha", "beta")), s1, cu)
+    assert_close(out2.reshape(N * T, H, -1), ref_o2, TOL["bf16"], scale, "second verify out")
