@@ -31,6 +31,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -110,7 +111,8 @@ class ClockSampler:
         self.index = index
         self.interval_ms = interval_ms
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks{tag}_rank{index}.csv")
+        out_dir = os.environ.get("KDA_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"kda_clocks{tag}_rank{index}.csv")
 
     def __enter__(self):
         try:
