@@ -123,28 +123,28 @@ __device__ __forceinline__ uint32_t ld_volatile(const uint32_t *p) {
 // so the next chunk's chain waits neither for the output MMA nor for a shared-memory store.
 namespace cons {
 constexpr uint32_t STAGE0 = 0, STAGE1 = SLOT;
-constexpr uint32_t SBT = 2 * SLOT;         // S_b^T [d][c] bf16 128 x 128 (64-column blocks of 16 KB)
-constexpr uint32_t MISC = SBT + 32768;     // barriers, flags
+constexpr uint32_t MISC = 2 * SLOT;        // barriers, flags
 constexpr uint32_t BYTES = MISC + 256;
 // TMEM: S^T fp32 (128 columns), two bf16 copies S_b^T (64 columns each, used by alternate chunks),
-// two M=64 output accumulators (row i in lane i % 16 + 32 (i / 16); 128 columns each).
+// two output accumulators O^T (lane = value channel, column = token; 64 of 128 columns used).
 constexpr uint32_t TM_S = 0, TM_SB0 = 128, TM_SB1 = 192, TM_O0 = 256, TM_O1 = 384, TM_COLS = 512;
 }  // namespace cons
 
 // Consumer roles, per chunk c (stage b = c & 1). Loader: once the producer has published chunk c
 // and chunk c - 2's MMAs have completed (o[b]), copy its image into stage b (full[b]); publish
 // consumption of chunk c - 2 at that point. MMA thread: wait for the image and for S_b^T(c) in TMEM,
-// issue the chain (commit s); wait for S_b^T(c) in shared memory and for the output warps to have
-// read accumulator b (chunk c - 2), issue O = P S_b (commit sr) and O += A U~ (commit o[b]). State
+// issue the chain (commit s); once the output warps have read accumulator b (chunk c - 2), issue
+// the transposed output O^T = S_b^T P^T + U~^T A^T from the same TMEM copy (commit o[b]). State
 // warps 0..3 (lane = value channel): after s, the new state's bf16 copy into TMEM ("tmem ready": the
-// critical path), after sr into shared memory ("smem ready"). Output warps 4..7: after o[b], the
-// outputs ("o free"). No CTA-wide barrier inside the loop.
+// critical path). Output warps 4..7: after o[b], the outputs ("o free"). No CTA-wide barrier inside
+// the loop. S_b^T(c) in TMEM copy c & 1 is rewritten only after the chain of chunk c + 1 has
+// completed, and so has O(c), issued before it by the same thread.
 __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t *sm, int hd) {
     using namespace cons;
     constexpr uint32_t I_C = idesc_bf16_f32(128, 128, false, 0, 0);   // S_b^T M^T (A in TMEM)
     constexpr uint32_t I_K = idesc_bf16_f32(128, 128, false, 1, 1);   // U~^T K^
-    constexpr uint32_t I_P = idesc_bf16_f32(64, 128, false, 0, 0);    // P S_b
-    constexpr uint32_t I_A = idesc_bf16_f32(64, 128, false, 0, 1);    // A U~
+    constexpr uint32_t I_OP = idesc_bf16_f32(128, 64, false, 0, 0);   // S_b^T P^T (A in TMEM)
+    constexpr uint32_t I_OA = idesc_bf16_f32(128, 64, false, 1, 0);   // U~^T A^T
     // full0, full1, s, sr, o0, o1, tmem ready, smem ready, o free 0, o free 1, teardown
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);
     uint32_t *s_flags = reinterpret_cast<uint32_t *>(sm + MISC + 96); // abort, tmem
@@ -207,8 +207,7 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
         if (requested == nchunks) st_release(p.consumed + hd, nchunks);
     } else if (tid == CTL) {
         // ------------------------------------------------ MMA thread
-        uint32_t ph_full[2] = {0, 0}, ph_t = 0, ph_s = 0, ph_free[2] = {0, 0};
-        const uint64_t dSBT = desc_k(sb + SBT, 16384, 0);
+        uint32_t ph_full[2] = {0, 0}, ph_t = 0, ph_free[2] = {0, 0};
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
             if (ld_volatile(&s_flags[0])) break;
@@ -230,20 +229,17 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
             for (uint32_t kk = 0; kk < 4; ++kk)  // ... + U~^T K^
                 mma_bf16_ss(tmem + TM_S, desc_mn_at(dU, kk), desc_mn_at(dK, kk), I_K, 1);
             mma_commit(&bars[2]);
-            if (!mbar_wait_bounded(&bars[7], ph_s, p.timeout_ns)) { fail(); break; }
-            ph_s ^= 1u;
             if (c >= 2) {  // the output warps have read this accumulator's previous chunk
                 if (!mbar_wait_bounded(&bars[8 + b], ph_free[b], p.timeout_ns)) { fail(); break; }
                 ph_free[b] ^= 1u;
             }
             tc_fence_after();
 #pragma unroll
-            for (uint32_t kk = 0; kk < 8; ++kk)  // O = P S_b ...
-                mma_bf16_ss(tm_o, desc_k_at(dP, 8192, kk), desc_k_at(dSBT, 16384, kk), I_P, kk > 0);
-            mma_commit(&bars[3]);                // S_b^T in shared memory has been read
+            for (uint32_t kk = 0; kk < 8; ++kk)  // O^T = S_b^T P^T ...
+                mma_bf16_ts(tm_o, tm_sb + 8 * kk, desc_k_at(dP, 8192, kk), I_OP, kk > 0);
 #pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)  // ... + A U~
-                mma_bf16_ss(tm_o, desc_k_at(dA, 8192, kk), desc_mn_at(dU, kk), I_A, 1);
+            for (uint32_t kk = 0; kk < 4; ++kk)  // ... + U~^T A^T
+                mma_bf16_ss(tm_o, desc_mn_at(dU, kk), desc_k_at(dA, 8192, kk), I_OA, 1);
             mma_commit(&bars[4 + b]);            // O and the stage are done
         }
         // teardown: every issued MMA completes before TMEM is freed
@@ -251,8 +247,8 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
         mbar_wait_bounded(&bars[10], 0, p.timeout_ns);
     } else if (warp < 4) {
         // ------------------------------------------------ state warps (lane = value channel d)
-        // per chunk: the new state -> its bf16 copy in TMEM (the next chain's A operand: the
-        // critical path), then, once P S_b has read the old one, into shared memory
+        // per chunk: the new state -> its bf16 copy in TMEM (the next chain's and the output's A
+        // operand)
         const int d_me = tid;  // 0..127
         auto wait_bar = [&](uint64_t *bar, uint32_t &ph) -> bool {
             const bool ok = mbar_wait_bounded(bar, ph, p.timeout_ns);
@@ -270,17 +266,7 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
             for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(w[hh][e]);
             tmem_st32(tmem + lane_base + tm_sb + 32 * hh, f);
         };
-        auto to_smem = [&]() {
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                for (int q8 = 0; q8 < 8; ++q8)
-                    *reinterpret_cast<uint4 *>(sm + SBT + tchunk(16384, d_me, 64 * hh + 8 * q8)) =
-                        make_uint4(w[hh][4 * q8], w[hh][4 * q8 + 1], w[hh][4 * q8 + 2], w[hh][4 * q8 + 3]);
-            fence_proxy_async_smem();
-            mbar_arrive(&bars[7]);
-        };
-        // initial state S[c][d] -> S^T in TMEM and both bf16 copies; empty sequences copy it out
+        // initial state S[c][d] -> S^T in TMEM and its bf16 copy; empty sequences copy it out
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             float v[2][32];
@@ -303,9 +289,8 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars[6]);
-            to_smem();
         }
-        uint32_t ph_s = 0, ph_sr = 0;
+        uint32_t ph_s = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
             const bool last = c + 1 == nchunks;
@@ -331,14 +316,13 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
                 tc_fence_before();
                 mbar_arrive(&bars[6]);
             }
-            if (!wait_bar(&bars[3], ph_sr)) break;
-            if (!last) to_smem();
         }
         tc_fence_before();
     } else if (tid < NT) {
         // ------------------------------------------------ output warps
-        // O of chunk c (M=64 accumulator: row i in lane i % 16 + 32 (i / 16)) -> bf16 outputs
-        const int i = 16 * quad + lane;
+        // O^T of chunk c (lane = value channel d, column = token) -> bf16 outputs; for each token a
+        // warp stores 32 consecutive channels (64 bytes)
+        const int d_me = 32 * quad + lane;
         uint32_t ph_o[2] = {0, 0};
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
@@ -350,26 +334,16 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
             const int64_t tc = bos + (int64_t)c * C;
             const int vc = (int)(eos - tc < C ? eos - tc : C);
             const uint32_t tm_o = b ? TM_O1 : TM_O0;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float vv[2][32];
-                tmem_ld32(tmem + lane_base + tm_o + 64 * hh, vv[0]);
-                tmem_ld32(tmem + lane_base + tm_o + 64 * hh + 32, vv[1]);
-                tmem_wait_ld();
-                if (lane < 16 && i < vc) {
-#pragma unroll
-                    for (int part = 0; part < 2; ++part) {
-                        const float *v = vv[part];
-                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(tc + i) * H + h) * D + 64 * hh + 32 * part);
-#pragma unroll
-                        for (int q8 = 0; q8 < 4; ++q8)
-                            dst[q8] = make_uint4(pack2(v[8 * q8], v[8 * q8 + 1]), pack2(v[8 * q8 + 2], v[8 * q8 + 3]),
-                                                 pack2(v[8 * q8 + 4], v[8 * q8 + 5]), pack2(v[8 * q8 + 6], v[8 * q8 + 7]));
-                    }
-                }
-            }
+            float vv[2][32];  // tokens 0..31, 32..63 of channel d_me
+            tmem_ld32(tmem + lane_base + tm_o, vv[0]);
+            tmem_ld32(tmem + lane_base + tm_o + 32, vv[1]);
+            tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(&bars[8 + b]);  // this accumulator may take chunk c + 2
+            mbar_arrive(&bars[8 + b]);  // read: this accumulator may take chunk c + 2
+            __nv_bfloat16 *dst = p.out + ((size_t)tc * H + h) * D + d_me;
+#pragma unroll
+            for (int t = 0; t < C; ++t)
+                if (t < vc) dst[(size_t)t * H * D] = __float2bfloat16_rn(vv[t >> 5][t & 31]);
         }
         tc_fence_before();
     }
