@@ -50,8 +50,8 @@ FLOP_PER_TOKEN_HEAD = 180224
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
 # dram__bytes_read.sum + dram__bytes_write.sum of one split_kernel launch on the headline workload,
 # from one ncu capture; reported only while the kernel's sources are the ones it was taken on.
-SPLIT_TRAFFIC_BYTES = 336.7744e6 + 59.280896e6
-SPLIT_TRAFFIC_SOURCES_SHA256 = "4ab0d089948fa8ab284b89981f34fde2a857a073451c478e224eea58f08458a5"
+SPLIT_TRAFFIC_BYTES = 336.781056e6 + 58.767872e6
+SPLIT_TRAFFIC_SOURCES_SHA256 = "534ceb571a66ac824dee92464968760a0b66e9dc647a0f8d49d7fb1b3d87a559"
 
 
 def measured_traffic():
