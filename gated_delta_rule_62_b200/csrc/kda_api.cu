@@ -124,7 +124,10 @@ kda_status_t run_prefill(kda::Problem &p, const int32_t *cu_seqlens_host, void *
         kda::split_eligible_seqs(p.num_seqs) &&
         workspace_bytes >= kda::split_workspace_bytes(heads)) {
         // few heads: consumer CTAs run the state chains, producer CTAs fill the other SMs
-        e = kda::launch_prefill_split(p, max_chunks, workspace, s, kda::kWaitTimeoutNs);
+        bool not_coresident = false;
+        e = kda::launch_prefill_split(p, max_chunks, workspace, s, kda::kWaitTimeoutNs, &not_coresident);
+        if (e == cudaSuccess && not_coresident)  // nothing enqueued: the single-role kernel runs
+            e = kda::launch_prefill_chunk(p, workspace, s, kda::kWaitTimeoutNs);
     } else if (kda::chunk_supported(p)) {
         // the planning kernel clears the status word
         e = kda::launch_prefill_chunk(p, workspace, s, kda::kWaitTimeoutNs);
@@ -523,6 +526,20 @@ kda_status_t kda_selftest_bounded_wait(void *workspace, size_t workspace_bytes,
     cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
     if (e == cudaSuccess) e = kda::launch_bounded_wait_probe(workspace, timeout_ns, s);
     if (e != cudaSuccess) return cuda_fail(e, "kda_selftest_bounded_wait: launch");
+    return launched(1);
+}
+
+kda_status_t kda_selftest_flag_wait(void *workspace, size_t workspace_bytes, uint64_t timeout_ns,
+                                    kda_stream_t stream) {
+    if (!workspace || workspace_bytes < kStatusBytes)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "workspace of at least %zu bytes is required",
+                    kStatusBytes);
+    if (timeout_ns == 0 || timeout_ns > 10000000000ull)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "timeout_ns must be in (0, 1e10]");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
+    if (e == cudaSuccess) e = kda::launch_flag_wait_probe(workspace, timeout_ns, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_selftest_flag_wait: launch");
     return launched(1);
 }
 

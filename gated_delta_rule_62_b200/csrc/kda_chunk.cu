@@ -469,16 +469,21 @@ __global__ void bounded_wait_probe(int32_t *status, uint64_t timeout_ns) {
         atomicOr(status, 1);
 }
 
+// Waits on a global word that nothing writes (cleared here, released at 1) with the split
+// kernel's inter-CTA flag wait; records the timeout in the status word and returns.
+__global__ void flag_wait_probe(int32_t *status, int32_t *flag, uint64_t timeout_ns) {
+    if (threadIdx.x == 0) {
+        if (!wait_flag_ge(flag, 1, timeout_ns)) atomicOr(status, 1);
+    }
+}
+
 template <int DS, bool PRO>
 cudaError_t launch_ds(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                       const CUtensorMap &mla, const ChunkParams &cp, unsigned grid,
                       cudaStream_t stream) {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(chunk_kernel<DS, PRO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)Smem<DS>::BYTES);
-    });
+    static PerDeviceOnce<> once;
+    const cudaError_t attr_err =
+        set_smem_limit_once(once, (const void *)chunk_kernel<DS, PRO>, (int)Smem<DS>::BYTES);
     if (attr_err != cudaSuccess) return attr_err;
     chunk_kernel<DS, PRO><<<grid, NT, Smem<DS>::BYTES, stream>>>(mq, mk, mv, mla, cp);
     return cudaGetLastError();
@@ -537,6 +542,13 @@ bool make_rows_map(CUtensorMap *m, void *base, uint64_t rows, uint32_t box_rows)
 
 cudaError_t launch_bounded_wait_probe(void *workspace, uint64_t timeout_ns, cudaStream_t stream) {
     bounded_wait_probe<<<1, 32, 0, stream>>>(static_cast<int32_t *>(workspace), timeout_ns);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_flag_wait_probe(void *workspace, uint64_t timeout_ns, cudaStream_t stream) {
+    // status word at byte 0, the never-released flag at byte 128 (both zeroed by the caller)
+    int32_t *ws = static_cast<int32_t *>(workspace);
+    flag_wait_probe<<<1, 32, 0, stream>>>(ws, ws + 32, timeout_ns);
     return cudaGetLastError();
 }
 

@@ -36,6 +36,29 @@ __device__ __forceinline__ int sync_compute_or(int pred) {
     return (int)r;
 }
 
+// ---------------------------------------------------------------- global flags between CTAs
+__device__ __forceinline__ int ld_acquire(const int32_t *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(int32_t *p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Bounded spin until *p >= target (acquire); false once timeout_ns have passed on %globaltimer.
+__device__ __forceinline__ bool wait_flag_ge(const int32_t *p, int target, uint64_t timeout_ns) {
+    if (ld_acquire(p) >= target) return true;
+    const uint64_t deadline = globaltimer_ns() + timeout_ns;
+    while (true) {
+        __nanosleep(100);
+        if (ld_acquire(p) >= target) return true;
+        if (globaltimer_ns() > deadline) return false;
+    }
+}
+
 // ---------------------------------------------------------------- tile addressing
 // bf16 tiles use the 128-byte swizzle: 128-byte rows of 64 elements, 8-row groups
 // 1024 bytes apart, 16-byte chunk index XOR (row % 8); 64-column blocks `bs` bytes apart.

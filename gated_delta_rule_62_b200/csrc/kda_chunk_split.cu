@@ -71,27 +71,6 @@ struct SplitParams {
     uint64_t timeout_ns;
 };
 
-__device__ __forceinline__ int ld_acquire(const int32_t *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release(int32_t *p, int v) {
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_global() {
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-// Bounded spin until *p >= target; false on timeout.
-__device__ __forceinline__ bool wait_flag_ge(const int32_t *p, int target, uint64_t timeout_ns) {
-    if (ld_acquire(p) >= target) return true;
-    const uint64_t deadline = globaltimer_ns() + timeout_ns;
-    while (true) {
-        __nanosleep(100);
-        if (ld_acquire(p) >= target) return true;
-        if (globaltimer_ns() > deadline) return false;
-    }
-}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until the committed TMA stores have finished reading shared memory / are complete.
 __device__ __forceinline__ void bulk_wait_read() {
@@ -771,25 +750,24 @@ size_t split_workspace_bytes(int64_t heads) {
 }
 
 cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *workspace,
-                                 cudaStream_t stream, uint64_t timeout_ns) {
+                                 cudaStream_t stream, uint64_t timeout_ns, bool *not_coresident) {
+    *not_coresident = false;
     const int64_t heads = (int64_t)p.num_seqs * p.H;
     const int sms = sm_count();
     int per_sm = 0;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)SPLIT_SMEM);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            (int)SPLIT_SMEM);
-    });
-    if (attr_err != cudaSuccess) return attr_err;
+    static PerDeviceOnce<> once_plain, once_pro;
     const void *kern = p.pro.flags ? (const void *)split_kernel<true> : (const void *)split_kernel<false>;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NTS, SPLIT_SMEM);
+    cudaError_t e = set_smem_limit_once(p.pro.flags ? once_pro : once_plain, kern, (int)SPLIT_SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NTS, SPLIT_SMEM);
     if (e != cudaSuccess) return e;
     const int grid = per_sm * sms;
-    if (per_sm < 1 || grid < 2 * heads) return cudaErrorInvalidConfiguration;
+    // Fewer resident blocks than the launch needs (fewer SMs visible, e.g. a partitioned
+    // context): nothing is enqueued and the caller runs the single-role kernel instead.
+    if (!split_coresident(per_sm, sms, heads)) {
+        *not_coresident = true;
+        return cudaSuccess;
+    }
 
     CUtensorMap mq, mk, mv, mla, mrl, mrs;
     const uint64_t T = (uint64_t)p.total_tokens, H = (uint64_t)p.H;

@@ -1,9 +1,9 @@
 // Fused KDA decode step: one token per (sequence, head), state updated in place.
 //
-// The per-token cost is constant ("Decoding throughput stays roughly flat as
-// context grows": shivam2003.com Kimi K3 article, section "Kimi Delta Attention:
-// the load-bearing choice"); the step is bound by streaming the fp32 state
-// through HBM once in and once out. With S' = Diag(alpha) S:
+// The per-token decode cost does not depend on how long the context is (the
+// shivam2003.com Kimi K3 article, section "Kimi Delta Attention: the load-bearing
+// choice"); the step is bound by streaming the fp32 state through HBM once in and
+// once out. With S' = Diag(alpha) S:
 //   a = S'^T k,  b = S'^T q,  u = beta (v - a),  S_new = S' + k u^T,
 //   o = S_new^T q = b + (k.q) u,
 // so one read of S feeds both column reductions and one write stores S_new.

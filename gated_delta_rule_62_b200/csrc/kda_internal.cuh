@@ -5,9 +5,22 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "host_plan.h"
 #include "kda.h"
 
 namespace kda {
+
+// Sets a kernel's dynamic shared-memory limit on the current device, once per device (the
+// attribute belongs to that device's context, so each GPU a process uses needs its own call).
+inline cudaError_t set_smem_limit_once(PerDeviceOnce<> &once, const void *func, int bytes) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int r = once.run(dev, [&] {
+        return (int)cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    });
+    return r == PerDeviceOnce<>::kBadDevice ? cudaErrorInvalidDevice : static_cast<cudaError_t>(r);
+}
 
 // ---- element access for the two input dtypes -------------------------------------------
 __device__ __forceinline__ float to_f32(float x) { return x; }
@@ -92,14 +105,17 @@ size_t chunk_workspace_bytes(int32_t num_seqs);
 cudaError_t launch_prefill_chunk(const Problem &p, void *workspace, cudaStream_t stream,
                                  uint64_t timeout_ns);
 cudaError_t launch_bounded_wait_probe(void *workspace, uint64_t timeout_ns, cudaStream_t stream);
+cudaError_t launch_flag_wait_probe(void *workspace, uint64_t timeout_ns, cudaStream_t stream);
 
 // Split-role chunk kernel (consumers run the state chain, producers the key-side half) for
 // workloads with few (sequence, head) pairs; it needs a larger workspace (a ring of chunk images).
 bool split_eligible(int64_t heads, kda_dtype_t dtype, int32_t dk, int32_t dv);
 bool split_eligible_seqs(int32_t num_seqs);
 size_t split_workspace_bytes(int64_t heads);
+// Enqueues the split-role kernel; if its blocks cannot all be resident on this device, enqueues
+// nothing, sets *not_coresident and returns cudaSuccess.
 cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *workspace,
-                                 cudaStream_t stream, uint64_t timeout_ns);
+                                 cudaStream_t stream, uint64_t timeout_ns, bool *not_coresident);
 
 // Records `msg` as the calling thread's kda_last_error() and returns `st`.
 kda_status_t record_error(kda_status_t st, const char *msg);

@@ -11,7 +11,10 @@
 // libkda holds it (kNoallocScratchBytes) until the process exits. In host code
 // its name is only a host-side stand-in for the symbol, not a device address, so
 // the address is looked up with cudaGetSymbolAddress once per device (with that
-// device current) and passed to the kernels as a plain pointer.
+// device current) and passed to the kernels as a plain pointer. That address is
+// kept for the life of the process; a cudaDeviceReset unloads the library's
+// device code and may move the array, so after a reset of a device this entry
+// point must not be used on it again in the same process.
 #include <cstdio>
 #include <mutex>
 
@@ -73,4 +76,18 @@ extern "C" KDA_API kda_status_t kda_prefill_noalloc(
     return kda_prefill(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev, cu_seqlens_host,
                        num_seqs, total_tokens, H, d_k, d_v, dtype, out, final_state, scratch,
                        kNoallocScratchBytes, stream);
+}
+
+// The status word of the last kda_prefill_noalloc on the current device sits at the start of the
+// scratch array; read it the way kda_read_device_status reads a caller's workspace.
+extern "C" KDA_API kda_status_t kda_prefill_noalloc_status(kda_stream_t stream) {
+    void *scratch = nullptr;
+    cudaError_t e = scratch_on_current_device(&scratch);
+    if (e != cudaSuccess) {
+        char msg[200];
+        snprintf(msg, sizeof msg, "kda_prefill_noalloc_status: scratch set-up (cudaGetSymbolAddress) failed: %s",
+                 cudaGetErrorString(e));
+        return kda::record_error(KDA_ERR_CUDA, msg);
+    }
+    return kda_read_device_status(scratch, stream);
 }

@@ -41,8 +41,10 @@ SIGNATURES = {
     "kda_version": (_i32, []),
     "kda_last_launch_count": (_i32, []),
     "kda_selftest_bounded_wait": (_i32, [_vp, _sz, ctypes.c_uint64, _vp]),
+    "kda_selftest_flag_wait": (_i32, [_vp, _sz, ctypes.c_uint64, _vp]),
     "kda_prefill_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                                    _i32, _i32, _vp, _vp, _vp]),
+    "kda_prefill_noalloc_status": (_i32, [_vp]),
     "kda_prefill_slots": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _i32, _i64,
                                  _i32, _i32, _i32, _i32, _vp, _vp, _sz, _vp]),
     "kda_decode_step_slots": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _i32,
@@ -440,6 +442,12 @@ def selftest_bounded_wait(workspace, timeout_ns: int, stream=None):
     """Launch the bounded-wait probe (a wait nothing releases); see kda.h."""
     _check(lib().kda_selftest_bounded_wait(_ptr(workspace), workspace.numel(), int(timeout_ns),
                                            _stream(stream)), "kda_selftest_bounded_wait")
+
+
+def selftest_flag_wait(workspace, timeout_ns: int, stream=None):
+    """Launch the flag-wait probe (a global flag nothing releases); see kda.h."""
+    _check(lib().kda_selftest_flag_wait(_ptr(workspace), workspace.numel(), int(timeout_ns),
+                                        _stream(stream)), "kda_selftest_flag_wait")
 
 
 def read_device_status(workspace, stream=None) -> int:

@@ -85,6 +85,14 @@ KDA_API size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens
 /*
  * Chunked prefill over packed variable-length sequences.
  *
+ * Defined by: the recurrence of "How the delta rule actually works" with the
+ * per-key-channel forgetting of "Kimi Delta Attention: the load-bearing choice"
+ * (shivam2003.com Kimi K3 article; that section also says the update is computed
+ * blockwise so it maps onto matrix units: the 64-token chunks here), and the
+ * state save/restore of "Serving infrastructure: supernodes and the prefill
+ * cache" (same article: a cached state lets a returning request pay only for
+ * its new suffix), which initial_state / final_state carry.
+ *
  *   q, k        [total_tokens, H, d_k]  dtype
  *   v           [total_tokens, H, d_v]  dtype
  *   log_alpha   [total_tokens, H, d_k]  fp32
@@ -143,6 +151,11 @@ KDA_API kda_status_t kda_prefill_recurrent(const void *q, const void *k, const v
  * One decode step: one new token for each of num_seqs sequences, state updated
  * in place (constant cost per token: the state of each head is read once and
  * written once).
+ *
+ * Defined by: the same per-token recurrence ("How the delta rule actually
+ * works", "Kimi Delta Attention: the load-bearing choice", shivam2003.com Kimi
+ * K3 article); the second section also gives the property this kernel is built
+ * around, a decode cost per token that stays the same however long the context.
  *
  *   q, k        [num_seqs, H, d_k]  dtype
  *   v           [num_seqs, H, d_v]  dtype
@@ -375,6 +388,18 @@ KDA_API kda_status_t kda_selftest_bounded_wait(void *workspace, size_t workspace
                                                uint64_t timeout_ns, kda_stream_t stream);
 
 /*
+ * Diagnostic: the same check for the other kind of wait in the prefill
+ * kernels, a spin on a flag in global memory that another thread block
+ * releases (the split-role kernel's hand-off between its thread blocks). One
+ * thread waits, with that kernel's bounded flag wait, for a word at byte 128 of
+ * `workspace` that this call zeroes and nothing then writes; after timeout_ns
+ * (in (0, 1e10]) it records KDA_ERR_TIMEOUT in the status word at the start of
+ * `workspace` (>= 256 bytes) and exits, leaving the context usable.
+ */
+KDA_API kda_status_t kda_selftest_flag_wait(void *workspace, size_t workspace_bytes,
+                                            uint64_t timeout_ns, kda_stream_t stream);
+
+/*
  * kda_prefill without a workspace argument, for callers that cannot allocate
  * device memory when they run a prefill (code inside an allocator or pool
  * callback, a serving loop whose memory is fixed at start-up). The pages
@@ -389,8 +414,10 @@ KDA_API kda_status_t kda_selftest_bounded_wait(void *workspace, size_t workspace
  * Every call shares the one array and rewrites all of it that it uses, so
  * calls that overlap on the GPU (different streams, or different host threads)
  * race and must be serialised by the caller. The device status word is kept in
- * that array and is not readable by the caller. Other arguments, results and
- * status codes are those of kda_prefill.
+ * that array; kda_prefill_noalloc_status reads it. The looked-up address is
+ * kept until the process exits: after cudaDeviceReset on a device, do not call
+ * this entry point on that device again in the same process. Other arguments,
+ * results and status codes are those of kda_prefill.
  */
 KDA_API kda_status_t kda_prefill_noalloc(const void *q, const void *k, const void *v,
                                          const float *log_alpha, const float *beta,
@@ -400,6 +427,16 @@ KDA_API kda_status_t kda_prefill_noalloc(const void *q, const void *k, const voi
                                          int32_t num_seqs, int64_t total_tokens, int32_t H,
                                          int32_t d_k, int32_t d_v, kda_dtype_t dtype,
                                          void *out, float *final_state, kda_stream_t stream);
+
+/*
+ * Status word of the last kda_prefill_noalloc on the current device (the
+ * device-side report that kda_read_device_status gives for a caller's
+ * workspace): KDA_OK, KDA_ERR_TIMEOUT if a bounded on-device wait of that call
+ * gave up (its outputs are then invalid), or KDA_ERR_CUDA if the scratch
+ * array's address cannot be looked up. Synchronises `stream`; call it on the
+ * stream of the kda_prefill_noalloc it checks. No counterpart in the pages.
+ */
+KDA_API kda_status_t kda_prefill_noalloc_status(kda_stream_t stream);
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 KDA_API int32_t kda_version(void);

@@ -25,3 +25,28 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(autouse=True, scope="session")
+def _canary_guards():
+    """On a GPU, every output the library writes in the tests sits between canary guard bands
+    that are checked after the call (tests/guards.py)."""
+    try:
+        import torch
+        has_gpu = torch.cuda.is_available()
+    except Exception:  # pragma: no cover
+        has_gpu = False
+    if has_gpu:
+        from gated_delta_rule_62_b200 import kda as K
+        from tests import guards
+        guards.install(K)
+    yield
+
+
+def pytest_terminal_summary(terminalreporter):
+    try:
+        from tests import guards
+    except Exception:  # pragma: no cover
+        return
+    if guards.checks():
+        terminalreporter.write_line(f"canary guard bands checked intact: {guards.checks()}")

@@ -74,3 +74,39 @@ def test_decode_256_sequences_from_prefill_state():
         scale = float(d["v"].abs().max())
         assert_close(out, ro, TOL["bf16"], scale, f"decode256 out step {t}")
         assert_close(state, ref_s, TOL["bf16"], scale, f"decode256 state step {t}")
+
+
+def test_decode_1024_steps_against_oracle_without_reseeding():
+    """The full decode workload: 256 sequences x 32 heads seeded by the 512-token GPU prefill, then
+    1,024 GPU decode steps. The oracle starts once from the GPU's seeded states and runs the same
+    1,024 tokens per sequence on its own (no re-seeding between steps), so accumulated drift is
+    compared. Oracle subset: 16 evenly spaced sequences x all 32 heads; every step's output and the
+    final state are compared element by element at the bf16 tolerance."""
+    wl = W.DECODE_256
+    steps_n = wl.decode_steps
+    inp = W.make_inputs(wl, DEV)
+    _, state = K.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], None,
+                         inp["cu_seqlens"], inp["cu_seqlens_dev"])
+    sub = torch.arange(0, wl.num_seqs, wl.num_seqs // 16, device=DEV)
+    assert sub.numel() == 16
+    seeded = f64(state[sub])
+    steps = W.make_decode_steps(wl, inp["_gen"], steps_n, DEV)
+    outs = torch.empty(steps_n, sub.numel(), wl.H, wl.dv, dtype=steps["v"].dtype, device=DEV)
+    for t in range(steps_n):
+        out = K.decode_step(steps["q"][t], steps["k"][t], steps["v"][t], steps["log_alpha"][t],
+                            steps["beta"][t], state)
+        outs[t] = out[sub]
+    torch.cuda.synchronize()
+    # the subset's tokens packed sequence-major: row n * steps_n + t is step t of sequence sub[n]
+    seq_major = {n: f64(steps[n][:, sub].transpose(0, 1).reshape(-1, *steps[n].shape[2:]))
+                 for n in ("q", "k", "v", "log_alpha", "beta")}
+    cu = np.arange(sub.numel() + 1, dtype=np.int64) * steps_n
+    ro, rs = oracle.forward(seq_major["q"], seq_major["k"], seq_major["v"], seq_major["log_alpha"],
+                            seq_major["beta"], seeded, cu)
+    scale = float(steps["v"].abs().max())
+    got = f64(outs.transpose(0, 1).reshape(-1, wl.H, wl.dv))
+    assert_close(got, ro, TOL["bf16"], scale, "decode 1024 steps: every output")
+    assert_close(state[sub], rs, TOL["bf16"], scale, "decode 1024 steps: final state")
+    # drift stays far inside the tolerance: the last step alone, for the record
+    last = got.reshape(sub.numel(), steps_n, wl.H, wl.dv)[:, -1]
+    assert float(np.abs(last - ro.reshape(sub.numel(), steps_n, wl.H, wl.dv)[:, -1]).max()) <= TOL["bf16"] * scale

@@ -4,17 +4,22 @@ Callers such as an allocator or memory-pool callback, or a serving loop whose
 device memory is fixed at start-up, cannot cudaMalloc a workspace when they run
 a prefill. kda_prefill_noalloc takes no workspace and uses a fixed scratch array
 inside the library instead. These tests call it through the C ABI and compare it
-with kda_prefill (which takes a caller-allocated workspace) on two calls in a row,
-so the second call also shows that what the first left in the shared scratch does
-not leak into its result. This file is named so that pytest collects it last.
+with kda_prefill (which takes a caller-allocated workspace) and with the fp64
+oracle on two calls in a row, so the second call also shows that what the first
+left in the shared scratch does not leak into its result; the status word the
+calls leave in that scratch must read KDA_OK. This file is named so that pytest
+collects it last.
 """
 import ctypes
+
+import numpy as np
 
 import pytest
 import torch
 
 from gated_delta_rule_62_b200 import kda as K
 from gated_delta_rule_62_b200 import workloads as W
+import oracle
 
 MAX_SEQS = 16320  # (64 KiB - 256 B status word) / 4 B per scheduled sequence
 
@@ -48,6 +53,7 @@ def test_noalloc_rejects_more_sequences_than_its_scratch_holds():
 @pytest.mark.gpu
 def test_noalloc_matches_prefill_on_two_calls_in_a_row():
     torch.cuda.set_device(0)
+    oracle.build()
     problems = [((300, 0, 65, 128, 1), 31), ((200, 77, 9), 32)]  # different N, lengths, seeds
     for lens, seed in problems:
         wl = W.custom(lens, 4, 128, 128, "bf16", seed=seed, init_state="normal")
@@ -63,3 +69,11 @@ def test_noalloc_matches_prefill_on_two_calls_in_a_row():
         assert torch.isfinite(out).all() and torch.isfinite(fs).all()
         assert float((out.float() - ref_out.float()).abs().max()) <= tol, lens
         assert float((fs - ref_fs).abs().max()) <= tol, lens
+        # and against the oracle directly, on the same input bits
+        f64 = W.to_f64_numpy
+        ro, rs = oracle.forward(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["log_alpha"]),
+                                f64(inp["beta"]), f64(inp["initial_state"]), inp["cu_seqlens"].numpy())
+        assert float(np.abs(f64(out) - ro).max()) <= tol, lens
+        assert float(np.abs(f64(fs) - rs).max()) <= tol, lens
+        assert K.lib().kda_prefill_noalloc_status(
+            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == K.KDA_OK
