@@ -379,17 +379,30 @@ def bench_speculative(args, K, stream, ws, decode_ms):
             "gpu_launches": 3 * nsteps}
 
 
-def bench_prefill_workload(wl, K, stream, steps, warmup, rank, prologue=0):
+def bench_prefill_workload(wl, K, stream, steps, warmup, rank, prologue=0, segments=0, inp=None):
     """Device-timed kda_prefill of one workload (inputs resident in HBM); returns a summary dict.
-    With ``prologue`` flags: kda_prefill_prologue on the same draws before activation."""
-    inp = W.make_inputs(wl, "cuda", seed=wl.seed + 7919 * rank, raw=bool(prologue))
+    With ``prologue`` flags: kda_prefill_prologue on the same draws before activation. With
+    ``segments`` > 0: kda_prefill_cp (context parallelism, each sequence cut into that many
+    segments)."""
+    if inp is None:
+        inp = W.make_inputs(wl, "cuda", seed=wl.seed + 7919 * rank, raw=bool(prologue))
     N, T, H = wl.num_seqs, wl.total_tokens, wl.H
     out = torch.empty(T, H, wl.dv, dtype=wl.torch_dtype, device="cuda")
     fs = torch.empty(N, H, wl.dk, wl.dv, dtype=torch.float32, device="cuda")
-    work = torch.empty(K.workspace_size(N, T, H, wl.dk, wl.dv, wl.torch_dtype), dtype=torch.uint8,
-                       device="cuda")
+    if segments:
+        import ctypes
+        wsz = int(K.lib().kda_prefill_cp_workspace_size(N, ctypes.c_void_p(inp["cu_seqlens"].data_ptr()), H,
+                                                        wl.dk, wl.dv, K.KDA_BF16, segments))
+    else:
+        wsz = K.workspace_size(N, T, H, wl.dk, wl.dv, wl.torch_dtype)
+    work = torch.empty(wsz, dtype=torch.uint8, device="cuda")
 
     def step():
+        if segments:
+            K.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["initial_state"],
+                      inp["cu_seqlens"], inp["cu_seqlens_dev"], out=out, final_state=fs, workspace=work,
+                      stream=stream, algo="cp", segments=segments)
+            return
         K.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["initial_state"],
                   inp["cu_seqlens"], inp["cu_seqlens_dev"], out=out, final_state=fs, workspace=work,
                   stream=stream, prologue=prologue, gate_scale=W.GATE_SCALE)
@@ -405,6 +418,8 @@ def bench_prefill_workload(wl, K, stream, steps, warmup, rank, prologue=0):
     torch.cuda.empty_cache()
     name = wl.name + (" raw inputs, fused prologue (q/k L2 norm, gate -softplus, beta sigmoid)"
                       if prologue else "")
+    if segments:
+        name += f" context-parallel, {segments} segments per sequence (kda_prefill_cp)"
     return {"workload": name, "tokens": T, "heads": H, "sequences": N, "ms_per_step": ms,
             "tokens_per_s": T / (ms * 1e-3),
             "tc_frac": FLOP_PER_TOKEN_HEAD * th / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
@@ -532,9 +547,14 @@ def run_ours(args, rank, local, ws):
     spec = None if args.no_decode else bench_speculative(args, K, stream, ws, dec["ms_per_step"])
     extra = None
     if not args.no_extra:
-        extra = [bench_prefill_workload(W.VARLEN_24, K, stream, 10, 3, rank),
-                 bench_prefill_workload(W.PREFILL_1M, K, stream, 6, 3, rank),
-                 bench_prefill_workload(wl, K, stream, 20, 3, rank, prologue=K.PROLOGUE_ALL)]
+        extra = [bench_prefill_workload(W.VARLEN_24, K, stream, 10, 3, rank)]
+        inp_1m = W.make_inputs(W.PREFILL_1M, "cuda", seed=W.PREFILL_1M.seed + 7919 * rank)
+        for segs in (0, 2, 4):  # the million-token prefill without and with context parallelism
+            extra.append(bench_prefill_workload(W.PREFILL_1M, K, stream, 6, 3, rank, segments=segs,
+                                                inp=inp_1m))
+        del inp_1m
+        torch.cuda.empty_cache()
+        extra.append(bench_prefill_workload(wl, K, stream, 20, 3, rank, prologue=K.PROLOGUE_ALL))
 
     if rank != 0:
         return

@@ -11,6 +11,12 @@
 
 #include <mutex>
 
+#ifdef __CUDACC__
+#define KDA_HD __host__ __device__
+#else
+#define KDA_HD
+#endif
+
 namespace kda {
 
 template <int MaxDevices = 64>
@@ -46,6 +52,41 @@ class PerDeviceOnce {
 // producer blocks as consumers. False means: run the single-role chunk kernel instead.
 inline bool split_coresident(int per_sm, int sms, long long heads) {
     return per_sm >= 1 && sms >= 1 && heads >= 1 && (long long)per_sm * sms >= 2 * heads;
+}
+
+// Context parallelism: a sequence of `chunks` 64-token chunks runs as seg_count(chunks, segments)
+// segments (at least one, so an empty sequence still has a chain that carries its state), segment
+// g covering chunks [seg_chunk_begin(chunks, G, g), seg_chunk_begin(chunks, G, g + 1)). The host
+// plans with these and the device plan kernel derives the same table from them.
+KDA_HD inline int seg_count(int chunks, int segments) {
+    const int g = chunks < segments ? chunks : segments;
+    return g < 1 ? 1 : g;
+}
+KDA_HD inline int seg_chunk_begin(int chunks, int G, int g) {
+    return (int)((long long)g * chunks / G);
+}
+
+// Totals of a segmentation of num_seqs sequences (token offsets cu[0..num_seqs]): the segments
+// (chains), the chunks of all segments after their sequence's first (one E tile per chunk and
+// head), and the most chunks in one segment.
+struct SegTotals {
+    int num_vseqs = 0;
+    long long e_chunks = 0;
+    int max_chunks = 0;
+};
+inline SegTotals seg_totals(const int *cu, int num_seqs, int segments) {
+    SegTotals t;
+    for (int n = 0; n < num_seqs; ++n) {
+        const int chunks = (cu[n + 1] - cu[n] + 63) / 64;
+        const int G = seg_count(chunks, segments);
+        t.num_vseqs += G;
+        for (int g = 0; g < G; ++g) {
+            const int len = seg_chunk_begin(chunks, G, g + 1) - seg_chunk_begin(chunks, G, g);
+            if (g >= 1) t.e_chunks += len;
+            if (len > t.max_chunks) t.max_chunks = len;
+        }
+    }
+    return t;
 }
 
 }  // namespace kda

@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <string>
 
@@ -44,6 +45,7 @@ bool supported_d(int32_t d) { return d == 32 || d == 64 || d == 128; }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 constexpr size_t kStatusBytes = 256;
+constexpr int32_t kMaxSegments = 64;
 
 // Checks shared by the prefill entry points. On success returns KDA_OK.
 kda_status_t check_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -102,6 +104,25 @@ kda::Problem make_problem(const void *q, const void *k, const void *v, const flo
     return p;
 }
 
+// Byte ranges of the problem's buffers, for the debug build's access checks (no effect otherwise).
+void set_ranges(kda::Problem &p, const void *workspace, size_t workspace_bytes, int64_t state_entries) {
+    const uint64_t esz = p.dtype == KDA_BF16 ? 2 : 4;
+    const uint64_t sbytes = (uint64_t)state_entries * p.H * p.dk * p.dv * 4;
+    p.dbg.out = kda::buf_range(p.out, (uint64_t)p.total_tokens * p.H * p.dv * esz);
+    p.dbg.init = kda::buf_range(p.initial_state, sbytes);
+    p.dbg.fin = kda::buf_range(p.final_state, sbytes);
+    p.dbg.beta = kda::buf_range(p.beta, (uint64_t)p.total_tokens * p.H * 4);
+    p.dbg.ws = kda::buf_range(workspace, workspace_bytes);
+#ifdef KDA_DEBUG
+    // Debug builds only: declare the output smaller than it is, so a test can see the checks
+    // skip and report the writes past that point (the buffer itself is large enough for them).
+    if (const char *e = getenv("KDA_DEBUG_SHRINK_OUT")) {
+        const uint64_t b = strtoull(e, nullptr, 10);
+        if (p.dbg.out.hi > p.dbg.out.lo + b) p.dbg.out.hi = p.dbg.out.lo + b;
+    }
+#endif
+}
+
 // Workspace check and kernel choice shared by kda_prefill and kda_prefill_slots.
 kda_status_t run_prefill(kda::Problem &p, const int32_t *cu_seqlens_host, void *workspace,
                          size_t workspace_bytes, cudaStream_t s, const char *who) {
@@ -113,6 +134,7 @@ kda_status_t run_prefill(kda::Problem &p, const int32_t *cu_seqlens_host, void *
                     workspace, workspace_bytes, need);
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(KDA_ERR_INVALID_ARGUMENT, "workspace is not 256-byte aligned");
+    set_ranges(p, workspace, workspace_bytes, p.slots.init_slot ? p.slots.slots : p.num_seqs);
     cudaError_t e;
     int32_t max_chunks = 0;
     for (int32_t n = 0; n < p.num_seqs; ++n) {
@@ -170,6 +192,7 @@ kda_status_t kda_prefill(const void *q, const void *k, const void *v, const floa
                          int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
                          int32_t d_v, kda_dtype_t dtype, void *out, float *final_state,
                          void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+    KDA_RANGE("kda_prefill");
     kda_status_t st = check_prefill(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev,
                                     cu_seqlens_host, num_seqs, total_tokens, H, d_k, d_v, dtype,
                                     out, final_state);
@@ -180,6 +203,71 @@ kda_status_t kda_prefill(const void *q, const void *k, const void *v, const floa
                        reinterpret_cast<cudaStream_t>(stream), "kda_prefill: launch");
 }
 
+size_t kda_prefill_cp_workspace_size(int32_t num_seqs, const int32_t *cu_seqlens_host, int32_t H,
+                                     int32_t d_k, int32_t d_v, kda_dtype_t dtype, int32_t segments) {
+    if (num_seqs < 0 || H <= 0 || !supported_d(d_k) || !supported_d(d_v) ||
+        (dtype != KDA_F32 && dtype != KDA_BF16) || segments < 1 || segments > kMaxSegments ||
+        (num_seqs > 0 && !cu_seqlens_host))
+        return 0;
+    const int64_t total = num_seqs > 0 ? (int64_t)cu_seqlens_host[num_seqs] : 0;
+    const size_t plain = kda_prefill_workspace_size(num_seqs, total, H, d_k, d_v, dtype);
+    if (num_seqs == 0 || dtype != KDA_BF16 || d_k != 128 || d_v != 128 || segments == 1) return plain;
+    const kda::SegTotals t = kda::seg_totals(cu_seqlens_host, num_seqs, segments);
+    const size_t cp = kda::split_workspace_bytes((int64_t)t.num_vseqs * H) +
+                      kda::seg_workspace_bytes(num_seqs, t.num_vseqs, t.e_chunks, H);
+    return cp > plain ? cp : plain;
+}
+
+kda_status_t kda_prefill_cp(const void *q, const void *k, const void *v, const float *log_alpha,
+                            const float *beta, const float *initial_state,
+                            const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                            int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
+                            int32_t d_v, kda_dtype_t dtype, void *out, float *final_state,
+                            int32_t segments, void *workspace, size_t workspace_bytes,
+                            kda_stream_t stream) {
+    KDA_RANGE("kda_prefill_cp");
+    if (segments < 1 || segments > kMaxSegments)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "segments=%d outside [1, %d]", segments, kMaxSegments);
+    kda_status_t st = check_prefill(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev,
+                                    cu_seqlens_host, num_seqs, total_tokens, H, d_k, d_v, dtype,
+                                    out, final_state);
+    if (st != KDA_OK || num_seqs == 0) return st;
+    kda::Problem p = make_problem(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev,
+                                  num_seqs, total_tokens, H, d_k, d_v, dtype, out, final_state);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const kda::SegTotals t = kda::seg_totals(cu_seqlens_host, num_seqs, segments);
+    if (!kda::chunk_supported(p) || t.num_vseqs == num_seqs)  // nothing to split: the plain prefill
+        return run_prefill(p, cu_seqlens_host, workspace, workspace_bytes, s, "kda_prefill_cp: launch");
+    const size_t split_bytes = kda::split_workspace_bytes((int64_t)t.num_vseqs * H);
+    const size_t need = split_bytes + kda::seg_workspace_bytes(num_seqs, t.num_vseqs, t.e_chunks, H);
+    if (!workspace || workspace_bytes < need)
+        return fail(KDA_ERR_INVALID_ARGUMENT,
+                    "workspace %p of %zu bytes < %zu required for %d segments (kda_prefill_cp_workspace_size)",
+                    workspace, workspace_bytes, need, segments);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(KDA_ERR_INVALID_ARGUMENT, "workspace is not 256-byte aligned");
+    set_ranges(p, workspace, workspace_bytes, num_seqs);
+    kda::SegPlan sp;
+    sp.segments = segments;
+    sp.max_chunks = t.max_chunks;
+    kda::seg_carve(sp, static_cast<uint8_t *>(workspace) + split_bytes, num_seqs, t.num_vseqs,
+                   t.e_chunks, H);
+    p.seg = &sp;
+    cudaError_t e = kda::launch_seg_plan(p, sp, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_prefill_cp: plan");
+    bool not_coresident = false;
+    e = kda::launch_prefill_split(p, t.max_chunks, workspace, s, kda::kWaitTimeoutNs, &not_coresident);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_prefill_cp: launch");
+    if (not_coresident) {  // too many chains to be resident at once: the plain prefill
+        p.seg = nullptr;
+        return run_prefill(p, cu_seqlens_host, workspace, workspace_bytes, s, "kda_prefill_cp: launch");
+    }
+    int32_t n = 3;  // plan, split init, split kernel
+    e = kda::launch_seg_scan_fixup(p, sp, static_cast<int32_t *>(workspace), s, &n);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_prefill_cp: scan / fix-up");
+    return launched(n);
+}
+
 kda_status_t kda_prefill_prologue(const void *q, const void *k, const void *v,
                                   const float *log_alpha, const float *beta,
                                   const float *initial_state, const int32_t *cu_seqlens_dev,
@@ -188,6 +276,7 @@ kda_status_t kda_prefill_prologue(const void *q, const void *k, const void *v,
                                   kda_dtype_t dtype, void *out, float *final_state, void *workspace,
                                   size_t workspace_bytes, uint32_t prologue_flags, float gate_scale,
                                   kda_stream_t stream) {
+    KDA_RANGE("kda_prefill_prologue");
     constexpr uint32_t kAll =
         KDA_PROLOGUE_QK_L2NORM | KDA_PROLOGUE_GATE_SOFTPLUS | KDA_PROLOGUE_BETA_SIGMOID;
     if (prologue_flags & ~kAll)
@@ -213,6 +302,7 @@ kda_status_t kda_prefill_slots(const void *q, const void *k, const void *v, cons
                                int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
                                int32_t d_v, kda_dtype_t dtype, void *out, void *workspace,
                                size_t workspace_bytes, kda_stream_t stream) {
+    KDA_RANGE("kda_prefill_slots");
     if (pool_slots < 0 || pool_slots > INT32_MAX)
         return fail(KDA_ERR_INVALID_ARGUMENT, "pool_slots=%lld outside [0, 2^31)", (long long)pool_slots);
     if (pool_slots > 0 && !state_pool)
@@ -242,12 +332,14 @@ kda_status_t kda_prefill_recurrent(const void *q, const void *k, const void *v,
                                    int64_t total_tokens, int32_t H, int32_t d_k, int32_t d_v,
                                    kda_dtype_t dtype, void *out, float *final_state,
                                    kda_stream_t stream) {
+    KDA_RANGE("kda_prefill_recurrent");
     kda_status_t st = check_prefill(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev,
                                     cu_seqlens_host, num_seqs, total_tokens, H, d_k, d_v, dtype,
                                     out, final_state);
     if (st != KDA_OK || num_seqs == 0) return st;
     kda::Problem p = make_problem(q, k, v, log_alpha, beta, initial_state, cu_seqlens_dev,
                                   num_seqs, total_tokens, H, d_k, d_v, dtype, out, final_state);
+    set_ranges(p, nullptr, 0, num_seqs);
     cudaError_t e = kda::launch_prefill_recurrent(p, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kda_prefill_recurrent: launch");
     return launched(1);
@@ -257,6 +349,7 @@ kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const 
                              const float *beta, float *state, int32_t num_seqs, int32_t H,
                              int32_t d_k, int32_t d_v, kda_dtype_t dtype, void *out,
                              void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+    KDA_RANGE("kda_decode_step");
     (void)workspace;
     (void)workspace_bytes;
     if (dtype != KDA_F32 && dtype != KDA_BF16)
@@ -279,6 +372,9 @@ kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const 
     kda::DecodeProblem p;
     p.q = q; p.k = k; p.v = v; p.log_alpha = log_alpha; p.beta = beta; p.state = state;
     p.num_seqs = num_seqs; p.H = H; p.dk = d_k; p.dv = d_v; p.dtype = dtype; p.out = out;
+    const uint64_t esz = dtype == KDA_BF16 ? 2 : 4;
+    p.dbg.out = kda::buf_range(out, (uint64_t)num_seqs * H * d_v * esz);
+    p.dbg.init = p.dbg.fin = kda::buf_range(state, (uint64_t)num_seqs * H * d_k * d_v * 4);
     cudaError_t e = kda::launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step: launch");
     return launched(1);
@@ -290,6 +386,7 @@ kda_status_t kda_decode_step_slots(const void *q, const void *k, const void *v,
                                    int32_t H, int32_t d_k, int32_t d_v, kda_dtype_t dtype,
                                    void *out, void *workspace, size_t workspace_bytes,
                                    kda_stream_t stream) {
+    KDA_RANGE("kda_decode_step_slots");
     if (pool_slots < 0 || pool_slots > INT32_MAX)
         return fail(KDA_ERR_INVALID_ARGUMENT, "pool_slots=%lld outside [0, 2^31)", (long long)pool_slots);
     if (dtype != KDA_F32 && dtype != KDA_BF16)
@@ -323,6 +420,9 @@ kda_status_t kda_decode_step_slots(const void *q, const void *k, const void *v,
     p.slots.init_slot = p.slots.final_slot = slot_dev;
     p.slots.slots = pool_slots;
     p.slots.status = static_cast<int32_t *>(workspace);
+    const uint64_t esz = dtype == KDA_BF16 ? 2 : 4;
+    p.dbg.out = kda::buf_range(out, (uint64_t)num_seqs * H * d_v * esz);
+    p.dbg.init = p.dbg.fin = kda::buf_range(state_pool, (uint64_t)pool_slots * H * d_k * d_v * 4);
     cudaError_t e = cudaMemsetAsync(workspace, 0, kStatusBytes, s);
     if (e == cudaSuccess) e = kda::launch_decode(p, s);
     if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step_slots: launch");
@@ -420,6 +520,7 @@ kda_status_t kda_decode_verify(const void *q, const void *k, const void *v, cons
                                int32_t d_k, int32_t d_v, kda_dtype_t dtype, void *out,
                                float *u_cache, void *workspace, size_t workspace_bytes,
                                kda_stream_t stream) {
+    KDA_RANGE("kda_decode_verify");
     const char *who = "kda_decode_verify";
     kda_status_t st = check_verify(who, state, pool_slots, slot_dev, num_seqs, T, H, d_k, d_v, dtype,
                                    workspace, workspace_bytes);
@@ -439,6 +540,7 @@ kda_status_t kda_decode_commit(const void *k, const float *log_alpha, const floa
                                const int32_t *accepted_dev, int32_t num_seqs, int32_t T, int32_t H,
                                int32_t d_k, int32_t d_v, kda_dtype_t dtype, void *workspace,
                                size_t workspace_bytes, kda_stream_t stream) {
+    KDA_RANGE("kda_decode_commit");
     const char *who = "kda_decode_commit";
     kda_status_t st = check_verify(who, state, pool_slots, slot_dev, num_seqs, T, H, d_k, d_v, dtype,
                                    workspace, workspace_bytes);
@@ -461,6 +563,7 @@ kda_status_t kda_decode_commit_verify(const void *prev_k, const float *prev_log_
                                       kda_dtype_t dtype, void *out, float *u_cache,
                                       void *workspace, size_t workspace_bytes,
                                       kda_stream_t stream) {
+    KDA_RANGE("kda_decode_commit_verify");
     const char *who = "kda_decode_commit_verify";
     kda_status_t st = check_verify(who, state, pool_slots, slot_dev, num_seqs, T, H, d_k, d_v, dtype,
                                    workspace, workspace_bytes);
@@ -494,6 +597,7 @@ const char *kda_status_string(kda_status_t s) {
         case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
         case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
         case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+        case KDA_ERR_INTERNAL: return "KDA_ERR_INTERNAL";
     }
     return "KDA_ERR_UNKNOWN";
 }
@@ -502,12 +606,19 @@ const char *kda_last_error(void) { return g_last_error.c_str(); }
 
 kda_status_t kda_read_device_status(const void *workspace, kda_stream_t stream) {
     if (!workspace) return fail(KDA_ERR_INVALID_ARGUMENT, "workspace is NULL");
-    int32_t word = 0;
+    int32_t rec[4] = {0, 0, 0, 0};  // status word; with kStatusBounds: site, address
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof word, cudaMemcpyDeviceToHost, s);
+    cudaError_t e = cudaMemcpyAsync(rec, workspace, sizeof rec, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "kda_read_device_status");
+    const int32_t word = rec[0];
     if (word == 0) return ok();
+    if (word & kda::kStatusBounds) {
+        unsigned long long addr = 0;
+        memcpy(&addr, rec + 2, sizeof addr);
+        return fail(KDA_ERR_INTERNAL, "device status word 0x%x: the debug build caught an access "
+                    "outside its buffer at site %d (address 0x%llx)", (unsigned)word, rec[1], addr);
+    }
     if (word & (kda::kStatusBadSlot | kda::kStatusBadAccept))
         return fail(KDA_ERR_INVALID_ARGUMENT, "device status word 0x%x: a state slot outside "
                     "[-1, pool_slots) or an accepted count outside [0, T]", (unsigned)word);

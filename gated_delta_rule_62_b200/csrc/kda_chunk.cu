@@ -84,6 +84,7 @@ struct ChunkParams {
     int32_t H;
     uint64_t timeout_ns;
     StateSlots ss;
+    DebugRanges dbg;  // buffer ranges (checked by debug builds only)
 };
 
 template <int DS, bool PRO>
@@ -129,6 +130,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const int nchunks = (int)((eos - bos + C - 1) / C);
     const float *s0b = init_state_block(p.s0, n, H, h, (size_t)D * D, p.ss);
     float *sTb = final_state_block(p.sT, n, H, h, (size_t)D * D, p.ss);
+    if (s0b && !KDA_ACCESS_OK(p.status, p.dbg.init, s0b, D * D * 4, 11)) s0b = nullptr;
+    if (sTb && !KDA_ACCESS_OK(p.status, p.dbg.fin, sTb, D * D * 4, 12)) sTb = nullptr;
     const int c_me = 32 * quad + lane;  // key channel = TMEM lane of this thread
 
     if (tid == 0) {
@@ -232,7 +235,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     // beta of the next chunk is loaded one chunk ahead (one value per thread < C)
     const bool raw_beta = PRO && (p.pro.flags & KDA_PROLOGUE_BETA_SIGMOID) != 0;
     auto load_beta = [&](int64_t t) {
-        const float b = p.beta[(size_t)t * H + h];
+        const float *bp = p.beta + (size_t)t * H + h;
+        if (!KDA_ACCESS_OK(p.status, p.dbg.beta, bp, 4, 14)) return 0.f;
+        const float b = *bp;
         return raw_beta ? beta_from_raw(b) : b;
     };
     float beta_next = 0.f;
@@ -380,7 +385,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 const int col = half * SCOLS + 32 * part;
                 const float *v = vv[part];
                 const int i = 16 * quad + lane;
-                if (lane < 16 && i < valid) {
+                if (lane < 16 && i < valid &&
+                    KDA_ACCESS_OK(p.status, p.dbg.out, p.out + ((size_t)(t0 + i) * H + h) * D + d0 + col, 64, 13)) {
                     uint4 *dst = reinterpret_cast<uint4 *>(
                         p.out + ((size_t)(t0 + i) * H + h) * D + d0 + col);
 #pragma unroll
@@ -592,6 +598,7 @@ cudaError_t launch_prefill_chunk(const Problem &p, void *workspace, cudaStream_t
     cp.pro = p.pro;
     cp.s0 = p.initial_state;
     cp.sT = p.final_state;
+    cp.dbg = p.dbg;
     cp.out = static_cast<__nv_bfloat16 *>(p.out);
     cp.status = status;
     cp.ss = p.slots;

@@ -69,6 +69,12 @@ struct SplitParams {
     int32_t *next_item;  // producers' work counter (items k = chunk * heads + head, chunk-major)
     int32_t H, heads, max_chunks;
     uint64_t timeout_ns;
+    // context parallelism (segments as separate chains), or all null
+    const int4 *vinfo;   // [segments] {sequence, segment index, segments of the sequence, E offset}
+    float *seg_state;    // [segments, H, D, D] each chain's end state (sequences of several segments)
+    float *seg_trans;    // [segments, H, D, D] transition product of segments after the first
+    uint8_t *e_tiles;    // [E chunks, H] E = P R tiles
+    DebugRanges dbg;     // buffer ranges (checked by debug builds only)
 };
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
@@ -131,11 +137,17 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
-    const int H = p.H, n = hd / H, h = hd % H;
-    const int64_t bos = p.cu_seqlens[n], eos = p.cu_seqlens[n + 1];
+    const int H = p.H, v = hd / H, h = hd % H;
+    const int64_t bos = p.cu_seqlens[v], eos = p.cu_seqlens[v + 1];
     const int nchunks = (int)((eos - bos + C - 1) / C);
-    const float *s0b = init_state_block(p.s0, n, H, h, (size_t)D * D, p.ss);
-    float *sTb = final_state_block(p.sT, n, H, h, (size_t)D * D, p.ss);
+    // v is a sequence, or with context parallelism the first segment of sequence vinfo[v].x: it
+    // starts from the sequence's initial state; its end state goes to the scan if more segments follow
+    const int4 vi = p.vinfo ? p.vinfo[v] : make_int4(v, 0, 1, 0);
+    const float *s0b = init_state_block(p.s0, vi.x, H, h, (size_t)D * D, p.ss);
+    float *sTb = vi.z > 1 ? p.seg_state + (size_t)hd * D * D
+                          : final_state_block(p.sT, vi.x, H, h, (size_t)D * D, p.ss);
+    if (s0b && !KDA_ACCESS_OK(p.status, p.dbg.init, s0b, D * D * 4, 1)) s0b = nullptr;
+    if (sTb && !KDA_ACCESS_OK(p.status, vi.z > 1 ? p.dbg.ws : p.dbg.fin, sTb, D * D * 4, 2)) sTb = nullptr;
 
     if (tid == 0) {
         s_flags[0] = 0;
@@ -322,7 +334,256 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
             __nv_bfloat16 *dst = p.out + ((size_t)tc * H + h) * D + d_me;
 #pragma unroll
             for (int t = 0; t < C; ++t)
-                if (t < vc) dst[(size_t)t * H * D] = __float2bfloat16_rn(vv[t >> 5][t & 31]);
+                if (t < vc && KDA_ACCESS_OK(p.status, p.dbg.out, dst + (size_t)t * H * D, 2, 3))
+                    dst[(size_t)t * H * D] = __float2bfloat16_rn(vv[t >> 5][t & 31]);
+        }
+        tc_fence_before();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- consumer of a later segment
+// Context parallelism: a segment g >= 1 of a long sequence runs its chain before the state it starts
+// from is known. Its chunks see the true state S_j = S0_j + R_j S_start, where S0 is the chain from
+// a zero state and R_j = F_{j-1} ... F_0 (F = I + M) the product of the segment's chunk transitions,
+// so the output is O_j = O0_j + P_j R_j S_start. This consumer runs both chains on the same images,
+//   S0^T += S0_b^T M^T + U~^T K^,   R^T += R_b^T M^T   (R^T starts at I),
+// writes O0 = P S0_b + A U~ to `out`, and E_j = P_j R_j (computed transposed, E^T = R_b^T P^T) as a
+// bf16 tile for the fix-up, and at its end S0 and R as fp32 for the scan. Every TMEM region is
+// single-buffered (the two chains need 256 columns more than the plain consumer): the bf16 copies
+// for chunk c + 1 are written once chunk c's outputs are complete.
+namespace segc {
+constexpr uint32_t TM_S = 0, TM_SB = 128, TM_R = 192, TM_RB = 320, TM_O = 384, TM_E = 448, TM_COLS = 512;
+}  // namespace segc
+
+__device__ void consumer_seg(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t *sm, int hd,
+                             int4 vi) {
+    using namespace cons;
+    using segc::TM_S; using segc::TM_SB; using segc::TM_R; using segc::TM_RB;
+    using segc::TM_O; using segc::TM_E; using segc::TM_COLS;
+    constexpr uint32_t I_C = idesc_bf16_f32(128, 128, false, 0, 0);   // X_b^T M^T (A in TMEM)
+    constexpr uint32_t I_K = idesc_bf16_f32(128, 128, false, 1, 1);   // U~^T K^
+    constexpr uint32_t I_OP = idesc_bf16_f32(128, 64, false, 0, 0);   // X_b^T P^T (A in TMEM)
+    constexpr uint32_t I_OA = idesc_bf16_f32(128, 64, false, 1, 0);   // U~^T A^T
+    // full0, full1, o0, o1, ready (bf16 copies written), free (O and E read), teardown
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);
+    uint32_t *s_flags = reinterpret_cast<uint32_t *>(sm + MISC + 96);  // abort, tmem
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3;
+    const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+    const int H = p.H, v = hd / H, h = hd % H;
+    const int64_t bos = p.cu_seqlens[v], eos = p.cu_seqlens[v + 1];
+    const int nchunks = (int)((eos - bos + C - 1) / C);
+    float *s_end = p.seg_state + (size_t)hd * D * D;
+    float *r_end = p.seg_trans + (size_t)hd * D * D;
+    const bool ends_ok = KDA_ACCESS_OK(p.status, p.dbg.ws, s_end, D * D * 4, 4) &&
+                         KDA_ACCESS_OK(p.status, p.dbg.ws, r_end, D * D * 4, 5);
+
+    if (tid == 0) {
+        s_flags[0] = 0;
+        for (int k = 0; k < 7; ++k) mbar_init(&bars[k], (k == 4 || k == 5) ? NT / 2 : 1);
+        fence_mbarrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&s_flags[1], TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_flags[1];
+    auto fail = [&]() {
+        s_flags[0] = 1;
+        atomicOr(p.status, 1);
+    };
+
+    if (tid == LDR) {
+        // ------------------------------------------------ loader thread (as in the plain consumer)
+        uint32_t ph_o[2] = {0, 0};
+        int requested = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1;
+            if (ld_volatile(&s_flags[0])) break;
+            if (!wait_flag_ge(p.filled + hd * RING + (c % RING), c + 1, p.timeout_ns)) { fail(); break; }
+            fence_proxy_async_global();
+            if (c >= 2) {
+                if (!mbar_wait_bounded(&bars[2 + b], ph_o[b], p.timeout_ns)) { fail(); break; }
+                ph_o[b] ^= 1u;
+                st_release(p.consumed + hd, c - 1);
+            }
+            const int32_t row0 = (int32_t)(((uint32_t)hd * RING + (uint32_t)(c % RING)) * SLOT_ROWS);
+            uint8_t *dst = sm + (b ? STAGE1 : STAGE0);
+            mbar_arrive_expect_tx(&bars[b], SLOT);
+#pragma unroll
+            for (uint32_t k = 0; k < SLOT_ROWS / RL_BOX; ++k)
+                tma_load_2d(dst + k * RL_BOX * ROW_BYTES, tm_rl, &bars[b], 0, row0 + (int32_t)(k * RL_BOX));
+            requested = c + 1;
+        }
+        for (int c = requested - 2 < 0 ? 0 : requested - 2; c < requested; ++c)
+            if (!mbar_wait_bounded(&bars[c & 1], (uint32_t)(c >> 1) & 1u, p.timeout_ns)) fail();
+        if (requested == nchunks) st_release(p.consumed + hd, nchunks);
+    } else if (tid == CTL) {
+        // ------------------------------------------------ MMA thread
+        uint32_t ph_full[2] = {0, 0}, ph_ready = 0, ph_free = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1;
+            if (ld_volatile(&s_flags[0])) break;
+            if (!mbar_wait_bounded(&bars[b], ph_full[b], p.timeout_ns)) { fail(); break; }
+            ph_full[b] ^= 1u;
+            if (!mbar_wait_bounded(&bars[4], ph_ready, p.timeout_ns)) { fail(); break; }
+            ph_ready ^= 1u;
+            tc_fence_after();
+            const uint32_t st = sb + (b ? STAGE1 : STAGE0);
+            const uint64_t dM = desc_k(st + SL_M, 16384, 0), dK = desc_mn(st + SL_KH, 8192, 0);
+            const uint64_t dU = desc_mn(st + SL_U, 8192, 0);
+            const uint64_t dP = desc_k(st + SL_P, 8192, 0), dA = desc_k(st + SL_A, 8192, 0);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 8; ++kk)  // S0^T += S0_b^T M^T ...
+                mma_bf16_ts(tmem + TM_S, tmem + TM_SB + 8 * kk, desc_k_at(dM, 16384, kk), I_C, 1);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)  // ... + U~^T K^
+                mma_bf16_ss(tmem + TM_S, desc_mn_at(dU, kk), desc_mn_at(dK, kk), I_K, 1);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 8; ++kk)  // R^T += R_b^T M^T
+                mma_bf16_ts(tmem + TM_R, tmem + TM_RB + 8 * kk, desc_k_at(dM, 16384, kk), I_C, 1);
+            if (c >= 1) {  // the output warps have read O and E of chunk c - 1
+                if (!mbar_wait_bounded(&bars[5], ph_free, p.timeout_ns)) { fail(); break; }
+                ph_free ^= 1u;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (uint32_t kk = 0; kk < 8; ++kk)  // O0^T = S0_b^T P^T ...
+                mma_bf16_ts(tmem + TM_O, tmem + TM_SB + 8 * kk, desc_k_at(dP, 8192, kk), I_OP, kk > 0);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)  // ... + U~^T A^T
+                mma_bf16_ss(tmem + TM_O, desc_mn_at(dU, kk), desc_k_at(dA, 8192, kk), I_OA, 1);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 8; ++kk)  // E^T = R_b^T P^T
+                mma_bf16_ts(tmem + TM_E, tmem + TM_RB + 8 * kk, desc_k_at(dP, 8192, kk), I_OP, kk > 0);
+            mma_commit(&bars[2 + b]);  // both chains, O, E and the stage are done
+        }
+        mma_commit(&bars[6]);
+        mbar_wait_bounded(&bars[6], 0, p.timeout_ns);
+    } else if (warp < 4) {
+        // ------------------------------------------------ state warps (lane = value channel d for
+        // S0^T, = column a of R for R^T); after chunk c's outputs: the bf16 copies for chunk c + 1
+        const int d_me = tid;  // 0..127
+        auto pack_store = [&](const float (&x)[2][32], uint32_t tm_b, int hh) {
+            float f[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                f[e] = __uint_as_float(pack2(x[e >> 4][2 * (e & 15)], x[e >> 4][2 * (e & 15) + 1]));
+            tmem_st32(tmem + lane_base + tm_b + 32 * hh, f);
+        };
+        // S0^T = 0, R^T = I and their bf16 copies, 32 columns at a time
+        for (int which = 0; which < 2; ++which) {
+            const uint32_t tm_x = which ? TM_R : TM_S, tm_b = which ? TM_RB : TM_SB;
+            for (int part = 0; part < 4; ++part) {
+                float x[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[e] = (which && 32 * part + e == d_me) ? 1.f : 0.f;
+                tmem_st32(tmem + lane_base + tm_x + 32 * part, x);
+                float f[32];  // columns 32 part .. + 31 as 16 bf16 pairs: half a 32-column copy store
+#pragma unroll
+                for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(pack2(x[2 * e], x[2 * e + 1]));
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(f[e]);
+                // bf16 copy column (32 part + 2e) / 2 = 16 part + e
+                asm volatile(
+                    "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+                    "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+                        tmem + lane_base + tm_b + 16 * part),
+                    "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]),
+                    "r"(w[7]), "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]),
+                    "r"(w[14]), "r"(w[15])
+                    : "memory");
+            }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars[4]);
+        uint32_t ph_o[2] = {0, 0};
+        for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1;
+            const bool last = c + 1 == nchunks;
+            if (ld_volatile(&s_flags[0])) break;
+            const bool ok = mbar_wait_bounded(&bars[2 + b], ph_o[b], p.timeout_ns);
+            ph_o[b] ^= 1u;
+            if (!ok) { fail(); break; }
+            tc_fence_after();
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t tm_x = which ? TM_R : TM_S, tm_b = which ? TM_RB : TM_SB;
+                float *dst_end = which ? r_end : s_end;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float x[2][32];
+                    tmem_ld32(tmem + lane_base + tm_x + 64 * hh, x[0]);
+                    tmem_ld32(tmem + lane_base + tm_x + 64 * hh + 32, x[1]);
+                    tmem_wait_ld();
+                    if (!last) {
+                        pack_store(x, tm_b, hh);
+                    } else if (ends_ok) {
+                        // row d_me of S0^T (or column d_me of R) -> element [c][d_me], c = 64 hh + e
+                        float *dst = dst_end + (size_t)(64 * hh) * D + d_me;
+#pragma unroll
+                        for (int e = 0; e < 64; ++e) dst[(size_t)e * D] = x[e >> 5][e & 31];
+                    }
+                }
+            }
+            if (!last) {
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bars[4]);
+            }
+        }
+        tc_fence_before();
+    } else if (tid < NT) {
+        // ------------------------------------------------ output warps: O0 -> out, E^T -> its tile
+        const int d_me = 32 * quad + lane;  // value channel of O0^T, row a of E^T
+        uint32_t ph_o[2] = {0, 0};
+        for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1;
+            if (ld_volatile(&s_flags[0])) break;
+            const bool ok = mbar_wait_bounded(&bars[2 + b], ph_o[b], p.timeout_ns);
+            ph_o[b] ^= 1u;
+            if (!ok) { fail(); break; }
+            tc_fence_after();
+            const int64_t tc = bos + (int64_t)c * C;
+            const int vc = (int)(eos - tc < C ? eos - tc : C);
+            // E^T first (row a = d_me, 64 tokens, as a 128-byte swizzled row of a [128][64] bf16
+            // tile), then O0: one accumulator's registers live at a time
+            uint8_t *et = p.e_tiles + ((size_t)(vi.w + c) * H + h) * 16384 + (uint32_t)(d_me >> 3) * 1024 +
+                          (uint32_t)(d_me & 7) * 128;
+            const bool et_ok = KDA_ACCESS_OK(p.status, p.dbg.ws, et, 128, 6);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                float ee[32];
+                tmem_ld32(tmem + lane_base + TM_E + 32 * part, ee);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const uint32_t q8 = 4 * part + q4;
+                    if (et_ok) st_chunk(et + ((q8 ^ (uint32_t)(d_me & 7)) << 4), ee + 8 * q4);
+                }
+            }
+            float oo[2][32];
+            tmem_ld32(tmem + lane_base + TM_O, oo[0]);
+            tmem_ld32(tmem + lane_base + TM_O + 32, oo[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&bars[5]);  // read: O and E may take chunk c + 1
+            __nv_bfloat16 *dst = p.out + ((size_t)tc * H + h) * D + d_me;
+#pragma unroll
+            for (int t = 0; t < C; ++t)
+                if (t < vc && KDA_ACCESS_OK(p.status, p.dbg.out, dst + (size_t)t * H * D, 2, 7))
+                    dst[(size_t)t * H * D] = __float2bfloat16_rn(oo[t >> 5][t & 31]);
         }
         tc_fence_before();
     }
@@ -469,7 +730,9 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         const Item it = decode(k);
         const int64_t t0 = it.bos + (int64_t)it.c * C;
         if (t0 + tid >= it.eos) return 0.f;
-        const float b = p.beta[(size_t)(t0 + tid) * H + it.h];
+        const float *bp = p.beta + (size_t)(t0 + tid) * H + it.h;
+        if (!KDA_ACCESS_OK(p.status, p.dbg.beta, bp, 4, 8)) return 0.f;
+        const float b = *bp;
         return (PRO && (p.pro.flags & KDA_PROLOGUE_BETA_SIGMOID)) ? beta_from_raw(b) : b;
     };
     // the previous image, published once its bulk stores are complete (control thread, during
@@ -716,9 +979,13 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     // 1024-byte aligned (128-byte swizzled tiles); offsetting the shared array itself keeps the
     // accesses in the shared state space (an integer round trip would make them generic)
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    if ((int)blockIdx.x < p.heads)
-        consumer(&tm_rl, p, sm, blockIdx.x);
-    else
+    if ((int)blockIdx.x < p.heads) {
+        const int4 vi = p.vinfo ? p.vinfo[blockIdx.x / p.H] : make_int4(0, 0, 1, 0);
+        if (vi.y > 0)
+            consumer_seg(&tm_rl, p, sm, blockIdx.x, vi);
+        else
+            consumer(&tm_rl, p, sm, blockIdx.x);
+    } else
         producer<PRO>(&tm_q, &tm_k, &tm_v, &tm_la, &tm_rs, p, sm, blockIdx.x - p.heads, gridDim.x - p.heads);
 }
 
@@ -752,7 +1019,8 @@ size_t split_workspace_bytes(int64_t heads) {
 cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *workspace,
                                  cudaStream_t stream, uint64_t timeout_ns, bool *not_coresident) {
     *not_coresident = false;
-    const int64_t heads = (int64_t)p.num_seqs * p.H;
+    // with context parallelism every segment is a chain of its own
+    const int64_t heads = (int64_t)(p.seg ? p.seg->num_vseqs : p.num_seqs) * p.H;
     const int sms = sm_count();
     int per_sm = 0;
     static PerDeviceOnce<> once_plain, once_pro;
@@ -790,7 +1058,12 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
     if (e != cudaSuccess) return e;
 
     SplitParams sp;
-    sp.cu_seqlens = p.cu_seqlens;
+    sp.cu_seqlens = p.seg ? p.seg->vcu : p.cu_seqlens;
+    sp.vinfo = p.seg ? p.seg->vinfo : nullptr;
+    sp.seg_state = p.seg ? p.seg->seg_state : nullptr;
+    sp.seg_trans = p.seg ? p.seg->seg_trans : nullptr;
+    sp.e_tiles = p.seg ? p.seg->e_tiles : nullptr;
+    sp.dbg = p.dbg;
     sp.beta = p.beta;
     sp.pro = p.pro;
     sp.s0 = p.initial_state;

@@ -32,7 +32,8 @@ template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
 decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta,
-              float *__restrict__ state, Tin *__restrict__ out, int H, const StateSlots ss) {
+              float *__restrict__ state, Tin *__restrict__ out, int H, const StateSlots ss,
+              const DebugRanges dbg) {
     using Sh = DecodeShape<DK, DV>;
     constexpr int CG = Sh::CG, NT = Sh::NT, R = Sh::R, RPT = Sh::RPT;
     __shared__ float s_k[DK], s_q[DK], s_a[DK];
@@ -45,6 +46,7 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     const int cg = tid % CG, rg = tid / CG;
     // this head's state: entry `head`, or its sequence's slot of the pool (none: zeros, not stored)
     float *blk = final_state_block(state, (int)(head / H), H, (int)(head % H), (size_t)(DK * DV), ss);
+    if (blk && !KDA_ACCESS_OK(ss.status, dbg.fin, blk, DK * DV * 4, 31)) blk = nullptr;
     float4 *S4 = reinterpret_cast<float4 *>(blk);
 
     // Issue the state loads first: they are the only long-latency traffic.
@@ -88,7 +90,8 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
         for (int r = 0; r < R; ++r) { a += s_red[0][r][tid]; b += s_red[1][r][tid]; }
         const float u = beta[head] * (to_f32(v[head * DV + tid]) - a);
         s_u[tid] = u;
-        out[head * DV + tid] = from_f32<Tin>(fmaf(s_kq, u, b));
+        if (KDA_ACCESS_OK(ss.status, dbg.out, out + head * DV + tid, sizeof(Tin), 32))
+            out[head * DV + tid] = from_f32<Tin>(fmaf(s_kq, u, b));
     }
     __syncthreads();
 
@@ -345,7 +348,7 @@ cudaError_t launch3(const DecodeProblem &p, cudaStream_t stream) {
     const unsigned blocks = (unsigned)p.num_seqs * (unsigned)p.H;
     decode_kernel<Tin, DK, DV><<<blocks, DecodeShape<DK, DV>::NT, 0, stream>>>(
         (const Tin *)p.q, (const Tin *)p.k, (const Tin *)p.v, p.log_alpha, p.beta, p.state,
-        (Tin *)p.out, p.H, p.slots);
+        (Tin *)p.out, p.H, p.slots, p.dbg);
     return cudaGetLastError();
 }
 

@@ -8,6 +8,23 @@
 #include "host_plan.h"
 #include "kda.h"
 
+// ---- optional NVTX ranges (build with -DKDA_NVTX): one named range per library call, so a
+// profiler's timeline shows which entry point enqueued which kernels. Off by default: no cost.
+#ifdef KDA_NVTX
+#include <nvtx3/nvToolsExt.h>
+namespace kda {
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+}  // namespace kda
+#define KDA_RANGE(name) ::kda::NvtxRange kda_nvtx_range_(name)
+#else
+#define KDA_RANGE(name) ((void)0)
+#endif
+
 namespace kda {
 
 // Sets a kernel's dynamic shared-memory limit on the current device, once per device (the
@@ -36,7 +53,41 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // Entry n of initial_state / final_state ([N, H, d_k, d_v]); or, with slot tables, slot
 // init_slot[n] / final_slot[n] of one pool ([slots, H, d_k, d_v]), -1 meaning none. A slot outside
 // [-1, slots) counts as -1 and sets kStatusBadSlot in the device status word.
-constexpr int32_t kStatusTimeout = 1, kStatusBadSlot = 2, kStatusBadAccept = 4;
+constexpr int32_t kStatusTimeout = 1, kStatusBadSlot = 2, kStatusBadAccept = 4, kStatusBounds = 8;
+
+// ---- debug builds (-DKDA_DEBUG): every global access at a computed address is checked against
+// the byte range of the buffer it belongs to. An access outside it is skipped, and the first one
+// is recorded in the device status word: bit kStatusBounds, then word 1 = the access site, words
+// 2-3 = the offending address. No trap, no assert: the kernel keeps running and the host reads
+// the record (kda_read_device_status -> KDA_ERR_INTERNAL). Release builds compile the checks away.
+struct BufRange {
+    uintptr_t lo = 0, hi = 0;  // [lo, hi); empty: not checked
+};
+struct DebugRanges {
+    BufRange out, init, fin, beta, ws;  // outputs, initial / final states, beta, workspace
+};
+__host__ __device__ inline BufRange buf_range(const void *p, uint64_t bytes) {
+    BufRange r;
+    r.lo = reinterpret_cast<uintptr_t>(p);
+    r.hi = p ? r.lo + bytes : 0;
+    return r;
+}
+#ifdef KDA_DEBUG
+static __device__ __noinline__ bool debug_access_ok(int32_t *status, const BufRange &r, const void *p,
+                                             uint32_t bytes, int site) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    if (r.hi == r.lo || (a >= r.lo && a + bytes <= r.hi)) return true;
+    if (status && !(atomicOr(status, kStatusBounds) & kStatusBounds)) {
+        status[1] = site;
+        reinterpret_cast<unsigned long long *>(status)[1] = (unsigned long long)a;
+    }
+    return false;
+}
+#define KDA_ACCESS_OK(status, range, ptr, bytes, site) \
+    ::kda::debug_access_ok((status), (range), (ptr), (bytes), (site))
+#else
+#define KDA_ACCESS_OK(status, range, ptr, bytes, site) true
+#endif
 struct StateSlots {
     const int32_t *init_slot = nullptr, *final_slot = nullptr;  // device tables (or null)
     int64_t slots = 0;
@@ -79,6 +130,25 @@ __device__ __forceinline__ float gate_from_raw(float g, float scale) {
 }
 __device__ __forceinline__ float beta_from_raw(float b) { return 1.f / (1.f + __expf(-b)); }
 
+// ---- context parallelism: long sequences split into segments run as separate chains ------
+// Device tables and buffers in the workspace (see kda_context.cu). A segment is a "virtual
+// sequence" v with token offsets vcu[v], vcu[v + 1]; vinfo[v] = {sequence n, segment index g,
+// segments of n, first chunk of its E tiles}. Segments g >= 1 start from a zero state; their
+// consumers also carry the segment's transition product and emit, per chunk, E = P R: the
+// chunk's output is its zero-start output plus E times the segment's true start state, which
+// the scan kernel finds after all chains are done and the fix-up kernel applies.
+struct SegPlan {
+    int32_t *vcu = nullptr;       // [N_v + 1]
+    int4 *vinfo = nullptr;        // [N_v]
+    int32_t *vfirst = nullptr;    // [N] first segment of each sequence
+    float *seg_state = nullptr;   // [N_v, H, d_k, d_v] fp32 end state of each segment's chain
+    float *seg_trans = nullptr;   // [N_v, H, d_k, d_k] fp32 transition product of segments g >= 1
+    uint8_t *s_start = nullptr;   // [N_v, H] 32 KB bf16 tiles: true start state of segments g >= 1
+    uint8_t *e_tiles = nullptr;   // [E chunks, H] 16 KB bf16 tiles
+    int32_t segments = 1, num_vseqs = 0, e_chunks = 0, max_chunks = 0;
+};
+constexpr uint32_t kSegStartTileBytes = 32768, kSegETileBytes = 16384;
+
 // ---- problem description passed from the API layer to the launchers --------------------
 struct Problem {
     const void *q, *k, *v;
@@ -93,6 +163,8 @@ struct Problem {
     float *final_state;          // or the state pool (with slots)
     StateSlots slots;
     Prologue pro;
+    const SegPlan *seg = nullptr;  // context parallelism (split kernel only), or none
+    DebugRanges dbg;               // buffer ranges for the debug build's access checks
 };
 
 // Each launcher enqueues its kernel(s) on `stream` and returns the launch's cudaError_t.
@@ -117,6 +189,16 @@ size_t split_workspace_bytes(int64_t heads);
 cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *workspace,
                                  cudaStream_t stream, uint64_t timeout_ns, bool *not_coresident);
 
+// Context parallelism (kda_context.cu): workspace bytes beyond the split kernel's for a plan, and
+// the launches around the split kernel: the plan kernel before it, then the segment scan (true
+// start and final states) and the output fix-up after it.
+size_t seg_workspace_bytes(int32_t num_seqs, int32_t num_vseqs, int64_t e_chunks, int32_t H);
+void seg_carve(SegPlan &sp, void *base, int32_t num_seqs, int32_t num_vseqs, int64_t e_chunks,
+               int32_t H);
+cudaError_t launch_seg_plan(const Problem &p, const SegPlan &sp, cudaStream_t stream);
+cudaError_t launch_seg_scan_fixup(const Problem &p, const SegPlan &sp, int32_t *status,
+                                  cudaStream_t stream, int32_t *launches);
+
 // Records `msg` as the calling thread's kda_last_error() and returns `st`.
 kda_status_t record_error(kda_status_t st, const char *msg);
 
@@ -131,6 +213,7 @@ struct DecodeProblem {
     kda_dtype_t dtype;
     void *out;
     StateSlots slots;
+    DebugRanges dbg;
 };
 cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream);
 

@@ -57,6 +57,7 @@ extern "C" KDA_API kda_status_t kda_prefill_noalloc(
     const float *initial_state, const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
     int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k, int32_t d_v,
     kda_dtype_t dtype, void *out, float *final_state, kda_stream_t stream) {
+    KDA_RANGE("kda_prefill_noalloc");
     if (num_seqs > kNoallocMaxSeqs) {
         char msg[160];
         snprintf(msg, sizeof msg, "kda_prefill_noalloc: num_seqs=%d exceeds the fixed scratch limit of %d",

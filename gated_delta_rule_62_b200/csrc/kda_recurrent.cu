@@ -25,7 +25,7 @@ recurrent_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin
                  const float *__restrict__ log_alpha, const float *__restrict__ beta,
                  const float *s0, const int32_t *__restrict__ cu_seqlens, int H,
                  int dv, Tin *__restrict__ out, float *sT, const StateSlots ss,
-                 const Prologue pro) {
+                 const Prologue pro, const DebugRanges dbg) {
     constexpr int R = DK / 32;  // key rows per lane
     const int n = blockIdx.x, h = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -34,6 +34,7 @@ recurrent_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin
 
     float S[R][kCols];
     const float *src = init_state_block(s0, n, H, h, (size_t)DK * dv, ss);
+    if (src && !KDA_ACCESS_OK(ss.status, dbg.init, src, DK * dv * 4, 41)) src = nullptr;
 #pragma unroll
     for (int m = 0; m < R; ++m)
 #pragma unroll
@@ -111,7 +112,9 @@ recurrent_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin
             const float o = fmaf(kq, u, pb[j]);
             if (lane == j) o_mine = o;
         }
-        if (lane < kCols) out[((size_t)t * H + h) * dv + col0 + lane] = from_f32<Tin>(o_mine);
+        if (lane < kCols &&
+            KDA_ACCESS_OK(ss.status, dbg.out, out + ((size_t)t * H + h) * dv + col0 + lane, sizeof(Tin), 43))
+            out[((size_t)t * H + h) * dv + col0 + lane] = from_f32<Tin>(o_mine);
 
 #pragma unroll
         for (int m = 0; m < R; ++m) { kc[m] = nk[m]; qc[m] = nq[m]; lc[m] = nl[m]; }
@@ -120,7 +123,7 @@ recurrent_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin
         bt = nb;
     }
     float *dst = final_state_block(sT, n, H, h, (size_t)DK * dv, ss);
-    if (dst) {
+    if (dst && KDA_ACCESS_OK(ss.status, dbg.fin, dst, DK * dv * 4, 42)) {
 #pragma unroll
         for (int m = 0; m < R; ++m)
 #pragma unroll
@@ -135,7 +138,7 @@ cudaError_t launch_typed(const Problem &p, cudaStream_t stream) {
     auto args = [&](auto kern) {
         kern<<<grid, 128, 0, stream>>>((const Tin *)p.q, (const Tin *)p.k, (const Tin *)p.v,
                                        p.log_alpha, p.beta, p.initial_state, p.cu_seqlens, p.H,
-                                       p.dv, (Tin *)p.out, p.final_state, p.slots, p.pro);
+                                       p.dv, (Tin *)p.out, p.final_state, p.slots, p.pro, p.dbg);
     };
     switch (p.dk) {
         case 32: args(recurrent_kernel<Tin, 32>); break;

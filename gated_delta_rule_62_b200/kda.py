@@ -17,9 +17,10 @@ from typing import Optional
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libkda.so")
+# KDA_LIB selects another build of the library (e.g. the bounds-checked libkda_debug.so).
+LIB_PATH = os.environ.get("KDA_LIB") or os.path.join(_PKG, "libkda.so")
 
-KDA_OK, KDA_ERR_INVALID_ARGUMENT, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
+KDA_OK, KDA_ERR_INVALID_ARGUMENT, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_INTERNAL = range(6)
 KDA_F32, KDA_BF16 = 0, 1
 
 _lock = threading.Lock()
@@ -45,6 +46,9 @@ SIGNATURES = {
     "kda_prefill_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                                    _i32, _i32, _vp, _vp, _vp]),
     "kda_prefill_noalloc_status": (_i32, [_vp]),
+    "kda_prefill_cp": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
+                              _i32, _vp, _vp, _i32, _vp, _sz, _vp]),
+    "kda_prefill_cp_workspace_size": (_sz, [_i32, _vp, _i32, _i32, _i32, _i32, _i32]),
     "kda_prefill_slots": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _i32, _i64,
                                  _i32, _i32, _i32, _i32, _vp, _vp, _sz, _vp]),
     "kda_decode_step_slots": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _i32,
@@ -129,7 +133,8 @@ def workspace_size(num_seqs: int, total_tokens: int, H: int, dk: int, dv: int, d
 
 def prefill(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, cu_seqlens_dev=None,
             out=None, final_state=None, workspace=None, output_final_state=True,
-            algo: str = "auto", stream=None, prologue: int = 0, gate_scale: float = 1.0):
+            algo: str = "auto", stream=None, prologue: int = 0, gate_scale: float = 1.0,
+            segments: int = 2):
     """Chunked KDA prefill over packed sequences (``kda_prefill``).
 
     prologue: KDA_PROLOGUE_* flags (``kda_prefill_prologue``): q, k, log_alpha, beta hold the
@@ -138,7 +143,8 @@ def prefill(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, cu_se
     q, k, log_alpha: [T, H, d_k] (or [B, T, H, d_k]); v: [T, H, d_v]; beta [T, H].
     cu_seqlens: host int32 offsets [N + 1] (default: one sequence, or B equal ones
     for 4-D inputs); cu_seqlens_dev: the same on the device (copied if omitted).
-    algo: "auto" (``kda_prefill``) or "recurrent" (``kda_prefill_recurrent``).
+    algo: "auto" (``kda_prefill``), "recurrent" (``kda_prefill_recurrent``) or "cp"
+    (``kda_prefill_cp``: context parallelism, each sequence cut into up to ``segments`` segments).
     Returns (out, final_state or None).
     """
     dense = q.dim() == 4
@@ -186,6 +192,18 @@ def prefill(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, cu_se
         if prologue:
             raise ValueError("the prologue runs through kda_prefill_prologue (algo='auto')")
         _check(L.kda_prefill_recurrent(*common, _stream(stream)), "kda_prefill_recurrent")
+    elif algo == "cp":
+        if prologue:
+            raise ValueError("the prologue runs through kda_prefill_prologue (algo='auto')")
+        cu_p = ctypes.c_void_p(cu_host.data_ptr())
+        need = int(L.kda_prefill_cp_workspace_size(N, cu_p, H, dk, dv, code, int(segments)))
+        if need == 0:
+            raise ValueError("kda_prefill_cp_workspace_size rejected the arguments")
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _need(workspace, "workspace", torch.uint8, 1)
+        _check(L.kda_prefill_cp(*common, int(segments), _ptr(workspace), workspace.numel(), _stream(stream)),
+               "kda_prefill_cp")
     elif algo == "auto":
         need = workspace_size(N, Ttot, H, dk, dv, dtype)
         if workspace is None:

@@ -63,7 +63,9 @@ typedef enum {
     KDA_ERR_INVALID_ARGUMENT = 1, /* bad pointer, size, shape, or cu_seqlens            */
     KDA_ERR_UNSUPPORTED = 2,      /* a dtype / head-size combination with no kernel       */
     KDA_ERR_CUDA = 3,             /* a CUDA runtime call or launch failed                 */
-    KDA_ERR_TIMEOUT = 4           /* a bounded on-device wait gave up (device status word) */
+    KDA_ERR_TIMEOUT = 4,          /* a bounded on-device wait gave up (device status word) */
+    KDA_ERR_INTERNAL = 5          /* a debug build (-DKDA_DEBUG) caught an access outside its
+                                     buffer (device status word); never set by release builds */
 } kda_status_t;
 
 typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
@@ -132,6 +134,48 @@ KDA_API kda_status_t kda_prefill(const void *q, const void *k, const void *v,
                          int32_t d_k, int32_t d_v, kda_dtype_t dtype,
                          void *out, float *final_state,
                          void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * kda_prefill with context parallelism inside the GPU: each sequence is cut
+ * into up to `segments` segments of whole 64-token chunks (fewer if it has
+ * fewer chunks), and their state chains run side by side instead of one after
+ * another.
+ *
+ * Defined by: the blockwise, context-parallel computation of the KDA update in
+ * "Kimi Delta Attention: the load-bearing choice" (shivam2003.com Kimi K3
+ * article). The state map of a segment is affine, S_end = F S_start + S0_end
+ * (F: the product of the segment's per-chunk transitions, S0: the segment run
+ * from a zero state), so segments after the first run from zero alongside the
+ * product F and a per-chunk correction term; a scan then finds each segment's
+ * true start state (and the final state) and a fix-up pass adds the start
+ * state's contribution to the outputs. The result is kda_prefill's up to
+ * rounding.
+ *
+ * Applies to bf16 inputs with d_k = d_v = 128; with segments = 1, other
+ * dtypes / head sizes, sequences too short to split, or more chains than the
+ * GPU can hold at once (2 * segments * H thread blocks resident), it runs
+ * kda_prefill's own path. The workspace must hold
+ * kda_prefill_cp_workspace_size(...) bytes (about 16 KiB per chunk and head of
+ * every segment after a sequence's first, plus the split kernel's ring).
+ * Arguments, layouts and status as kda_prefill; segments in [1, 64].
+ */
+KDA_API kda_status_t kda_prefill_cp(const void *q, const void *k, const void *v,
+                            const float *log_alpha, const float *beta,
+                            const float *initial_state,
+                            const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                            int32_t num_seqs, int64_t total_tokens, int32_t H,
+                            int32_t d_k, int32_t d_v, kda_dtype_t dtype,
+                            void *out, float *final_state, int32_t segments,
+                            void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * Workspace bytes kda_prefill_cp needs for these sequences (it reads
+ * cu_seqlens_host[0..num_seqs]) and `segments`; at least
+ * kda_prefill_workspace_size. 0 for arguments kda_prefill_cp rejects.
+ */
+KDA_API size_t kda_prefill_cp_workspace_size(int32_t num_seqs, const int32_t *cu_seqlens_host,
+                                             int32_t H, int32_t d_k, int32_t d_v,
+                                             kda_dtype_t dtype, int32_t segments);
 
 /*
  * The same operation as kda_prefill, always on the token-serial kernel: one

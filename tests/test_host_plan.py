@@ -52,6 +52,24 @@ int main() {
     CHECK(!kda::split_coresident(1, 20, 16));    // few SMs visible (a partitioned context)
     CHECK(kda::split_coresident(2, 16, 16));
     CHECK(!kda::split_coresident(1, 148, 0));
+    // segmentation: at least one segment, never more than the chunks, contiguous cover
+    CHECK(kda::seg_count(0, 4) == 1 && kda::seg_count(1, 4) == 1 && kda::seg_count(3, 4) == 3);
+    CHECK(kda::seg_count(100, 4) == 4 && kda::seg_count(100, 1) == 1);
+    for (int chunks = 1; chunks < 300; ++chunks)
+        for (int segs = 1; segs < 12; ++segs) {
+            const int G = kda::seg_count(chunks, segs);
+            CHECK(kda::seg_chunk_begin(chunks, G, 0) == 0 && kda::seg_chunk_begin(chunks, G, G) == chunks);
+            for (int g = 0; g < G; ++g) {
+                const int len = kda::seg_chunk_begin(chunks, G, g + 1) - kda::seg_chunk_begin(chunks, G, g);
+                CHECK(len >= 1 && len <= (chunks + G - 1) / G);
+            }
+        }
+    // totals over a ragged pack: 2500 (40 chunks, 3 segments), 1, 0, 700 (11 chunks), 129 (3)
+    const int cu[6] = {0, 2500, 2501, 2501, 3201, 3330};
+    const kda::SegTotals t = kda::seg_totals(cu, 5, 3);
+    CHECK(t.num_vseqs == 3 + 1 + 1 + 3 + 3);
+    CHECK(t.e_chunks == (40 - 13) + (11 - 3) + (3 - 1));
+    CHECK(t.max_chunks == 14);
     std::printf("ok\n");
     return 0;
 }

@@ -19,6 +19,8 @@ BUDGET = [
     ("kda_chunk.cu", "chunk_kernelILi128ELb0E", 255),
     ("kda_chunk.cu", "chunk_kernelILi64ELb0E", 255),
     ("kda_chunk.cu", "chunk_kernelILi128ELb1E", 255),
+    ("kda_context.cu", "seg_fixup_kernel", 255),
+    ("kda_context.cu", "seg_scan_kernel", 255),
     ("kda_decode.cu", "decode_kernelI13__nv_bfloat16Li128ELi128E", 64),
     ("kda_decode.cu", "spec_kernelI13__nv_bfloat16Li128ELi128ELb0ELb1E", 72),
     ("kda_decode.cu", "spec_kernelI13__nv_bfloat16Li128ELi128ELb1ELb0E", 72),
