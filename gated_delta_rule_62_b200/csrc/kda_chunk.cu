@@ -56,7 +56,7 @@ struct Smem {
     static constexpr uint32_t LT = LA + 32768;              // L -> T fp32 [64][LT_LD]
     static constexpr uint32_t PB = LT + 64 * LT_LD * 4;     // 32 x PB_LD fp32
     static constexpr uint32_t MISC = PB + 32 * PB_LD * 4;   // beta, gamma, psum, flags, barriers
-    static constexpr uint32_t MISC_BYTES = 64 * 4 + 128 * 4 + 8 * 128 * 4 + 64 + 64;
+    static constexpr uint32_t MISC_BYTES = 64 * 4 + 128 * 4 + 9 * 128 * 4 + 64 + 64;
     static constexpr uint32_t BYTES = MISC + MISC_BYTES + 1024;  // + alignment slack
 };
 
@@ -108,8 +108,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float *s_beta = reinterpret_cast<float *>(sm + SM::MISC);  // [64]
     float *s_gamma = s_beta + 64;                               // [128]
-    float *s_psum = s_gamma + 128;                              // [8][128]
-    uint32_t *s_flags = reinterpret_cast<uint32_t *>(s_psum + 1024);  // abort, exact path, tmem
+    float *s_psum = s_gamma + 128;                              // [8 + 1][128]
+    uint32_t *s_flags = reinterpret_cast<uint32_t *>(s_psum + 9 * 128);  // abort, exact path, tmem
     uint64_t *bars = reinterpret_cast<uint64_t *>(s_flags + 16);     // qk, la, v, mma
     uint64_t *bar_qk = bars, *bar_la = bars + 1, *bar_v = bars + 2, *bar_mma = bars + 3;
     float *LA = reinterpret_cast<float *>(sm + SM::LA);
@@ -289,7 +289,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         tc_fence_after();
 
         // ---- A (D1 rows 0..63) to bf16, L (rows 64..127, times beta_i, j < i) to fp32
-        if (!safe) extract_al(tmem + lane_base + TM::D1 + 32 * half, sm + SM::AQK, LT, s_beta, c_me, half);
+        if (!safe) extract_al(tmem + lane_base + TM::D1 + 32 * half, sm + SM::AQK, LT, s_beta, c_me, 32 * half);
         tc_fence_before();
         __syncthreads();
         if (s_flags[0]) break;
@@ -530,19 +530,6 @@ bool make_token_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, ui
     return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE,
               swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-
-bool make_rows_map(CUtensorMap *m, void *base, uint64_t rows, uint32_t box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {256, rows};
-    cuuint64_t strides[1] = {512};
-    cuuint32_t box[2] = {256, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

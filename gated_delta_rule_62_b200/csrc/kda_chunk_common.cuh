@@ -19,10 +19,12 @@ constexpr int D = 128;   // d_k = d_v
 constexpr int NT = 256;  // compute threads per CTA
 constexpr float kFastLimit = 60.f;  // max in-chunk decay exponent for the factored path
 
-// Barrier over the NT compute threads (warps 0 .. NT/32 - 1) only: hardware barrier 1, so a
+// Barrier over the NTC compute threads (warps 0 .. NTC/32 - 1) only: hardware barrier 1, so a
 // CTA may run further warps (a control warp) that never join it.
-__device__ __forceinline__ void sync_compute() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
+template <int NTC = NT>
+__device__ __forceinline__ void sync_compute() { asm volatile("bar.sync 1, %0;" ::"n"(NTC) : "memory"); }
 // The same barrier, returning whether any compute thread passed a non-zero `pred`.
+template <int NTC = NT>
 __device__ __forceinline__ int sync_compute_or(int pred) {
     uint32_t r;
     asm volatile(
@@ -31,7 +33,7 @@ __device__ __forceinline__ int sync_compute_or(int pred) {
         "bar.red.or.pred p, 1, %2, q;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)pred), "n"(NT)
+        : "r"((uint32_t)pred), "n"(NTC)
         : "memory");
     return (int)r;
 }
@@ -171,6 +173,7 @@ __device__ __forceinline__ void frag_to_tt(uint8_t *TT, int r0, int c0, const fl
 // C^-1]] at 16 and then at 32, on the tensor cores (tf32 mma.sync). LT keeps the fp32 blocks
 // later stages need. Called by the NT compute threads (synchronised among themselves with
 // sync_compute); ends with the TT stores issued (no barrier).
+template <int NTC = NT>
 static __device__ __forceinline__ void invert_unit_lower(float *LT, float *PB, uint8_t *TT, const float *beta,
                                                          int tid) {
     const int warp = tid >> 5, lane = tid & 31;
@@ -199,7 +202,7 @@ static __device__ __forceinline__ void invert_unit_lower(float *LT, float *PB, u
             st_bf(TT + telem(8192, b0 + i, b0 + lane), x[i] * bl);
         }
     }
-    sync_compute();
+    sync_compute<NTC>();
     if (warp < 2) {
         // warp 0: T10 = -T11 (L10 T00); warp 1: T32 = -T33 (L32 T22)
         const int r0 = warp ? 48 : 16, c0 = warp ? 32 : 0;
@@ -213,7 +216,7 @@ static __device__ __forceinline__ void invert_unit_lower(float *LT, float *PB, u
         warp_store16(LT + r0 * LT_LD + c0, LT_LD, acc2, -1.f);
         frag_to_tt(TT, r0, c0, acc2, -1.f, beta);
     }
-    sync_compute();
+    sync_compute<NTC>();
     // rows 32..63 x cols 0..31: P = L[32:64, 0:32] T[0:32, 0:32];  T[32:64, 0:32] = -T[32:64, 32:64] P
     const int rt = (warp >> 1) & 1, ct = warp & 1;
     if (warp < 4) {
@@ -221,7 +224,7 @@ static __device__ __forceinline__ void invert_unit_lower(float *LT, float *PB, u
         warp_mm16(acc, LT + (32 + 16 * rt) * LT_LD, LT_LD, LT + 16 * ct, LT_LD, 32);
         warp_store16(PB + (16 * rt) * PB_LD + 16 * ct, PB_LD, acc, 1.f);
     }
-    sync_compute();
+    sync_compute<NTC>();
     if (warp < 4) {
         float acc[2][4] = {};
         warp_mm16(acc, LT + (32 + 16 * rt) * LT_LD + 32, LT_LD, PB + 16 * ct, PB_LD, 32);
@@ -231,40 +234,55 @@ static __device__ __forceinline__ void invert_unit_lower(float *LT, float *PB, u
 
 
 // ---------------------------------------------------------------- gating of one chunk
-// The NT compute threads (synchronised among themselves with sync_compute). In: QK holds raw
-// q (rows 0..63) and k (rows 64..127) as a K-major tile with
-// 16 KB blocks, LA the chunk's raw log_alpha [t][c] fp32, s_beta the chunk's beta (0 past `valid`).
+// The NTC compute threads (synchronised among themselves with sync_compute<NTC>). In: QK holds
+// raw q (rows 0..63) and k (rows 64..127) as a K-major tile with 16 KB blocks, LA the chunk's raw
+// log_alpha [t][c] fp32, s_beta the chunk's beta (0 past `valid`).
 // Out: QK holds Q~ and K~ in place, KI holds K- (factored path) or K^ (exact path), s_gamma =
 // e^(g_{C-1}); the exact path also writes A into AQK and beta-scaled L into LT (zeros elsewhere).
-// Thread mapping: channels 4 lane .. 4 lane + 3, token octet = warp (tokens 8 warp .. 8 warp + 7);
-// s_psum holds [8][D] floats.
+// Thread mapping: channels 4 lane .. 4 lane + 3 of the TPG = C / (NTC / 32) tokens of group
+// `warp` (tokens TPG warp .. TPG warp + TPG - 1); s_psum holds [NTC / 32 + 1][D] floats (the
+// groups' totals, turned in place into exclusive prefixes by a scan, plus the chunk totals).
 // If KH is not null it also receives K^ = k e^(g_{C-1} - g) on both paths. If src_free is not
 // null, the writes to KI, KH and AQK first wait (bounded by timeout_ns) for that mbarrier's
 // phase with parity src_parity: another thread may still be reading those tiles.
-// Returns 1 for the exact path, 0 for the factored path, -1 if *s_abort was set or the wait
-// timed out (which sets *s_abort).
+// Returns 1 for the exact path, 0 for the factored path, -1 if the wait timed out (which sets
+// *s_abort). Every compute thread passes every barrier inside (the path is decided by a barrier
+// reduction, and a failed wait only sets a flag), so no thread is left waiting at one.
 // PRO: the prologue (raw q, k rows and raw gates, per pro.flags) is compiled in; without it the
 // function is the plain gating.
-template <bool PRO = false>
+// SCRATCH: only the exact path waits for src_free (it writes AQK and LT); the factored path
+// writes nothing but QK, KI (K-) and KH (K^), so KI and KH may be scratch regions outside the
+// previous image (KH may be LA itself: it is written after the last read of LA). On the exact
+// path KI is not written at all (its D1 is never issued).
+template <bool PRO = false, int NTC = NT, bool SCRATCH = false>
 __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK, float *LA,
                                           float *LT, const float *s_beta, float *s_gamma,
                                           float *s_psum, uint32_t *s_abort, int valid,
                                           int tid, uint8_t *KH = nullptr,
                                           uint64_t *src_free = nullptr, uint32_t src_parity = 0,
                                           uint64_t timeout_ns = 0, const Prologue pro = Prologue()) {
+    constexpr int G = NTC / 32, TPG = C / G;  // token groups (one per warp), tokens per group
+    static_assert(G * TPG == C && TPG >= 1 && TPG <= 8, "gating thread mapping");
     const int warp = tid >> 5, lane = tid & 31;
-    const int to = warp, c4 = 4 * lane;  // token octet 8 to .. 8 to + 7, channels c4 .. c4 + 3
+    const int to = warp, c4 = 4 * lane;  // group `to`: tokens TPG to .. + TPG - 1; channels c4 .. c4 + 3
+    const uint32_t cx = (uint32_t)(c4 & 63) >> 3;
+    // Byte offset of token row t, channels c4 .. c4 + 3, in a 128-byte-swizzled tile (64-column
+    // blocks `bs` bytes apart): telem(bs, t, c4) with the block term left to the caller.
+    auto row_off = [&](int t) {
+        return (uint32_t)(t >> 3) * 1024 + (uint32_t)(t & 7) * 128 + ((cx ^ (uint32_t)(t & 7)) << 4) +
+               (uint32_t)(c4 & 7) * 2;
+    };
     if (PRO && (pro.flags & KDA_PROLOGUE_QK_L2NORM)) {
-        // Raw q and k rows -> x / sqrt(x.x + eps), in place. A warp holds its 8 tokens' whole
-        // rows (lane: 4 channels), addressed as in the operand loop below.
-        const uint32_t cx = (uint32_t)(c4 & 63) >> 3;
-        uint8_t *const q0 = QK + (uint32_t)(c4 >> 6) * 16384 + (uint32_t)to * 1024 + (uint32_t)(c4 & 7) * 2;
+        // Raw q and k rows -> x / sqrt(x.x + eps), in place. A warp holds its tokens' whole rows
+        // (lane: 4 channels), addressed as in the operand loop below.
+        uint8_t *const q0 = QK + (uint32_t)(c4 >> 6) * 16384;
         auto widen = [](uint32_t u) { return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u)); };
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (8 * to + i >= valid) break;  // the same for the whole warp
-            const uint32_t off = (uint32_t)i * 128 + ((cx ^ (uint32_t)i) << 4);
-            uint2 *qp = reinterpret_cast<uint2 *>(q0 + off), *kp = reinterpret_cast<uint2 *>(q0 + 8192 + off);
+        for (int i = 0; i < TPG; ++i) {
+            const int t = TPG * to + i;
+            if (t >= valid) break;  // the same for the whole warp
+            uint2 *qp = reinterpret_cast<uint2 *>(q0 + row_off(t));
+            uint2 *kp = reinterpret_cast<uint2 *>(q0 + 8192 + row_off(t));
             const uint2 qu = *qp, ku = *kp;
             const float2 qa = widen(qu.x), qb = widen(qu.y), ka = widen(ku.x), kb = widen(ku.y);
             float sq = qa.x * qa.x + qa.y * qa.y + qb.x * qb.x + qb.y * qb.y;
@@ -279,12 +297,12 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
             *kp = make_uint2(pack2(ka.x * rk, ka.y * rk), pack2(kb.x * rk, kb.y * rk));
         }
     }
-    // ---- gates: log_alpha of 8 tokens x 4 channels into registers, octet totals
-    float4 la[8];
+    // ---- gates: log_alpha of TPG tokens x 4 channels into registers, group totals
+    float4 la[TPG];
     float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int t = 8 * to + i;
+    for (int i = 0; i < TPG; ++i) {
+        const int t = TPG * to + i;
         la[i] = (t < valid) ? *reinterpret_cast<const float4 *>(LA + t * D + c4)
                             : make_float4(0.f, 0.f, 0.f, 0.f);
         if (PRO && (pro.flags & KDA_PROLOGUE_GATE_SOFTPLUS) && t < valid) {
@@ -298,56 +316,54 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
         tot.w += la[i].w;
     }
     *reinterpret_cast<float4 *>(s_psum + to * D + c4) = tot;
-    // An octet decaying by more than e^(kFastLimit/8) in some channel sends the chunk down the
+    // A group decaying by more than e^(kFastLimit/G) in some channel sends the chunk down the
     // exact path; otherwise the whole chunk decays by at most e^kFastLimit.
     // (NaN gates also take the exact path: the comparisons are false for NaN.)
-    const float lim = 0.125f * kFastLimit;
+    const float lim = kFastLimit / (float)G;
     const int unsafe = !(-tot.x <= lim) || !(-tot.y <= lim) || !(-tot.z <= lim) || !(-tot.w <= lim);
-    const bool safe = sync_compute_or(unsafe) != 0;
-    if (*s_abort) return -1;
-    if (src_free && !mbar_wait_bounded(src_free, src_parity, timeout_ns)) {
-        *s_abort = 1;
-        return -1;
-    }
-    float4 goff = make_float4(0.f, 0.f, 0.f, 0.f), gC = goff;
+    const bool safe = sync_compute_or<NTC>(unsafe) != 0;
+    bool failed = false;
+    // Per channel, the groups' totals -> exclusive prefixes (in place) and the chunk total (row
+    // G), by one thread per channel: each thread then reads two values instead of all G rows.
+    if (tid < D) {
+        float run = 0.f;
 #pragma unroll
-    for (int o = 0; o < 8; ++o) {
-        const float4 a = *reinterpret_cast<const float4 *>(s_psum + o * D + c4);
-        if (o < to) {
-            goff.x += a.x;
-            goff.y += a.y;
-            goff.z += a.z;
-            goff.w += a.w;
+        for (int o = 0; o < G; ++o) {
+            const float a = s_psum[o * D + tid];
+            s_psum[o * D + tid] = run;
+            run += a;
         }
-        gC.x += a.x;
-        gC.y += a.y;
-        gC.z += a.z;
-        gC.w += a.w;
+        s_psum[G * D + tid] = run;
+        s_gamma[tid] = __expf(run);
     }
-    if (to == 0)
-        *reinterpret_cast<float4 *>(s_gamma + c4) =
-            make_float4(__expf(gC.x), __expf(gC.y), __expf(gC.z), __expf(gC.w));
+    if (src_free && (!SCRATCH || safe) && !mbar_wait_bounded(src_free, src_parity, timeout_ns)) {
+        *s_abort = 1;
+        failed = true;  // the writes below go on (shared memory only); the caller stops
+    }
+    sync_compute<NTC>();
+    const float4 goff = *reinterpret_cast<const float4 *>(s_psum + to * D + c4);
+    const float4 gC = *reinterpret_cast<const float4 *>(s_psum + G * D + c4);
 
     if (safe) {
         // Exact path: A and L pairwise from raw q, k and the full g (no factored exponentials).
         {
             float4 g = goff;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < TPG; ++i) {
                 g.x += la[i].x;
                 g.y += la[i].y;
                 g.z += la[i].z;
                 g.w += la[i].w;
-                *reinterpret_cast<float4 *>(LA + (8 * to + i) * D + c4) = g;
+                *reinterpret_cast<float4 *>(LA + (TPG * to + i) * D + c4) = g;
             }
         }
-        for (int e = tid; e < 64 * 64; e += NT) {
+        for (int e = tid; e < 64 * 64; e += NTC) {
             const int i = e >> 6, j = e & 63;
             st_bf(AQK + telem(8192, i, j), 0.f);
             LT[i * LT_LD + j] = 0.f;
         }
-        sync_compute();
-        for (int e = warp; e < 64 * 64; e += NT / 32) {
+        sync_compute<NTC>();
+        for (int e = warp; e < 64 * 64; e += NTC / 32) {
             const int i = e >> 6, j = e & 63;
             if (j > i || i >= valid) continue;
             float a = 0.f, l = 0.f;
@@ -369,17 +385,17 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
                 if (j < i) LT[i * LT_LD + j] = s_beta[i] * l;
             }
         }
-        sync_compute();  // raw q, k are read above and overwritten below
+        sync_compute<NTC>();  // raw q, k are read above and overwritten below
     }
 
     // ---- gated operands. With alpha = e^log_alpha, prefix products P_i and suffix
-    // products R_i (within the octet): e^g_i = e^goff P_i; e^-g_i = e^(-goff-tot) R_i;
+    // products R_i (within the group): e^g_i = e^goff P_i; e^-g_i = e^(-goff-tot) R_i;
     // e^(g_C - g_i) = e^(g_C-goff-tot) R_i. Q~, K~ overwrite q, k in place; the KI tile
     // gets K- (fast path) or K^ (exact path).
     {
-        float4 al[8];
+        float4 al[TPG];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < TPG; ++i)
             al[i] = make_float4(__expf(la[i].x), __expf(la[i].y), __expf(la[i].z), __expf(la[i].w));
         const float4 eA = make_float4(__expf(goff.x), __expf(goff.y), __expf(goff.z), __expf(goff.w));
         const float4 eH = make_float4(__expf(gC.x - goff.x - tot.x), __expf(gC.y - goff.y - tot.y),
@@ -387,24 +403,21 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
         const float4 eB = safe ? eH
                                : make_float4(__expf(-goff.x - tot.x), __expf(-goff.y - tot.y),
                                              __expf(-goff.z - tot.z), __expf(-goff.w - tot.w));
-        float4 R[8];
+        float4 R[TPG];
         float4 run = make_float4(1.f, 1.f, 1.f, 1.f);
 #pragma unroll
-        for (int i = 7; i >= 0; --i) {
+        for (int i = TPG - 1; i >= 0; --i) {
             R[i] = run;
             run.x *= al[i].x;
             run.y *= al[i].y;
             run.z *= al[i].z;
             run.w *= al[i].w;
         }
-        // Token t = 8 to + i: t >> 3 = to and t & 7 = i (known at compile time), so
-        // telem(bs, t, c4) = base_bs + to 1024 + i 128 + ((cx ^ i) << 4) + (c4 & 7) 2; K~ rows
-        // (64 + t) sit 8 row groups further. Four channels = one 8-byte access.
-        const uint32_t cx = (uint32_t)(c4 & 63) >> 3;
-        const uint32_t row0 = (uint32_t)to * 1024 + (uint32_t)(c4 & 7) * 2;
-        uint8_t *const q0 = QK + (uint32_t)(c4 >> 6) * 16384 + row0;
-        uint8_t *const i0 = KI + (uint32_t)(c4 >> 6) * 8192 + row0;
-        uint8_t *const h0 = KH ? KH + (uint32_t)(c4 >> 6) * 8192 + row0 : nullptr;
+        // K~ rows (64 + t) sit 8 row groups (8 KB) after the Q~ rows. Four channels = one 8-byte
+        // access.
+        uint8_t *const q0 = QK + (uint32_t)(c4 >> 6) * 16384;
+        uint8_t *const i0 = KI + (uint32_t)(c4 >> 6) * 8192;
+        uint8_t *const h0 = KH ? KH + (uint32_t)(c4 >> 6) * 8192 : nullptr;
         auto unpack4 = [](uint2 u) {
             const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
             const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
@@ -413,50 +426,58 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
         auto pack4 = [](float a, float b, float c, float d) { return make_uint2(pack2(a, b), pack2(c, d)); };
         float4 P = eA;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int t = 8 * to + i;
+        for (int i = 0; i < TPG; ++i) {
+            const int t = TPG * to + i;
             P.x *= al[i].x;
             P.y *= al[i].y;
             P.z *= al[i].z;
             P.w *= al[i].w;
-            const uint32_t off = (uint32_t)i * 128 + ((cx ^ (uint32_t)i) << 4);
+            const uint32_t off = row_off(t);
             uint2 *qp = reinterpret_cast<uint2 *>(q0 + off);
             uint2 *kp = reinterpret_cast<uint2 *>(q0 + 8192 + off);
             float4 qv = unpack4(*qp), kv = unpack4(*kp);
             if (t >= valid) qv = kv = make_float4(0.f, 0.f, 0.f, 0.f);
             *qp = pack4(qv.x * P.x, qv.y * P.y, qv.z * P.z, qv.w * P.w);
             *kp = pack4(kv.x * P.x, kv.y * P.y, kv.z * P.z, kv.w * P.w);
-            *reinterpret_cast<uint2 *>(i0 + off) =
-                pack4(kv.x * (eB.x * R[i].x), kv.y * (eB.y * R[i].y), kv.z * (eB.z * R[i].z), kv.w * (eB.w * R[i].w));
+            if (!SCRATCH || !safe)
+                *reinterpret_cast<uint2 *>(i0 + off) =
+                    pack4(kv.x * (eB.x * R[i].x), kv.y * (eB.y * R[i].y), kv.z * (eB.z * R[i].z), kv.w * (eB.w * R[i].w));
             if (KH)
                 *reinterpret_cast<uint2 *>(h0 + off) =
                     pack4(kv.x * (eH.x * R[i].x), kv.y * (eH.y * R[i].y), kv.z * (eH.z * R[i].z), kv.w * (eH.w * R[i].w));
         }
     }
-    return safe ? 1 : 0;
+    return failed ? -1 : (safe ? 1 : 0);
 }
 
 // ---------------------------------------------------------------- TMEM epilogues
 // D1 (M=128: rows 0..63 = Q~ K-^T, rows 64..127 = K~ K-^T) -> A (bf16, j <= i) into AQK and
-// L (fp32, times beta_i, j < i) into LT. Thread: TMEM lane r, columns [32 half, 32 half + 32).
+// L (fp32, times beta_i, j < i) into LT. Thread: TMEM lane r, NC columns from col0 (taddr points
+// at column col0 of D1).
+template <int NC = 32>
 __device__ __forceinline__ void extract_al(uint32_t taddr, uint8_t *AQK, float *LT,
-                                           const float *s_beta, int r, int half) {
-    float v[32];
-    tmem_ld32(taddr, v);
+                                           const float *s_beta, int r, int col0) {
+    static_assert(NC == 16 || NC == 32, "extract_al columns");
+    float v[NC];
+    if constexpr (NC == 32) {
+        tmem_ld32(taddr, v);
+    } else {
+        tmem_ld16(taddr, v);
+    }
     tmem_wait_ld();
     if (r < 64) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = (32 * half + e <= r) ? v[e] : 0.f;
+        for (int e = 0; e < NC; ++e) v[e] = (col0 + e <= r) ? v[e] : 0.f;
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8)
-            st_chunk(AQK + tchunk(8192, r, 32 * half + 8 * q8), v + 8 * q8);
+        for (int q8 = 0; q8 < NC / 8; ++q8)
+            st_chunk(AQK + tchunk(8192, r, col0 + 8 * q8), v + 8 * q8);
     } else {
         const int i = r - 64;
         const float b = s_beta[i];
-        float4 *dst = reinterpret_cast<float4 *>(LT + i * LT_LD + 32 * half);
+        float4 *dst = reinterpret_cast<float4 *>(LT + i * LT_LD + col0);
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-            const int j = 32 * half + 4 * e4;
+        for (int e4 = 0; e4 < NC / 4; ++e4) {
+            const int j = col0 + 4 * e4;
             dst[e4] = make_float4(j + 0 < i ? b * v[4 * e4 + 0] : 0.f,
                                   j + 1 < i ? b * v[4 * e4 + 1] : 0.f,
                                   j + 2 < i ? b * v[4 * e4 + 2] : 0.f,
@@ -510,8 +531,5 @@ __device__ __forceinline__ void scale_tmem_row(uint32_t taddr, float gm) {
 // 3-D TMA map over [T][H][inner] with a box of (box_inner, 1, 64 tokens); false on failure.
 bool make_token_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint32_t esize,
                     uint64_t inner, uint64_t H, uint64_t T, uint32_t box_inner, bool swizzle);
-// 2-D TMA map over `rows` 512-byte rows (256 bf16 each, copied verbatim: no swizzle) with a box of
-// box_rows rows; false on failure.
-bool make_rows_map(CUtensorMap *m, void *base, uint64_t rows, uint32_t box_rows);
 
 }  // namespace kda

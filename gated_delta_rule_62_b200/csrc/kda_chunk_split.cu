@@ -49,10 +49,10 @@ constexpr int RING = 8;
 constexpr uint32_t SL_M = 0, SL_KH = 32768, SL_U = 49152, SL_P = 65536, SL_A = 81920;
 constexpr uint32_t SLOT = 90112;
 static_assert(SLOT % 1024 == 0, "slot layout");
-// The ring moves with tiled TMA over a [rows][256] bf16 view (512-byte rows copied verbatim):
-// an image is SLOT_ROWS rows, loaded as one box and stored in 8 KB pieces of RS_BOX rows.
-constexpr uint32_t ROW_BYTES = 512, SLOT_ROWS = SLOT / ROW_BYTES, RL_BOX = SLOT_ROWS, RS_BOX = 8192 / ROW_BYTES;
-static_assert(SLOT % ROW_BYTES == 0 && RL_BOX <= 256, "ring load box");
+// The ring moves with plain (1-D) bulk copies: a consumer loads a whole image in one copy, a
+// producer stores it in six, one per contiguous piece of its shared memory. (One SM moves about
+// 75 bytes per cycle from L2 into shared memory this way, and about 30 the other way; the 2-D
+// tensor copies of 512-byte rows used before loaded at about a third of that.)
 
 struct SplitParams {
     const int32_t *cu_seqlens;
@@ -74,24 +74,57 @@ struct SplitParams {
     float *seg_state;    // [segments, H, D, D] each chain's end state (sequences of several segments)
     float *seg_trans;    // [segments, H, D, D] transition product of segments after the first
     uint8_t *e_tiles;    // [E chunks, H] E = P R tiles
+    int32_t *e_live;     // [segments, H] chunks of a later segment whose E tile is live
     DebugRanges dbg;     // buffer ranges (checked by debug builds only)
 };
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// global -> shared, completing on `bar` (complete_tx); both addresses 16-byte aligned, bytes % 16 == 0
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+// shared -> global, tracked by the issuing thread's bulk async-group
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
+                 "r"(bytes)
+                 : "memory");
+}
 // Waits until the committed TMA stores have finished reading shared memory / are complete.
 __device__ __forceinline__ void bulk_wait_read() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Every split CTA runs the NT compute threads (warps 0..7) plus two control warps: lane 0 of
-// warp 8 issues the tensor-core MMAs (and, in a producer, the TMA loads and stores and the
-// hand-off flags); lane 0 of warp 9 brings a consumer its chunk images. None of their waits
-// stalls a compute warp. (Ten warps leave at most three per SM sub-partition, so they cost no
-// more registers per thread than nine.)
-constexpr int NTS = NT + 64;
-constexpr int CTL = NT;       // the MMA / control thread
-constexpr int LDR = NT + 32;  // the consumer's loader thread
+// Every split CTA runs NTC compute threads (warps 0..15) plus two control warps: lane 0 of
+// warp 16 issues the tensor-core MMAs (and, in a producer, the TMA loads); lane 0 of warp 17
+// brings a consumer its chunk images, or takes a producer's finished images to the ring (slot
+// wait, stores, hand-off flag). None of their waits stalls a compute warp. Sixteen compute warps (four per SM sub-partition) halve each phase's
+// per-thread work against eight: the per-chunk work is latency-bound, not issue-bound.
+constexpr int NTC = 2 * NT;    // compute threads: 16 warps
+constexpr int NTS = NTC + 64;
+constexpr int CTL = NTC;       // the MMA / control thread
+constexpr int LDR = NTC + 32;  // the consumer's loader thread
+constexpr int STR = NTC + 32;  // the producer's store thread
+// Barrier of a producer's compute threads and its control warp (warps 0 .. 16), which leaves out
+// the store thread's warp: its waits on the ring never hold up the others.
+constexpr int NWORK = NTC + 32;
+__device__ __forceinline__ void sync_work() { asm volatile("bar.sync 2, %0;" ::"n"(NWORK) : "memory"); }
+__device__ __forceinline__ int sync_work_or(int pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, 2, %2, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "n"(NWORK)
+        : "memory");
+    return (int)r;
+}
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -124,7 +157,7 @@ constexpr uint32_t TM_S = 0, TM_SB0 = 128, TM_SB1 = 192, TM_O0 = 256, TM_O1 = 38
 // critical path). Output warps 4..7: after o[b], the outputs ("o free"). No CTA-wide barrier inside
 // the loop. S_b^T(c) in TMEM copy c & 1 is rewritten only after the chain of chunk c + 1 has
 // completed, and so has O(c), issued before it by the same thread.
-__device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t *sm, int hd) {
+__device__ void consumer(const SplitParams &p, uint8_t *sm, int hd) {
     using namespace cons;
     constexpr uint32_t I_C = idesc_bf16_f32(128, 128, false, 0, 0);   // S_b^T M^T (A in TMEM)
     constexpr uint32_t I_K = idesc_bf16_f32(128, 128, false, 1, 1);   // U~^T K^
@@ -151,7 +184,7 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
 
     if (tid == 0) {
         s_flags[0] = 0;
-        for (int k = 0; k < 11; ++k) mbar_init(&bars[k], (k >= 6 && k <= 9) ? NT / 2 : 1);
+        for (int k = 0; k < 11; ++k) mbar_init(&bars[k], (k >= 6 && k <= 9) ? NTC / 2 : 1);
         fence_mbarrier_init();
     }
     if (warp == 0) {
@@ -184,12 +217,9 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
                 ph_o[b] ^= 1u;
                 st_release(p.consumed + hd, c - 1);
             }
-            const int32_t row0 = (int32_t)(((uint32_t)hd * RING + (uint32_t)(c % RING)) * SLOT_ROWS);
-            uint8_t *dst = sm + (b ? STAGE1 : STAGE0);
+            const uint8_t *src = p.ring + ((size_t)hd * RING + (size_t)(c % RING)) * SLOT;
             mbar_arrive_expect_tx(&bars[b], SLOT);
-#pragma unroll
-            for (uint32_t k = 0; k < SLOT_ROWS / RL_BOX; ++k)
-                tma_load_2d(dst + k * RL_BOX * ROW_BYTES, tm_rl, &bars[b], 0, row0 + (int32_t)(k * RL_BOX));
+            bulk_load(sm + (b ? STAGE1 : STAGE0), src, SLOT, &bars[b]);
             requested = c + 1;
         }
         // the last images land before the CTA exits (the MMA thread may have stopped early)
@@ -236,44 +266,43 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
         // teardown: every issued MMA completes before TMEM is freed
         mma_commit(&bars[10]);
         mbar_wait_bounded(&bars[10], 0, p.timeout_ns);
-    } else if (warp < 4) {
+    } else if (warp < 8) {
         // ------------------------------------------------ state warps (lane = value channel d)
         // per chunk: the new state -> its bf16 copy in TMEM (the next chain's and the output's A
-        // operand)
-        const int d_me = tid;  // 0..127
+        // operand). Warps w and w + 4 share lanes 32 (w % 4) .. + 31: columns [64 hh, 64 hh + 64).
+        const int d_me = 32 * quad + lane;
+        const int hh = warp >> 2;
         auto wait_bar = [&](uint64_t *bar, uint32_t &ph) -> bool {
             const bool ok = mbar_wait_bounded(bar, ph, p.timeout_ns);
             ph ^= 1u;
             if (!ok) fail();
             return ok;
         };
-        uint32_t w[2][32];  // this thread's row of S_b^T, bf16 pairs (c, c + 1)
-        // S^T row d, columns [64 h, 64 h + 64) in v -> packed w[h] -> TMEM copy at tm_sb
-        auto pack_store = [&](const float (&v)[2][32], int hh, uint32_t tm_sb) {
+        // 32 fp32 columns (state columns 64 hh + 32 part ..) -> 16 bf16 pairs of the copy at tm_sb
+        auto pack_store = [&](const float (&v)[32], int part, uint32_t tm_sb) {
+            uint32_t w[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) w[hh][e] = pack2(v[e >> 4][2 * (e & 15)], v[e >> 4][2 * (e & 15) + 1]);
-            float f[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(w[hh][e]);
-            tmem_st32(tmem + lane_base + tm_sb + 32 * hh, f);
+            for (int e = 0; e < 16; ++e) w[e] = pack2(v[2 * e], v[2 * e + 1]);
+            tmem_st16(tmem + lane_base + tm_sb + 32 * hh + 16 * part, w);
         };
         // initial state S[c][d] -> S^T in TMEM and its bf16 copy; empty sequences copy it out
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            float v[2][32];
+        {
             const float *src = s0b ? s0b + (size_t)(64 * hh) * D + d_me : nullptr;
 #pragma unroll
-            for (int e = 0; e < 64; ++e) v[e >> 5][e & 31] = src ? src[(size_t)e * D] : 0.f;
-            if (nchunks == 0) {
-                if (sTb) {
-                    float *dst = sTb + (size_t)(64 * hh) * D + d_me;
+            for (int part = 0; part < 2; ++part) {
+                float v[32];
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) dst[(size_t)e * D] = v[e >> 5][e & 31];
+                for (int e = 0; e < 32; ++e) v[e] = src ? src[(size_t)(32 * part + e) * D] : 0.f;
+                if (nchunks == 0) {
+                    if (sTb) {
+                        float *dst = sTb + (size_t)(64 * hh + 32 * part) * D + d_me;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) dst[(size_t)e * D] = v[e];
+                    }
+                } else {
+                    tmem_st32(tmem + lane_base + TM_S + 64 * hh + 32 * part, v);
+                    pack_store(v, part, TM_SB0);
                 }
-            } else {
-                tmem_st32(tmem + lane_base + TM_S + 64 * hh, v[0]);
-                tmem_st32(tmem + lane_base + TM_S + 64 * hh + 32, v[1]);
-                pack_store(v, hh, TM_SB0);
             }
         }
         if (nchunks > 0) {
@@ -288,32 +317,30 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
             if (ld_volatile(&s_flags[0])) break;
             if (!wait_bar(&bars[2], ph_s)) break;
             tc_fence_after();
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float v[2][32];
-                tmem_ld32(tmem + lane_base + TM_S + 64 * hh, v[0]);
-                tmem_ld32(tmem + lane_base + TM_S + 64 * hh + 32, v[1]);
-                tmem_wait_ld();
-                if (!last) {
-                    pack_store(v, hh, b ? TM_SB0 : TM_SB1);  // the next chunk's copy
-                } else if (sTb) {
-                    float *dst = sTb + (size_t)(64 * hh) * D + d_me;
-#pragma unroll
-                    for (int e = 0; e < 64; ++e) dst[(size_t)e * D] = v[e >> 5][e & 31];
-                }
-            }
+            float v[2][32];
+            tmem_ld32(tmem + lane_base + TM_S + 64 * hh, v[0]);
+            tmem_ld32(tmem + lane_base + TM_S + 64 * hh + 32, v[1]);
+            tmem_wait_ld();
             if (!last) {
+                pack_store(v[0], 0, b ? TM_SB0 : TM_SB1);  // the next chunk's copy
+                pack_store(v[1], 1, b ? TM_SB0 : TM_SB1);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&bars[6]);
+            } else if (sTb) {
+                float *dst = sTb + (size_t)(64 * hh) * D + d_me;
+#pragma unroll
+                for (int e = 0; e < 64; ++e) dst[(size_t)e * D] = v[e >> 5][e & 31];
             }
         }
         tc_fence_before();
-    } else if (tid < NT) {
+    } else if (tid < NTC) {
         // ------------------------------------------------ output warps
-        // O^T of chunk c (lane = value channel d, column = token) -> bf16 outputs; for each token a
-        // warp stores 32 consecutive channels (64 bytes)
+        // O^T of chunk c (lane = value channel d, column = token) -> bf16 outputs; warps w and
+        // w + 4 (w = 8..11) take tokens [32 th, 32 th + 32); for each token a warp stores 32
+        // consecutive channels (64 bytes)
         const int d_me = 32 * quad + lane;
+        const int th = (warp >> 2) & 1;
         uint32_t ph_o[2] = {0, 0};
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
@@ -322,20 +349,19 @@ __device__ void consumer(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t
             ph_o[b] ^= 1u;
             if (!ok) { fail(); break; }
             tc_fence_after();
-            const int64_t tc = bos + (int64_t)c * C;
-            const int vc = (int)(eos - tc < C ? eos - tc : C);
+            const int64_t tc = bos + (int64_t)c * C + 32 * th;
+            const int vc = (int)(eos - tc < 32 ? eos - tc : 32);
             const uint32_t tm_o = b ? TM_O1 : TM_O0;
-            float vv[2][32];  // tokens 0..31, 32..63 of channel d_me
-            tmem_ld32(tmem + lane_base + tm_o, vv[0]);
-            tmem_ld32(tmem + lane_base + tm_o + 32, vv[1]);
+            float vv[32];  // tokens 32 th .. 32 th + 31 of channel d_me
+            tmem_ld32(tmem + lane_base + tm_o + 32 * th, vv);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&bars[8 + b]);  // read: this accumulator may take chunk c + 2
             __nv_bfloat16 *dst = p.out + ((size_t)tc * H + h) * D + d_me;
 #pragma unroll
-            for (int t = 0; t < C; ++t)
+            for (int t = 0; t < 32; ++t)
                 if (t < vc && KDA_ACCESS_OK(p.status, p.dbg.out, dst + (size_t)t * H * D, 2, 3))
-                    dst[(size_t)t * H * D] = __float2bfloat16_rn(vv[t >> 5][t & 31]);
+                    dst[(size_t)t * H * D] = __float2bfloat16_rn(vv[t]);
         }
         tc_fence_before();
     }
@@ -360,8 +386,7 @@ namespace segc {
 constexpr uint32_t TM_S = 0, TM_SB = 128, TM_R = 192, TM_RB = 320, TM_O = 384, TM_E = 448, TM_COLS = 512;
 }  // namespace segc
 
-__device__ void consumer_seg(const CUtensorMap *tm_rl, const SplitParams &p, uint8_t *sm, int hd,
-                             int4 vi) {
+__device__ void consumer_seg(const SplitParams &p, uint8_t *sm, int hd, int4 vi) {
     using namespace cons;
     using segc::TM_S; using segc::TM_SB; using segc::TM_R; using segc::TM_RB;
     using segc::TM_O; using segc::TM_E; using segc::TM_COLS;
@@ -371,7 +396,8 @@ __device__ void consumer_seg(const CUtensorMap *tm_rl, const SplitParams &p, uin
     constexpr uint32_t I_OA = idesc_bf16_f32(128, 64, false, 1, 0);   // U~^T A^T
     // full0, full1, o0, o1, ready (bf16 copies written), free (O and E read), teardown
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + MISC);
-    uint32_t *s_flags = reinterpret_cast<uint32_t *>(sm + MISC + 96);  // abort, tmem
+    // abort, tmem, first chunk whose R chain and E are not computed (R has decayed away)
+    uint32_t *s_flags = reinterpret_cast<uint32_t *>(sm + MISC + 96);
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3;
@@ -379,6 +405,7 @@ __device__ void consumer_seg(const CUtensorMap *tm_rl, const SplitParams &p, uin
     const int H = p.H, v = hd / H, h = hd % H;
     const int64_t bos = p.cu_seqlens[v], eos = p.cu_seqlens[v + 1];
     const int nchunks = (int)((eos - bos + C - 1) / C);
+    auto r_live = [&](int c) { return c < (int)ld_volatile(&s_flags[2]); };
     float *s_end = p.seg_state + (size_t)hd * D * D;
     float *r_end = p.seg_trans + (size_t)hd * D * D;
     const bool ends_ok = KDA_ACCESS_OK(p.status, p.dbg.ws, s_end, D * D * 4, 4) &&
@@ -386,7 +413,8 @@ __device__ void consumer_seg(const CUtensorMap *tm_rl, const SplitParams &p, uin
 
     if (tid == 0) {
         s_flags[0] = 0;
-        for (int k = 0; k < 7; ++k) mbar_init(&bars[k], (k == 4 || k == 5) ? NT / 2 : 1);
+        s_flags[2] = 0x7fffffffu;
+        for (int k = 0; k < 7; ++k) mbar_init(&bars[k], (k == 4 || k == 5) ? NTC / 2 : 1);
         fence_mbarrier_init();
     }
     if (warp == 0) {
@@ -416,12 +444,9 @@ __device__ void consumer_seg(const CUtensorMap *tm_rl, const SplitParams &p, uin
                 ph_o[b] ^= 1u;
                 st_release(p.consumed + hd, c - 1);
             }
-            const int32_t row0 = (int32_t)(((uint32_t)hd * RING + (uint32_t)(c % RING)) * SLOT_ROWS);
-            uint8_t *dst = sm + (b ? STAGE1 : STAGE0);
+            const uint8_t *src = p.ring + ((size_t)hd * RING + (size_t)(c % RING)) * SLOT;
             mbar_arrive_expect_tx(&bars[b], SLOT);
-#pragma unroll
-            for (uint32_t k = 0; k < SLOT_ROWS / RL_BOX; ++k)
-                tma_load_2d(dst + k * RL_BOX * ROW_BYTES, tm_rl, &bars[b], 0, row0 + (int32_t)(k * RL_BOX));
+            bulk_load(sm + (b ? STAGE1 : STAGE0), src, SLOT, &bars[b]);
             requested = c + 1;
         }
         for (int c = requested - 2 < 0 ? 0 : requested - 2; c < requested; ++c)
@@ -448,9 +473,12 @@ __device__ void consumer_seg(const CUtensorMap *tm_rl, const SplitParams &p, uin
 #pragma unroll
             for (uint32_t kk = 0; kk < 4; ++kk)  // ... + U~^T K^
                 mma_bf16_ss(tmem + TM_S, desc_mn_at(dU, kk), desc_mn_at(dK, kk), I_K, 1);
+            const bool live = r_live(c);  // read after `ready`: the state warps set it before arriving
+            if (live) {
 #pragma unroll
-            for (uint32_t kk = 0; kk < 8; ++kk)  // R^T += R_b^T M^T
-                mma_bf16_ts(tmem + TM_R, tmem + TM_RB + 8 * kk, desc_k_at(dM, 16384, kk), I_C, 1);
+                for (uint32_t kk = 0; kk < 8; ++kk)  // R^T += R_b^T M^T
+                    mma_bf16_ts(tmem + TM_R, tmem + TM_RB + 8 * kk, desc_k_at(dM, 16384, kk), I_C, 1);
+            }
             if (c >= 1) {  // the output warps have read O and E of chunk c - 1
                 if (!mbar_wait_bounded(&bars[5], ph_free, p.timeout_ns)) { fail(); break; }
                 ph_free ^= 1u;
@@ -462,53 +490,45 @@ __device__ void consumer_seg(const CUtensorMap *tm_rl, const SplitParams &p, uin
 #pragma unroll
             for (uint32_t kk = 0; kk < 4; ++kk)  // ... + U~^T A^T
                 mma_bf16_ss(tmem + TM_O, desc_mn_at(dU, kk), desc_k_at(dA, 8192, kk), I_OA, 1);
+            if (live) {
 #pragma unroll
-            for (uint32_t kk = 0; kk < 8; ++kk)  // E^T = R_b^T P^T
-                mma_bf16_ts(tmem + TM_E, tmem + TM_RB + 8 * kk, desc_k_at(dP, 8192, kk), I_OP, kk > 0);
+                for (uint32_t kk = 0; kk < 8; ++kk)  // E^T = R_b^T P^T
+                    mma_bf16_ts(tmem + TM_E, tmem + TM_RB + 8 * kk, desc_k_at(dP, 8192, kk), I_OP, kk > 0);
+            }
             mma_commit(&bars[2 + b]);  // both chains, O, E and the stage are done
         }
         mma_commit(&bars[6]);
         mbar_wait_bounded(&bars[6], 0, p.timeout_ns);
-    } else if (warp < 4) {
+    } else if (warp < 8) {
         // ------------------------------------------------ state warps (lane = value channel d for
-        // S0^T, = column a of R for R^T); after chunk c's outputs: the bf16 copies for chunk c + 1
-        const int d_me = tid;  // 0..127
-        auto pack_store = [&](const float (&x)[2][32], uint32_t tm_b, int hh) {
-            float f[32];
+        // S0^T, = column a of R for R^T; warps w and w + 4 take columns [64 hh, 64 hh + 64)); after
+        // chunk c's outputs: the bf16 copies for chunk c + 1
+        const int d_me = 32 * quad + lane;
+        const int hh = warp >> 2;
+        auto pack_store = [&](const float (&x)[32], uint32_t tm_b, int part) {
+            uint32_t w[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-                f[e] = __uint_as_float(pack2(x[e >> 4][2 * (e & 15)], x[e >> 4][2 * (e & 15) + 1]));
-            tmem_st32(tmem + lane_base + tm_b + 32 * hh, f);
+            for (int e = 0; e < 16; ++e) w[e] = pack2(x[2 * e], x[2 * e + 1]);
+            tmem_st16(tmem + lane_base + tm_b + 32 * hh + 16 * part, w);
         };
-        // S0^T = 0, R^T = I and their bf16 copies, 32 columns at a time
+        // S0^T = 0, R^T = I and their bf16 copies
+#pragma unroll 1
         for (int which = 0; which < 2; ++which) {
             const uint32_t tm_x = which ? TM_R : TM_S, tm_b = which ? TM_RB : TM_SB;
-            for (int part = 0; part < 4; ++part) {
+#pragma unroll 1
+            for (int part = 0; part < 2; ++part) {
                 float x[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = (which && 32 * part + e == d_me) ? 1.f : 0.f;
-                tmem_st32(tmem + lane_base + tm_x + 32 * part, x);
-                float f[32];  // columns 32 part .. + 31 as 16 bf16 pairs: half a 32-column copy store
-#pragma unroll
-                for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(pack2(x[2 * e], x[2 * e + 1]));
-                uint32_t w[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(f[e]);
-                // bf16 copy column (32 part + 2e) / 2 = 16 part + e
-                asm volatile(
-                    "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-                    "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-                        tmem + lane_base + tm_b + 16 * part),
-                    "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]),
-                    "r"(w[7]), "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]),
-                    "r"(w[14]), "r"(w[15])
-                    : "memory");
+                for (int e = 0; e < 32; ++e) x[e] = (which && 64 * hh + 32 * part + e == d_me) ? 1.f : 0.f;
+                tmem_st32(tmem + lane_base + tm_x + 64 * hh + 32 * part, x);
+                pack_store(x, tm_b, part);
             }
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars[4]);
         uint32_t ph_o[2] = {0, 0};
+        int dead_from = 0x7fffffff;  // the state warps' copy of s_flags[2]
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
             const bool last = c + 1 == nchunks;
@@ -517,24 +537,45 @@ __device__ void consumer_seg(const CUtensorMap *tm_rl, const SplitParams &p, uin
             ph_o[b] ^= 1u;
             if (!ok) { fail(); break; }
             tc_fence_after();
-#pragma unroll
+            uint32_t rmax = 0;  // max |R| over this thread's columns (as float bits)
+#pragma unroll 1
             for (int which = 0; which < 2; ++which) {
+                if (which && !last && c + 1 > dead_from) continue;  // R decayed away: no copy needed
                 const uint32_t tm_x = which ? TM_R : TM_S, tm_b = which ? TM_RB : TM_SB;
                 float *dst_end = which ? r_end : s_end;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float x[2][32];
-                    tmem_ld32(tmem + lane_base + tm_x + 64 * hh, x[0]);
-                    tmem_ld32(tmem + lane_base + tm_x + 64 * hh + 32, x[1]);
+#pragma unroll 1
+                for (int part = 0; part < 2; ++part) {
+                    float x[32];
+                    tmem_ld32(tmem + lane_base + tm_x + 64 * hh + 32 * part, x);
                     tmem_wait_ld();
-                    if (!last) {
-                        pack_store(x, tm_b, hh);
-                    } else if (ends_ok) {
-                        // row d_me of S0^T (or column d_me of R) -> element [c][d_me], c = 64 hh + e
-                        float *dst = dst_end + (size_t)(64 * hh) * D + d_me;
+                    if (which) {
 #pragma unroll
-                        for (int e = 0; e < 64; ++e) dst[(size_t)e * D] = x[e >> 5][e & 31];
+                        for (int e = 0; e < 32; ++e) rmax = max(rmax, __float_as_uint(fabsf(x[e])));
                     }
+                    if (!last) {
+                        pack_store(x, tm_b, part);
+                    } else if (ends_ok) {
+                        // row d_me of S0^T (or column d_me of R) -> element [c][d_me]
+                        float *dst = dst_end + (size_t)(64 * hh + 32 * part) * D + d_me;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) dst[(size_t)e * D] = x[e];
+                    }
+                }
+            }
+            if (!last && dead_from == 0x7fffffff) {
+                // has R decayed away? (all 256 state threads: named barrier 3 with an OR)
+                uint32_t any_alive;
+                asm volatile(
+                    "{\n\t.reg .pred p, q;\n\t"
+                    "setp.ge.f32 q, %1, %2;\n\t"
+                    "bar.red.or.pred p, 3, 256, q;\n\t"
+                    "selp.u32 %0, 1, 0, p;\n\t}"
+                    : "=r"(any_alive)
+                    : "f"(__uint_as_float(rmax)), "f"(kSegDeadR)
+                    : "memory");
+                if (!any_alive) {
+                    dead_from = c + 1;
+                    if (tid == 0) s_flags[2] = (uint32_t)dead_from;  // seen by the MMA thread after `ready`
                 }
             }
             if (!last) {
@@ -543,10 +584,14 @@ __device__ void consumer_seg(const CUtensorMap *tm_rl, const SplitParams &p, uin
                 mbar_arrive(&bars[4]);
             }
         }
+        if (tid == 0 && !ld_volatile(&s_flags[0]))
+            p.e_live[hd] = dead_from < nchunks ? dead_from : nchunks;
         tc_fence_before();
-    } else if (tid < NT) {
-        // ------------------------------------------------ output warps: O0 -> out, E^T -> its tile
+    } else if (tid < NTC) {
+        // ------------------------------------------------ output warps: O0 -> out, E^T -> its tile;
+        // warps w and w + 4 (w = 8..11) take tokens [32 th, 32 th + 32)
         const int d_me = 32 * quad + lane;  // value channel of O0^T, row a of E^T
+        const int th = (warp >> 2) & 1;
         uint32_t ph_o[2] = {0, 0};
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
@@ -555,35 +600,34 @@ __device__ void consumer_seg(const CUtensorMap *tm_rl, const SplitParams &p, uin
             ph_o[b] ^= 1u;
             if (!ok) { fail(); break; }
             tc_fence_after();
-            const int64_t tc = bos + (int64_t)c * C;
-            const int vc = (int)(eos - tc < C ? eos - tc : C);
-            // E^T first (row a = d_me, 64 tokens, as a 128-byte swizzled row of a [128][64] bf16
-            // tile), then O0: one accumulator's registers live at a time
+            const int64_t tc = bos + (int64_t)c * C + 32 * th;
+            const int vc = (int)(eos - tc < 32 ? eos - tc : 32);
+            // E^T row a = d_me, tokens 32 th .. + 31: four 16-byte chunks of a 128-byte swizzled
+            // row of the [128][64] bf16 tile
             uint8_t *et = p.e_tiles + ((size_t)(vi.w + c) * H + h) * 16384 + (uint32_t)(d_me >> 3) * 1024 +
                           (uint32_t)(d_me & 7) * 128;
             const bool et_ok = KDA_ACCESS_OK(p.status, p.dbg.ws, et, 128, 6);
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                float ee[32];
-                tmem_ld32(tmem + lane_base + TM_E + 32 * part, ee);
+            float x[32];
+            // E of a chunk after R decayed away was not computed (a late view of the flag only
+            // writes a tile the fix-up never reads: it stops at the segment's live count)
+            if (r_live(c)) {
+                tmem_ld32(tmem + lane_base + TM_E + 32 * th, x);
                 tmem_wait_ld();
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
-                    const uint32_t q8 = 4 * part + q4;
-                    if (et_ok) st_chunk(et + ((q8 ^ (uint32_t)(d_me & 7)) << 4), ee + 8 * q4);
+                    const uint32_t q8 = 4 * th + q4;
+                    if (et_ok) st_chunk(et + ((q8 ^ (uint32_t)(d_me & 7)) << 4), x + 8 * q4);
                 }
             }
-            float oo[2][32];
-            tmem_ld32(tmem + lane_base + TM_O, oo[0]);
-            tmem_ld32(tmem + lane_base + TM_O + 32, oo[1]);
+            tmem_ld32(tmem + lane_base + TM_O + 32 * th, x);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&bars[5]);  // read: O and E may take chunk c + 1
             __nv_bfloat16 *dst = p.out + ((size_t)tc * H + h) * D + d_me;
 #pragma unroll
-            for (int t = 0; t < C; ++t)
+            for (int t = 0; t < 32; ++t)
                 if (t < vc && KDA_ACCESS_OK(p.status, p.dbg.out, dst + (size_t)t * H * D, 2, 7))
-                    dst[(size_t)t * H * D] = __float2bfloat16_rn(oo[t >> 5][t & 31]);
+                    dst[(size_t)t * H * D] = __float2bfloat16_rn(x[t]);
         }
         tc_fence_before();
     }
@@ -608,7 +652,8 @@ constexpr uint32_t AQK = ZB + 8192;       // A [i][j]    /
 constexpr uint32_t LT = AQK + 8192;       // L -> T fp32 [64][LT_LD]
 constexpr uint32_t PB = LT + 64 * LT_LD * 4;   // 32 x PB_LD fp32
 constexpr uint32_t MISC = PB + 32 * PB_LD * 4; // beta, gamma, psum, flags, barriers
-constexpr uint32_t BYTES = MISC + 64 * 4 + 128 * 4 + 8 * 128 * 4 + 64 + 64;
+constexpr uint32_t PSUM_FLOATS = (NTC / 32 + 1) * 128;  // group totals per compute warp, chunk totals
+constexpr uint32_t BYTES = MISC + 64 * 4 + 128 * 4 + PSUM_FLOATS * 4 + 64 + 64 + 4 * 32;
 // TMEM: D1 = [Q~; K~] K-^T (M=128, 64 columns), W (M=64), D3 = [U~; -A W], D4 = -K^^T W
 constexpr uint32_t TM_D1 = 0, TM_W = 128, TM_D3 = 256, TM_D4 = 384, TM_COLS = 512;
 }  // namespace prod
@@ -618,8 +663,7 @@ constexpr uint32_t TM_D1 = 0, TM_W = 128, TM_D3 = 256, TM_D4 = 384, TM_COLS = 51
 // ring slot and publishes the image. The phases of one item are separated by CTA barriers.
 template <bool PRO>
 __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
-                         const CUtensorMap *tm_la, const CUtensorMap *tm_rs, const SplitParams &p,
-                         uint8_t *sm, int pid, int nprod) {
+                         const CUtensorMap *tm_la, const SplitParams &p, uint8_t *sm, int pid, int nprod) {
     using namespace prod;
     constexpr uint32_t I_D1 = idesc_bf16_f32(128, 64);
     constexpr uint32_t I_W = idesc_bf16_f32(64, 128, false, 0, 1);
@@ -628,15 +672,17 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     float *s_beta = reinterpret_cast<float *>(sm + MISC);
     float *s_gamma = s_beta + 64;
     float *s_psum = s_gamma + 128;
-    uint32_t *s_flags = reinterpret_cast<uint32_t *>(s_psum + 1024);  // abort, tmem, gate
-    uint64_t *bars = reinterpret_cast<uint64_t *>(s_flags + 16);     // qk0, qk1, la, v, mma, src
+    uint32_t *s_flags = reinterpret_cast<uint32_t *>(s_psum + PSUM_FLOATS);  // abort, tmem, gate
+    // qk0, qk1, la, v, mma, src (the image's sources may be rewritten), img (an image is ready)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(s_flags + 16);
     float *LTp = reinterpret_cast<float *>(sm + LT);
     float *PBp = reinterpret_cast<float *>(sm + PB);
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = (warp >> 2) & 1;
+    // TMEM epilogues: warp w reads lanes 32 (w % 4) .. + 31, column part w / 4 of four
+    const int quad = warp & 3, part = warp >> 2;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
-    const bool compute = tid < NT, ctl = tid == CTL;
+    const bool compute = tid < NTC, ctl = tid == CTL;
     const int H = p.H;
     // Dynamic assignment: items k = chunk * heads + head are claimed from one counter in that
     // (chunk-major) order, so every head advances at the producers' common rate. A producer's
@@ -667,17 +713,38 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             if ((int64_t)c * C < len) return k;
         }
     };
-    int *s_items = reinterpret_cast<int *>(s_flags + 4);  // first two items; then the one after next
+    // Item n's record, rec[n % 4]: {head, chunk, head within the sequence, first token, valid
+    // tokens} (head < 0: no item n). The control thread decodes each item it claims once; nothing
+    // else reads cu_seqlens, so no thread stalls on a global load for it. Record n + 2 is written
+    // during item n's inverse and read from item n + 1 on (behind the barrier that ends the inverse).
+    struct ItemRec {
+        int hd, c, h, t0, valid, pad[3];
+    };
+    ItemRec *s_rec = reinterpret_cast<ItemRec *>(bars + 8);
+    auto put_rec = [&](int n, int k) {  // control thread
+        ItemRec r;
+        r.hd = -1;
+        if (k >= 0) {
+            const Item it = decode(k);
+            r.hd = it.hd;
+            r.c = it.c;
+            r.h = it.h;
+            const int64_t t0 = it.bos + (int64_t)it.c * C;
+            r.t0 = (int)t0;
+            r.valid = (int)(it.eos - t0 < C ? it.eos - t0 : C);
+        }
+        s_rec[n & 3] = r;
+    };
 
     if (tid == 0) {
         s_flags[0] = 0;
-        for (int k = 0; k < 6; ++k) mbar_init(&bars[k], 1);
+        s_flags[7] = 0xffffffffu;  // *s_nimg = -1: items still running
+        for (int k = 0; k < 7; ++k) mbar_init(&bars[k], 1);
         fence_mbarrier_init();
         prefetch_tmap(tm_q);
         prefetch_tmap(tm_k);
         prefetch_tmap(tm_v);
         prefetch_tmap(tm_la);
-        prefetch_tmap(tm_rs);
     }
     if (warp == 0) {
         tmem_alloc(&s_flags[1], TM_COLS);
@@ -696,10 +763,8 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 
     // control thread; each buffer's previous contents were read by generic loads or bulk stores
     // that have completed (see the call sites)
-    auto issue_qk = [&](int k, int b) {
-        const Item it = decode(k);
-        const int h = it.h;
-        const int64_t t0 = it.bos + (int64_t)it.c * C;
+    auto issue_qk = [&](const ItemRec &r, int b) {
+        const int h = r.h, t0 = r.t0;
         uint8_t *qk = sm + (b ? QK1 : QK0);
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&bars[b], 32768);
@@ -708,46 +773,34 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         tma_load_3d(qk + 16384, tm_q, &bars[b], 64, h, (int32_t)t0);
         tma_load_3d(qk + 24576, tm_k, &bars[b], 64, h, (int32_t)t0);
     };
-    auto issue_la = [&](int k) {
-        const Item it = decode(k);
-        const int h = it.h;
-        const int64_t t0 = it.bos + (int64_t)it.c * C;
+    auto issue_la = [&](const ItemRec &r) {
+        const int h = r.h, t0 = r.t0;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&bars[2], 32768);
         tma_load_3d(sm + LA, tm_la, &bars[2], 0, h, (int32_t)t0);
     };
-    auto issue_v = [&](int k) {
-        const Item it = decode(k);
-        const int h = it.h;
-        const int64_t t0 = it.bos + (int64_t)it.c * C;
+    auto issue_v = [&](const ItemRec &r) {
+        const int h = r.h, t0 = r.t0;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&bars[3], 16384);
         tma_load_3d(sm + VB, tm_v, &bars[3], 0, h, (int32_t)t0);
         tma_load_3d(sm + VB + 8192, tm_v, &bars[3], 64, h, (int32_t)t0);
     };
-    auto load_beta = [&](int k) -> float {  // tid < C
-        if (k < 0) return 0.f;
-        const Item it = decode(k);
-        const int64_t t0 = it.bos + (int64_t)it.c * C;
-        if (t0 + tid >= it.eos) return 0.f;
-        const float *bp = p.beta + (size_t)(t0 + tid) * H + it.h;
+    auto load_beta = [&](const ItemRec &r) -> float {  // tid < C
+        if (r.hd < 0 || tid >= r.valid) return 0.f;
+        const float *bp = p.beta + (size_t)(r.t0 + tid) * H + r.h;
         if (!KDA_ACCESS_OK(p.status, p.dbg.beta, bp, 4, 8)) return 0.f;
         const float b = *bp;
         return (PRO && (p.pro.flags & KDA_PROLOGUE_BETA_SIGMOID)) ? beta_from_raw(b) : b;
     };
-    // the previous image, published once its bulk stores are complete (control thread, during
-    // the next item's gating)
-    int32_t *rel_flag = nullptr;
-    int rel_val = 0;
-    auto release = [&]() {
-        if (rel_flag) {
-            bulk_wait_all();
-            fence_proxy_async_global();
-            __threadfence();
-            st_release(rel_flag, rel_val);
-            rel_flag = nullptr;
-        }
-    };
+    // Hand-off of image n to the store thread: entry n % 2 = {head, chunk, QK buffer}, then an
+    // arrival on the img barrier. Entry n % 2 is rewritten only for image n + 2, after the store
+    // thread has released image n + 1's sources, which it does only after reading entry n; for
+    // the same reason the img barrier is never more than one phase ahead of the store thread.
+    // The end of the items is not an arrival (that could complete a second phase before the store
+    // thread has waited for the last image) but a count, *s_nimg = images handed over in all.
+    volatile int32_t *s_store = reinterpret_cast<volatile int32_t *>(s_flags + 8);
+    volatile int32_t *s_nimg = reinterpret_cast<volatile int32_t *>(s_flags + 7);
 
     uint32_t ph_qk[2] = {0, 0}, ph_la = 0, ph_v = 0, ph_mma = 0, ph_src = 0;
     bool pend_qk[2] = {false, false}, pend_la = false, pend_v = false;
@@ -758,45 +811,96 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     };
 
     if (ctl) {
-        s_items[0] = claim();
-        s_items[1] = s_items[0] >= 0 ? claim() : -1;
-        if (s_items[0] >= 0) {
-            issue_qk(s_items[0], 0);
-            issue_la(s_items[0]);
+        const int k0 = claim();
+        put_rec(0, k0);
+        put_rec(1, k0 >= 0 ? claim() : -1);
+        if (k0 >= 0) {
+            issue_qk(s_rec[0], 0);
+            issue_la(s_rec[0]);
         }
     }
     __syncthreads();
-    int item = s_items[0], nxt = s_items[1];
-    if (item >= 0) pend_qk[0] = pend_la = true;
-    float beta_next = (tid < C) ? load_beta(item) : 0.f;
-    int b = 0;
-    while (item >= 0) {
-        const Item it = decode(item);
-        const int hd = it.hd, c = it.c;
-        const int64_t t0 = it.bos + (int64_t)c * C;
-        const int valid = (int)(it.eos - t0 < C ? it.eos - t0 : C);
+    if (warp == STR / 32) {
+        if (tid == STR) {
+            // ------------------------------------------------ store thread
+            // Per image, in item order: wait until the compute threads have written it (img), wait
+            // for its ring slot's previous chunk to have been taken, store it (six bulk copies),
+            // let the sources be rewritten once the copies have read them (src), and publish it
+            // once they are complete.
+            mbar_arrive(&bars[5]);  // the first item's gating may write the image's sources
+            uint32_t ph_img = 0;
+            for (int n = 0;; ++n) {
+                // image n handed over, or the item loop ended with n images handed over
+                bool have = false, ended = false;
+                const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
+                while (true) {
+                    if (mbar_try_wait(&bars[6], ph_img)) { have = true; break; }
+                    const int ni = *s_nimg;
+                    if (ni >= 0 && ni <= n) { ended = true; break; }
+                    if (globaltimer_ns() > deadline) break;
+                    __nanosleep(64);
+                }
+                if (!have) {
+                    if (!ended) fail();
+                    break;
+                }
+                ph_img ^= 1u;
+                volatile int32_t *e = s_store + 4 * (n & 1);
+                const int hd = e[0], c = e[1];
+                if (c >= RING && !wait_flag_ge(p.consumed + hd, c - RING + 1, p.timeout_ns)) {
+                    fail();
+                    mbar_arrive(&bars[5]);  // nothing was stored; let the compute threads see the stop
+                    break;
+                }
+                uint8_t *slot = p.ring + ((size_t)hd * RING + (size_t)(c % RING)) * SLOT;
+                const uint32_t b_img = (uint32_t)e[2];
+                const uint8_t *qkb = sm + (b_img ? QK1 : QK0);
+                bulk_store(slot + SL_M, sm + KI, 32768);       // M: K- and -W regions, contiguous
+                bulk_store(slot + SL_KH, sm + KH, 16384);
+                bulk_store(slot + SL_U, sm + VB, 16384);
+                bulk_store(slot + SL_P, qkb, 8192);             // P, columns 0..63 (over Q~)
+                bulk_store(slot + SL_P + 8192, qkb + 16384, 8192);  // and 64..127
+                bulk_store(slot + SL_A, sm + AQK, 8192);
+                bulk_commit();
+                bulk_wait_read();
+                mbar_arrive(&bars[5]);  // the sources may be rewritten
+                bulk_wait_all();
+                fence_proxy_async_global();
+                __threadfence();
+                st_release(p.filled + hd * RING + (c % RING), c + 1);
+            }
+            bulk_wait_all();
+        }
+    } else {
+    if (s_rec[0].hd >= 0) pend_qk[0] = pend_la = true;
+    float beta_next = (tid < C) ? load_beta(s_rec[0]) : 0.f;
+    int b = 0, n_img = 0;
+    for (int n = 0; s_rec[n & 3].hd >= 0; ++n) {
+        const ItemRec cur = s_rec[n & 3], nx = s_rec[(n + 1) & 3];
+        const int hd = cur.hd, c = cur.c, valid = cur.valid;
         uint8_t *qk = sm + (b ? QK1 : QK0);
         if (tid < C) s_beta[tid] = beta_next;
-        if (ctl) {  // the previous image's sources (K-, K^, A, ...) are rewritten by the gating
-            bulk_wait_read();
-            mbar_arrive(&bars[5]);
-        }
         wait_bar(&bars[b], ph_qk[b]);
         wait_bar(&bars[2], ph_la);
         pend_qk[b] = pend_la = false;
 
-        if (tid < C) beta_next = load_beta(nxt);
-        if (ctl) release();  // the previous item's image, while the compute threads gate
+        if (tid < C) beta_next = load_beta(nx);
+        // K- goes to the L/T scratch (free until the A/L extraction, which follows D1) and K^ to the
+        // log_alpha buffer (free once the gating has read it; the next chunk's log_alpha is loaded
+        // after K^ has been copied to its image slot). So the factored gating writes nothing the
+        // previous image's stores may still be reading, and its wait for them (src) moves after D1.
+        const uint32_t src_par = ph_src;
         if (compute) {
-            const int gate = gate_chunk<PRO>(qk, sm + KI, sm + AQK, reinterpret_cast<float *>(sm + LA), LTp,
-                                        s_beta, s_gamma, s_psum, s_flags, valid, tid, sm + KH,
-                                        &bars[5], ph_src, p.timeout_ns, p.pro);
+            const int gate = gate_chunk<PRO, NTC, true>(qk, reinterpret_cast<uint8_t *>(LTp), sm + AQK,
+                                                        reinterpret_cast<float *>(sm + LA), LTp, s_beta,
+                                                        s_gamma, s_psum, s_flags, valid, tid, sm + LA, &bars[5],
+                                                        src_par, p.timeout_ns, p.pro);
             if (gate < 0) atomicOr(p.status, 1);
             if (tid == 0) s_flags[2] = (uint32_t)(gate + 1);
             fence_proxy_async_smem();
         }
         ph_src ^= 1u;
-        const bool stop = __syncthreads_or(ld_volatile(&s_flags[0]) != 0) != 0;
+        const bool stop = sync_work_or(ld_volatile(&s_flags[0]) != 0) != 0;
         const int gate = (int)s_flags[2] - 1;
         if (gate < 0 || stop) break;
         const bool safe = gate == 1;
@@ -806,36 +910,44 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 #pragma unroll
                 for (uint32_t kk = 0; kk < 8; ++kk)
                     mma_bf16_ss(tmem + TM_D1, desc_k(smem_u32(qk), 16384, kk),
-                                desc_k(sb + KI, 8192, kk), I_D1, kk > 0);
+                                desc_k(sb + LT, 8192, kk), I_D1, kk > 0);
             }
             mma_commit(&bars[4]);
-            // V of this chunk; q/k and log_alpha of the next one (the gating is done with them)
-            issue_v(item);
-            if (nxt >= 0) {
-                issue_qk(nxt, b ^ 1);
-                issue_la(nxt);
-            }
+            // once the previous image's stores have read their sources (V's buffer holds its U~,
+            // the other QK buffer its P): V of this chunk and q/k of the next one
+            if (!mbar_wait_bounded(&bars[5], src_par, p.timeout_ns)) fail();
+            issue_v(cur);
+            if (nx.hd >= 0) issue_qk(nx, b ^ 1);
         }
         pend_v = true;
-        if (nxt >= 0) pend_qk[b ^ 1] = pend_la = true;
+        if (nx.hd >= 0) pend_qk[b ^ 1] = true;
         wait_bar(&bars[4], ph_mma);
         tc_fence_after();
-        if (compute && !safe) extract_al(tmem + lane_base + TM_D1 + 32 * half, sm + AQK, LTp, s_beta, 32 * quad + lane, half);
+        if (compute) {
+            // A, and K^ for D4, go to image sources: the previous image's stores must have read them
+            if (!mbar_wait_bounded(&bars[5], src_par, p.timeout_ns)) fail();
+            for (int e = tid; e < 16384 / 16; e += NTC)  // K^: log_alpha buffer -> its image slot
+                reinterpret_cast<uint4 *>(sm + KH)[e] = reinterpret_cast<const uint4 *>(sm + LA)[e];
+            if (!safe)
+                extract_al<16>(tmem + lane_base + TM_D1 + 16 * part, sm + AQK, LTp, s_beta, 32 * quad + lane,
+                               16 * part);
+        }
         tc_fence_before();
         // L and A to the inverse: a barrier of the compute threads only (the control thread is
         // still issuing the prefetches); the CTA-wide stop check follows the inverse
-        if (compute) sync_compute();
+        if (compute) sync_compute<NTC>();
 
         // the item after the next one, claimed while the compute threads invert (the atomic's
         // latency stays off their path); read by all after the following barriers
-        if (ctl) s_items[2] = nxt >= 0 ? claim() : -1;
+        if (ctl) put_rec(n + 2, nx.hd >= 0 ? claim() : -1);
         if (compute) {
-            invert_unit_lower(LTp, PBp, sm + TT, s_beta, tid);
+            invert_unit_lower<NTC>(LTp, PBp, sm + TT, s_beta, tid);
             fence_proxy_async_smem();
         }
-        if (__syncthreads_or(ld_volatile(&s_flags[0]) != 0)) break;
+        if (sync_work_or(ld_volatile(&s_flags[0]) != 0)) break;
 
         if (ctl) {
+            if (nx.hd >= 0) issue_la(nx);  // K^ has left the log_alpha buffer (copied before the inverse)
             tc_fence_after();
 #pragma unroll
             for (uint32_t kk = 0; kk < 4; ++kk)  // W = T' K~
@@ -843,14 +955,15 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
                             desc_mn(smem_u32(qk) + 8192, 16384, kk), I_W, kk > 0);
             mma_commit(&bars[4]);
         }
+        if (nx.hd >= 0) pend_la = true;
         wait_bar(&bars[4], ph_mma);
         tc_fence_after();
         if (compute) {
-            rows64_to_tile<64>(tmem + lane_base + TM_W + 64 * half, sm + WN, 8192, 64 * half, quad, lane, -1.f);
+            rows64_to_tile<32>(tmem + lane_base + TM_W + 32 * part, sm + WN, 8192, 32 * part, quad, lane, -1.f);
             fence_proxy_async_smem();
         }
         tc_fence_before();
-        __syncthreads();
+        sync_work();
 
         // D3 = [T'; 0] V + [0; A] (-W) = [U~; -A W] and D4 = K^^T (-W)
         if (ctl) {
@@ -873,85 +986,58 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         tc_fence_after();
         if (compute) {
             const int r = 32 * quad + lane;  // TMEM lane
-            // D3 rows 0..63: U~ [j][d] over V; rows 64..127: P = Q~ - A W over Q~ (both 32-column
-            // loads in flight before one wait)
-            float vv[2][32];
-            tmem_ld32(tmem + lane_base + TM_D3 + 64 * half, vv[0]);
-            tmem_ld32(tmem + lane_base + TM_D3 + 64 * half + 32, vv[1]);
+            const int col = 32 * part;       // this thread's 32 columns of D3 and D4
+            // D3 rows 0..63: U~ [j][d] over V; rows 64..127: P = Q~ - A W over Q~; D4 -> M =
+            // diag(gamma - 1) - K^^T W [c][c'] over K- and -W (both loads in flight before one wait)
+            float v[32], m[32];
+            tmem_ld32(tmem + lane_base + TM_D3 + col, v);
+            tmem_ld32(tmem + lane_base + TM_D4 + col, m);
             tmem_wait_ld();
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int col = 64 * half + 32 * part;
-                float *v = vv[part];
-                if (r < 64) {
-#pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8)
-                        st_chunk(sm + VB + tchunk(8192, r, col + 8 * q8), v + 8 * q8);
-                } else {
-#pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8) {
-                        uint8_t *qp = qk + tchunk(16384, r - 64, col + 8 * q8);
-                        const uint4 raw = *reinterpret_cast<const uint4 *>(qp);
-                        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
-                            v[8 * q8 + 2 * e] += f.x;
-                            v[8 * q8 + 2 * e + 1] += f.y;
-                        }
-                        st_chunk(qp, v + 8 * q8);
-                    }
-                }
-            }
-            // D4 -> M = diag(gamma - 1) - K^^T W [c][c'] over K- and -W
-            const float gm1 = s_gamma[r] - 1.f;
-            tmem_ld32(tmem + lane_base + TM_D4 + 64 * half, vv[0]);
-            tmem_ld32(tmem + lane_base + TM_D4 + 64 * half + 32, vv[1]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int col = 64 * half + 32 * part;
-                float *v = vv[part];
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    if (col + e == r) v[e] += gm1;
+            if (r < 64) {
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8)
-                    st_chunk(sm + KI + tchunk(16384, r, col + 8 * q8), v + 8 * q8);
+                    st_chunk(sm + VB + tchunk(8192, r, col + 8 * q8), v + 8 * q8);
+            } else {
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    uint8_t *qp = qk + tchunk(16384, r - 64, col + 8 * q8);
+                    const uint4 raw = *reinterpret_cast<const uint4 *>(qp);
+                    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
+                        v[8 * q8 + 2 * e] += f.x;
+                        v[8 * q8 + 2 * e + 1] += f.y;
+                    }
+                    st_chunk(qp, v + 8 * q8);
+                }
             }
+            const float gm1 = s_gamma[r] - 1.f;
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                if (col + e == r) m[e] += gm1;
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8)
+                st_chunk(sm + KI + tchunk(16384, r, col + 8 * q8), m + 8 * q8);
             fence_proxy_async_smem();  // written by generic stores; the copy-out is async
         }
-        if (ctl && c >= RING) {  // the slot's previous chunk must have been taken
-            if (!wait_flag_ge(p.consumed + hd, c - RING + 1, p.timeout_ns)) fail();
-        }
         tc_fence_before();
-        if (__syncthreads_or(ld_volatile(&s_flags[0]) != 0)) break;
-
-        // copy the image out with bulk stores (layout at the top of this file); published at the
-        // next item (see release)
+        if (sync_work_or(ld_volatile(&s_flags[0]) != 0)) break;
+        // the image is in shared memory (written by generic stores, each followed by a proxy
+        // fence): hand it to the store thread
         if (ctl) {
-            const int32_t row0 = (int32_t)(((uint32_t)hd * RING + (uint32_t)(c % RING)) * SLOT_ROWS);
-            // 8 KB pieces (RS_BOX rows): source, image offset
-            const uint8_t *src[11] = {sm + KI, sm + KI + 8192, sm + KI + 16384, sm + KI + 24576,
-                                      sm + KH, sm + KH + 8192, sm + VB, sm + VB + 8192,
-                                      qk, qk + 16384,  // P, columns 0..63 and 64..127
-                                      sm + AQK};
-            const uint32_t off[11] = {SL_M, SL_M + 8192, SL_M + 16384, SL_M + 24576, SL_KH, SL_KH + 8192,
-                                      SL_U, SL_U + 8192, SL_P, SL_P + 8192, SL_A};
-#pragma unroll
-            for (int k = 0; k < 11; ++k) tma_store_2d(tm_rs, src[k], 0, row0 + (int32_t)(off[k] / ROW_BYTES));
-            bulk_commit();
-            rel_flag = p.filled + hd * RING + (c % RING);
-            rel_val = c + 1;
+            volatile int32_t *e = s_store + 4 * (n_img & 1);
+            e[0] = hd;
+            e[1] = c;
+            e[2] = b;
+            mbar_arrive(&bars[6]);
         }
-        item = nxt;
-        nxt = s_items[2];
+        ++n_img;
         b ^= 1;
     }
 
     if (ctl) {
-        if (!s_flags[0]) release();
-        bulk_wait_all();
+        *s_nimg = n_img;  // no more images: the store thread ends after image n_img - 1
         for (int k = 0; k < 2; ++k)
             if (pend_qk[k]) mbar_wait_bounded(&bars[k], ph_qk[k], p.timeout_ns);
         if (pend_la) mbar_wait_bounded(&bars[2], ph_la, p.timeout_ns);
@@ -959,6 +1045,7 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         mma_commit(&bars[4]);
         mbar_wait_bounded(&bars[4], ph_mma, p.timeout_ns);
     }
+    }  // the work warps
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -973,7 +1060,6 @@ template <bool PRO>
 __global__ void __launch_bounds__(NTS, 1)
 split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_la,
-             const __grid_constant__ CUtensorMap tm_rl, const __grid_constant__ CUtensorMap tm_rs,
              const SplitParams p) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned (128-byte swizzled tiles); offsetting the shared array itself keeps the
@@ -982,11 +1068,11 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     if ((int)blockIdx.x < p.heads) {
         const int4 vi = p.vinfo ? p.vinfo[blockIdx.x / p.H] : make_int4(0, 0, 1, 0);
         if (vi.y > 0)
-            consumer_seg(&tm_rl, p, sm, blockIdx.x, vi);
+            consumer_seg(p, sm, blockIdx.x, vi);
         else
-            consumer(&tm_rl, p, sm, blockIdx.x);
+            consumer(p, sm, blockIdx.x);
     } else
-        producer<PRO>(&tm_q, &tm_k, &tm_v, &tm_la, &tm_rs, p, sm, blockIdx.x - p.heads, gridDim.x - p.heads);
+        producer<PRO>(&tm_q, &tm_k, &tm_v, &tm_la, p, sm, blockIdx.x - p.heads, gridDim.x - p.heads);
 }
 
 // Zeroes the status word and the ring flags.
@@ -1037,7 +1123,7 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
         return cudaSuccess;
     }
 
-    CUtensorMap mq, mk, mv, mla, mrl, mrs;
+    CUtensorMap mq, mk, mv, mla;
     const uint64_t T = (uint64_t)p.total_tokens, H = (uint64_t)p.H;
     if (!make_token_map(&mq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, H, T, 64, true) ||
         !make_token_map(&mk, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, H, T, 64, true) ||
@@ -1046,10 +1132,7 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
         return cudaErrorInvalidValue;
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    uint8_t *ring = ws + 1024 + flags_bytes(heads);
-    const uint64_t ring_rows = (uint64_t)heads * RING * SLOT_ROWS;
-    if (!make_rows_map(&mrl, ring, ring_rows, RL_BOX) || !make_rows_map(&mrs, ring, ring_rows, RS_BOX))
-        return cudaErrorInvalidValue;
+    uint8_t *ring = ws + 1024 + flags_bytes(heads);  // 1024-byte aligned: slots are too (SLOT % 1024 == 0)
     int32_t *status = reinterpret_cast<int32_t *>(ws);
     int32_t *flags = reinterpret_cast<int32_t *>(ws + 1024);
     const int nflags = (int)(heads * (RING + 2));
@@ -1063,6 +1146,7 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
     sp.seg_state = p.seg ? p.seg->seg_state : nullptr;
     sp.seg_trans = p.seg ? p.seg->seg_trans : nullptr;
     sp.e_tiles = p.seg ? p.seg->e_tiles : nullptr;
+    sp.e_live = p.seg ? p.seg->e_live : nullptr;
     sp.dbg = p.dbg;
     sp.beta = p.beta;
     sp.pro = p.pro;
@@ -1080,7 +1164,7 @@ cudaError_t launch_prefill_split(const Problem &p, int32_t max_chunks, void *wor
     sp.heads = (int32_t)heads;
     sp.max_chunks = max_chunks;
     sp.timeout_ns = timeout_ns;
-    void *args[] = {&mq, &mk, &mv, &mla, &mrl, &mrs, &sp};
+    void *args[] = {&mq, &mk, &mv, &mla, &sp};
     return cudaLaunchCooperativeKernel(kern, dim3(grid), dim3(NTS), args,
                                        SPLIT_SMEM, stream);
 }

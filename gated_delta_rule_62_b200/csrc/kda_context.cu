@@ -142,6 +142,7 @@ struct FixParams {
     const int32_t *vcu;
     const int4 *vinfo;
     const uint8_t *s_start, *e_tiles;
+    const int32_t *e_live;
     __nv_bfloat16 *out;
     int32_t *status;
     int32_t H, num_vseqs, ranges;  // ranges: chunk ranges per (segment, head) in the grid
@@ -159,9 +160,11 @@ seg_fixup_kernel(const FixParams p) {
     if (v >= p.num_vseqs) return;
     const int4 vi = p.vinfo[v];
     const int64_t bos = p.vcu[v], eos = p.vcu[v + 1];
-    const int nchunks = (int)((eos - bos + C - 1) / C);
-    const int c0 = r * FIX_CHUNKS, c1 = min(nchunks, c0 + FIX_CHUNKS);
-    if (vi.y < 1 || c0 >= c1) return;  // the block's whole range is empty: nothing allocated yet
+    if (vi.y < 1) return;  // a first segment: its outputs are final
+    // chunks whose E tile is live (the segment's transition product had not decayed away)
+    const int live = min((int)((eos - bos + C - 1) / C), p.e_live[(size_t)v * H + h]);
+    const int c0 = r * FIX_CHUNKS, c1 = min(live, c0 + FIX_CHUNKS);
+    if (c0 >= c1) return;  // the block's whole range is empty: nothing allocated yet
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + FIX_MISC);  // a, e0, e1, mma
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + FIX_MISC + 64);
@@ -275,6 +278,7 @@ size_t seg_workspace_bytes(int32_t num_seqs, int32_t num_vseqs, int64_t e_chunks
     b += 2 * (size_t)num_vseqs * H * D * D * 4;              // end states, transition products
     b += (size_t)num_vseqs * H * kSegStartTileBytes;         // start-state tiles
     b += (size_t)e_chunks * H * kSegETileBytes;              // E tiles
+    b += round1k((size_t)num_vseqs * H * 4);                 // live E chunks per segment-head
     return b;
 }
 
@@ -293,6 +297,8 @@ void seg_carve(SegPlan &sp, void *base, int32_t num_seqs, int32_t num_vseqs, int
     sp.s_start = p;
     p += (size_t)num_vseqs * H * kSegStartTileBytes;
     sp.e_tiles = p;
+    p += (size_t)e_chunks * H * kSegETileBytes;
+    sp.e_live = reinterpret_cast<int32_t *>(p);
     sp.num_vseqs = num_vseqs;
     sp.e_chunks = (int32_t)e_chunks;
 }
@@ -321,6 +327,7 @@ cudaError_t launch_seg_scan_fixup(const Problem &p, const SegPlan &sp, int32_t *
     fp.vinfo = sp.vinfo;
     fp.s_start = sp.s_start;
     fp.e_tiles = sp.e_tiles;
+    fp.e_live = sp.e_live;
     fp.out = static_cast<__nv_bfloat16 *>(p.out);
     fp.status = status;
     fp.H = p.H;

@@ -145,9 +145,15 @@ struct SegPlan {
     float *seg_trans = nullptr;   // [N_v, H, d_k, d_k] fp32 transition product of segments g >= 1
     uint8_t *s_start = nullptr;   // [N_v, H] 32 KB bf16 tiles: true start state of segments g >= 1
     uint8_t *e_tiles = nullptr;   // [E chunks, H] 16 KB bf16 tiles
+    int32_t *e_live = nullptr;    // [N_v, H] chunks of a later segment whose E tile is live
     int32_t segments = 1, num_vseqs = 0, e_chunks = 0, max_chunks = 0;
 };
 constexpr uint32_t kSegStartTileBytes = 32768, kSegETileBytes = 16384;
+// A later segment's transition product R (max |entry|) below this has decayed past any effect on
+// the outputs: under the value contract (beta in [0, 1], unit keys) every chunk's transition is a
+// contraction, so R only shrinks further, and the rest of the segment's E = P R and its share of
+// the start state are below 128^2 * 2^-40 of the inputs' scale. Its chain and E tiles stop there.
+constexpr float kSegDeadR = 9.094947e-13f;  // 2^-40
 
 // ---- problem description passed from the API layer to the launchers --------------------
 struct Problem {

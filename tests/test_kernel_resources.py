@@ -1,7 +1,7 @@
 """Register and spill budget of the hot kernels, from ptxas's resource report (no GPU needed).
 
-Each bound is the occupancy the kernel is designed for: the split-role kernel's 10 warps fit at
-<= 168 registers; two 512-thread decode blocks per SM need <= 64; the speculative kernels' 128-thread
+Each bound is the occupancy the kernel is designed for: the split-role kernel's 18 warps (16
+compute, 2 control; up to five per SM sub-partition) fit at <= 96 registers; two 512-thread decode blocks per SM need <= 64; the speculative kernels' 128-thread
 blocks keep >= 7 per SM at <= 72. No hot kernel may spill."""
 import concurrent.futures as cf
 import os
@@ -14,8 +14,8 @@ from gated_delta_rule_62_b200 import build as B
 
 # (source, mangled-name fragment, max registers)
 BUDGET = [
-    ("kda_chunk_split.cu", "split_kernelILb0E", 168),
-    ("kda_chunk_split.cu", "split_kernelILb1E", 168),
+    ("kda_chunk_split.cu", "split_kernelILb0E", 96),
+    ("kda_chunk_split.cu", "split_kernelILb1E", 96),
     ("kda_chunk.cu", "chunk_kernelILi128ELb0E", 255),
     ("kda_chunk.cu", "chunk_kernelILi64ELb0E", 255),
     ("kda_chunk.cu", "chunk_kernelILi128ELb1E", 255),
