@@ -295,7 +295,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         if (s_flags[0]) break;
 
         // ---- T' = (I + L)^-1 diag(beta), bf16, into the TT tile
-        invert_unit_lower(LT, PB, sm + SM::TT, s_beta, tid);
+        invert_unit_lower(LT, PB, sm + SM::TT, s_beta, tid, tid >> 5);
         fence_proxy_async_smem();
         __syncthreads();
 

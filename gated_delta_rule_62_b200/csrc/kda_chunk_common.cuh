@@ -173,11 +173,13 @@ __device__ __forceinline__ void frag_to_tt(uint8_t *TT, int r0, int c0, const fl
 // C^-1]] at 16 and then at 32, on the tensor cores (tf32 mma.sync). LT keeps the fp32 blocks
 // later stages need. Called by the NT compute threads (synchronised among themselves with
 // sync_compute); ends with the TT stores issued (no barrier).
+// `warp` is the caller's logical warp index for the inverse: 0..3 do its work, any other value
+// (e.g. -1 for a warp that does other work meanwhile) only joins its barriers.
 template <int NTC = NT>
 static __device__ __forceinline__ void invert_unit_lower(float *LT, float *PB, uint8_t *TT, const float *beta,
-                                                         int tid) {
-    const int warp = tid >> 5, lane = tid & 31;
-    if (warp < 4 && lane < 16) {
+                                                         int tid, int warp) {
+    const int lane = tid & 31;
+    if (warp >= 0 && warp < 4 && lane < 16) {
         const int b0 = 16 * warp;
         const float *Lb = LT + b0 * LT_LD + b0;
         // all 120 sub-diagonal values first (independent loads), then a dependency chain of 15
@@ -203,7 +205,7 @@ static __device__ __forceinline__ void invert_unit_lower(float *LT, float *PB, u
         }
     }
     sync_compute<NTC>();
-    if (warp < 2) {
+    if (warp >= 0 && warp < 2) {
         // warp 0: T10 = -T11 (L10 T00); warp 1: T32 = -T33 (L32 T22)
         const int r0 = warp ? 48 : 16, c0 = warp ? 32 : 0;
         float *P = PB + warp * 16 * PB_LD;
@@ -219,13 +221,13 @@ static __device__ __forceinline__ void invert_unit_lower(float *LT, float *PB, u
     sync_compute<NTC>();
     // rows 32..63 x cols 0..31: P = L[32:64, 0:32] T[0:32, 0:32];  T[32:64, 0:32] = -T[32:64, 32:64] P
     const int rt = (warp >> 1) & 1, ct = warp & 1;
-    if (warp < 4) {
+    if (warp >= 0 && warp < 4) {
         float acc[2][4] = {};
         warp_mm16(acc, LT + (32 + 16 * rt) * LT_LD, LT_LD, LT + 16 * ct, LT_LD, 32);
         warp_store16(PB + (16 * rt) * PB_LD + 16 * ct, PB_LD, acc, 1.f);
     }
     sync_compute<NTC>();
-    if (warp < 4) {
+    if (warp >= 0 && warp < 4) {
         float acc[2][4] = {};
         warp_mm16(acc, LT + (32 + 16 * rt) * LT_LD + 32, LT_LD, PB + 16 * ct, PB_LD, 32);
         frag_to_tt(TT, 32 + 16 * rt, 16 * ct, acc, -1.f, beta);
@@ -398,11 +400,20 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
         for (int i = 0; i < TPG; ++i)
             al[i] = make_float4(__expf(la[i].x), __expf(la[i].y), __expf(la[i].z), __expf(la[i].w));
         const float4 eA = make_float4(__expf(goff.x), __expf(goff.y), __expf(goff.z), __expf(goff.w));
-        const float4 eH = make_float4(__expf(gC.x - goff.x - tot.x), __expf(gC.y - goff.y - tot.y),
-                                      __expf(gC.z - goff.z - tot.z), __expf(gC.w - goff.w - tot.w));
-        const float4 eB = safe ? eH
-                               : make_float4(__expf(-goff.x - tot.x), __expf(-goff.y - tot.y),
-                                             __expf(-goff.z - tot.z), __expf(-goff.w - tot.w));
+        // e^(g_C - goff - tot) and e^(-goff - tot): on the factored path the first is the second
+        // times gamma (the scan's e^(g_C)); the exact path needs only the first, which cannot
+        // overflow, and uses it for both.
+        float4 eH, eB;
+        if (safe) {
+            eH = make_float4(__expf(gC.x - goff.x - tot.x), __expf(gC.y - goff.y - tot.y),
+                             __expf(gC.z - goff.z - tot.z), __expf(gC.w - goff.w - tot.w));
+            eB = eH;
+        } else {
+            eB = make_float4(__expf(-goff.x - tot.x), __expf(-goff.y - tot.y), __expf(-goff.z - tot.z),
+                             __expf(-goff.w - tot.w));
+            const float4 gm = *reinterpret_cast<const float4 *>(s_gamma + c4);
+            eH = make_float4(eB.x * gm.x, eB.y * gm.y, eB.z * gm.z, eB.w * gm.w);
+        }
         float4 R[TPG];
         float4 run = make_float4(1.f, 1.f, 1.f, 1.f);
 #pragma unroll
@@ -439,12 +450,11 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
             if (t >= valid) qv = kv = make_float4(0.f, 0.f, 0.f, 0.f);
             *qp = pack4(qv.x * P.x, qv.y * P.y, qv.z * P.z, qv.w * P.w);
             *kp = pack4(kv.x * P.x, kv.y * P.y, kv.z * P.z, kv.w * P.w);
+            const float4 kr = make_float4(kv.x * R[i].x, kv.y * R[i].y, kv.z * R[i].z, kv.w * R[i].w);
             if (!SCRATCH || !safe)
-                *reinterpret_cast<uint2 *>(i0 + off) =
-                    pack4(kv.x * (eB.x * R[i].x), kv.y * (eB.y * R[i].y), kv.z * (eB.z * R[i].z), kv.w * (eB.w * R[i].w));
+                *reinterpret_cast<uint2 *>(i0 + off) = pack4(kr.x * eB.x, kr.y * eB.y, kr.z * eB.z, kr.w * eB.w);
             if (KH)
-                *reinterpret_cast<uint2 *>(h0 + off) =
-                    pack4(kv.x * (eH.x * R[i].x), kv.y * (eH.y * R[i].y), kv.z * (eH.z * R[i].z), kv.w * (eH.w * R[i].w));
+                *reinterpret_cast<uint2 *>(h0 + off) = pack4(kr.x * eH.x, kr.y * eH.y, kr.z * eH.z, kr.w * eH.w);
         }
     }
     return failed ? -1 : (safe ? 1 : 0);

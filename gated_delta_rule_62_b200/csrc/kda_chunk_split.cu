@@ -205,7 +205,6 @@ __device__ void consumer(const SplitParams &p, uint8_t *sm, int hd) {
         // Chunk c goes to stage c & 1 once the producer has published it (acquired ahead, so
         // the acquire's latency overlaps the wait) and chunk c - 2's MMAs have completed (o[b]);
         // that completion also means chunk c - 2's image had landed: its slot may be refilled.
-        uint32_t ph_o[2] = {0, 0};
         int requested = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
@@ -213,8 +212,8 @@ __device__ void consumer(const SplitParams &p, uint8_t *sm, int hd) {
             if (!wait_flag_ge(p.filled + hd * RING + (c % RING), c + 1, p.timeout_ns)) { fail(); break; }
             fence_proxy_async_global();
             if (c >= 2) {
-                if (!mbar_wait_bounded(&bars[4 + b], ph_o[b], p.timeout_ns)) { fail(); break; }
-                ph_o[b] ^= 1u;
+                // chunk c - 2 is use (c - 2) / 2 of o[b]: phase parity ((c - 2) >> 1) & 1
+                if (!mbar_wait_bounded(&bars[4 + b], (uint32_t)((c - 2) >> 1) & 1u, p.timeout_ns)) { fail(); break; }
                 st_release(p.consumed + hd, c - 1);
             }
             const uint8_t *src = p.ring + ((size_t)hd * RING + (size_t)(c % RING)) * SLOT;
@@ -228,12 +227,11 @@ __device__ void consumer(const SplitParams &p, uint8_t *sm, int hd) {
         if (requested == nchunks) st_release(p.consumed + hd, nchunks);
     } else if (tid == CTL) {
         // ------------------------------------------------ MMA thread
-        uint32_t ph_full[2] = {0, 0}, ph_t = 0, ph_free[2] = {0, 0};
+        uint32_t ph_t = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
             if (ld_volatile(&s_flags[0])) break;
-            if (!mbar_wait_bounded(&bars[b], ph_full[b], p.timeout_ns)) { fail(); break; }
-            ph_full[b] ^= 1u;
+            if (!mbar_wait_bounded(&bars[b], (uint32_t)(c >> 1) & 1u, p.timeout_ns)) { fail(); break; }
             if (!mbar_wait_bounded(&bars[6], ph_t, p.timeout_ns)) { fail(); break; }
             ph_t ^= 1u;
             tc_fence_after();
@@ -251,8 +249,7 @@ __device__ void consumer(const SplitParams &p, uint8_t *sm, int hd) {
                 mma_bf16_ss(tmem + TM_S, desc_mn_at(dU, kk), desc_mn_at(dK, kk), I_K, 1);
             mma_commit(&bars[2]);
             if (c >= 2) {  // the output warps have read this accumulator's previous chunk
-                if (!mbar_wait_bounded(&bars[8 + b], ph_free[b], p.timeout_ns)) { fail(); break; }
-                ph_free[b] ^= 1u;
+                if (!mbar_wait_bounded(&bars[8 + b], (uint32_t)((c - 2) >> 1) & 1u, p.timeout_ns)) { fail(); break; }
             }
             tc_fence_after();
 #pragma unroll
@@ -341,12 +338,10 @@ __device__ void consumer(const SplitParams &p, uint8_t *sm, int hd) {
         // consecutive channels (64 bytes)
         const int d_me = 32 * quad + lane;
         const int th = (warp >> 2) & 1;
-        uint32_t ph_o[2] = {0, 0};
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
             if (ld_volatile(&s_flags[0])) break;
-            const bool ok = mbar_wait_bounded(&bars[4 + b], ph_o[b], p.timeout_ns);
-            ph_o[b] ^= 1u;
+            const bool ok = mbar_wait_bounded(&bars[4 + b], (uint32_t)(c >> 1) & 1u, p.timeout_ns);
             if (!ok) { fail(); break; }
             tc_fence_after();
             const int64_t tc = bos + (int64_t)c * C + 32 * th;
@@ -432,7 +427,6 @@ __device__ void consumer_seg(const SplitParams &p, uint8_t *sm, int hd, int4 vi)
 
     if (tid == LDR) {
         // ------------------------------------------------ loader thread (as in the plain consumer)
-        uint32_t ph_o[2] = {0, 0};
         int requested = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
@@ -440,8 +434,7 @@ __device__ void consumer_seg(const SplitParams &p, uint8_t *sm, int hd, int4 vi)
             if (!wait_flag_ge(p.filled + hd * RING + (c % RING), c + 1, p.timeout_ns)) { fail(); break; }
             fence_proxy_async_global();
             if (c >= 2) {
-                if (!mbar_wait_bounded(&bars[2 + b], ph_o[b], p.timeout_ns)) { fail(); break; }
-                ph_o[b] ^= 1u;
+                if (!mbar_wait_bounded(&bars[2 + b], (uint32_t)((c - 2) >> 1) & 1u, p.timeout_ns)) { fail(); break; }
                 st_release(p.consumed + hd, c - 1);
             }
             const uint8_t *src = p.ring + ((size_t)hd * RING + (size_t)(c % RING)) * SLOT;
@@ -454,12 +447,11 @@ __device__ void consumer_seg(const SplitParams &p, uint8_t *sm, int hd, int4 vi)
         if (requested == nchunks) st_release(p.consumed + hd, nchunks);
     } else if (tid == CTL) {
         // ------------------------------------------------ MMA thread
-        uint32_t ph_full[2] = {0, 0}, ph_ready = 0, ph_free = 0;
+        uint32_t ph_ready = 0, ph_free = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
             if (ld_volatile(&s_flags[0])) break;
-            if (!mbar_wait_bounded(&bars[b], ph_full[b], p.timeout_ns)) { fail(); break; }
-            ph_full[b] ^= 1u;
+            if (!mbar_wait_bounded(&bars[b], (uint32_t)(c >> 1) & 1u, p.timeout_ns)) { fail(); break; }
             if (!mbar_wait_bounded(&bars[4], ph_ready, p.timeout_ns)) { fail(); break; }
             ph_ready ^= 1u;
             tc_fence_after();
@@ -527,14 +519,12 @@ __device__ void consumer_seg(const SplitParams &p, uint8_t *sm, int hd, int4 vi)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars[4]);
-        uint32_t ph_o[2] = {0, 0};
         int dead_from = 0x7fffffff;  // the state warps' copy of s_flags[2]
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
             const bool last = c + 1 == nchunks;
             if (ld_volatile(&s_flags[0])) break;
-            const bool ok = mbar_wait_bounded(&bars[2 + b], ph_o[b], p.timeout_ns);
-            ph_o[b] ^= 1u;
+            const bool ok = mbar_wait_bounded(&bars[2 + b], (uint32_t)(c >> 1) & 1u, p.timeout_ns);
             if (!ok) { fail(); break; }
             tc_fence_after();
             uint32_t rmax = 0;  // max |R| over this thread's columns (as float bits)
@@ -592,12 +582,10 @@ __device__ void consumer_seg(const SplitParams &p, uint8_t *sm, int hd, int4 vi)
         // warps w and w + 4 (w = 8..11) take tokens [32 th, 32 th + 32)
         const int d_me = 32 * quad + lane;  // value channel of O0^T, row a of E^T
         const int th = (warp >> 2) & 1;
-        uint32_t ph_o[2] = {0, 0};
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
             if (ld_volatile(&s_flags[0])) break;
-            const bool ok = mbar_wait_bounded(&bars[2 + b], ph_o[b], p.timeout_ns);
-            ph_o[b] ^= 1u;
+            const bool ok = mbar_wait_bounded(&bars[2 + b], (uint32_t)(c >> 1) & 1u, p.timeout_ns);
             if (!ok) { fail(); break; }
             tc_fence_after();
             const int64_t tc = bos + (int64_t)c * C + 32 * th;
@@ -941,7 +929,8 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         // latency stays off their path); read by all after the following barriers
         if (ctl) put_rec(n + 2, nx.hd >= 0 ? claim() : -1);
         if (compute) {
-            invert_unit_lower<NTC>(LTp, PBp, sm + TT, s_beta, tid);
+            // warps 0..3, one per SM sub-partition
+            invert_unit_lower<NTC>(LTp, PBp, sm + TT, s_beta, tid, warp);
             fence_proxy_async_smem();
         }
         if (sync_work_or(ld_volatile(&s_flags[0]) != 0)) break;

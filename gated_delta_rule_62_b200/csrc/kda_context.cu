@@ -192,33 +192,32 @@ seg_fixup_kernel(const FixParams p) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    // thread 0 owns the copies: pending[k] is set while copy k (0: A, 1 / 2: E stages) may be in flight
-    bool ok = true, pending[3] = {false, false, false};
-    uint32_t ph_e[2] = {0, 0};
+    // thread 0 owns the copies: bit k of `pending` is set while copy k (0: A, 1 / 2: E stages) may
+    // be in flight. E stage s serves chunks c with (c - c0) % 2 == s, use (c - c0) / 2.
+    bool ok = true;
+    uint32_t pending = 0;
     if (tid == 0) {
         mbar_arrive_expect_tx(&bars[0], kSegStartTileBytes);
         bulk_load(sm + FIX_A, p.s_start + ((size_t)v * H + h) * kSegStartTileBytes, kSegStartTileBytes, &bars[0]);
-        pending[0] = true;
+        pending = 1u;
         for (int k = 0; k < 2 && c0 + k < c1; ++k) {
             mbar_arrive_expect_tx(&bars[1 + k], kSegETileBytes);
             bulk_load(sm + (k ? FIX_E1 : FIX_E0), e_tile(c0 + k), kSegETileBytes, &bars[1 + k]);
-            pending[1 + k] = true;
+            pending |= 2u << k;
         }
         ok = mbar_wait_bounded(&bars[0], 0, p.timeout_ns);
-        if (ok) pending[0] = false;
+        if (ok) pending &= ~1u;
     }
     uint32_t ph_mma = 0;
     const uint32_t sb = smem_u32(sm);
     const int d = tid;
+    int brk = -1;  // the chunk the loop broke off at (its copy and the next one may be in flight)
     for (int c = c0; c < c1; ++c) {
         const int s = (c - c0) & 1;
         if (tid == 0) {
             if (ok) {
-                ok = mbar_wait_bounded(&bars[1 + s], ph_e[s], p.timeout_ns);
-                if (ok) {
-                    pending[1 + s] = false;
-                    ph_e[s] ^= 1u;
-                }
+                ok = mbar_wait_bounded(&bars[1 + s], (uint32_t)((c - c0) >> 1) & 1u, p.timeout_ns);
+                if (ok) pending &= ~(2u << s);
             }
             if (ok) {
                 tc_fence_after();
@@ -234,13 +233,14 @@ seg_fixup_kernel(const FixParams p) {
         ph_mma ^= 1u;
         if (__syncthreads_or(!done || (tid == 0 && !ok))) {
             if (tid == 0) atomicOr(p.status, 1);
+            brk = c;
             break;
         }
         tc_fence_after();
         if (tid == 0 && c + 2 < c1) {  // stage s is free: the MMA that read it has completed
             mbar_arrive_expect_tx(&bars[1 + s], kSegETileBytes);
             bulk_load(sm + (s ? FIX_E1 : FIX_E0), e_tile(c + 2), kSegETileBytes, &bars[1 + s]);
-            pending[1 + s] = true;
+            pending |= 2u << s;
         }
         float x[2][32];
         tmem_ld32(tmem + lane_base, x[0]);
@@ -258,10 +258,14 @@ seg_fixup_kernel(const FixParams p) {
             }
         __syncthreads();  // the accumulator is read before the next chunk's MMA rewrites it
     }
-    if (tid == 0) {  // copies still in flight (after a timeout) land before the block exits
-        if (pending[0]) mbar_wait_bounded(&bars[0], 0, p.timeout_ns);
-        for (int k = 0; k < 2; ++k)
-            if (pending[1 + k]) mbar_wait_bounded(&bars[1 + k], ph_e[k], p.timeout_ns);
+    if (tid == 0 && pending) {  // copies still in flight (after a timeout) land before the block exits
+        if (pending & 1u) mbar_wait_bounded(&bars[0], 0, p.timeout_ns);
+        // only after a break: the copies of chunks brk and brk + 1 (one per stage) may be in
+        // flight; chunk c's copy completes use (c - c0) / 2 of stage (c - c0) % 2's barrier
+        for (int cc = brk; cc >= 0 && cc <= brk + 1 && cc < c1; ++cc) {
+            const int k = (cc - c0) & 1;
+            if (pending & (2u << k)) mbar_wait_bounded(&bars[1 + k], (uint32_t)((cc - c0) >> 1) & 1u, p.timeout_ns);
+        }
     }
     __syncthreads();
     if (warp == 0) {
