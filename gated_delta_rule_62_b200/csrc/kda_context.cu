@@ -130,14 +130,6 @@ constexpr int FIX_CHUNKS = 64;
 constexpr uint32_t FIX_A = 0, FIX_E0 = 32768, FIX_E1 = 49152, FIX_MISC = 65536;
 constexpr uint32_t FIX_SMEM = FIX_MISC + 128 + 1024;
 
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
 struct FixParams {
     const int32_t *vcu;
     const int4 *vinfo;
