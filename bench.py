@@ -50,8 +50,8 @@ FLOP_PER_TOKEN_HEAD = 180224
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
 # dram__bytes_read.sum + dram__bytes_write.sum of one split_kernel launch on the headline workload,
 # from one ncu capture; reported only while the kernel's sources are the ones it was taken on.
-SPLIT_TRAFFIC_BYTES = 336.781056e6 + 58.767872e6
-SPLIT_TRAFFIC_SOURCES_SHA256 = "42f80fc283b15a5f3059454ef4cd74b41d578fbf479c479d624e84fc6a095a72"
+SPLIT_TRAFFIC_BYTES = 336.772608e6 + 59.311872e6
+SPLIT_TRAFFIC_SOURCES_SHA256 = "94bf48a27fe1df27b132ba4cdabbadc912e9fe61d5e70353f0e2c03af3b143ce"
 
 
 def measured_traffic():
@@ -66,10 +66,10 @@ DECODE_BYTES_PER_TOKEN_HEAD = 2 * 128 * 128 * 4 + 3 * 128 * 2 + 128 * 4 + 4 + 12
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of each decode-side kernel on the
 # decode workload (ncu, one capture each), reported while kda_decode.cu and kda_internal.cuh hash
 # to the sources they were taken on.
-DECODE_SIDE_TRAFFIC = {"decode": 547.409152e6 + 479.214336e6, "verify": 581.512192e6 + 10.139392e6,
-                       "commit": 602.596608e6 + 480.340992e6,
-                       "commit_verify": 802.48832e6 + 505.373952e6}
-DECODE_SIDE_SOURCES_SHA256 = "a0901424501414022377629fe654c9a9d34e9e5a922a5e5d3ae32419e8122e94"
+DECODE_SIDE_TRAFFIC = {"decode": 547.412759e6 + 476.568460e6, "verify": 580.620688e6 + 6.144944e6,
+                       "commit": 604.566640e6 + 477.464256e6,
+                       "commit_verify": 800.792272e6 + 502.303952e6}
+DECODE_SIDE_SOURCES_SHA256 = "c2fdce9b14ee2d939e5ee1bb9c35bba1c78f13c73015416e4bcd8603ccc48e07"
 
 
 def decode_side_traffic(kernel):
