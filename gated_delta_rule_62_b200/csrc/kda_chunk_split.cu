@@ -94,8 +94,9 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 // Every split CTA runs NTC compute threads (warps 0..15) plus two control warps: lane 0 of
 // warp 16 issues the tensor-core MMAs (and, in a producer, the TMA loads); lane 0 of warp 17
 // brings a consumer its chunk images, or takes a producer's finished images to the ring (slot
-// wait, stores, hand-off flag). None of their waits stalls a compute warp. Sixteen compute warps (four per SM sub-partition) halve each phase's
-// per-thread work against eight: the per-chunk work is latency-bound, not issue-bound.
+// wait, stores, hand-off flag). None of their waits stalls a compute warp. Sixteen compute warps
+// (four per SM sub-partition) halve each phase's per-thread work against eight: the per-chunk work
+// is latency-bound, not issue-bound.
 constexpr int NTC = 2 * NT;    // compute threads: 16 warps
 constexpr int NTS = NTC + 64;
 constexpr int CTL = NTC;       // the MMA / control thread
@@ -142,8 +143,9 @@ constexpr uint32_t TM_S = 0, TM_SB0 = 128, TM_SB1 = 192, TM_O0 = 256, TM_O1 = 38
 // consumption of chunk c - 2 at that point. MMA thread: wait for the image and for S_b^T(c) in TMEM,
 // issue the chain (commit s); once the output warps have read accumulator b (chunk c - 2), issue
 // the transposed output O^T = S_b^T P^T + U~^T A^T from the same TMEM copy (commit o[b]). State
-// warps 0..3 (lane = value channel): after s, the new state's bf16 copy into TMEM ("tmem ready": the
-// critical path). Output warps 4..7: after o[b], the outputs ("o free"). No CTA-wide barrier inside
+// warps 0..7 (lane = value channel, two column halves): after s, the new state's bf16 copy into
+// TMEM ("tmem ready": the critical path). Output warps 8..15 (32 tokens each): after o[b], the
+// outputs ("o free"). No CTA-wide barrier inside
 // the loop. S_b^T(c) in TMEM copy c & 1 is rewritten only after the chain of chunk c + 1 has
 // completed, and so has O(c), issued before it by the same thread.
 __device__ void consumer(const SplitParams &p, uint8_t *sm, int hd) {
@@ -636,8 +638,9 @@ constexpr uint32_t TM_D1 = 0, TM_W = 128, TM_D3 = 256, TM_D4 = 384, TM_COLS = 51
 }  // namespace prod
 
 // Producer roles: the compute threads run the gating, the TMEM epilogues and the inverse; the
-// control thread issues the TMA loads, the MMAs and the image's bulk stores, waits for a free
-// ring slot and publishes the image. The phases of one item are separated by CTA barriers.
+// control thread claims the items and issues the TMA loads and the MMAs; the store thread waits
+// for a free ring slot, copies each finished image out with bulk stores and publishes it. The
+// phases of one item are separated by barriers of the compute threads and the control warp.
 template <bool PRO>
 __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
                          const CUtensorMap *tm_la, const SplitParams &p, uint8_t *sm, int pid, int nprod) {
