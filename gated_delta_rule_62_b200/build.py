@@ -1,6 +1,6 @@
 """Build libkda.so in-tree with nvcc for sm_100a (B200).
 
-    python -m gated_delta_rule_62_b200.build [--force] [--verbose] [--debug] [--nvtx]
+    python -m gated_delta_rule_62_b200.build [--force] [--verbose] [--debug] [--nvtx] [--tc-inverse]
 
 Each ``csrc/*.cu`` is compiled to an object under ``_build/`` (in parallel) and
 linked with the static CUDA runtime into ``gated_delta_rule_62_b200/libkda.so``.
@@ -10,6 +10,9 @@ Works without a GPU (nvcc cross-compiles).
 access at a computed address is checked against its buffer's byte range, and an
 access outside it is skipped and reported through the device status word
 (KDA_ERR_INTERNAL). ``--nvtx`` adds an NVTX range per library call (-DKDA_NVTX).
+``--tc-inverse`` builds ``libkda_tcinv.so``, whose split-role prefill inverts the 64x64 unit
+lower-triangular matrix with three rounds of tcgen05 MMAs (-DKDA_TC_INVERSE) instead of the
+warp-level tf32 merges; it is correct and slower, and kept for that comparison.
 Load another build than ``libkda.so`` by setting KDA_LIB to its path.
 """
 from __future__ import annotations
@@ -29,6 +32,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libkda.so")
 DEBUG_LIB = os.path.join(PKG, "libkda_debug.so")
+TCINV_LIB = os.path.join(PKG, "libkda_tcinv.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -58,11 +62,11 @@ def up_to_date(lib: str = LIB) -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, debug: bool = False,
-          nvtx: bool = False) -> str:
-    lib = DEBUG_LIB if debug else LIB
+          nvtx: bool = False, tc_inverse: bool = False) -> str:
+    lib = DEBUG_LIB if debug else (TCINV_LIB if tc_inverse else LIB)
     if not force and not nvtx and up_to_date(lib):
         return lib
-    objdir = os.path.join(BUILD, "debug" if debug else ("nvtx" if nvtx else "release"))
+    objdir = os.path.join(BUILD, "debug" if debug else ("tcinv" if tc_inverse else ("nvtx" if nvtx else "release")))
     os.makedirs(objdir, exist_ok=True)
     cc = nvcc()
     extra = ["-Xptxas", "-v"] if ptxas_info else []
@@ -70,6 +74,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, 
         extra += ["-DKDA_DEBUG"]
     if nvtx:
         extra += ["-DKDA_NVTX"]
+    if tc_inverse:
+        extra += ["-DKDA_TC_INVERSE"]
 
     def compile_one(src):
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
@@ -99,5 +105,7 @@ if __name__ == "__main__":
     ap.add_argument("--ptxas-info", action="store_true")
     ap.add_argument("--debug", action="store_true")
     ap.add_argument("--nvtx", action="store_true")
+    ap.add_argument("--tc-inverse", action="store_true")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose, ptxas_info=a.ptxas_info, debug=a.debug, nvtx=a.nvtx))
+    print(build(force=a.force, verbose=a.verbose, ptxas_info=a.ptxas_info, debug=a.debug, nvtx=a.nvtx,
+                tc_inverse=a.tc_inverse))

@@ -235,6 +235,89 @@ static __device__ __forceinline__ void invert_unit_lower(float *LT, float *PB, u
 }
 
 
+// ---------------------------------------------------------------- the same inverse on tcgen05
+// With D = I + (the 16x16 diagonal blocks of L) and L_off = L outside those blocks,
+// I + L = D (I + N) with N = D^-1 L_off. N's blocks lie strictly below the block diagonal, so
+// N^4 = 0 and (I + N)^-1 = (I + N^2)(I - N):
+//   T = (I + L)^-1 = (I + N^2)(I - N) D^-1,
+// three rounds of dependent bf16 MMAs with fp32 accumulation, which the caller issues:
+//   [N | D^-1] = D^-1 [L_off | I];   W1 = D^-1 - N D^-1 (onto D^-1, A negated), N2 = N N;
+//   T = W1 + N2 W1 (onto W1).
+// Every operand is a 64x64 bf16 tile in the natural row layout (tchunk, one 64-column block),
+// which is both a K-major A operand and an MN-major B operand. Rounding: D^-1, L_off, N, N2 and
+// W1 are rounded to bf16 once each as operands (the accumulators stay fp32); T' = T diag(beta)
+// is rounded to bf16 anyway for the MMAs that use it, and that rounding dominates (checked
+// against the mma.sync tf32 merges above).
+
+// Step 0, before the first MMA: D^-1 into t_dinv (the four diagonal blocks by forward
+// substitution, lanes 0..15 of logical warps 0..3; the other blocks zero), L_off into t_loff and
+// the identity into t_eye. Called by the NTC compute threads; ends with the tile stores issued
+// (no barrier).
+template <int NTC = NT>
+static __device__ __forceinline__ void inv_tc_setup(const float *LT, uint8_t *t_dinv, uint8_t *t_loff,
+                                                    int tid, int warp, uint8_t *t_eye) {
+    static_assert(NTC > 128, "the tile writers are the warps after the first four");
+    const int lane = tid & 31;
+    if (warp >= 0 && warp < 4) {
+        if (lane < 16) {
+            const int b0 = 16 * warp;
+            const float *Lb = LT + b0 * LT_LD + b0;
+            float lv[120];
+#pragma unroll
+            for (int j = 0, e = 0; j < 15; ++j)
+#pragma unroll
+                for (int i = j + 1; i < 16; ++i, ++e) lv[e] = Lb[i * LT_LD + j];
+            float x[16];  // column `lane` of the block's inverse
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = (i == lane) ? 1.f : 0.f;
+#pragma unroll
+            for (int j = 0, e = 0; j < 15; ++j)
+#pragma unroll
+                for (int i = j + 1; i < 16; ++i, ++e) x[i] = fmaf(-lv[e], x[j], x[i]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) st_bf(t_dinv + telem(8192, b0 + i, b0 + lane), x[i]);
+        }
+        return;
+    }
+    // 16-byte chunks (8 columns, inside one 16-column block): L_off everywhere, zeros of D^-1
+    // outside the diagonal blocks (the forward substitution writes those chunks)
+    const float zero[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int q = tid - 128; q < 512; q += NTC - 128) {
+        const int r = q >> 3, c0 = (q & 7) * 8;
+        if ((r >> 4) == (c0 >> 4)) {
+            st_chunk(t_loff + tchunk(8192, r, c0), zero);
+        } else {
+            const float4 a = *reinterpret_cast<const float4 *>(LT + r * LT_LD + c0);
+            const float4 b = *reinterpret_cast<const float4 *>(LT + r * LT_LD + c0 + 4);
+            const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            st_chunk(t_loff + tchunk(8192, r, c0), v);
+            st_chunk(t_dinv + tchunk(8192, r, c0), zero);
+        }
+        float e[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) e[x] = (c0 + x == r) ? 1.f : 0.f;
+        st_chunk(t_eye + tchunk(8192, r, c0), e);
+    }
+}
+
+// 16 columns col0.. of an M=64 accumulator (row 16 quad + lane in lanes 0..15 of each quadrant;
+// taddr includes the warp's lane base) -> the same rows and columns of a 64x64 bf16 tile, as
+// op(row, col, value).
+template <typename Op>
+__device__ __forceinline__ void acc64_cols16_to_tile(uint32_t taddr, uint8_t *tile, int col0, int quad,
+                                                     int lane, Op op) {
+    float v[16];
+    tmem_ld16(taddr + (uint32_t)col0, v);
+    tmem_wait_ld();
+    if (lane < 16) {
+        const int row = 16 * quad + lane;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = op(row, col0 + e, v[e]);
+        st_chunk(tile + tchunk(8192, row, col0), v);
+        st_chunk(tile + tchunk(8192, row, col0 + 8), v + 8);
+    }
+}
+
 // ---------------------------------------------------------------- gating of one chunk
 // The NTC compute threads (synchronised among themselves with sync_compute<NTC>). In: QK holds
 // raw q (rows 0..63) and k (rows 64..127) as a K-major tile with 16 KB blocks, LA the chunk's raw

@@ -635,6 +635,13 @@ constexpr uint32_t PSUM_FLOATS = (NTC / 32 + 1) * 128;  // group totals per comp
 constexpr uint32_t BYTES = MISC + 64 * 4 + 128 * 4 + PSUM_FLOATS * 4 + 64 + 64 + 4 * 32;
 // TMEM: D1 = [Q~; K~] K-^T (M=128, 64 columns), W (M=64), D3 = [U~; -A W], D4 = -K^^T W
 constexpr uint32_t TM_D1 = 0, TM_W = 128, TM_D3 = 256, TM_D4 = 384, TM_COLS = 512;
+// Tiles of the tensor-core inverse (build option KDA_TC_INVERSE; 64x64 bf16, 8 KB each), over
+// regions dead during it. The
+// identity sits 8 KB after L_off, so [L_off | I] is one MN-major B operand of two 64-column
+// blocks; N overwrites the identity once the first MMA has read it.
+constexpr uint32_t IV_DINV = KI, IV_LOFF = KI + 8192, IV_EYE = IV_LOFF + 8192, IV_N = IV_EYE;
+constexpr uint32_t IV_N2 = LT, IV_W1 = LT + 8192;
+static_assert(IV_EYE == WN && IV_N2 % 1024 == 0 && IV_W1 + 8192 <= MISC, "inverse tiles");
 }  // namespace prod
 
 // Producer roles: the compute threads run the gating, the TMEM epilogues and the inverse; the
@@ -649,6 +656,11 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     constexpr uint32_t I_W = idesc_bf16_f32(64, 128, false, 0, 1);
     constexpr uint32_t I_3 = idesc_bf16_f32(128, 128, false, 0, 1);
     constexpr uint32_t I_4 = idesc_bf16_f32(128, 128, false, 1, 1);
+#ifdef KDA_TC_INVERSE
+    constexpr uint32_t I_IV = idesc_bf16_f32(64, 64, false, 0, 1);   // inverse steps
+    constexpr uint32_t I_IVN = idesc_bf16_f32(64, 64, true, 0, 1);   // the same, A negated
+    constexpr uint32_t I_IV2 = idesc_bf16_f32(64, 128, false, 0, 1); // D^-1 [L_off | I]
+#endif
     float *s_beta = reinterpret_cast<float *>(sm + MISC);
     float *s_gamma = s_beta + 64;
     float *s_psum = s_gamma + 128;
@@ -656,7 +668,9 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     // qk0, qk1, la, v, mma, src (the image's sources may be rewritten), img (an image is ready)
     uint64_t *bars = reinterpret_cast<uint64_t *>(s_flags + 16);
     float *LTp = reinterpret_cast<float *>(sm + LT);
+#ifndef KDA_TC_INVERSE
     float *PBp = reinterpret_cast<float *>(sm + PB);
+#endif
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // TMEM epilogues: warp w reads lanes 32 (w % 4) .. + 31, column part w / 4 of four
@@ -880,6 +894,12 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             fence_proxy_async_smem();
         }
         ph_src ^= 1u;
+#ifdef KDA_TC_INVERSE
+        // the item after the next one, claimed while the compute threads run the gating (the
+        // control thread has a part in every round of the inverse); read by all after the
+        // following barriers. Record n + 2's slot was last read at the top of item n - 2.
+        if (ctl) put_rec(n + 2, nx.hd >= 0 ? claim() : -1);
+#endif
         const bool stop = sync_work_or(ld_volatile(&s_flags[0]) != 0) != 0;
         const int gate = (int)s_flags[2] - 1;
         if (gate < 0 || stop) break;
@@ -917,6 +937,73 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         // still issuing the prefetches); the CTA-wide stop check follows the inverse
         if (compute) sync_compute<NTC>();
 
+#ifdef KDA_TC_INVERSE
+        // (build option) T' = (I + L)^-1 diag(beta) on the tensor cores, three rounds of MMAs (inv_tc_setup):
+        //   1: [N | D^-1] = D^-1 [L_off | I]            (one N = 128 MMA: D^-1 lands in TMEM)
+        //   2: W1 = D^-1 - N D^-1 (onto D^-1), N2 = N N
+        //   3: T = W1 + N2 W1 (onto W1) = (I + N2)(I - N) D^-1
+        // Tiles: D^-1 and L_off over K- (dead since D1), I and then N over -W (written after W),
+        // N2 and W1 over the L/T scratch (L is read in step 0). Accumulators: the W and D3
+        // columns, free until those MMAs.
+        if (compute) {
+            inv_tc_setup<NTC>(LTp, sm + IV_DINV, sm + IV_LOFF, tid, warp, sm + IV_EYE);
+            fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        sync_work();
+        if (ctl) {
+            tc_fence_after();
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)
+                mma_bf16_ss(tmem + TM_W, desc_k(sb + IV_DINV, 8192, kk), desc_mn(sb + IV_LOFF, 8192, kk), I_IV2, kk > 0);
+            mma_commit(&bars[4]);
+        }
+        wait_bar(&bars[4], ph_mma);
+        tc_fence_after();
+        if (compute) {
+            acc64_cols16_to_tile(tmem + lane_base + TM_W, sm + IV_N, 16 * part, quad, lane,
+                                 [](int, int, float x) { return x; });
+            fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        sync_work();
+        if (ctl) {
+            tc_fence_after();
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)  // W1 = D^-1 - N D^-1
+                mma_bf16_ss(tmem + TM_W + 64, desc_k(sb + IV_N, 8192, kk), desc_mn(sb + IV_DINV, 8192, kk), I_IVN, 1);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)  // N2 = N N
+                mma_bf16_ss(tmem + TM_D3, desc_k(sb + IV_N, 8192, kk), desc_mn(sb + IV_N, 8192, kk), I_IV, kk > 0);
+            mma_commit(&bars[4]);
+        }
+        wait_bar(&bars[4], ph_mma);
+        tc_fence_after();
+        if (compute) {
+            acc64_cols16_to_tile(tmem + lane_base + TM_W + 64, sm + IV_W1, 16 * part, quad, lane,
+                                 [](int, int, float x) { return x; });
+            acc64_cols16_to_tile(tmem + lane_base + TM_D3, sm + IV_N2, 16 * part, quad, lane,
+                                 [](int, int, float x) { return x; });
+            fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        sync_work();
+        if (ctl) {
+            tc_fence_after();
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; ++kk)  // T = W1 + N2 W1
+                mma_bf16_ss(tmem + TM_W + 64, desc_k(sb + IV_N2, 8192, kk), desc_mn(sb + IV_W1, 8192, kk), I_IV, 1);
+            mma_commit(&bars[4]);
+        }
+        wait_bar(&bars[4], ph_mma);
+        tc_fence_after();
+        if (compute) {
+            acc64_cols16_to_tile(tmem + lane_base + TM_W + 64, sm + TT, 16 * part, quad, lane,
+                                 [s_beta](int, int c, float x) { return x * s_beta[c]; });
+            fence_proxy_async_smem();
+        }
+        tc_fence_before();
+#else
         // the item after the next one, claimed while the compute threads invert (the atomic's
         // latency stays off their path); read by all after the following barriers
         if (ctl) put_rec(n + 2, nx.hd >= 0 ? claim() : -1);
@@ -925,6 +1012,7 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
             invert_unit_lower<NTC>(LTp, PBp, sm + TT, s_beta, tid, warp);
             fence_proxy_async_smem();
         }
+#endif
         if (sync_work_or(ld_volatile(&s_flags[0]) != 0)) break;
 
         if (ctl) {

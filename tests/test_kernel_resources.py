@@ -16,6 +16,7 @@ from gated_delta_rule_62_b200 import build as B
 BUDGET = [
     ("kda_chunk_split.cu", "split_kernelILb0E", 96),
     ("kda_chunk_split.cu", "split_kernelILb1E", 96),
+    ("kda_chunk_split.cu@-DKDA_TC_INVERSE", "split_kernelILb0E", 96),  # the build option
     ("kda_chunk.cu", "chunk_kernelILi128ELb0E", 255),
     ("kda_chunk.cu", "chunk_kernelILi64ELb0E", 255),
     ("kda_chunk.cu", "chunk_kernelILi128ELb1E", 255),
@@ -28,9 +29,10 @@ BUDGET = [
 ]
 
 
-def _ptxas_report(src, tmp):
-    obj = os.path.join(tmp, src + ".o")
-    cmd = [B.nvcc(), *B.ARCH, *B.NVCC_FLAGS, "-Xptxas", "-v", "-c", os.path.join(B.CSRC, src), "-o", obj]
+def _ptxas_report(spec, tmp):
+    src, *defs = spec.split("@")  # source, then any -D flags of a build option
+    obj = os.path.join(tmp, spec.replace("@", "_").replace("-", "") + ".o")
+    cmd = [B.nvcc(), *B.ARCH, *B.NVCC_FLAGS, *defs, "-Xptxas", "-v", "-c", os.path.join(B.CSRC, src), "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     assert r.returncode == 0, r.stderr[-2000:]
     props, name = {}, None
