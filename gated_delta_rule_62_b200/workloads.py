@@ -87,7 +87,11 @@ PREFILL_1M = Workload("prefill_B1_T1048576_H16_d128_bf16", 1004, (1 << 20,), 16,
 VARLEN_24 = Workload("varlen_24seq_logU512-65536_H32_d128_bf16_resume", 1005,
                      varlen_lengths(), 32, 128, 128, "bf16", init_state="normal")
 
-WORKLOADS = {w.name: w for w in (TINY_F32, PREFILL_8K, DECODE_256, PREFILL_1M, VARLEN_24)}
+# Not a benchmark line: 64 of the decode workload's 512-token seeding prefills (2,048 chains, the
+# fused kernel's regime), 1.8 GB on the device, for profiler captures that replay each launch.
+PREFILL_64x512 = Workload("prefill_N64_T512_H32_d128_bf16", 1006, (512,) * 64, 32, 128, 128, "bf16")
+
+WORKLOADS = {w.name: w for w in (TINY_F32, PREFILL_8K, DECODE_256, PREFILL_1M, VARLEN_24, PREFILL_64x512)}
 
 
 def custom(seqlens, H, dk, dv, dtype="bf16", seed=7, init_state="zero", name=None) -> Workload:
