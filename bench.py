@@ -8,7 +8,8 @@ solve, WY build, state recall/correction, output, state update, varlen state
 I/O) of the 8192-token, 32-head, d=128 bf16 workload through ``kda_prefill``.
 ``value`` is tokens/s with inputs resident in HBM; ``e2e`` is the same metric
 with the step's inputs copied from pinned host memory and its outputs read back
-inside the timed region. The decode step (256 sequences x 32 heads, fp32 state
+inside the timed region (beside it, the uploads alone timed the same way: the host
+link's bound on that number). The decode step (256 sequences x 32 heads, fp32 state
 of 512 MiB streamed once in and once out) is measured in the same run and
 reported under ``decode``; speculative decode on the same states (verify 4 draft
 tokens, commit them, and the fused commit + verify step) under
@@ -529,7 +530,21 @@ def run_ours(args, rank, local, ws):
         end.synchronize()
         return start.elapsed_time(end) / steps
 
-    e2e_ms = e2e_serial_ms = None
+    def timed_upload(steps):  # the step's host -> device copies alone: the link's own bound
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(s_up)
+        for i in range(steps):
+            dev = bufs[i % 2]
+            with torch.cuda.stream(s_up):
+                for n in names:
+                    dev[n].copy_(host[n], non_blocking=True)
+                if host_s0 is not None:
+                    bufs_s0[i % 2].copy_(host_s0, non_blocking=True)
+        end.record(s_up)
+        end.synchronize()
+        return start.elapsed_time(end) / steps
+
+    e2e_ms = e2e_serial_ms = upload_ms = None
     if not args.no_e2e:
         n_e2e = max(4, args.steps // 2)
         for _ in range(2):
@@ -540,6 +555,9 @@ def run_ours(args, rank, local, ws):
         torch.cuda.synchronize()
         barrier(ws)
         e2e_serial_ms = max_over_ranks(timed_e2e(False, n_e2e), ws)
+        torch.cuda.synchronize()
+        barrier(ws)
+        upload_ms = max_over_ranks(timed_upload(n_e2e), ws)
         torch.cuda.synchronize()
     del host, bufs, bufs_s0, outs, fss
 
@@ -588,7 +606,11 @@ def run_ours(args, rank, local, ws):
             "copies": "pipelined: step i+1's upload overlaps step i's kernel and download "
                       "(two buffer sets, three streams)",
             "serial_ms_per_step": e2e_serial_ms,
-            "serial_value": T * ws / (e2e_serial_ms * 1e-3)},
+            "serial_value": T * ws / (e2e_serial_ms * 1e-3),
+            # the uploads alone, timed the same way: the host link's bound on this step
+            "upload_only_ms_per_step": upload_ms,
+            "upload_gbs": h2d / (upload_ms * 1e-3) / 1e9,
+            "frac_of_upload_bound": upload_ms / e2e_ms},
         "decode": dec,
         "speculative_decode": spec,
         "other_prefill_workloads": extra,
