@@ -44,6 +44,12 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     const size_t head = blockIdx.x;  // n * H + h
     const int tid = threadIdx.x;
     const int cg = tid % CG, rg = tid / CG;
+    // Launched with programmatic stream serialization: the next decode step's blocks may become
+    // resident while this grid drains, and this grid's while the previous one drains. Nothing is
+    // read before the wait, which returns once the previous kernel in the stream has completed
+    // and its writes are visible (without that launch attribute both are no-ops).
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // this head's state: entry `head`, or its sequence's slot of the pool (none: zeros, not stored)
     float *blk = final_state_block(state, (int)(head / H), H, (int)(head % H), (size_t)(DK * DV), ss);
     if (blk && !KDA_ACCESS_OK(ss.status, dbg.fin, blk, DK * DV * 4, 31)) blk = nullptr;
@@ -345,11 +351,19 @@ cudaError_t launch_verify3(const VerifyProblem &p, cudaStream_t stream) {
 
 template <typename Tin, int DK, int DV>
 cudaError_t launch3(const DecodeProblem &p, cudaStream_t stream) {
-    const unsigned blocks = (unsigned)p.num_seqs * (unsigned)p.H;
-    decode_kernel<Tin, DK, DV><<<blocks, DecodeShape<DK, DV>::NT, 0, stream>>>(
-        (const Tin *)p.q, (const Tin *)p.k, (const Tin *)p.v, p.log_alpha, p.beta, p.state,
-        (Tin *)p.out, p.H, p.slots, p.dbg);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.num_seqs * (unsigned)p.H);
+    cfg.blockDim = dim3(DecodeShape<DK, DV>::NT);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_kernel<Tin, DK, DV>, (const Tin *)p.q, (const Tin *)p.k,
+                              (const Tin *)p.v, p.log_alpha, p.beta, p.state, (Tin *)p.out, p.H, p.slots,
+                              p.dbg);
 }
 
 template <template <typename, int, int> class L, typename P>
