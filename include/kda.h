@@ -29,7 +29,12 @@
  *   - Ownership: the caller allocates and frees every buffer, including the
  *     workspace. The library does not allocate, free or synchronise inside
  *     kda_prefill / kda_decode_step: both only enqueue work on `stream` and
- *     return. Buffers must stay valid until the stream has run the work.
+ *     return. Buffers must stay valid until the stream has run the work. The
+ *     prefill, decode and speculative-decode calls can therefore be captured
+ *     into a CUDA graph (after one call outside the capture, which sets each
+ *     kernel's shared-memory limit) and replayed on the same buffers; the decode
+ *     step's kernel is launched with programmatic stream serialization, so
+ *     consecutive steps overlap their launch, in a stream or in a graph.
  *   - Aliasing: final_state may alias initial_state (in-place resume); the
  *     decode state is updated in place; out must not alias any input.
  *   - Errors: arguments are checked on the host before anything is enqueued;

@@ -6,6 +6,9 @@ allocation whose GUARD bytes before and after it are filled with a canary byte. 
 the stream is synchronised and both bands must still hold the canary; a kernel that writes past
 either end of a buffer fails the test that made the call.
 
+Calls made while a CUDA graph is being captured go straight to the binding (a band check
+synchronises the device, which a capture does not allow).
+
 ``install(K)`` replaces the binding's entry points (prefill, decode_step, prefill_slots,
 decode_step_slots, decode_verify, decode_commit, decode_commit_verify) by guarded versions with
 the same signatures: outputs the caller did not pass are allocated guarded, in-place states are
@@ -70,6 +73,8 @@ def _guard_prefill(orig):
 
     @functools.wraps(orig)
     def f(*args, **kwargs):
+        if torch.cuda.is_current_stream_capturing():  # no synchronising check inside a CUDA graph
+            return orig(*args, **kwargs)
         b = sig.bind(*args, **kwargs)
         a = b.arguments
         bands = _Bands()
@@ -93,6 +98,8 @@ def _guard_inplace(orig, name, outs, states):
 
     @functools.wraps(orig)
     def f(*args, **kwargs):
+        if torch.cuda.is_current_stream_capturing():  # no synchronising check inside a CUDA graph
+            return orig(*args, **kwargs)
         b = sig.bind(*args, **kwargs)
         a = b.arguments
         bands = _Bands()
