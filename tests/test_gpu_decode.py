@@ -110,3 +110,30 @@ def test_decode_1024_steps_against_oracle_without_reseeding():
     # drift stays far inside the tolerance: the last step alone, for the record
     last = got.reshape(sub.numel(), steps_n, wl.H, wl.dv)[:, -1]
     assert float(np.abs(last - ro.reshape(sub.numel(), steps_n, wl.H, wl.dv)[:, -1]).max()) <= TOL["bf16"] * scale
+
+
+def test_back_to_back_steps_and_other_kernels_between():
+    """Decode steps launched back to back (the programmatic launch lets a step's blocks become
+    resident while the previous step drains), and with PyTorch kernels between them that rewrite
+    the state and the next inputs: each step must see the writes of everything before it."""
+    step = getattr(K.decode_step, "__wrapped__", K.decode_step)  # no guard copies between the calls
+    wl = W.custom((1,) * 64, 8, 128, 128, "bf16", seed=91)
+    g = torch.Generator(device=DEV).manual_seed(91)
+    state = torch.randn(64, 8, 128, 128, device=DEV, generator=g) * 0.1
+    steps = W.make_decode_steps(wl, g, 12, DEV)
+    ref_s = f64(state)
+    outs = torch.empty(12, 64, 8, 128, dtype=torch.bfloat16, device=DEV)
+    ref_o = []
+    for t in range(12):
+        d = {n: steps[n][t] for n in steps}
+        if t % 4 == 3:  # another kernel between two steps: halve the state, rescale v
+            state.mul_(0.5)
+            ref_s = ref_s * 0.5
+            d["v"].mul_(2)
+        step(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], state, out=outs[t])
+        ro, ref_s = _oracle_step(d, ref_s)
+        ref_o.append(ro)
+    torch.cuda.synchronize()
+    scale = float(torch.stack([steps["v"][t] for t in range(12)]).abs().max())
+    assert_close(outs, np.stack(ref_o), TOL["bf16"], scale, "back-to-back decode outputs")
+    assert_close(state, ref_s, TOL["bf16"], scale, "back-to-back decode state")
