@@ -153,6 +153,28 @@ __device__ __forceinline__ void warp_store16(float *X, int px, const float (&acc
     }
 }
 
+// Column `col` of (I + L)^-1 for one 16x16 diagonal block (L strictly lower, fp32 rows LT_LD
+// apart from Lb, which is 16-byte aligned) by forward substitution in row order:
+// x_i = [i == col] - sum_{j<i} L_ij x_j. Each row's values come in as 16-byte broadcast loads
+// (36 for the block), and every row sum runs as two interleaved partial sums.
+__device__ __forceinline__ void unit_lower16_column(const float *Lb, int col, float (&x)[16]) {
+    x[0] = (col == 0) ? 1.f : 0.f;
+#pragma unroll
+    for (int i = 1; i < 16; ++i) {
+        float s0 = (col == i) ? 1.f : 0.f, s1 = 0.f;
+#pragma unroll
+        for (int j4 = 0; 4 * j4 < i; ++j4) {
+            const float4 l = *reinterpret_cast<const float4 *>(Lb + i * LT_LD + 4 * j4);
+            const int j = 4 * j4;
+            s0 = fmaf(-l.x, x[j], s0);
+            if (j + 1 < i) s1 = fmaf(-l.y, x[j + 1], s1);
+            if (j + 2 < i) s0 = fmaf(-l.z, x[j + 2], s0);
+            if (j + 3 < i) s1 = fmaf(-l.w, x[j + 3], s1);
+        }
+        x[i] = s0 + s1;
+    }
+}
+
 // Writes rows of a 16x16 fragment tile as bf16 T' = T diag(beta) into the TT tile at (r0, c0).
 __device__ __forceinline__ void frag_to_tt(uint8_t *TT, int r0, int c0, const float (&acc)[2][4],
                                            float s, const float *beta) {
@@ -181,20 +203,8 @@ static __device__ __forceinline__ void invert_unit_lower(float *LT, float *PB, u
     const int lane = tid & 31;
     if (warp >= 0 && warp < 4 && lane < 16) {
         const int b0 = 16 * warp;
-        const float *Lb = LT + b0 * LT_LD + b0;
-        // all 120 sub-diagonal values first (independent loads), then a dependency chain of 15
-        float lv[120];
-#pragma unroll
-        for (int j = 0, e = 0; j < 15; ++j)
-#pragma unroll
-            for (int i = j + 1; i < 16; ++i, ++e) lv[e] = Lb[i * LT_LD + j];
         float x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = (i == lane) ? 1.f : 0.f;
-#pragma unroll
-        for (int j = 0, e = 0; j < 15; ++j)
-#pragma unroll
-            for (int i = j + 1; i < 16; ++i, ++e) x[i] = fmaf(-lv[e], x[j], x[i]);
+        unit_lower16_column(LT + b0 * LT_LD + b0, lane, x);
         __syncwarp(0x0000ffffu);
         float *Tb = LT + b0 * LT_LD + b0;
         const float bl = beta[b0 + lane];
@@ -261,19 +271,8 @@ static __device__ __forceinline__ void inv_tc_setup(const float *LT, uint8_t *t_
     if (warp >= 0 && warp < 4) {
         if (lane < 16) {
             const int b0 = 16 * warp;
-            const float *Lb = LT + b0 * LT_LD + b0;
-            float lv[120];
-#pragma unroll
-            for (int j = 0, e = 0; j < 15; ++j)
-#pragma unroll
-                for (int i = j + 1; i < 16; ++i, ++e) lv[e] = Lb[i * LT_LD + j];
             float x[16];  // column `lane` of the block's inverse
-#pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = (i == lane) ? 1.f : 0.f;
-#pragma unroll
-            for (int j = 0, e = 0; j < 15; ++j)
-#pragma unroll
-                for (int i = j + 1; i < 16; ++i, ++e) x[i] = fmaf(-lv[e], x[j], x[i]);
+            unit_lower16_column(LT + b0 * LT_LD + b0, lane, x);
 #pragma unroll
             for (int i = 0; i < 16; ++i) st_bf(t_dinv + telem(8192, b0 + i, b0 + lane), x[i]);
         }
@@ -518,6 +517,15 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
             return make_float4(a.x, a.y, b.x, b.y);
         };
         auto pack4 = [](float a, float b, float c, float d) { return make_uint2(pack2(a, b), pack2(c, d)); };
+        // all of this thread's q and k first: each element is rewritten in place by the thread
+        // that reads it, so no load has to wait behind a store
+        uint2 qraw[TPG], kraw[TPG];
+#pragma unroll
+        for (int i = 0; i < TPG; ++i) {
+            const uint32_t off = row_off(TPG * to + i);
+            qraw[i] = *reinterpret_cast<const uint2 *>(q0 + off);
+            kraw[i] = *reinterpret_cast<const uint2 *>(q0 + 8192 + off);
+        }
         float4 P = eA;
 #pragma unroll
         for (int i = 0; i < TPG; ++i) {
@@ -529,7 +537,7 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
             const uint32_t off = row_off(t);
             uint2 *qp = reinterpret_cast<uint2 *>(q0 + off);
             uint2 *kp = reinterpret_cast<uint2 *>(q0 + 8192 + off);
-            float4 qv = unpack4(*qp), kv = unpack4(*kp);
+            float4 qv = unpack4(qraw[i]), kv = unpack4(kraw[i]);
             if (t >= valid) qv = kv = make_float4(0.f, 0.f, 0.f, 0.f);
             *qp = pack4(qv.x * P.x, qv.y * P.y, qv.z * P.z, qv.w * P.w);
             *kp = pack4(kv.x * P.x, kv.y * P.y, kv.z * P.z, kv.w * P.w);
