@@ -328,7 +328,8 @@ __device__ __forceinline__ void acc64_cols16_to_tile(uint32_t taddr, uint8_t *ti
 // groups' totals, turned in place into exclusive prefixes by a scan, plus the chunk totals).
 // If KH is not null it also receives K^ = k e^(g_{C-1} - g) on both paths. If src_free is not
 // null, the writes to KI, KH and AQK first wait (bounded by timeout_ns) for that mbarrier's
-// phase with parity src_parity: another thread may still be reading those tiles.
+// phase with parity src_parity, and then for src_free2's phase with parity src_parity2 if that
+// is not null: other threads or the tensor core may still be reading those tiles.
 // Returns 1 for the exact path, 0 for the factored path, -1 if the wait timed out (which sets
 // *s_abort). Every compute thread passes every barrier inside (the path is decided by a barrier
 // reduction, and a failed wait only sets a flag), so no thread is left waiting at one.
@@ -344,7 +345,8 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
                                           float *s_psum, uint32_t *s_abort, int valid,
                                           int tid, uint8_t *KH = nullptr,
                                           uint64_t *src_free = nullptr, uint32_t src_parity = 0,
-                                          uint64_t timeout_ns = 0, const Prologue pro = Prologue()) {
+                                          uint64_t timeout_ns = 0, const Prologue pro = Prologue(),
+                                          uint64_t *src_free2 = nullptr, uint32_t src_parity2 = 0) {
     constexpr int G = NTC / 32, TPG = C / G;  // token groups (one per warp), tokens per group
     static_assert(G * TPG == C && TPG >= 1 && TPG <= 8, "gating thread mapping");
     const int warp = tid >> 5, lane = tid & 31;
@@ -420,7 +422,9 @@ __device__ __forceinline__ int gate_chunk(uint8_t *QK, uint8_t *KI, uint8_t *AQK
         s_psum[G * D + tid] = run;
         s_gamma[tid] = __expf(run);
     }
-    if (src_free && (!SCRATCH || safe) && !mbar_wait_bounded(src_free, src_parity, timeout_ns)) {
+    if (src_free && (!SCRATCH || safe) &&
+        (!mbar_wait_bounded(src_free, src_parity, timeout_ns) ||
+         (src_free2 && !mbar_wait_bounded(src_free2, src_parity2, timeout_ns)))) {
         *s_abort = 1;
         failed = true;  // the writes below go on (shared memory only); the caller stops
     }

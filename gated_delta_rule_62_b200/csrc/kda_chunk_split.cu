@@ -632,7 +632,7 @@ constexpr uint32_t LT = AQK + 8192;       // L -> T fp32 [64][LT_LD]
 constexpr uint32_t PB = LT + 64 * LT_LD * 4;   // 32 x PB_LD fp32
 constexpr uint32_t MISC = PB + 32 * PB_LD * 4; // beta, gamma, psum, flags, barriers
 constexpr uint32_t PSUM_FLOATS = (NTC / 32 + 1) * 128;  // group totals per compute warp, chunk totals
-constexpr uint32_t BYTES = MISC + 64 * 4 + 128 * 4 + PSUM_FLOATS * 4 + 64 + 64 + 4 * 32;
+constexpr uint32_t BYTES = MISC + 64 * 4 + 2 * 128 * 4 + PSUM_FLOATS * 4 + 64 + 10 * 8 + 4 * 32;
 // TMEM: D1 = [Q~; K~] K-^T (M=128, 64 columns), W (M=64), D3 = [U~; -A W], D4 = -K^^T W
 constexpr uint32_t TM_D1 = 0, TM_W = 128, TM_D3 = 256, TM_D4 = 384, TM_COLS = 512;
 // Tiles of the tensor-core inverse (build option KDA_TC_INVERSE; 64x64 bf16, 8 KB each), over
@@ -663,9 +663,10 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 #endif
     float *s_beta = reinterpret_cast<float *>(sm + MISC);
     float *s_gamma = s_beta + 64;
-    float *s_psum = s_gamma + 128;
+    float *s_psum = s_gamma + 2 * 128;  // s_gamma: one row of 128 per item in flight
     uint32_t *s_flags = reinterpret_cast<uint32_t *>(s_psum + PSUM_FLOATS);  // abort, tmem, gate
-    // qk0, qk1, la, v, mma, src (the image's sources may be rewritten), img (an image is ready)
+    // qk0, qk1, la, v (TMA loads), mma (W, D3/D4), srcM, img2, img1, src1 (hand-off of an image's two
+    // parts), d1 (D1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(s_flags + 16);
     float *LTp = reinterpret_cast<float *>(sm + LT);
 #ifndef KDA_TC_INVERSE
@@ -710,11 +711,11 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     // Item n's record, rec[n % 4]: {head, chunk, head within the sequence, first token, valid
     // tokens} (head < 0: no item n). The control thread decodes each item it claims once; nothing
     // else reads cu_seqlens, so no thread stalls on a global load for it. Record n + 2 is written
-    // during item n's inverse and read from item n + 1 on (behind the barrier that ends the inverse).
+    // during item n's gating and read from iteration n + 1 on (behind the barrier that ends it).
     struct ItemRec {
         int hd, c, h, t0, valid, pad[3];
     };
-    ItemRec *s_rec = reinterpret_cast<ItemRec *>(bars + 8);
+    ItemRec *s_rec = reinterpret_cast<ItemRec *>(bars + 10);
     auto put_rec = [&](int n, int k) {  // control thread
         ItemRec r;
         r.hd = -1;
@@ -733,7 +734,7 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     if (tid == 0) {
         s_flags[0] = 0;
         s_flags[7] = 0xffffffffu;  // *s_nimg = -1: items still running
-        for (int k = 0; k < 7; ++k) mbar_init(&bars[k], 1);
+        for (int k = 0; k < 10; ++k) mbar_init(&bars[k], 1);
         fence_mbarrier_init();
         prefetch_tmap(tm_q);
         prefetch_tmap(tm_k);
@@ -787,22 +788,22 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         const float b = *bp;
         return (PRO && (p.pro.flags & KDA_PROLOGUE_BETA_SIGMOID)) ? beta_from_raw(b) : b;
     };
-    // Hand-off of image n to the store thread: entry n % 2 = {head, chunk, QK buffer}, then an
-    // arrival on the img barrier. Entry n % 2 is rewritten only for image n + 2, after the store
-    // thread has released image n + 1's sources, which it does only after reading entry n; for
-    // the same reason the img barrier is never more than one phase ahead of the store thread.
-    // The end of the items is not an arrival (that could complete a second phase before the store
-    // thread has waited for the last image) but a count, *s_nimg = images handed over in all.
+    // Hand-off of image n to the store thread, in two parts: the key-side part (K^ and A, final
+    // once item n's A/L extraction is done) and the rest (M, U~, P, after item n's epilogue, one
+    // iteration later). Entry n % 2 = {head, chunk, QK buffer} is written with the first part and
+    // rewritten for image n + 2 only after the store thread has read image n + 1's first part
+    // (src1), by which time it has finished image n. img1 / img2: one arrival per part; src1 /
+    // srcM: the store thread has read the first part's sources / the rest's M, which may then be
+    // rewritten. The rest's P and U~ buffers take the next items' loads, which the store thread
+    // issues itself once it has read them (before M's copy, so the loads do not queue behind
+    // it): V of item n + 1 over U~, q/k of item n + 2 over P. Neither
+    // barrier gets two phases ahead of its waiters (each part of image n + 1 is handed over only
+    // after a wait for the same part of image n). The end of the items is not an arrival but a
+    // count, *s_nimg = images handed over in all.
     volatile int32_t *s_store = reinterpret_cast<volatile int32_t *>(s_flags + 8);
     volatile int32_t *s_nimg = reinterpret_cast<volatile int32_t *>(s_flags + 7);
-
-    uint32_t ph_qk[2] = {0, 0}, ph_la = 0, ph_v = 0, ph_mma = 0, ph_src = 0;
-    bool pend_qk[2] = {false, false}, pend_la = false, pend_v = false;
-    auto wait_bar = [&](uint64_t *bar, uint32_t &ph) {
-        const bool ok = mbar_wait_bounded(bar, ph, p.timeout_ns);
-        ph ^= 1u;
-        if (!ok) fail();
-    };
+    uint64_t *const b_mma = &bars[4], *const b_srcM = &bars[5], *const b_img2 = &bars[6];
+    uint64_t *const b_img1 = &bars[7], *const b_src1 = &bars[8], *const b_d1 = &bars[9];
 
     if (ctl) {
         const int k0 = claim();
@@ -817,135 +818,281 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     if (warp == STR / 32) {
         if (tid == STR) {
             // ------------------------------------------------ store thread
-            // Per image, in item order: wait until the compute threads have written it (img), wait
-            // for its ring slot's previous chunk to have been taken, store it (six bulk copies),
-            // let the sources be rewritten once the copies have read them (src), and publish it
-            // once they are complete.
-            mbar_arrive(&bars[5]);  // the first item's gating may write the image's sources
-            uint32_t ph_img = 0;
+            // Per image, in item order: the first part once handed over (after a wait for its
+            // ring slot's previous chunk to have been taken), then the rest; each part's sources
+            // are released once the copies have read them, and the image is published once all
+            // its copies are complete.
+            auto wait_part = [&](uint64_t *bar, uint32_t ph) -> bool {
+                const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
+                while (true) {
+                    if (mbar_try_wait(bar, ph)) return true;
+                    if (ld_volatile(&s_flags[0]) != 0 || globaltimer_ns() > deadline) return false;
+                    __nanosleep(64);
+                }
+            };
+            // Loads it issues: V of item i on bars[3] (phase i), q/k of item i on bars[i % 2] (phase
+            // i / 2); the last of each is waited for before the thread ends.
+            int last_v = -1, last_qk0 = -1, last_qk1 = -1;
+            auto load_v = [&](int i) {
+                if (s_rec[i & 3].hd < 0) return;
+                issue_v(s_rec[i & 3]);
+                last_v = i;
+            };
+            auto load_qk = [&](int i) {
+                if (s_rec[i & 3].hd < 0) return;
+                issue_qk(s_rec[i & 3], i & 1);
+                (i & 1 ? last_qk1 : last_qk0) = i;
+            };
+            load_v(0);   // into free buffers
+            load_qk(1);
+            uint32_t ph1 = 0, ph2 = 0;
             for (int n = 0;; ++n) {
-                // image n handed over, or the item loop ended with n images handed over
+                // image n's first part handed over, or the item loop ended with n images
                 bool have = false, ended = false;
                 const uint64_t deadline = globaltimer_ns() + p.timeout_ns;
                 while (true) {
-                    if (mbar_try_wait(&bars[6], ph_img)) { have = true; break; }
+                    if (mbar_try_wait(b_img1, ph1)) { have = true; break; }
                     const int ni = *s_nimg;
                     if (ni >= 0 && ni <= n) { ended = true; break; }
-                    if (globaltimer_ns() > deadline) break;
+                    if (ld_volatile(&s_flags[0]) != 0 || globaltimer_ns() > deadline) break;
                     __nanosleep(64);
                 }
                 if (!have) {
                     if (!ended) fail();
                     break;
                 }
-                ph_img ^= 1u;
+                ph1 ^= 1u;
                 volatile int32_t *e = s_store + 4 * (n & 1);
                 const int hd = e[0], c = e[1];
-                if (c >= RING && !wait_flag_ge(p.consumed + hd, c - RING + 1, p.timeout_ns)) {
+                const uint32_t b_img = (uint32_t)e[2];
+                bool ok = c < RING || wait_flag_ge(p.consumed + hd, c - RING + 1, p.timeout_ns);
+                uint8_t *slot = p.ring + ((size_t)hd * RING + (size_t)(c % RING)) * SLOT;
+                if (ok) {
+                    bulk_store(slot + SL_KH, sm + KH, 16384);
+                    bulk_store(slot + SL_A, sm + AQK, 8192);
+                    bulk_commit();
+                    bulk_wait_read();
+                }
+                mbar_arrive(b_src1);  // (also on failure: the compute threads then see the stop)
+                ok = ok && wait_part(b_img2, ph2);
+                ph2 ^= 1u;
+                if (ok) {  // P and U~ first: their buffers take the next items' loads
+                    const uint8_t *qkb = sm + (b_img ? QK1 : QK0);
+                    bulk_store(slot + SL_P, qkb, 8192);             // P, columns 0..63 (over Q~)
+                    bulk_store(slot + SL_P + 8192, qkb + 16384, 8192);  // and 64..127
+                    bulk_store(slot + SL_U, sm + VB, 16384);
+                    bulk_commit();
+                    bulk_wait_read();
+                    load_v(n + 1);
+                    load_qk(n + 2);
+                    bulk_store(slot + SL_M, sm + KI, 32768);       // M: K- and W regions, contiguous
+                    bulk_commit();
+                    bulk_wait_read();
+                }
+                mbar_arrive(b_srcM);
+                if (!ok) {
                     fail();
-                    mbar_arrive(&bars[5]);  // nothing was stored; let the compute threads see the stop
                     break;
                 }
-                uint8_t *slot = p.ring + ((size_t)hd * RING + (size_t)(c % RING)) * SLOT;
-                const uint32_t b_img = (uint32_t)e[2];
-                const uint8_t *qkb = sm + (b_img ? QK1 : QK0);
-                bulk_store(slot + SL_M, sm + KI, 32768);       // M: K- and -W regions, contiguous
-                bulk_store(slot + SL_KH, sm + KH, 16384);
-                bulk_store(slot + SL_U, sm + VB, 16384);
-                bulk_store(slot + SL_P, qkb, 8192);             // P, columns 0..63 (over Q~)
-                bulk_store(slot + SL_P + 8192, qkb + 16384, 8192);  // and 64..127
-                bulk_store(slot + SL_A, sm + AQK, 8192);
-                bulk_commit();
-                bulk_wait_read();
-                mbar_arrive(&bars[5]);  // the sources may be rewritten
                 bulk_wait_all();
                 fence_proxy_async_global();
                 __threadfence();
                 st_release(p.filled + hd * RING + (c % RING), c + 1);
             }
             bulk_wait_all();
+            if (last_v >= 0) mbar_wait_bounded(&bars[3], (uint32_t)(last_v & 1), p.timeout_ns);
+            if (last_qk0 >= 0) mbar_wait_bounded(&bars[0], (uint32_t)((last_qk0 >> 1) & 1), p.timeout_ns);
+            if (last_qk1 >= 0) mbar_wait_bounded(&bars[1], (uint32_t)((last_qk1 >> 1) & 1), p.timeout_ns);
         }
     } else {
-    if (s_rec[0].hd >= 0) pend_qk[0] = pend_la = true;
+    // Phase parities of the waited barriers and the control thread's loads in flight (q/k of item
+    // 0, log_alpha), as bits of one word (the loop is at the register limit): parity of bars[k]
+    // at bit k (k = 0..4: qk0, qk1, la, v, mma; bit 5: d1), load in flight at bit 8 + k. V and
+    // the later q/k loads are the store thread's, which waits for its own.
+    constexpr int B_MMA = 4, B_D1 = 5, PEND = 8;
+    uint32_t phs = 0;
+    auto wait_bar = [&](uint64_t *bar, int bit) {
+        const bool ok = mbar_wait_bounded(bar, (phs >> bit) & 1u, p.timeout_ns);
+        phs ^= 1u << bit;
+        if (!ok) fail();
+    };
+    auto pend = [&](int k, bool on) { phs = on ? (phs | (1u << (PEND + k))) : (phs & ~(1u << (PEND + k))); };
+    if (s_rec[0].hd >= 0) {
+        pend(0, true);
+        pend(2, true);
+    }
     float beta_next = (tid < C) ? load_beta(s_rec[0]) : 0.f;
-    int b = 0, n_img = 0;
-    for (int n = 0; s_rec[n & 3].hd >= 0; ++n) {
-        const ItemRec cur = s_rec[n & 3], nx = s_rec[(n + 1) & 3];
-        const int hd = cur.hd, c = cur.c, valid = cur.valid;
-        uint8_t *qk = sm + (b ? QK1 : QK0);
-        if (tid < C) s_beta[tid] = beta_next;
-        wait_bar(&bars[b], ph_qk[b]);
-        wait_bar(&bars[2], ph_la);
-        pend_qk[b] = pend_la = false;
+    int n_img = 0;
+    // Iteration n runs the early phases of item n (E) and the late phases of item n - 1 (P), so
+    // that each item's MMAs run while the compute threads work on the other item:
+    //   a. P: W -> its tile; D3/D4(P) issued
+    //   b. E: gating (D3/D4(P) run); D1(E) issued
+    //   c. P: epilogue (D1(E) runs); the rest of image P to the store thread
+    //   d. E: K^ to its tile, A and L; image E's first part to the store thread; log_alpha of E + 1
+    //   e. E: inverse; W(E) issued
+    // Item E's buffers: QK[n % 2], s_gamma[n % 2]; item P's: the others. Every phase ends with a
+    // barrier of the compute threads and the control warp.
+    for (int n = 0;; ++n) {
+        const ItemRec &cur = s_rec[n & 3], &nx = s_rec[(n + 1) & 3];  // read where used
+        const bool hasE = cur.hd >= 0, hasP = n > 0;
+        if (!hasE && !hasP) break;
+        uint8_t *const qkE = sm + ((n & 1) ? QK1 : QK0), *const qkP = sm + ((n & 1) ? QK0 : QK1);
+        float *const gamE = s_gamma + 128 * (n & 1), *const gamP = s_gamma + 128 * ((n - 1) & 1);
+        const uint32_t parP = (uint32_t)((n - 1) & 1), parPP = (uint32_t)(n & 1);  // phases of images n - 1, n - 2
+        uint32_t ph_d34 = 0;
 
-        if (tid < C) beta_next = load_beta(nx);
-        // K- goes to the L/T scratch (free until the A/L extraction, which follows D1) and K^ to the
-        // log_alpha buffer (free once the gating has read it; the next chunk's log_alpha is loaded
-        // after K^ has been copied to its image slot). So the factored gating writes nothing the
-        // previous image's stores may still be reading, and its wait for them (src) moves after D1.
-        const uint32_t src_par = ph_src;
-        if (compute) {
-            const int gate = gate_chunk<PRO, NTC, true>(qk, reinterpret_cast<uint8_t *>(LTp), sm + AQK,
-                                                        reinterpret_cast<float *>(sm + LA), LTp, s_beta,
-                                                        s_gamma, s_psum, s_flags, valid, tid, sm + LA, &bars[5],
-                                                        src_par, p.timeout_ns, p.pro);
-            if (gate < 0) atomicOr(p.status, 1);
-            if (tid == 0) s_flags[2] = (uint32_t)(gate + 1);
-            fence_proxy_async_smem();
-        }
-        ph_src ^= 1u;
-#ifdef KDA_TC_INVERSE
-        // the item after the next one, claimed while the compute threads run the gating (the
-        // control thread has a part in every round of the inverse); read by all after the
-        // following barriers. Record n + 2's slot was last read at the top of item n - 2.
-        if (ctl) put_rec(n + 2, nx.hd >= 0 ? claim() : -1);
-#endif
-        const bool stop = sync_work_or(ld_volatile(&s_flags[0]) != 0) != 0;
-        const int gate = (int)s_flags[2] - 1;
-        if (gate < 0 || stop) break;
-        const bool safe = gate == 1;
-        if (ctl) {
+        // ---- a. item n - 1: W -> its tile (over M's second half of image n - 2), then D3/D4:
+        // D3 = [T'; 0] V + [0; A] (-W) = [U~; -A W] and D4 = K^^T (-W)
+        if (hasP) {
+            wait_bar(b_mma, B_MMA);
             tc_fence_after();
-            if (!safe) {
+            if (compute) {
+                if (n >= 2 && !mbar_wait_bounded(b_srcM, parPP, p.timeout_ns)) fail();
+                rows64_to_tile<32>(tmem + lane_base + TM_W + 32 * part, sm + WN, 8192, 32 * part, quad, lane, -1.f);
+                fence_proxy_async_smem();
+            }
+            tc_fence_before();
+            sync_work();
+            if (ctl) {
+                if (!mbar_wait_bounded(&bars[3], (phs >> 3) & 1u, p.timeout_ns)) fail();
+                tc_fence_after();
+#pragma unroll
+                for (uint32_t kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tmem + TM_D3, desc_k(sb + TT, 16384, kk), desc_mn(sb + VB, 8192, kk), I_3, kk > 0);
+#pragma unroll
+                for (uint32_t kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tmem + TM_D3, desc_k(sb + ZB, 16384, kk), desc_mn(sb + WN, 8192, kk), I_3, 1);
+#pragma unroll
+                for (uint32_t kk = 0; kk < 4; ++kk)
+                    mma_bf16_ss(tmem + TM_D4, desc_mn(sb + KH, 8192, kk), desc_mn(sb + WN, 8192, kk), I_4, kk > 0);
+                mma_commit(b_mma);
+            }
+            phs ^= 1u << 3;
+            ph_d34 = (phs >> B_MMA) & 1u;
+        }
+
+        // ---- b. item n: the gating. K- goes to the L/T scratch and K^ to the log_alpha buffer,
+        // so the factored path writes nothing item n - 1 still needs; the exact path also writes A
+        // over item n - 1's, so it first waits for D3 (which reads it) and for the store thread.
+        if (hasE) {
+            if (tid < C) s_beta[tid] = beta_next;
+            wait_bar(&bars[n & 1], n & 1);
+            wait_bar(&bars[2], 2);
+            pend(n & 1, false);
+            pend(2, false);
+            if (tid < C) beta_next = load_beta(nx);
+            if (compute) {
+                const int g = gate_chunk<PRO, NTC, true>(qkE, reinterpret_cast<uint8_t *>(LTp), sm + AQK,
+                                                         reinterpret_cast<float *>(sm + LA), LTp, s_beta, gamE,
+                                                         s_psum, s_flags, cur.valid, tid, sm + LA,
+                                                         hasP ? b_mma : nullptr, ph_d34, p.timeout_ns, p.pro,
+                                                         hasP ? b_src1 : nullptr, parP);
+                if (g < 0) atomicOr(p.status, 1);
+                if (tid == 0) s_flags[2] = (uint32_t)(g + 1);
+                fence_proxy_async_smem();
+            }
+            // the item after the next one, claimed while the compute threads run the gating; read
+            // by all after the following barriers. Its record slot last served item n - 2.
+            if (ctl) put_rec(n + 2, nx.hd >= 0 ? claim() : -1);
+        }
+        if (sync_work_or(ld_volatile(&s_flags[0]) != 0)) break;
+        const int gate = hasE ? (int)s_flags[2] - 1 : 0;
+        if (gate < 0) break;
+        const bool exactE = gate == 1;
+        if (ctl && hasE) {
+            tc_fence_after();
+            if (!exactE) {
 #pragma unroll
                 for (uint32_t kk = 0; kk < 8; ++kk)
-                    mma_bf16_ss(tmem + TM_D1, desc_k(smem_u32(qk), 16384, kk),
-                                desc_k(sb + LT, 8192, kk), I_D1, kk > 0);
+                    mma_bf16_ss(tmem + TM_D1, desc_k(smem_u32(qkE), 16384, kk), desc_k(sb + LT, 8192, kk), I_D1,
+                                kk > 0);
             }
-            mma_commit(&bars[4]);
-            // once the previous image's stores have read their sources (V's buffer holds its U~,
-            // the other QK buffer its P): V of this chunk and q/k of the next one
-            if (!mbar_wait_bounded(&bars[5], src_par, p.timeout_ns)) fail();
-            issue_v(cur);
-            if (nx.hd >= 0) issue_qk(nx, b ^ 1);
+            mma_commit(b_d1);
         }
-        pend_v = true;
-        if (nx.hd >= 0) pend_qk[b ^ 1] = true;
-        wait_bar(&bars[4], ph_mma);
+
+        // ---- c. item n - 1: the epilogue. D3 rows 0..63: U~ [j][d] over V; rows 64..127: P =
+        // Q~ - A W over Q~; D4 -> M = diag(gamma - 1) - K^^T W [c][c'] over K- and W.
+        if (hasP) {
+            wait_bar(b_mma, B_MMA);
+            tc_fence_after();
+            if (compute) {
+                const int r = 32 * quad + lane;  // TMEM lane
+                const int col = 32 * part;       // this thread's 32 columns of D3 and D4
+                float v[32], m[32];  // both loads in flight before one wait
+                tmem_ld32(tmem + lane_base + TM_D3 + col, v);
+                tmem_ld32(tmem + lane_base + TM_D4 + col, m);
+                tmem_wait_ld();
+                if (r < 64) {
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8)
+                        st_chunk(sm + VB + tchunk(8192, r, col + 8 * q8), v + 8 * q8);
+                } else {
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        uint8_t *qp = qkP + tchunk(16384, r - 64, col + 8 * q8);
+                        const uint4 raw = *reinterpret_cast<const uint4 *>(qp);
+                        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
+                            v[8 * q8 + 2 * e] += f.x;
+                            v[8 * q8 + 2 * e + 1] += f.y;
+                        }
+                        st_chunk(qp, v + 8 * q8);
+                    }
+                }
+                const float gm1 = gamP[r] - 1.f;
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    if (col + e == r) m[e] += gm1;
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8)
+                    st_chunk(sm + KI + tchunk(16384, r, col + 8 * q8), m + 8 * q8);
+                fence_proxy_async_smem();  // written by generic stores; the copy-out is async
+            }
+            tc_fence_before();
+            if (sync_work_or(ld_volatile(&s_flags[0]) != 0)) break;
+            if (ctl) mbar_arrive(b_img2);
+        }
+        if (!hasE) break;  // the last item's late phases were the last work
+
+        // ---- d. item n: K^ to its tile and A, L from D1 (over item n - 1's K^ and A, once the
+        // store thread has taken them; D4 and D3, which read them too, are complete)
+        wait_bar(b_d1, B_D1);
         tc_fence_after();
         if (compute) {
-            // A, and K^ for D4, go to image sources: the previous image's stores must have read them
-            if (!mbar_wait_bounded(&bars[5], src_par, p.timeout_ns)) fail();
+            if (hasP && !mbar_wait_bounded(b_src1, parP, p.timeout_ns)) fail();
             for (int e = tid; e < 16384 / 16; e += NTC)  // K^: log_alpha buffer -> its image slot
                 reinterpret_cast<uint4 *>(sm + KH)[e] = reinterpret_cast<const uint4 *>(sm + LA)[e];
-            if (!safe)
+            if (!exactE)
                 extract_al<16>(tmem + lane_base + TM_D1 + 16 * part, sm + AQK, LTp, s_beta, 32 * quad + lane,
                                16 * part);
+            fence_proxy_async_smem();
         }
         tc_fence_before();
-        // L and A to the inverse: a barrier of the compute threads only (the control thread is
-        // still issuing the prefetches); the CTA-wide stop check follows the inverse
-        if (compute) sync_compute<NTC>();
+        if (sync_work_or(ld_volatile(&s_flags[0]) != 0)) break;
+        if (ctl) {
+            if (nx.hd >= 0) issue_la(nx);  // K^ has left the log_alpha buffer
+            volatile int32_t *e = s_store + 4 * (n & 1);
+            e[0] = cur.hd;
+            e[1] = cur.c;
+            e[2] = n & 1;
+            mbar_arrive(b_img1);
+        }
+        if (nx.hd >= 0) pend(2, true);
+        ++n_img;
 
+        // ---- e. item n: T' = (I + L)^-1 diag(beta), then W = T' K~
 #ifdef KDA_TC_INVERSE
-        // (build option) T' = (I + L)^-1 diag(beta) on the tensor cores, three rounds of MMAs (inv_tc_setup):
+        // (build option) on the tensor cores, three rounds of MMAs (inv_tc_setup):
         //   1: [N | D^-1] = D^-1 [L_off | I]            (one N = 128 MMA: D^-1 lands in TMEM)
         //   2: W1 = D^-1 - N D^-1 (onto D^-1), N2 = N N
         //   3: T = W1 + N2 W1 (onto W1) = (I + N2)(I - N) D^-1
-        // Tiles: D^-1 and L_off over K- (dead since D1), I and then N over -W (written after W),
-        // N2 and W1 over the L/T scratch (L is read in step 0). Accumulators: the W and D3
-        // columns, free until those MMAs.
+        // Tiles: D^-1 and L_off over K-, I and then N over W (both regions hold image n - 1's M
+        // until the store thread has read it), N2 and W1 over the L/T scratch (L is read in step
+        // 0). Accumulators: the W and D3 columns, free until those MMAs.
         if (compute) {
+            if (hasP && !mbar_wait_bounded(b_srcM, parP, p.timeout_ns)) fail();
             inv_tc_setup<NTC>(LTp, sm + IV_DINV, sm + IV_LOFF, tid, warp, sm + IV_EYE);
             fence_proxy_async_smem();
         }
@@ -956,9 +1103,9 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 #pragma unroll
             for (uint32_t kk = 0; kk < 4; ++kk)
                 mma_bf16_ss(tmem + TM_W, desc_k(sb + IV_DINV, 8192, kk), desc_mn(sb + IV_LOFF, 8192, kk), I_IV2, kk > 0);
-            mma_commit(&bars[4]);
+            mma_commit(b_mma);
         }
-        wait_bar(&bars[4], ph_mma);
+        wait_bar(b_mma, B_MMA);
         tc_fence_after();
         if (compute) {
             acc64_cols16_to_tile(tmem + lane_base + TM_W, sm + IV_N, 16 * part, quad, lane,
@@ -975,9 +1122,9 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 #pragma unroll
             for (uint32_t kk = 0; kk < 4; ++kk)  // N2 = N N
                 mma_bf16_ss(tmem + TM_D3, desc_k(sb + IV_N, 8192, kk), desc_mn(sb + IV_N, 8192, kk), I_IV, kk > 0);
-            mma_commit(&bars[4]);
+            mma_commit(b_mma);
         }
-        wait_bar(&bars[4], ph_mma);
+        wait_bar(b_mma, B_MMA);
         tc_fence_after();
         if (compute) {
             acc64_cols16_to_tile(tmem + lane_base + TM_W + 64, sm + IV_W1, 16 * part, quad, lane,
@@ -993,9 +1140,9 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
 #pragma unroll
             for (uint32_t kk = 0; kk < 4; ++kk)  // T = W1 + N2 W1
                 mma_bf16_ss(tmem + TM_W + 64, desc_k(sb + IV_N2, 8192, kk), desc_mn(sb + IV_W1, 8192, kk), I_IV, 1);
-            mma_commit(&bars[4]);
+            mma_commit(b_mma);
         }
-        wait_bar(&bars[4], ph_mma);
+        wait_bar(b_mma, B_MMA);
         tc_fence_after();
         if (compute) {
             acc64_cols16_to_tile(tmem + lane_base + TM_W + 64, sm + TT, 16 * part, quad, lane,
@@ -1004,9 +1151,6 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         }
         tc_fence_before();
 #else
-        // the item after the next one, claimed while the compute threads invert (the atomic's
-        // latency stays off their path); read by all after the following barriers
-        if (ctl) put_rec(n + 2, nx.hd >= 0 ? claim() : -1);
         if (compute) {
             // warps 0..3, one per SM sub-partition
             invert_unit_lower<NTC>(LTp, PBp, sm + TT, s_beta, tid, warp);
@@ -1014,105 +1158,22 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
         }
 #endif
         if (sync_work_or(ld_volatile(&s_flags[0]) != 0)) break;
-
         if (ctl) {
-            if (nx.hd >= 0) issue_la(nx);  // K^ has left the log_alpha buffer (copied before the inverse)
             tc_fence_after();
 #pragma unroll
             for (uint32_t kk = 0; kk < 4; ++kk)  // W = T' K~
-                mma_bf16_ss(tmem + TM_W, desc_k(sb + TT, 8192, kk),
-                            desc_mn(smem_u32(qk) + 8192, 16384, kk), I_W, kk > 0);
-            mma_commit(&bars[4]);
+                mma_bf16_ss(tmem + TM_W, desc_k(sb + TT, 8192, kk), desc_mn(smem_u32(qkE) + 8192, 16384, kk), I_W,
+                            kk > 0);
+            mma_commit(b_mma);
         }
-        if (nx.hd >= 0) pend_la = true;
-        wait_bar(&bars[4], ph_mma);
-        tc_fence_after();
-        if (compute) {
-            rows64_to_tile<32>(tmem + lane_base + TM_W + 32 * part, sm + WN, 8192, 32 * part, quad, lane, -1.f);
-            fence_proxy_async_smem();
-        }
-        tc_fence_before();
-        sync_work();
-
-        // D3 = [T'; 0] V + [0; A] (-W) = [U~; -A W] and D4 = K^^T (-W)
-        if (ctl) {
-            if (!mbar_wait_bounded(&bars[3], ph_v, p.timeout_ns)) fail();
-            tc_fence_after();
-#pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_D3, desc_k(sb + TT, 16384, kk), desc_mn(sb + VB, 8192, kk), I_3, kk > 0);
-#pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_D3, desc_k(sb + ZB, 16384, kk), desc_mn(sb + WN, 8192, kk), I_3, 1);
-#pragma unroll
-            for (uint32_t kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(tmem + TM_D4, desc_mn(sb + KH, 8192, kk), desc_mn(sb + WN, 8192, kk), I_4, kk > 0);
-            mma_commit(&bars[4]);
-        }
-        ph_v ^= 1u;
-        pend_v = false;
-        wait_bar(&bars[4], ph_mma);
-        tc_fence_after();
-        if (compute) {
-            const int r = 32 * quad + lane;  // TMEM lane
-            const int col = 32 * part;       // this thread's 32 columns of D3 and D4
-            // D3 rows 0..63: U~ [j][d] over V; rows 64..127: P = Q~ - A W over Q~; D4 -> M =
-            // diag(gamma - 1) - K^^T W [c][c'] over K- and -W (both loads in flight before one wait)
-            float v[32], m[32];
-            tmem_ld32(tmem + lane_base + TM_D3 + col, v);
-            tmem_ld32(tmem + lane_base + TM_D4 + col, m);
-            tmem_wait_ld();
-            if (r < 64) {
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8)
-                    st_chunk(sm + VB + tchunk(8192, r, col + 8 * q8), v + 8 * q8);
-            } else {
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    uint8_t *qp = qk + tchunk(16384, r - 64, col + 8 * q8);
-                    const uint4 raw = *reinterpret_cast<const uint4 *>(qp);
-                    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
-                        v[8 * q8 + 2 * e] += f.x;
-                        v[8 * q8 + 2 * e + 1] += f.y;
-                    }
-                    st_chunk(qp, v + 8 * q8);
-                }
-            }
-            const float gm1 = s_gamma[r] - 1.f;
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-                if (col + e == r) m[e] += gm1;
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8)
-                st_chunk(sm + KI + tchunk(16384, r, col + 8 * q8), m + 8 * q8);
-            fence_proxy_async_smem();  // written by generic stores; the copy-out is async
-        }
-        tc_fence_before();
-        if (sync_work_or(ld_volatile(&s_flags[0]) != 0)) break;
-        // the image is in shared memory (written by generic stores, each followed by a proxy
-        // fence): hand it to the store thread
-        if (ctl) {
-            volatile int32_t *e = s_store + 4 * (n_img & 1);
-            e[0] = hd;
-            e[1] = c;
-            e[2] = b;
-            mbar_arrive(&bars[6]);
-        }
-        ++n_img;
-        b ^= 1;
     }
 
     if (ctl) {
         *s_nimg = n_img;  // no more images: the store thread ends after image n_img - 1
-        for (int k = 0; k < 2; ++k)
-            if (pend_qk[k]) mbar_wait_bounded(&bars[k], ph_qk[k], p.timeout_ns);
-        if (pend_la) mbar_wait_bounded(&bars[2], ph_la, p.timeout_ns);
-        if (pend_v) mbar_wait_bounded(&bars[3], ph_v, p.timeout_ns);
-        mma_commit(&bars[4]);
-        mbar_wait_bounded(&bars[4], ph_mma, p.timeout_ns);
+        for (int k = 0; k < 3; k += 2)  // q/k of item 0, log_alpha
+            if ((phs >> (PEND + k)) & 1u) mbar_wait_bounded(&bars[k], (phs >> k) & 1u, p.timeout_ns);
+        mma_commit(b_mma);
+        mbar_wait_bounded(b_mma, (phs >> B_MMA) & 1u, p.timeout_ns);
     }
     }  // the work warps
     tc_fence_before();
