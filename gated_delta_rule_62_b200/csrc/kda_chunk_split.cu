@@ -38,7 +38,10 @@ namespace {
 using namespace sm100;
 using namespace chunk;
 
-constexpr int RING = 8;
+// Ring depth, in chunks per head. Producers work about RING / 2 chunks ahead of the consumers;
+// a deeper ring keeps a slow consumer from stalling the producers' two items in flight (16 and
+// 8 measured the same where the consumers keep up).
+constexpr int RING = 16;
 // Chunk image (bytes), the same in a ring slot and in a consumer stage (bf16, 128-byte
 // swizzled tiles):
 //   [0, 32K)     M [c][c'] (K-major A operand, 128 rows, 64-column blocks of 16 KB)
