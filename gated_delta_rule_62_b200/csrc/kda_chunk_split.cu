@@ -38,10 +38,10 @@ namespace {
 using namespace sm100;
 using namespace chunk;
 
-// Ring depth, in chunks per head. Producers work about RING / 2 chunks ahead of the consumers;
-// a deeper ring keeps a slow consumer from stalling the producers' two items in flight (16 and
-// 8 measured the same where the consumers keep up).
-constexpr int RING = 16;
+// Ring depth, in chunks per head. 8 keeps the ring (22.5 MiB for 32 heads) resident in L2 next to
+// the streaming inputs; with 16 it spilled (DRAM writes per 8192 x 32 launch: 58 -> 267 MB) for
+// no gain in time.
+constexpr int RING = 8;
 // Chunk image (bytes), the same in a ring slot and in a consumer stage (bf16, 128-byte
 // swizzled tiles):
 //   [0, 32K)     M [c][c'] (K-major A operand, 128 rows, 64-column blocks of 16 KB)

@@ -80,7 +80,7 @@ typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
 /*
  * Bytes of device workspace that let kda_prefill take its fastest path for this
  * problem (a multiple of 256). Problems with few (sequence, head) pairs get room
- * for the split-role kernel's ring of chunk images (1.4 MiB per pair); any
+ * for the split-role kernel's ring of chunk images (704 KiB per pair); any
  * workspace of at least 256 + 4 * num_seqs bytes (rounded up to 256) is accepted,
  * and a smaller one than returned here selects the single-role kernel. Host
  * function: queries the current device's SM count; returns 0 only for
