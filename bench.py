@@ -51,8 +51,8 @@ FLOP_PER_TOKEN_HEAD = 180224
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
 # dram__bytes_read.sum + dram__bytes_write.sum of one split_kernel launch on the headline workload,
 # from one ncu capture; reported only while the kernel's sources are the ones it was taken on.
-SPLIT_TRAFFIC_BYTES = 336.774912e6 + 58.243840e6
-SPLIT_TRAFFIC_SOURCES_SHA256 = "34acba495bb3d2818013416b7ff4e3a997b229c4380d0fac297f968426637e40"
+SPLIT_TRAFFIC_BYTES = 336.793344e6 + 57.800960e6
+SPLIT_TRAFFIC_SOURCES_SHA256 = "b2f297d2fee5ee9f2806f9329fd306755629ad35a8b38e3168ab78114da37288"
 
 
 def measured_traffic():
