@@ -19,13 +19,19 @@
 namespace kda {
 namespace {
 
+// Value columns evolve independently, so d_v = 128 splits into two blocks of 64 columns (256
+// threads: four blocks per SM in flight instead of two of 512); the row groups R, and with them
+// the order of every sum, stay those of one 512-thread block over all columns.
 template <int DK, int DV>
 struct DecodeShape {
-    static constexpr int CG = DV / 4;                            // float4 column groups per row
-    static constexpr int NT = (CG * DK < 512) ? CG * DK : 512;   // threads per block
+    static constexpr int SW = DV == 128 ? 64 : DV;               // value columns per block
+    static constexpr int NSLICE = DV / SW;                       // blocks per head
+    static constexpr int CG = SW / 4;                            // float4 column groups per row
+    static constexpr int NTMAX = DV == 128 ? 256 : 512;
+    static constexpr int NT = (CG * DK < NTMAX) ? CG * DK : NTMAX;  // threads per block
     static constexpr int R = NT / CG;                            // row groups
     static constexpr int RPT = DK / R;                           // rows per thread
-    static_assert(NT % 32 == 0 && DK % R == 0, "bad decode shape");
+    static_assert(NT % 32 == 0 && DK % R == 0 && DV % SW == 0, "bad decode shape");
 };
 
 template <typename Tin, int DK, int DV>
@@ -35,13 +41,14 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
               float *__restrict__ state, Tin *__restrict__ out, int H, const StateSlots ss,
               const DebugRanges dbg) {
     using Sh = DecodeShape<DK, DV>;
-    constexpr int CG = Sh::CG, NT = Sh::NT, R = Sh::R, RPT = Sh::RPT;
+    constexpr int SW = Sh::SW, CG = Sh::CG, NT = Sh::NT, R = Sh::R, RPT = Sh::RPT;
     __shared__ float s_k[DK], s_q[DK], s_a[DK];
-    __shared__ __align__(16) float s_red[2][R][DV];
-    __shared__ __align__(16) float s_u[DV];
+    __shared__ __align__(16) float s_red[2][R][SW];
+    __shared__ __align__(16) float s_u[SW];
     __shared__ float s_kq;
 
     const size_t head = blockIdx.x;  // n * H + h
+    const int col0 = blockIdx.y * SW;  // this block's value columns
     const int tid = threadIdx.x;
     const int cg = tid % CG, rg = tid / CG;
     // Launched with programmatic stream serialization: the next decode step's blocks may become
@@ -53,13 +60,13 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     // this head's state: entry `head`, or its sequence's slot of the pool (none: zeros, not stored)
     float *blk = final_state_block(state, (int)(head / H), H, (int)(head % H), (size_t)(DK * DV), ss);
     if (blk && !KDA_ACCESS_OK(ss.status, dbg.fin, blk, DK * DV * 4, 31)) blk = nullptr;
-    float4 *S4 = reinterpret_cast<float4 *>(blk);
+    float4 *S4 = blk ? reinterpret_cast<float4 *>(blk + col0) : nullptr;
 
     // Issue the state loads first: they are the only long-latency traffic.
     float4 s[RPT];
 #pragma unroll
     for (int i = 0; i < RPT; ++i)
-        s[i] = blk ? __ldcs(&S4[(size_t)(rg + i * R) * CG + cg]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        s[i] = S4 ? __ldcs(&S4[(size_t)(rg + i * R) * (DV / 4) + cg]) : make_float4(0.f, 0.f, 0.f, 0.f);
 
     for (int c = tid; c < DK; c += NT) {
         s_k[c] = to_f32(k[head * DK + c]);
@@ -90,14 +97,14 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     }
     __syncthreads();
 
-    if (tid < DV) {
+    if (tid < SW) {
         float a = 0.f, b = 0.f;
 #pragma unroll 8
         for (int r = 0; r < R; ++r) { a += s_red[0][r][tid]; b += s_red[1][r][tid]; }
-        const float u = beta[head] * (to_f32(v[head * DV + tid]) - a);
+        const size_t o = head * DV + col0 + tid;
+        const float u = beta[head] * (to_f32(v[o]) - a);
         s_u[tid] = u;
-        if (KDA_ACCESS_OK(ss.status, dbg.out, out + head * DV + tid, sizeof(Tin), 32))
-            out[head * DV + tid] = from_f32<Tin>(fmaf(s_kq, u, b));
+        if (KDA_ACCESS_OK(ss.status, dbg.out, out + o, sizeof(Tin), 32)) out[o] = from_f32<Tin>(fmaf(s_kq, u, b));
     }
     __syncthreads();
 
@@ -107,7 +114,7 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
         const float kc = s_k[rg + i * R];
         s[i].x = fmaf(kc, u4.x, s[i].x); s[i].y = fmaf(kc, u4.y, s[i].y);
         s[i].z = fmaf(kc, u4.z, s[i].z); s[i].w = fmaf(kc, u4.w, s[i].w);
-        if (blk) __stcs(&S4[(size_t)(rg + i * R) * CG + cg], s[i]);
+        if (S4) __stcs(&S4[(size_t)(rg + i * R) * (DV / 4) + cg], s[i]);
     }
 }
 
@@ -352,7 +359,7 @@ cudaError_t launch_verify3(const VerifyProblem &p, cudaStream_t stream) {
 template <typename Tin, int DK, int DV>
 cudaError_t launch3(const DecodeProblem &p, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)p.num_seqs * (unsigned)p.H);
+    cfg.gridDim = dim3((unsigned)p.num_seqs * (unsigned)p.H, DecodeShape<DK, DV>::NSLICE);
     cfg.blockDim = dim3(DecodeShape<DK, DV>::NT);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
