@@ -123,6 +123,26 @@ def test_adversarial_decay(pattern, lens, H):
     assert_close(fs, ref_s, TOL["bf16"], vmax(inp), f"{pattern} state")
 
 
+# 8192 tokens x 4 heads: 512 chunk items over the split kernel's producers, several per producer,
+# so an exact-path item (which writes A over the previous item's, after waiting for it) follows
+# factored and exact ones inside one producer's two-item pipeline.
+@pytest.mark.parametrize("pattern", ["alternate_chunks", "mix_0_-20"])
+def test_exact_path_items_in_one_producer(pattern):
+    wl = W.custom((8192,), 4, 128, 128, "bf16", seed=17, init_state="normal")
+    inp = W.make_inputs(wl, DEV)
+    la = inp["log_alpha"]
+    if pattern == "alternate_chunks":  # even chunks decay by e^-1280 (exact path), odd ones not at all
+        chunk = torch.arange(la.shape[0], device=DEV) // 64
+        la.copy_(torch.where((chunk % 2 == 0)[:, None, None], torch.full_like(la, -20.0), torch.zeros_like(la)))
+    else:
+        g = torch.Generator(device=DEV).manual_seed(5)
+        la.copy_(torch.where(torch.rand(la.shape, device=DEV, generator=g) < 0.5, 0.0, -20.0))
+    out, fs = gpu_prefill(inp)
+    ref_o, ref_s = oracle_forward(inp)
+    assert_close(out, ref_o, TOL["bf16"], vmax(inp), f"{pattern} out")
+    assert_close(fs, ref_s, TOL["bf16"], vmax(inp), f"{pattern} state")
+
+
 def test_noop_gates_keep_state():
     """alpha = 1, beta = 0 on the GPU: the state passes through unchanged."""
     wl = W.custom((130,), 2, 128, 128, "bf16", seed=12, init_state="normal")
