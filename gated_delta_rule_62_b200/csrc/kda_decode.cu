@@ -131,9 +131,11 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
 // with the decode kernel's row groups: each column's sums run over the same rows in the same
 // order, and small blocks (128 threads for d_v = 128) let several heads' token loops overlap
 // on one SM while others wait for their states.
-template <int DK, int DV>
+// WIDE (the commit-only launch, which has no sums over rows): the decode kernel's column blocks,
+// whose rows a warp reads in longer pieces.
+template <int DK, int DV, bool WIDE = false>
 struct VerifyShape {
-    static constexpr int SW = DV < 32 ? DV : 32;       // value columns per block
+    static constexpr int SW = WIDE ? DecodeShape<DK, DV>::SW : (DV < 32 ? DV : 32);  // value columns per block
     static constexpr int NSLICE = DV / SW;
     static constexpr int CG = SW / 4;                  // float4 column groups per row
     static constexpr int R = DecodeShape<DK, DV>::R;   // row groups, as in the decode kernel
@@ -147,9 +149,9 @@ struct VerifyShape {
 // [T_prev][DK] as pairs and u [T_prev][SW] (commit). Every region starts on a 16-byte boundary.
 // The pairs feed the paired fp32 instructions (two columns of the state per instruction), whose
 // lanes round exactly as the scalar ones: results stay those of the decode kernel, bit for bit.
-template <int DK, int DV>
+template <int DK, int DV, bool WIDE = false>
 struct SpecSmem {
-    static constexpr int SW = VerifyShape<DK, DV>::SW;
+    static constexpr int SW = VerifyShape<DK, DV, WIDE>::SW;
     int k, q, a, v, b, ck, ca, cu, total;
     __host__ __device__ constexpr SpecSmem(int T, int TP)
         : k(0), q(2 * T * DK), a(4 * T * DK), v(6 * T * DK), b(6 * T * DK + T * SW),
@@ -176,15 +178,15 @@ __device__ __forceinline__ float4 exp4(float4 x) {
 // COMMIT: advance the state by accepted[n] tokens of the previous draft (k, alpha, u) and store
 // it; VERIFY: run the T draft tokens from the (advanced) state, writing out and u_cache.
 template <typename Tin, int DK, int DV, bool COMMIT, bool VERIFY>
-__global__ void __launch_bounds__(VerifyShape<DK, DV>::NT) spec_kernel(const VerifyProblem p) {
-    using Sh = VerifyShape<DK, DV>;
+__global__ void __launch_bounds__(VerifyShape<DK, DV, COMMIT && !VERIFY>::NT) spec_kernel(const VerifyProblem p) {
+    using Sh = VerifyShape<DK, DV, COMMIT && !VERIFY>;
     constexpr int SW = Sh::SW, CG = Sh::CG, NT = Sh::NT, R = Sh::R, RPT = Sh::RPT;
     extern __shared__ __align__(16) float s_in[];
     __shared__ __align__(16) float2 s_red[R][SW];  // (S'^T k, S'^T q) partials per row group
     __shared__ __align__(16) float s_u[SW];
     __shared__ float s_kq;
     const int T = VERIFY ? p.T : 0, TP = COMMIT ? p.T_prev : 0, H = p.H;
-    const SpecSmem<DK, DV> L(T, TP);
+    const SpecSmem<DK, DV, COMMIT && !VERIFY> L(T, TP);
     float2 *s_k = reinterpret_cast<float2 *>(s_in + L.k), *s_q = reinterpret_cast<float2 *>(s_in + L.q),
            *s_a = reinterpret_cast<float2 *>(s_in + L.a);
     float *s_v = s_in + L.v, *s_b = s_in + L.b, *c_u = s_in + L.cu;
@@ -337,9 +339,9 @@ __global__ void __launch_bounds__(VerifyShape<DK, DV>::NT) spec_kernel(const Ver
 
 template <typename Tin, int DK, int DV, bool COMMIT, bool VERIFY>
 cudaError_t launch_spec(const VerifyProblem &p, cudaStream_t stream) {
-    using VS = VerifyShape<DK, DV>;
+    using VS = VerifyShape<DK, DV, COMMIT && !VERIFY>;
     auto kern = spec_kernel<Tin, DK, DV, COMMIT, VERIFY>;
-    const SpecSmem<DK, DV> L(VERIFY ? p.T : 0, COMMIT ? p.T_prev : 0);
+    const SpecSmem<DK, DV, COMMIT && !VERIFY> L(VERIFY ? p.T : 0, COMMIT ? p.T_prev : 0);
     if (L.cu % 4 != 0) return cudaErrorInvalidValue;  // float4 reads of the u rows
     const size_t smem = (size_t)L.total * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
