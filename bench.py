@@ -67,10 +67,10 @@ DECODE_BYTES_PER_TOKEN_HEAD = 2 * 128 * 128 * 4 + 3 * 128 * 2 + 128 * 4 + 4 + 12
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of each decode-side kernel on the
 # decode workload (ncu, one capture each), reported while kda_decode.cu and kda_internal.cuh hash
 # to the sources they were taken on.
-DECODE_SIDE_TRAFFIC = {"decode": 547.586e6 + 477.467e6, "verify": 580.507e6 + 5.873e6,
-                       "commit": 603.117e6 + 477.143e6,
-                       "commit_verify": 801.749e6 + 502.264e6}
-DECODE_SIDE_SOURCES_SHA256 = "0d0bef4abea69a9a2ec91560ffa31de7be0b1a92157e1e02ccb65cdc2cd8cd4a"
+DECODE_SIDE_TRAFFIC = {"decode": 547.598e6 + 477.494e6, "verify": 580.534e6 + 5.976e6,
+                       "commit": 591.556e6 + 475.534e6,
+                       "commit_verify": 801.722e6 + 502.169e6}
+DECODE_SIDE_SOURCES_SHA256 = "acacbb0fe0ec21eb1a777d768e3e51901ad5783020300f3fc7625988517b8e0a"
 
 
 def decode_side_traffic(kernel):
