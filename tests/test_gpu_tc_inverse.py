@@ -3,7 +3,7 @@
 Its split-role prefill computes T = (I + L)^-1 of each chunk with three rounds of tcgen05 MMAs,
 T = (I + N^2)(I - N) D^-1 with N = D^-1 L_off, instead of the warp-level tf32 block merges. The
 default build keeps the merges (they are faster: the MMA rounds add about 2,000 cycles to every
-producer item). This build must still match the oracle on every kernel family."""
+producer item). The option's library must still match the oracle on every kernel family."""
 import os
 import subprocess
 import sys
