@@ -13,7 +13,8 @@
 //     A and L, T' = (I + L)^-1 diag(beta), W = T' K~, then U~ and -A W in one M=128 MMA
 //     ([T'; 0] V + [0; A] (-W)) and -K^^T W in another, and from those U~, P and M as
 //     ready-to-use shared-memory images (bf16) in a ring of RING slots per head in the
-//     workspace (L2 resident).
+//     workspace (L2 resident). Each producer keeps two items in flight, so that one item's
+//     MMAs run while the compute warps work on the other (see the producer).
 //   consumer CTAs (one per head): the chain. Per chunk: S += M S_b + K^^T U~ (S_b = the
 //     state's bf16 copy, fed from tensor memory), O = P S_b + A U~ behind it; the outputs leave
 //     while the next chunk's chain runs. The fp32 state stays in TMEM for the whole sequence.
@@ -648,9 +649,11 @@ static_assert(IV_EYE == WN && IV_N2 % 1024 == 0 && IV_W1 + 8192 <= MISC, "invers
 }  // namespace prod
 
 // Producer roles: the compute threads run the gating, the TMEM epilogues and the inverse; the
-// control thread claims the items and issues the TMA loads and the MMAs; the store thread waits
-// for a free ring slot, copies each finished image out with bulk stores and publishes it. The
-// phases of one item are separated by barriers of the compute threads and the control warp.
+// control thread claims the items, issues the MMAs, the log_alpha loads and the first item's
+// q/k; the store thread waits for a free ring slot, copies each image out in two parts with bulk
+// stores, issues the next items' V and q/k loads into the buffers it has just read, and
+// publishes the image. The phases are separated by barriers of the compute threads and the
+// control warp.
 template <bool PRO>
 __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
                          const CUtensorMap *tm_la, const SplitParams &p, uint8_t *sm, int pid, int nprod) {
