@@ -62,14 +62,16 @@ struct Smem {
     static constexpr uint32_t BYTES = MISC + MISC_BYTES + 1024;  // + alignment slack
 };
 
-// TMEM columns (fp32, 128 lanes). DS <= 64: O has its own columns; DS = 128: O reuses W's.
+// TMEM columns (fp32, 128 lanes). DS <= 64: O has its own columns; DS = 128: O takes D1's
+// columns and the 64 after them, free once A and L are out of D1, so O = Q~ S runs during the
+// inverse.
 template <int DS>
 struct Tmem {
     static constexpr uint32_t S = 0;
-    static constexpr uint32_t D1 = 128;
-    static constexpr uint32_t U = 192;
+    static constexpr uint32_t U = DS <= 64 ? 192 : 128;
     static constexpr uint32_t W = U + DS;
-    static constexpr uint32_t O = DS <= 64 ? W + 128 : W;
+    static constexpr uint32_t D1 = DS <= 64 ? 128 : W + 128;
+    static constexpr uint32_t O = DS <= 64 ? W + 128 : D1;
     static constexpr uint32_t COLS = 512;
     static_assert(O + DS <= COLS && W + 128 <= COLS, "TMEM overflow");
 };
@@ -295,6 +297,13 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         tc_fence_before();
         __syncthreads();
         if (s_flags[0]) break;
+        if (DS > 64 && tid == 0) {  // O = Q~ S over D1's columns, while the inverse runs
+            tc_fence_after();
+#pragma unroll
+            for (uint32_t kk = 0; kk < 8; ++kk)
+                mma_bf16_ss(tmem + TM::O, desc_k(sb + SM::QK, 16384, kk),
+                            desc_mn(sb + SM::S, 16384, kk), I_UT, kk > 0);
+        }
 
         // ---- T' = (I + L)^-1 diag(beta), bf16, into the TT tile
         invert_unit_lower(LT, PB, sm + SM::TT, s_beta, tid, tid >> 5);
@@ -319,10 +328,10 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         tc_fence_after();
         if (tid == 0 && has_next) {
             issue_v(t0 + C);
-            if (DS <= 64) issue_qk(t0 + C);  // Q~ and K~ are consumed
+            issue_qk(t0 + C);  // Q~ and K~ are consumed (O = Q~ S was issued before W)
         }
         v_pending = has_next;
-        if (DS <= 64) qk_pending = has_next;
+        qk_pending = has_next;
 
         // ---- W (TMEM, M=64: row 16*quad + lane for lane < 16) -> bf16 tile [i][c]
         rows64_to_tile<64>(tmem + lane_base + TM::W + 64 * half, sm + SM::W, 8192, 64 * half, quad, lane);
@@ -337,20 +346,10 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             for (uint32_t kk = 0; kk < 8; ++kk)  // U = U~ - W S
                 mma_bf16_ss(tmem + TM::U, desc_k(sb + SM::W, 8192, kk),
                             desc_mn(sb + SM::S, 16384, kk), I_UWS, 1);
-            if (DS > 64) {  // O = Q~ S (W's columns are free now)
-#pragma unroll
-                for (uint32_t kk = 0; kk < 8; ++kk)
-                    mma_bf16_ss(tmem + TM::O, desc_k(sb + SM::QK, 16384, kk),
-                                desc_mn(sb + SM::S, 16384, kk), I_UT, kk > 0);
-            }
             mma_commit(bar_mma);
         }
         wait_bar(bar_mma, ph_mma);
         tc_fence_after();
-        if (DS > 64) {
-            if (tid == 0 && has_next) issue_qk(t0 + C);
-            qk_pending = has_next;
-        }
 
         // ---- U (TMEM, M=64) -> bf16 tile [j][d]
         rows64_to_tile<SCOLS>(tmem + lane_base + TM::U + half * SCOLS, sm + SM::U, 8192, half * SCOLS, quad, lane);
