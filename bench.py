@@ -51,8 +51,8 @@ FLOP_PER_TOKEN_HEAD = 180224
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
 # dram__bytes_read.sum + dram__bytes_write.sum of one split_kernel launch on the headline workload,
 # from one ncu capture; reported only while the kernel's sources are the ones it was taken on.
-SPLIT_TRAFFIC_BYTES = 336.793344e6 + 57.800960e6
-SPLIT_TRAFFIC_SOURCES_SHA256 = "a7662d03785d999c792f9ec934d72fe199b60be2b14563594b901852d3f07ccb"
+SPLIT_TRAFFIC_BYTES = 336.741120e6 + 51.381760e6
+SPLIT_TRAFFIC_SOURCES_SHA256 = "93fdc61cadc5583014e5934869761f77e0add4e6d44ac973e6d3bd6dfe1394d0"
 
 
 def measured_traffic():

@@ -89,6 +89,11 @@ __device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t 
                  "r"(bytes)
                  : "memory");
 }
+// Output element store with the streaming (evict-first) cache hint: outputs are not read again
+// here, so they should not push the ring's images out of L2.
+__device__ __forceinline__ void st_stream_bf16(__nv_bfloat16 *dst, float x) {
+    __stcs(reinterpret_cast<unsigned short *>(dst), __bfloat16_as_ushort(__float2bfloat16_rn(x)));
+}
 // Waits until the committed TMA stores have finished reading shared memory / are complete.
 __device__ __forceinline__ void bulk_wait_read() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
@@ -212,8 +217,8 @@ __device__ void consumer(const SplitParams &p, uint8_t *sm, int hd) {
                 st_release(p.consumed + hd, c - 1);
             }
             const uint8_t *src = p.ring + ((size_t)hd * RING + (size_t)(c % RING)) * SLOT;
-            mbar_arrive_expect_tx(&bars[b], SLOT);
-            bulk_load(sm + (b ? STAGE1 : STAGE0), src, SLOT, &bars[b]);
+            mbar_arrive_expect_tx(&bars[b], SLOT);  // an image is dead once read: evict-first
+            bulk_load_pol(sm + (b ? STAGE1 : STAGE0), src, SLOT, &bars[b], l2_evict_first());
             requested = c + 1;
         }
         // the last images land before the CTA exits (the MMA thread may have stopped early)
@@ -351,7 +356,7 @@ __device__ void consumer(const SplitParams &p, uint8_t *sm, int hd) {
 #pragma unroll
             for (int t = 0; t < 32; ++t)
                 if (t < vc && KDA_ACCESS_OK(p.status, p.dbg.out, dst + (size_t)t * H * D, 2, 3))
-                    dst[(size_t)t * H * D] = __float2bfloat16_rn(vv[t]);
+                    st_stream_bf16(dst + (size_t)t * H * D, vv[t]);
         }
         tc_fence_before();
     }
@@ -433,8 +438,8 @@ __device__ void consumer_seg(const SplitParams &p, uint8_t *sm, int hd, int4 vi)
                 st_release(p.consumed + hd, c - 1);
             }
             const uint8_t *src = p.ring + ((size_t)hd * RING + (size_t)(c % RING)) * SLOT;
-            mbar_arrive_expect_tx(&bars[b], SLOT);
-            bulk_load(sm + (b ? STAGE1 : STAGE0), src, SLOT, &bars[b]);
+            mbar_arrive_expect_tx(&bars[b], SLOT);  // an image is dead once read: evict-first
+            bulk_load_pol(sm + (b ? STAGE1 : STAGE0), src, SLOT, &bars[b], l2_evict_first());
             requested = c + 1;
         }
         for (int c = requested - 2 < 0 ? 0 : requested - 2; c < requested; ++c)
@@ -610,7 +615,7 @@ __device__ void consumer_seg(const SplitParams &p, uint8_t *sm, int hd, int4 vi)
 #pragma unroll
             for (int t = 0; t < 32; ++t)
                 if (t < vc && KDA_ACCESS_OK(p.status, p.dbg.out, dst + (size_t)t * H * D, 2, 7))
-                    dst[(size_t)t * H * D] = __float2bfloat16_rn(x[t]);
+                    st_stream_bf16(dst + (size_t)t * H * D, x[t]);
         }
         tc_fence_before();
     }
@@ -763,29 +768,30 @@ __device__ void producer(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const
     };
 
     // control thread; each buffer's previous contents were read by generic loads or bulk stores
-    // that have completed (see the call sites)
+    // that have completed (see the call sites). Inputs are read once: evict-first, so that the
+    // stream of them does not push the ring's images out of L2.
     auto issue_qk = [&](const ItemRec &r, int b) {
         const int h = r.h, t0 = r.t0;
         uint8_t *qk = sm + (b ? QK1 : QK0);
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&bars[b], 32768);
-        tma_load_3d(qk, tm_q, &bars[b], 0, h, (int32_t)t0);
-        tma_load_3d(qk + 8192, tm_k, &bars[b], 0, h, (int32_t)t0);
-        tma_load_3d(qk + 16384, tm_q, &bars[b], 64, h, (int32_t)t0);
-        tma_load_3d(qk + 24576, tm_k, &bars[b], 64, h, (int32_t)t0);
+        tma_load_3d_pol(qk, tm_q, &bars[b], 0, h, (int32_t)t0, l2_evict_first());
+        tma_load_3d_pol(qk + 8192, tm_k, &bars[b], 0, h, (int32_t)t0, l2_evict_first());
+        tma_load_3d_pol(qk + 16384, tm_q, &bars[b], 64, h, (int32_t)t0, l2_evict_first());
+        tma_load_3d_pol(qk + 24576, tm_k, &bars[b], 64, h, (int32_t)t0, l2_evict_first());
     };
     auto issue_la = [&](const ItemRec &r) {
         const int h = r.h, t0 = r.t0;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&bars[2], 32768);
-        tma_load_3d(sm + LA, tm_la, &bars[2], 0, h, (int32_t)t0);
+        tma_load_3d_pol(sm + LA, tm_la, &bars[2], 0, h, (int32_t)t0, l2_evict_first());
     };
     auto issue_v = [&](const ItemRec &r) {
         const int h = r.h, t0 = r.t0;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&bars[3], 16384);
-        tma_load_3d(sm + VB, tm_v, &bars[3], 0, h, (int32_t)t0);
-        tma_load_3d(sm + VB + 8192, tm_v, &bars[3], 64, h, (int32_t)t0);
+        tma_load_3d_pol(sm + VB, tm_v, &bars[3], 0, h, (int32_t)t0, l2_evict_first());
+        tma_load_3d_pol(sm + VB + 8192, tm_v, &bars[3], 64, h, (int32_t)t0, l2_evict_first());
     };
     auto load_beta = [&](const ItemRec &r) -> float {  // tid < C
         if (r.hd < 0 || tid >= r.valid) return 0.f;
