@@ -51,8 +51,8 @@ FLOP_PER_TOKEN_HEAD = 180224
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
 # dram__bytes_read.sum + dram__bytes_write.sum of one split_kernel launch on the headline workload,
 # from one ncu capture; reported only while the kernel's sources are the ones it was taken on.
-SPLIT_TRAFFIC_BYTES = 336.741120e6 + 51.381760e6
-SPLIT_TRAFFIC_SOURCES_SHA256 = "93fdc61cadc5583014e5934869761f77e0add4e6d44ac973e6d3bd6dfe1394d0"
+SPLIT_TRAFFIC_BYTES = 336.748544e6 + 49.859584e6
+SPLIT_TRAFFIC_SOURCES_SHA256 = "ddc082409a8fd43cccaf9bcce4873eaadbcbdbef286dcd6068fc345e9687afee"
 
 
 def measured_traffic():

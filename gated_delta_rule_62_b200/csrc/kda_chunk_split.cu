@@ -1207,14 +1207,21 @@ split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     // 1024-byte aligned (128-byte swizzled tiles); offsetting the shared array itself keeps the
     // accesses in the shared state space (an integer round trip would make them generic)
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    if ((int)blockIdx.x < p.heads) {
-        const int4 vi = p.vinfo ? p.vinfo[blockIdx.x / p.H] : make_int4(0, 0, 1, 0);
+    // The consumers are the last `heads` blocks. Measured on two B200s (plain 1M-token, 16-head
+    // prefill): consumers as the first blocks 24.5 and 31.9 ms, as the last blocks 20.7 and 20.8 ms,
+    // spread evenly over the grid 29.3 ms (first GPU). The first blocks of a launch are
+    // spread over the whole chip, so consumers among them probably share their part of the chip
+    // (and its path to L2) with busy producers; the last blocks fill the SMs left over.
+    const int first_cons = (int)gridDim.x - p.heads;
+    if ((int)blockIdx.x >= first_cons) {
+        const int hd = (int)blockIdx.x - first_cons;
+        const int4 vi = p.vinfo ? p.vinfo[hd / p.H] : make_int4(0, 0, 1, 0);
         if (vi.y > 0)
-            consumer_seg(p, sm, blockIdx.x, vi);
+            consumer_seg(p, sm, hd, vi);
         else
-            consumer(p, sm, blockIdx.x);
+            consumer(p, sm, hd);
     } else
-        producer<PRO>(&tm_q, &tm_k, &tm_v, &tm_la, p, sm, blockIdx.x - p.heads, gridDim.x - p.heads);
+        producer<PRO>(&tm_q, &tm_k, &tm_v, &tm_la, p, sm, blockIdx.x, first_cons);
 }
 
 // Zeroes the status word and the ring flags.
