@@ -51,8 +51,8 @@ FLOP_PER_TOKEN_HEAD = 180224
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 128 * 2 + 128 * 4 + 4 + 128 * 2
 # dram__bytes_read.sum + dram__bytes_write.sum of one split_kernel launch on the headline workload,
 # from one ncu capture; reported only while the kernel's sources are the ones it was taken on.
-SPLIT_TRAFFIC_BYTES = 336.748544e6 + 49.859584e6
-SPLIT_TRAFFIC_SOURCES_SHA256 = "ddc082409a8fd43cccaf9bcce4873eaadbcbdbef286dcd6068fc345e9687afee"
+SPLIT_TRAFFIC_BYTES = 336.804608e6 + 50.913024e6
+SPLIT_TRAFFIC_SOURCES_SHA256 = "7683404149faad35199e5ccbd9a0e4dd95ec1ce1c2eee23bbcabf33862b6a71d"
 
 
 def measured_traffic():

@@ -217,8 +217,8 @@ __device__ void consumer(const SplitParams &p, uint8_t *sm, int hd) {
                 st_release(p.consumed + hd, c - 1);
             }
             const uint8_t *src = p.ring + ((size_t)hd * RING + (size_t)(c % RING)) * SLOT;
-            mbar_arrive_expect_tx(&bars[b], SLOT);  // an image is dead once read: evict-first
-            bulk_load_pol(sm + (b ? STAGE1 : STAGE0), src, SLOT, &bars[b], l2_evict_first());
+            mbar_arrive_expect_tx(&bars[b], SLOT);
+            bulk_load(sm + (b ? STAGE1 : STAGE0), src, SLOT, &bars[b]);
             requested = c + 1;
         }
         // the last images land before the CTA exits (the MMA thread may have stopped early)
@@ -438,8 +438,8 @@ __device__ void consumer_seg(const SplitParams &p, uint8_t *sm, int hd, int4 vi)
                 st_release(p.consumed + hd, c - 1);
             }
             const uint8_t *src = p.ring + ((size_t)hd * RING + (size_t)(c % RING)) * SLOT;
-            mbar_arrive_expect_tx(&bars[b], SLOT);  // an image is dead once read: evict-first
-            bulk_load_pol(sm + (b ? STAGE1 : STAGE0), src, SLOT, &bars[b], l2_evict_first());
+            mbar_arrive_expect_tx(&bars[b], SLOT);
+            bulk_load(sm + (b ? STAGE1 : STAGE0), src, SLOT, &bars[b]);
             requested = c + 1;
         }
         for (int c = requested - 2 < 0 ? 0 : requested - 2; c < requested; ++c)

@@ -95,23 +95,13 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
 }
 
 // ---------------------------------------------------------------- L2 eviction priority
-// Cache policies for the copies below: data read or written once is marked evict-first so
-// that it does not push out lines another CTA still needs.
+// Cache policy for the copies below: data read once is marked evict-first so that it does not
+// push out lines another CTA still needs.
 __device__ __forceinline__ uint64_t l2_evict_first() {
     uint64_t pol;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
     return pol;
 }
-// bulk_load with an L2 cache policy
-__device__ __forceinline__ void bulk_load_pol(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
-                                              uint64_t pol) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
-            "r"(smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
-        : "memory");
-}
-
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
